@@ -1,0 +1,373 @@
+// Host layer of the C ABI: argument validation, array sizes, layout derivation and
+// kernel dispatch.  No allocation, no synchronisation, no global state.
+#include <cstring>
+
+#include "kvq_internal.cuh"
+
+using namespace kvq;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int dtype_bytes(int dt) { return dt == KVQ_F32 ? 4 : 2; }
+
+bool valid_dtype(int dt) { return dt == KVQ_F32 || dt == KVQ_F16 || dt == KVQ_BF16; }
+
+// Per-side check: returns KVQ_OK / KVQ_ERR_INVALID / KVQ_ERR_UNSUPPORTED.
+kvq_status check_side(const kvq_format* f, int which) {
+  const int scheme = which == KVQ_KEYS ? f->k_scheme : f->v_scheme;
+  const int bits = which == KVQ_KEYS ? f->k_bits : f->v_bits;
+  const int axis = which == KVQ_KEYS ? f->k_axis : f->v_axis;
+  const int nout = which == KVQ_KEYS ? f->k_outliers : f->v_outliers;
+  const int want_axis = which == KVQ_KEYS ? KVQ_AXIS_CHANNEL : KVQ_AXIS_TOKEN;
+  switch (scheme) {
+    case KVQ_NONE:
+      return nout == 0 ? KVQ_OK : KVQ_ERR_INVALID;
+    case KVQ_SYM8:
+      if (bits != 8 || nout != 0) return KVQ_ERR_INVALID;
+      if (axis < KVQ_AXIS_TENSOR || axis > KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID;
+      return KVQ_OK;
+    case KVQ_ASYM:
+      if (bits != 2 && bits != 4 && bits != 8) return KVQ_ERR_INVALID;
+      if (nout != 0) return KVQ_ERR_INVALID;
+      if (axis < KVQ_AXIS_TENSOR || axis > KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID;
+      return axis == want_axis ? KVQ_OK : KVQ_ERR_UNSUPPORTED;
+    case KVQ_NUQ:
+      if (bits != 3 || nout < 0 || nout > 8) return KVQ_ERR_INVALID;
+      if (axis < KVQ_AXIS_TENSOR || axis > KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID;
+      if (which == KVQ_KEYS && nout > f->group_tokens) return KVQ_ERR_INVALID;
+      return axis == want_axis ? KVQ_OK : KVQ_ERR_UNSUPPORTED;
+    case KVQ_MIXED: {
+      if (which != KVQ_KEYS) return KVQ_ERR_UNSUPPORTED;
+      if (f->src_dtype == KVQ_F32) return KVQ_ERR_UNSUPPORTED;
+      const int lo = f->head_dim - f->mixed_hi - f->mixed_mid;
+      if (f->mixed_hi < 0 || f->mixed_mid < 0 || lo < 0) return KVQ_ERR_INVALID;
+      if (f->mixed_hi % 8 || f->mixed_mid % 8 || lo % 16) return KVQ_ERR_INVALID;
+      return KVQ_OK;
+    }
+    default:
+      return KVQ_ERR_INVALID;
+  }
+}
+
+int64_t code_row_bytes(const kvq_format* f, int which) {
+  const int scheme = which == KVQ_KEYS ? f->k_scheme : f->v_scheme;
+  const int bits = which == KVQ_KEYS ? f->k_bits : f->v_bits;
+  const int D = f->head_dim;
+  switch (scheme) {
+    case KVQ_NONE: return (int64_t)D * dtype_bytes(f->src_dtype);
+    case KVQ_SYM8: return D;
+    case KVQ_ASYM: return (int64_t)D * bits / 8;
+    case KVQ_NUQ: return 3 * (int64_t)D / 8;
+    case KVQ_MIXED: {
+      const int lo = D - f->mixed_hi - f->mixed_mid;
+      return 2 * f->mixed_hi + f->mixed_mid / 2 + lo / 4;
+    }
+  }
+  return 0;
+}
+
+// (scale elements, zero elements) per slab
+void meta_elems(const kvq_format* f, int which, int64_t C, int64_t* ns, int64_t* nz) {
+  const int scheme = which == KVQ_KEYS ? f->k_scheme : f->v_scheme;
+  const int axis = which == KVQ_KEYS ? f->k_axis : f->v_axis;
+  const int64_t ng = C / f->group_tokens, D = f->head_dim;
+  *ns = *nz = 0;
+  if (scheme == KVQ_SYM8) {
+    *ns = axis == KVQ_AXIS_TENSOR ? ng : axis == KVQ_AXIS_TOKEN ? C : ng * D;
+  } else if (scheme == KVQ_ASYM || scheme == KVQ_NUQ) {
+    *ns = *nz = axis == KVQ_AXIS_CHANNEL ? ng * D : C;
+  } else if (scheme == KVQ_MIXED) {
+    *ns = *nz = ng * (D - f->mixed_hi);
+  }
+}
+
+int meta_elem_bytes(const kvq_format* f, int which) {
+  const int scheme = which == KVQ_KEYS ? f->k_scheme : f->v_scheme;
+  return scheme == KVQ_SYM8 ? 4 : 2;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kvq_version(void) { return (KVQ_VERSION_MAJOR << 16) | KVQ_VERSION_MINOR; }
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported format or shape";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_format_check(const kvq_format* f) {
+  if (!f) return KVQ_ERR_INVALID;
+  const int D = f->head_dim, g = f->group_tokens;
+  if (D != 32 && D != 64 && D != 128 && D != 256) return KVQ_ERR_INVALID;
+  if (g < 16 || g > 256 || g % 16 || (int64_t)g * D > 32768) return KVQ_ERR_INVALID;
+  if (!valid_dtype(f->src_dtype)) return KVQ_ERR_INVALID;
+  if (f->n_sink < 0 || f->n_sink > 4096 || f->residual_cap < 0 || f->residual_cap > (1 << 20))
+    return KVQ_ERR_INVALID;
+  if (f->rope != 0 && f->rope != 1) return KVQ_ERR_INVALID;
+  if (f->rope && !(f->rope_base > 1.0f)) return KVQ_ERR_INVALID;
+  if (f->rope && D < 64) return KVQ_ERR_UNSUPPORTED;
+  kvq_status a = check_side(f, KVQ_KEYS);
+  if (a == KVQ_ERR_INVALID) return a;
+  kvq_status b = check_side(f, KVQ_VALUES);
+  if (b == KVQ_ERR_INVALID) return b;
+  if (a != KVQ_OK) return a;
+  return b;
+}
+
+size_t kvq_cache_array_bytes(const kvq_format* f, int32_t B, int32_t H, int64_t C, int32_t id) {
+  if (kvq_format_check(f) != KVQ_OK || B <= 0 || H <= 0 || C < 0 || C % f->group_tokens)
+    return 0;
+  const int64_t slabs = (int64_t)B * H, D = f->head_dim, g = f->group_tokens, ng = C / g;
+  const int64_t raw = dtype_bytes(f->src_dtype);
+  int64_t ns, nz;
+  const bool kout = f->k_scheme == KVQ_NUQ && f->k_outliers > 0;
+  const bool vout = f->v_scheme == KVQ_NUQ && f->v_outliers > 0;
+  switch (id) {
+    case KVQ_ARR_K_CODES: return slabs * C * code_row_bytes(f, KVQ_KEYS);
+    case KVQ_ARR_V_CODES: return slabs * C * code_row_bytes(f, KVQ_VALUES);
+    case KVQ_ARR_K_SCALE: meta_elems(f, KVQ_KEYS, C, &ns, &nz); return slabs * ns * meta_elem_bytes(f, KVQ_KEYS);
+    case KVQ_ARR_K_ZERO: meta_elems(f, KVQ_KEYS, C, &ns, &nz); return slabs * nz * 2;
+    case KVQ_ARR_V_SCALE: meta_elems(f, KVQ_VALUES, C, &ns, &nz); return slabs * ns * meta_elem_bytes(f, KVQ_VALUES);
+    case KVQ_ARR_V_ZERO: meta_elems(f, KVQ_VALUES, C, &ns, &nz); return slabs * nz * 2;
+    case KVQ_ARR_K_ORDER: return f->k_scheme == KVQ_MIXED ? slabs * ng * D : 0;
+    case KVQ_ARR_K_OUT_ROWPTR: return kout ? slabs * ng * (g + 1) * 4 : 0;
+    case KVQ_ARR_K_OUT_COL: return kout ? slabs * ng * D * f->k_outliers : 0;
+    case KVQ_ARR_K_OUT_VAL: return kout ? slabs * ng * D * f->k_outliers * 2 : 0;
+    case KVQ_ARR_V_OUT_COL: return vout ? slabs * C * f->v_outliers : 0;
+    case KVQ_ARR_V_OUT_VAL: return vout ? slabs * C * f->v_outliers * 2 : 0;
+    case KVQ_ARR_K_LUT: return f->k_scheme == KVQ_NUQ ? 16 : 0;
+    case KVQ_ARR_V_LUT: return f->v_scheme == KVQ_NUQ ? 16 : 0;
+    case KVQ_ARR_SINK_K:
+    case KVQ_ARR_SINK_V: return slabs * f->n_sink * D * raw;
+    case KVQ_ARR_RES_K:
+    case KVQ_ARR_RES_V: return slabs * f->residual_cap * D * raw;
+  }
+  return 0;
+}
+
+}  // extern "C"
+
+namespace kvq {
+
+kvq_status make_layout(const kvq_format* f, const kvq_cache* c, Layout* L) {
+  kvq_status st = kvq_format_check(f);
+  if (st != KVQ_OK) return st;
+  if (!c || c->batch <= 0 || c->kv_heads <= 0 || c->capacity < 0 ||
+      c->capacity % f->group_tokens)
+    return KVQ_ERR_INVALID;
+  std::memset(L, 0, sizeof(*L));
+  L->D = f->head_dim;
+  L->g = f->group_tokens;
+  L->src_dtype = f->src_dtype;
+  L->raw_bytes = dtype_bytes(f->src_dtype);
+  L->B = c->batch;
+  L->Hkv = c->kv_heads;
+  L->C = c->capacity;
+  L->ng = (int)(c->capacity / f->group_tokens);
+  L->n_sink = f->n_sink;
+  L->res_cap = f->residual_cap;
+  L->rope = f->rope;
+  L->rope_base = f->rope_base;
+  L->mixed_hi = f->mixed_hi;
+  L->mixed_mid = f->mixed_mid;
+  L->mixed_lo = f->head_dim - f->mixed_hi - f->mixed_mid;
+  L->mixed_group_bytes = (int)(f->group_tokens * code_row_bytes(f, KVQ_KEYS));
+  for (int w = 0; w < 2; ++w) {
+    Side& s = L->side[w];
+    s.scheme = w == 0 ? f->k_scheme : f->v_scheme;
+    s.bits = w == 0 ? f->k_bits : f->v_bits;
+    s.axis = w == 0 ? f->k_axis : f->v_axis;
+    s.nout = s.scheme == KVQ_NUQ ? (w == 0 ? f->k_outliers : f->v_outliers) : 0;
+    s.code_row_bytes = (int)code_row_bytes(f, w);
+    s.code_slab_bytes = s.code_row_bytes * c->capacity;
+    int64_t ns, nz;
+    meta_elems(f, w, c->capacity, &ns, &nz);
+    s.meta_slab_elems = ns;
+    s.codes = w == 0 ? c->k_codes : c->v_codes;
+    s.scale = w == 0 ? c->k_scale : c->v_scale;
+    s.zero = w == 0 ? c->k_zero : c->v_zero;
+    s.lut = reinterpret_cast<const __half*>(w == 0 ? c->k_lut : c->v_lut);
+    if (!s.codes || !aligned16(s.codes)) return KVQ_ERR_INVALID;
+    if (ns && (!s.scale || !aligned16(s.scale))) return KVQ_ERR_INVALID;
+    if (nz && (!s.zero || !aligned16(s.zero))) return KVQ_ERR_INVALID;
+    if (s.scheme == KVQ_NUQ && (!s.lut || !aligned16(s.lut))) return KVQ_ERR_INVALID;
+  }
+  L->k_order = reinterpret_cast<uint8_t*>(c->k_order);
+  if (f->k_scheme == KVQ_MIXED && (!L->k_order || !aligned16(L->k_order))) return KVQ_ERR_INVALID;
+  if (f->k_scheme == KVQ_NUQ && f->k_outliers > 0) {
+    L->k_out_rowptr = reinterpret_cast<int32_t*>(c->k_out_rowptr);
+    L->k_out_col = reinterpret_cast<uint8_t*>(c->k_out_col);
+    L->k_out_val = reinterpret_cast<__half*>(c->k_out_val);
+    if (!L->k_out_rowptr || !L->k_out_col || !L->k_out_val || !aligned16(L->k_out_rowptr) ||
+        !aligned16(L->k_out_col) || !aligned16(L->k_out_val))
+      return KVQ_ERR_INVALID;
+  }
+  if (f->v_scheme == KVQ_NUQ && f->v_outliers > 0) {
+    L->v_out_col = reinterpret_cast<uint8_t*>(c->v_out_col);
+    L->v_out_val = reinterpret_cast<__half*>(c->v_out_val);
+    if (!L->v_out_col || !L->v_out_val || !aligned16(L->v_out_col) || !aligned16(L->v_out_val))
+      return KVQ_ERR_INVALID;
+  }
+  L->sink[0] = c->sink_k;
+  L->sink[1] = c->sink_v;
+  L->res[0] = c->res_k;
+  L->res[1] = c->res_v;
+  return KVQ_OK;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+}  // namespace kvq
+
+extern "C" {
+
+static kvq_status quantize_common(int which, const kvq_format* f, const kvq_cache* c,
+                                  const void* src, int64_t sb, int64_t sh, int64_t st,
+                                  int64_t t0, int64_t n, int32_t* d_status, void* stream) {
+  Layout L;
+  kvq_status s = make_layout(f, c, &L);
+  if (s != KVQ_OK) return s;
+  if (n < 0 || t0 < 0 || t0 % L.g || t0 + n > L.C) return KVQ_ERR_INVALID;
+  if (n == 0) return KVQ_OK;
+  if (!src || !aligned16(src)) return KVQ_ERR_INVALID;
+  const int64_t eb = dtype_bytes(L.src_dtype);
+  if (st < L.D || sb < 0 || sh < 0) return KVQ_ERR_INVALID;
+  if ((st * eb) % 16 || (sh * eb) % 16 || (sb * eb) % 16) return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  cudaError_t e = launch_quantize(L, which, src, sb, sh, st, t0, n, d_status,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_quantize_keys(const kvq_format* f, const kvq_cache* c, const void* src,
+                             int64_t sb, int64_t sh, int64_t st, int64_t t0, int64_t n,
+                             int32_t* d_status, void* stream) {
+  return quantize_common(KVQ_KEYS, f, c, src, sb, sh, st, t0, n, d_status, stream);
+}
+
+kvq_status kvq_quantize_values(const kvq_format* f, const kvq_cache* c, const void* src,
+                               int64_t sb, int64_t sh, int64_t st, int64_t t0, int64_t n,
+                               int32_t* d_status, void* stream) {
+  return quantize_common(KVQ_VALUES, f, c, src, sb, sh, st, t0, n, d_status, stream);
+}
+
+kvq_status kvq_dequantize(const kvq_format* f, const kvq_cache* c, int32_t which, int64_t t0,
+                          int64_t n, void* out, int32_t out_dtype, int32_t* d_status,
+                          void* stream) {
+  Layout L;
+  kvq_status s = make_layout(f, c, &L);
+  if (s != KVQ_OK) return s;
+  if (which != KVQ_KEYS && which != KVQ_VALUES) return KVQ_ERR_INVALID;
+  if (n < 0 || t0 < 0 || t0 + n > L.C) return KVQ_ERR_INVALID;
+  if (!valid_dtype(out_dtype)) return KVQ_ERR_INVALID;
+  if (n == 0) return KVQ_OK;
+  if (!out || !aligned16(out)) return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  cudaError_t e = launch_dequantize(L, which, t0, n, out, out_dtype, d_status,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_key_salience(const kvq_format* f, const void* q, int64_t qsb, int64_t qsh,
+                            int64_t qst, const void* k, int64_t ksb, int64_t ksh, int64_t kst,
+                            int32_t B, int32_t Hq, int32_t Hkv, int32_t R, double* sal,
+                            uint8_t* order, int64_t osb, int64_t osh, int32_t* d_status,
+                            void* stream) {
+  kvq_status s = kvq_format_check(f);
+  if (s != KVQ_OK) return s;
+  if (!q || !k || !order || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || R <= 0)
+    return KVQ_ERR_INVALID;
+  const int D = f->head_dim;
+  if (qst < D || kst < D || qsb < 0 || qsh < 0 || ksb < 0 || ksh < 0 || osb < 0 || osh < 0)
+    return KVQ_ERR_INVALID;
+  if (sal && (reinterpret_cast<uintptr_t>(sal) & 7)) return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  Layout L;
+  std::memset(&L, 0, sizeof(L));
+  L.D = D;
+  L.src_dtype = f->src_dtype;
+  cudaError_t e = launch_salience(L, q, qsb, qsh, qst, k, ksb, ksh, kst, B, Hq, Hkv, R, sal,
+                                  order, osb, osh, d_status,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+static kvq_status decode_args(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,
+                              int64_t t_quant, int32_t t_res, int32_t num_splits) {
+  kvq_status s = kvq_format_check(f);
+  if (s != KVQ_OK) return s;
+  if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv) return KVQ_ERR_INVALID;
+  if ((int64_t)(Hq / Hkv) * f->head_dim > 2048 || Hq / Hkv > 16) return KVQ_ERR_UNSUPPORTED;
+  if (t_quant < 0 || t_res < 0 || t_res > f->residual_cap || num_splits < 0)
+    return KVQ_ERR_INVALID;
+  if (f->n_sink + t_quant + t_res <= 0) return KVQ_ERR_INVALID;
+  return KVQ_OK;
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,
+                                  int64_t t_quant, int32_t t_res, int32_t num_splits) {
+  if (decode_args(f, B, Hq, Hkv, t_quant, t_res, num_splits) != KVQ_OK) return 0;
+  Layout L;
+  std::memset(&L, 0, sizeof(L));
+  L.D = f->head_dim;
+  L.g = f->group_tokens;
+  L.B = B;
+  L.Hkv = Hkv;
+  L.n_sink = f->n_sink;
+  L.side[0].scheme = f->k_scheme;
+  L.side[0].bits = f->k_bits;
+  L.side[0].axis = f->k_axis;
+  L.side[0].nout = f->k_scheme == KVQ_NUQ ? f->k_outliers : 0;
+  L.side[1].scheme = f->v_scheme;
+  L.side[1].bits = f->v_bits;
+  L.side[1].axis = f->v_axis;
+  L.side[1].nout = f->v_scheme == KVQ_NUQ ? f->v_outliers : 0;
+  L.rope = f->rope;
+  L.src_dtype = f->src_dtype;
+  DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
+  return workspace_bytes(L, Hq, p);
+}
+
+kvq_status kvq_decode_attention(const kvq_format* f, const kvq_cache* c, const void* q,
+                                int32_t q_dtype, int32_t Hq, int64_t t_quant, int32_t t_res,
+                                float scale, void* out, int32_t out_dtype, void* ws,
+                                size_t ws_bytes, int32_t num_splits, int32_t* d_status,
+                                void* stream) {
+  Layout L;
+  kvq_status s = make_layout(f, c, &L);
+  if (s != KVQ_OK) return s;
+  s = decode_args(f, L.B, Hq, L.Hkv, t_quant, t_res, num_splits);
+  if (s != KVQ_OK) return s;
+  if (t_quant > L.C) return KVQ_ERR_INVALID;
+  if (!q || !aligned16(q) || !out || !aligned16(out) || !valid_dtype(q_dtype) ||
+      !valid_dtype(out_dtype) || !(scale > 0.0f))
+    return KVQ_ERR_INVALID;
+  if (L.n_sink && (!L.sink[0] || !L.sink[1] || !aligned16(L.sink[0]) || !aligned16(L.sink[1])))
+    return KVQ_ERR_INVALID;
+  if (t_res && (!L.res[0] || !L.res[1] || !aligned16(L.res[0]) || !aligned16(L.res[1])))
+    return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
+  if (!ws || !aligned16(ws)) return KVQ_ERR_INVALID;
+  if (ws_bytes < workspace_bytes(L, Hq, p)) return KVQ_ERR_WORKSPACE;
+  cudaError_t e = launch_decode(L, p, q, q_dtype, Hq, t_quant, t_res, scale, out, out_dtype, ws,
+                                d_status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,407 @@
+// Split-KV decode attention: the generic path (any format, CUDA cores, fp32), the
+// cross-split combine, planning and dispatch.
+//
+//   out[h] = sum_t softmax_t(scale * q[h] . k^_t) v^_t      [AXES] "Separate the two
+//   error paths"; over sink + packed + residual tokens ([KVQ] "Approach", [MIX] Fig. 4).
+//
+// Partial softmax states are kept in the log2 domain (the query is pre-multiplied by
+// scale * log2(e)): per split and query head, m = max score, l = sum 2^(s - m),
+// o[d] = sum 2^(s - m) v[d].  The combine merges the splits with the usual
+// log-sum-exp rescaling.  Splits never wait on one another.
+#include <cmath>
+
+#include "decode_common.cuh"
+
+namespace kvq {
+
+// Fast tensor-core path (decode_mma.cu)
+bool mma_path_ok(const Layout& L, int Hq);
+int mma_ctas_per_sm();
+cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
+                              int Hq, int64_t t_quant, int t_res, float scale, float* ws_m,
+                              float* ws_l, float* ws_o, int32_t* d_status, cudaStream_t s);
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecArgs {
+  Layout L;
+  const void* q;
+  int q_dtype, Hq;
+  int64_t t_quant;
+  int t_res;
+  float qscale;          // softmax scale * log2(e)
+  int S, split_groups, n_packed, raw_slot;
+  float* ws_m;
+  float* ws_l;
+  float* ws_o;
+  int32_t* status;
+};
+
+template <int NC, int GM_>
+struct WarpState {
+  // query and accumulators of up to GM heads, NC channels per lane (c = lane + 32 j)
+  static constexpr int GM = GM_;
+  float q[GM][NC];
+  float o[GM][NC];
+  float m[GM], l[GM];
+};
+
+// Process one token of the current KV head: kh / vh are the lane's key / value
+// channels (already reconstructed and, for keys, rotated).
+template <int NC, int GM>
+__device__ __forceinline__ void consume_token(WarpState<NC, GM>& st, int G, const float* kh,
+                                              const float* vh) {
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    if (hh < G) {
+      float part = 0.0f;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) part = fmaf(st.q[hh][j], kh[j], part);
+      const float s = warp_sum(part);
+      if (s > st.m[hh]) {
+        const float corr = exp2f(st.m[hh] - s);   // 0 when m = -inf
+        st.l[hh] = st.l[hh] * corr + 1.0f;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) st.o[hh][j] = fmaf(st.o[hh][j], corr, vh[j]);
+        st.m[hh] = s;
+      } else {
+        const float p = exp2f(s - st.m[hh]);
+        st.l[hh] += p;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) st.o[hh][j] = fmaf(p, vh[j], st.o[hh][j]);
+      }
+    }
+  }
+}
+
+// Rotate-half RoPE of the lane's key channels at absolute position pos: channel pairs
+// (c, c + D/2) are both owned by the lane (j and j + NC/2).
+template <int NC>
+__device__ __forceinline__ void rope(float* kh, const double* theta, int64_t pos) {
+#pragma unroll
+  for (int j = 0; j < NC / 2; ++j) {
+    double sn, cs;
+    sincos((double)pos * theta[j], &sn, &cs);
+    const float c = (float)cs, s = (float)sn;
+    const float x1 = kh[j], x2 = kh[j + NC / 2];
+    kh[j] = x1 * c - x2 * s;
+    kh[j + NC / 2] = x2 * c + x1 * s;
+  }
+}
+
+template <int NC, int GM>
+__global__ void __launch_bounds__(kWarps * 32) decode_generic_kernel(DecArgs a) {
+  extern __shared__ __align__(16) float smem[];
+  const Layout& L = a.L;
+  const int D = L.D;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = a.Hq / L.Hkv;
+  const int64_t sl = (int64_t)b * L.Hkv + h;
+  int* inv = reinterpret_cast<int*>(smem);                 // [D] channel -> slot (MIXED)
+  float* wst = smem + 256;                                  // [kWarps][G][D + 2]
+
+  WarpState<NC, GM> st;
+  int bad = 0;
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    st.m[hh] = -INFINITY;
+    st.l[hh] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      st.o[hh][j] = 0.0f;
+      float x = 0.0f;
+      if (hh < G) {
+        x = load_elem(a.q, ((int64_t)b * a.Hq + h * G + hh) * D + lane + 32 * j, a.q_dtype);
+        bad |= !isfinite(x);
+      }
+      st.q[hh][j] = x * a.qscale;
+    }
+  }
+  double theta[NC / 2 > 0 ? NC / 2 : 1];
+  if (L.rope) {
+#pragma unroll
+    for (int j = 0; j < NC / 2; ++j)
+      theta[j] = pow((double)L.rope_base, -2.0 * (double)(lane + 32 * j) / (double)D);
+  }
+  float kh[NC], vh[NC];
+
+  if (split < a.n_packed) {
+    const int64_t ngv = (a.t_quant + L.g - 1) / L.g;
+    const int64_t g0 = (int64_t)split * a.split_groups;
+    const int64_t g1 = min(ngv, g0 + a.split_groups);
+    const Side& SK = L.side[0];
+    const Side& SV = L.side[1];
+    for (int64_t gi = g0; gi < g1; ++gi) {
+      if (SK.scheme == KVQ_MIXED) {
+        __syncthreads();
+        for (int j = threadIdx.x; j < D; j += blockDim.x) inv[L.k_order[(sl * L.ng + gi) * D + j]] = j;
+        __syncthreads();
+      }
+      const int64_t tb = gi * L.g, te = min(a.t_quant, tb + L.g);
+      for (int64_t t = tb + warp; t < te; t += kWarps) {
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+          const int c = lane + 32 * j;
+          kh[j] = SK.scheme == KVQ_MIXED ? mixed_slot_value(L, sl, t, inv[c]) : deq_dense(L, 0, sl, t, c);
+          vh[j] = deq_dense(L, 1, sl, t, c);
+        }
+        if (SK.nout > 0) {
+          const int rr = (int)(t - tb);
+          const int32_t* rp = L.k_out_rowptr + (sl * L.ng + gi) * (L.g + 1);
+          const int64_t e0 = (sl * L.ng + gi) * (int64_t)D * SK.nout;
+          for (int e = rp[rr]; e < rp[rr + 1]; ++e) {
+            const int c = L.k_out_col[e0 + e];
+            const float v = __half2float(L.k_out_val[e0 + e]);
+#pragma unroll
+            for (int j = 0; j < NC; ++j)
+              if (c == lane + 32 * j) kh[j] = v;
+          }
+        }
+        if (SV.nout > 0) {
+          for (int e = 0; e < SV.nout; ++e) {
+            const int64_t idx = (sl * L.C + t) * SV.nout + e;
+            const int c = L.v_out_col[idx];
+            const float v = __half2float(L.v_out_val[idx]);
+#pragma unroll
+            for (int j = 0; j < NC; ++j)
+              if (c == lane + 32 * j) vh[j] = v;
+          }
+        }
+        if (L.rope) rope<NC>(kh, theta, L.n_sink + t);
+        consume_token<NC, GM>(st, G, kh, vh);
+      }
+    }
+  } else if (split == a.raw_slot) {
+    const int nraw = L.n_sink + a.t_res;
+    for (int r = warp; r < nraw; r += kWarps) {
+      const bool sink = r < L.n_sink;
+      const int64_t row = sink ? r : r - L.n_sink;
+      const void* kb = sink ? L.sink[0] : L.res[0];
+      const void* vb = sink ? L.sink[1] : L.res[1];
+      const int64_t rows = sink ? L.n_sink : L.res_cap;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) {
+        const int64_t i = (sl * rows + row) * D + lane + 32 * j;
+        kh[j] = load_elem(kb, i, L.src_dtype);
+        vh[j] = load_elem(vb, i, L.src_dtype);
+      }
+      const int64_t pos = sink ? r : L.n_sink + a.t_quant + row;
+      if (L.rope) rope<NC>(kh, theta, pos);
+      consume_token<NC, GM>(st, G, kh, vh);
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+
+  // merge the warps' states and write this split's partial state
+  float* mine = wst + (size_t)warp * G * (D + 2);
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    if (hh < G) {
+#pragma unroll
+      for (int j = 0; j < NC; ++j) mine[hh * (D + 2) + lane + 32 * j] = st.o[hh][j];
+      if (lane == 0) {
+        mine[hh * (D + 2) + D] = st.m[hh];
+        mine[hh * (D + 2) + D + 1] = st.l[hh];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int hh = i / D, d = i % D;
+    float M = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wst[((size_t)w * G + hh) * (D + 2) + D]);
+    float l = 0.0f, o = 0.0f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float* p = wst + ((size_t)w * G + hh) * (D + 2);
+      const float f = p[D] == -INFINITY ? 0.0f : exp2f(p[D] - M);
+      l = fmaf(p[D + 1], f, l);
+      o = fmaf(p[d], f, o);
+    }
+    const int64_t slot = ((int64_t)b * a.Hq + h * G + hh) * a.S + split;
+    a.ws_o[slot * D + d] = o;
+    if (d == 0) {
+      a.ws_m[slot] = M;
+      a.ws_l[slot] = l;
+    }
+  }
+}
+
+struct CombArgs {
+  int D, Hq, S;
+  const float* m;
+  const float* l;
+  const float* o;
+  void* out;
+  int out_dtype;
+};
+
+__global__ void __launch_bounds__(256) combine_kernel(CombArgs a) {
+  const int hq = blockIdx.x, b = blockIdx.y;
+  const int64_t row = (int64_t)b * a.Hq + hq;
+  const float* m = a.m + row * a.S;
+  const float* l = a.l + row * a.S;
+  float M = -INFINITY;
+  for (int s = 0; s < a.S; ++s) M = fmaxf(M, m[s]);
+  for (int d = threadIdx.x; d < a.D; d += blockDim.x) {
+    float L = 0.0f, o = 0.0f;
+    for (int s = 0; s < a.S; ++s) {
+      const float f = m[s] == -INFINITY ? 0.0f : exp2f(m[s] - M);
+      L = fmaf(l[s], f, L);
+      o = fmaf(a.o[(row * a.S + s) * a.D + d], f, o);
+    }
+    store_elem(a.out, row * a.D + d, a.out_dtype, o / L);
+  }
+}
+
+template <int NC, int GM>
+cudaError_t launch_generic_g(const DecArgs& a, int grid_x, cudaStream_t s) {
+  const int G = a.Hq / a.L.Hkv;
+  const size_t smem = 256 * sizeof(float) + (size_t)kWarps * G * (a.L.D + 2) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(decode_generic_kernel<NC, GM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(grid_x, a.L.Hkv, a.L.B);
+  decode_generic_kernel<NC, GM><<<grid, kWarps * 32, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// G (query heads per KV head) is at most 16 and G * D at most 2048.
+template <int NC>
+cudaError_t launch_generic(const DecArgs& a, int grid_x, cudaStream_t s) {
+  const int G = a.Hq / a.L.Hkv;
+  if (G <= 1) return launch_generic_g<NC, 1>(a, grid_x, s);
+  if (G <= 2) return launch_generic_g<NC, 2>(a, grid_x, s);
+  if (G <= 4) return launch_generic_g<NC, 4>(a, grid_x, s);
+  if (G <= 8) return launch_generic_g<NC, 8>(a, grid_x, s);
+  if constexpr (NC <= 4) {
+    if (G <= 16) return launch_generic_g<NC, 16>(a, grid_x, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+}  // namespace
+
+bool fast_path_ok(const Layout& L, int Hq) { return mma_path_ok(L, Hq); }
+
+DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int num_splits) {
+  DecodePlan p;
+  const int64_t ngv = (t_quant + L.g - 1) / L.g;
+  const bool raw = L.n_sink + t_res > 0;
+  const int64_t heads = (int64_t)L.B * L.Hkv;
+  p.fast = (ngv > 0 && fast_path_ok(L, Hq)) ? 1 : 0;
+  int sp = 0, sg = 1;
+  if (ngv > 0) {
+    int64_t want;
+    if (num_splits > 0) {
+      want = num_splits;
+    } else {
+      const int sms = device_sm_count();
+      const int64_t target = p.fast ? (int64_t)sms * mma_ctas_per_sm() : (int64_t)sms * 8;
+      want = (target + heads - 1) / heads;
+    }
+    want = std::max<int64_t>(1, std::min<int64_t>(want, ngv));
+    sg = (int)((ngv + want - 1) / want);
+    sp = (int)((ngv + sg - 1) / sg);
+  }
+  p.n_packed_splits = sp;
+  p.split_groups = sg;
+  p.raw_slot = raw ? sp : -1;
+  p.S = sp + (raw ? 1 : 0);
+  p.grid_ctas = (int)(p.S * heads);
+  return p;
+}
+
+size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p) {
+  const size_t rows = (size_t)L.B * Hq * p.S;
+  return align16(rows * 4) * 2 + align16(rows * L.D * 4);
+}
+
+cudaError_t launch_decode(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
+                          int64_t t_quant, int t_res, float scale, void* out, int out_dtype,
+                          void* ws, int32_t* d_status, cudaStream_t s) {
+  const size_t rows = (size_t)L.B * Hq * p.S;
+  float* ws_m = reinterpret_cast<float*>(ws);
+  float* ws_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align16(rows * 4));
+  float* ws_o = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4));
+  DecArgs a;
+  a.L = L;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.Hq = Hq;
+  a.t_quant = t_quant;
+  a.t_res = t_res;
+  a.qscale = scale * kLog2e;
+  a.S = p.S;
+  a.split_groups = p.split_groups;
+  a.n_packed = p.n_packed_splits;
+  a.raw_slot = p.raw_slot;
+  a.ws_m = ws_m;
+  a.ws_l = ws_l;
+  a.ws_o = ws_o;
+  a.status = d_status;
+  cudaError_t e = cudaSuccess;
+  if (p.fast) {
+    e = launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
+  } else {
+    switch (L.D) {
+      case 32: e = launch_generic<1>(a, p.S, s); break;
+      case 64: e = launch_generic<2>(a, p.S, s); break;
+      case 128: e = launch_generic<4>(a, p.S, s); break;
+      default: e = launch_generic<8>(a, p.S, s); break;
+    }
+  }
+  if (e != cudaSuccess) return e;
+  CombArgs c;
+  c.D = L.D;
+  c.Hq = Hq;
+  c.S = p.S;
+  c.m = ws_m;
+  c.l = ws_l;
+  c.o = ws_o;
+  c.out = out;
+  c.out_dtype = out_dtype;
+  dim3 grid(Hq, L.B);
+  combine_kernel<<<grid, L.D < 256 ? L.D : 256, 0, s>>>(c);
+  return cudaGetLastError();
+}
+
+// Generic kernel entry used by the fast path for its raw (sink + residual) slot.
+cudaError_t launch_decode_raw_generic(const Layout& L, const DecodePlan& p, const void* q,
+                                      int q_dtype, int Hq, int64_t t_quant, int t_res, float scale,
+                                      float* ws_m, float* ws_l, float* ws_o, int32_t* d_status,
+                                      cudaStream_t s) {
+  DecArgs a;
+  a.L = L;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.Hq = Hq;
+  a.t_quant = t_quant;
+  a.t_res = t_res;
+  a.qscale = scale * kLog2e;
+  a.S = p.S;
+  a.split_groups = p.split_groups;
+  a.n_packed = 0;          // no packed splits: only CTA x = raw_slot does work
+  a.raw_slot = 0;
+  a.ws_m = ws_m;
+  a.ws_l = ws_l;
+  a.ws_o = ws_o;
+  a.status = d_status;
+  // write into slot p.raw_slot: offset the partial arrays so that split index 0 maps there
+  a.ws_m = ws_m + p.raw_slot;
+  a.ws_l = ws_l + p.raw_slot;
+  a.ws_o = ws_o + (size_t)p.raw_slot * L.D;
+  switch (L.D) {
+    case 32: return launch_generic<1>(a, 1, s);
+    case 64: return launch_generic<2>(a, 1, s);
+    case 128: return launch_generic<4>(a, 1, s);
+    default: return launch_generic<8>(a, 1, s);
+  }
+}
+
+}  // namespace kvq

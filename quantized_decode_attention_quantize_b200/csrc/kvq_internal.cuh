@@ -1,0 +1,165 @@
+// Internal declarations shared by the kernels and the host layer of libkvq.
+// Not part of the public ABI (include/kvq.h is).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// ---------------------------------------------------------------------------
+// Layout: everything a kernel needs to address the cache, derived on the host
+// from kvq_format + kvq_cache and passed by value.
+// ---------------------------------------------------------------------------
+struct Side {
+  int scheme, bits, axis, nout;
+  int64_t code_slab_bytes;   // bytes of codes per (b, kv-head) slab
+  int64_t meta_slab_elems;   // scale / zero elements per slab
+  int code_row_bytes;        // packed bytes per token row (MIXED: per row of all planes)
+  void* codes;
+  void* scale;
+  void* zero;
+  const __half* lut;
+};
+
+struct Layout {
+  int D, g, src_dtype, B, Hkv;
+  int64_t C;                 // capacity (tokens), multiple of g
+  int ng;                    // C / g
+  int n_sink, res_cap, rope;
+  float rope_base;
+  int mixed_hi, mixed_mid, mixed_lo, mixed_group_bytes;
+  Side side[2];
+  uint8_t* k_order;
+  int32_t* k_out_rowptr;
+  uint8_t* k_out_col;
+  __half* k_out_val;
+  uint8_t* v_out_col;
+  __half* v_out_val;
+  void* sink[2];
+  void* res[2];
+  int raw_bytes;             // element size of src_dtype
+};
+
+// Host helpers (api.cpp)
+kvq_status make_layout(const kvq_format* f, const kvq_cache* c, Layout* L);
+
+// Launchers (each .cu file), return cudaError_t of the launch.
+cudaError_t launch_quantize(const Layout& L, int which, const void* src, int64_t sb,
+                            int64_t sh, int64_t st, int64_t t0, int64_t n,
+                            int32_t* d_status, cudaStream_t s);
+cudaError_t launch_dequantize(const Layout& L, int which, int64_t t0, int64_t n, void* out,
+                              int out_dtype, int32_t* d_status, cudaStream_t s);
+cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t qsh,
+                            int64_t qst, const void* k, int64_t ksb, int64_t ksh, int64_t kst,
+                            int B, int Hq, int Hkv, int R, double* sal, uint8_t* order,
+                            int64_t osb, int64_t osh, int32_t* d_status, cudaStream_t s);
+
+struct DecodePlan {
+  int S;                // partial slots per query head
+  int split_groups;     // packed groups per packed split (generic path)
+  int n_packed_splits;  // splits over the packed region
+  int raw_slot;         // slot index of the raw (sink + residual) segment, -1 if none
+  int fast;             // 1 when the tensor-core K4/V2 kernel runs the packed region
+  int grid_ctas;        // CTAs of the split kernel
+};
+DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int num_splits);
+size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p);
+bool fast_path_ok(const Layout& L, int Hq);
+cudaError_t launch_decode(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
+                          int Hq, int64_t t_quant, int t_res, float scale, void* out,
+                          int out_dtype, void* ws, int32_t* d_status, cudaStream_t s);
+int device_sm_count();
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float load_elem(const void* p, int64_t i, int dtype) {
+  if (dtype == KVQ_F32) return reinterpret_cast<const float*>(p)[i];
+  if (dtype == KVQ_F16) return __half2float(reinterpret_cast<const __half*>(p)[i]);
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ void store_elem(void* p, int64_t i, int dtype, float v) {
+  if (dtype == KVQ_F32) reinterpret_cast<float*>(p)[i] = v;
+  else if (dtype == KVQ_F16) reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  else reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t b) {
+  return __half2float(__ushort_as_half(b));
+}
+
+__device__ __forceinline__ void flag(int32_t* st, int bits) {
+  if (st) atomicOr(st, bits);
+}
+
+// Asymmetric b-bit metadata: z = fp16 toward -inf of mn, s = fp16 toward +inf of
+// fl32(fl32(mx - z) / (2^b - 1)), s = 1 when that is zero.
+__device__ __forceinline__ bool asym_params(float mn, float mx, int bits, __half* s_out,
+                                            __half* z_out) {
+  __half z = __float2half_rd(mn);
+  float zf = __half2float(z);
+  float d = __fsub_rn(mx, zf);
+  float t = __fdiv_rn(d, (float)((1 << bits) - 1));
+  __half s = __float2half_ru(t);
+  float sf = __half2float(s);
+  if (sf == 0.0f) s = __float2half_rn(1.0f);
+  *s_out = s;
+  *z_out = z;
+  return isfinite(zf) && isfinite(__half2float(s));
+}
+
+__device__ __forceinline__ int asym_code(float x, float s, float z, int maxc) {
+  float q = __fdiv_rn(__fsub_rn(x, z), s);
+  float r = rintf(q);
+  r = fminf(fmaxf(r, 0.0f), (float)maxc);
+  return (int)r;
+}
+
+// nuq3 metadata: z = fp16 nearest of fl32(fl32(mx + mn) * 0.5),
+// s = fp16 toward +inf of max(fl32(mx - z), fl32(z - mn)), s = 1 when zero.
+__device__ __forceinline__ bool nuq_params(float mn, float mx, __half* s_out, __half* z_out) {
+  float h = __fmul_rn(__fadd_rn(mx, mn), 0.5f);
+  __half z = __float2half_rn(h);
+  float zf = __half2float(z);
+  float a = __fsub_rn(mx, zf);
+  float b = __fsub_rn(zf, mn);
+  __half s = __float2half_ru(fmaxf(a, b));
+  if (__half2float(s) == 0.0f) s = __float2half_rn(1.0f);
+  *s_out = s;
+  *z_out = z;
+  return isfinite(zf) && isfinite(__half2float(s));
+}
+
+// Nearest of the eight centroids via the seven fp32 midpoints (an exact midpoint
+// goes to the lower centroid).
+__device__ __forceinline__ int nuq_code(float x, float s, float z, const float* mids) {
+  float y = __fdiv_rn(__fsub_rn(x, z), s);
+  int c = 0;
+#pragma unroll
+  for (int j = 0; j < 7; ++j) c += (y > mids[j]) ? 1 : 0;
+  return c;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace kvq

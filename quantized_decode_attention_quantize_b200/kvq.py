@@ -1,0 +1,209 @@
+"""ctypes binding of libkvq.so (include/kvq.h).
+
+Argument marshalling only: every entry point forwards to the C ABI with the same
+name; device memory and streams come from PyTorch.  There is no fallback: when the
+shared library is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+# enums of include/kvq.h
+KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA, KVQ_ERR_WORKSPACE = range(5)
+KVQ_DEV_NONFINITE, KVQ_DEV_RANGE = 1, 2
+F32, F16, BF16 = 0, 1, 2
+NONE, SYM8, ASYM, NUQ, MIXED = range(5)
+TENSOR, TOKEN, CHANNEL = range(3)
+KEYS, VALUES = 0, 1
+
+ARRAYS = [
+    "k_codes", "k_scale", "k_zero", "k_order",
+    "k_out_rowptr", "k_out_col", "k_out_val",
+    "v_codes", "v_scale", "v_zero",
+    "v_out_col", "v_out_val",
+    "k_lut", "v_lut",
+    "sink_k", "sink_v", "res_k", "res_v",
+]
+
+TORCH_DTYPE = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
+KVQ_DTYPE = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+
+
+class kvq_format(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "head_dim", "group_tokens", "src_dtype",
+        "k_scheme", "k_bits", "k_axis", "k_outliers",
+        "v_scheme", "v_bits", "v_axis", "v_outliers",
+        "mixed_hi", "mixed_mid", "n_sink", "residual_cap", "rope")] + [("rope_base", ctypes.c_float)]
+
+
+class kvq_cache(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
+                ("capacity", ctypes.c_int64)] + [(n, ctypes.c_void_p) for n in ARRAYS]
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn}: {status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libkvq.so (raises when it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} not built; run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        FP, CP = ctypes.POINTER(kvq_format), ctypes.POINTER(kvq_cache)
+        sig = {
+            "kvq_version": (I32, []),
+            "kvq_status_string": (ctypes.c_char_p, [I32]),
+            "kvq_format_check": (I32, [FP]),
+            "kvq_cache_array_bytes": (SZ, [FP, I32, I32, I64, I32]),
+            "kvq_quantize_keys": (I32, [FP, CP, P, I64, I64, I64, I64, I64, P, P]),
+            "kvq_quantize_values": (I32, [FP, CP, P, I64, I64, I64, I64, I64, P, P]),
+            "kvq_dequantize": (I32, [FP, CP, I32, I64, I64, P, I32, P, P]),
+            "kvq_key_salience": (I32, [FP, P, I64, I64, I64, P, I64, I64, I64, I32, I32, I32, I32,
+                                       P, P, I64, I64, P, P]),
+            "kvq_decode_workspace_bytes": (SZ, [FP, I32, I32, I32, I64, I32, I32]),
+            "kvq_decode_attention": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, I32,
+                                           P, SZ, I32, P, P]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(st):
+    return lib().kvq_status_string(int(st)).decode()
+
+
+def _check(fn, st):
+    if st != KVQ_OK:
+        raise KvqError(fn, st)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_format(d: dict) -> kvq_format:
+    f = kvq_format()
+    for name, _ in kvq_format._fields_:
+        setattr(f, name, d[name])
+    return f
+
+
+def format_check(fmt: kvq_format) -> int:
+    return lib().kvq_format_check(ctypes.byref(fmt))
+
+
+def cache_array_bytes(fmt: kvq_format, B, H, C, array_id) -> int:
+    return lib().kvq_cache_array_bytes(ctypes.byref(fmt), B, H, C, array_id)
+
+
+class Cache:
+    """Device arrays of a packed cache (torch uint8 tensors), owned by this object."""
+
+    def __init__(self, fmt: kvq_format, B: int, H: int, C: int, device="cuda", k_lut=None,
+                 v_lut=None):
+        self.fmt, self.B, self.H, self.C = fmt, B, H, C
+        self.tensors = {}
+        self.struct = kvq_cache(batch=B, kv_heads=H, capacity=C)
+        for i, name in enumerate(ARRAYS):
+            n = cache_array_bytes(fmt, B, H, C, i)
+            if n:
+                t = torch.zeros(n, dtype=torch.uint8, device=device)
+                self.tensors[name] = t
+                setattr(self.struct, name, t.data_ptr())
+        for name, lut in (("k_lut", k_lut), ("v_lut", v_lut)):
+            if name in self.tensors and lut is not None:
+                self.tensors[name].copy_(torch.tensor(lut, dtype=torch.float16).view(torch.uint8))
+
+    def array(self, name):
+        return self.tensors[name]
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def quantize_keys(fmt, cache: Cache, src: torch.Tensor, t0: int, n: int, status=None, stream=None):
+    """src [B, H, n, D] (strided over the first three dims, channels contiguous)."""
+    st = lib().kvq_quantize_keys(ctypes.byref(fmt), cache.ref(), _ptr(src), src.stride(0),
+                                 src.stride(1), src.stride(2), t0, n, _ptr(status), _stream(stream))
+    _check("kvq_quantize_keys", st)
+
+
+def quantize_values(fmt, cache: Cache, src: torch.Tensor, t0: int, n: int, status=None,
+                    stream=None):
+    st = lib().kvq_quantize_values(ctypes.byref(fmt), cache.ref(), _ptr(src), src.stride(0),
+                                   src.stride(1), src.stride(2), t0, n, _ptr(status),
+                                   _stream(stream))
+    _check("kvq_quantize_values", st)
+
+
+def dequantize(fmt, cache: Cache, which: int, t0: int, n: int, out_dtype=F32, out=None,
+               status=None, stream=None):
+    if out is None:
+        out = torch.empty((cache.B, cache.H, n, fmt.head_dim), dtype=TORCH_DTYPE[out_dtype],
+                          device="cuda")
+    st = lib().kvq_dequantize(ctypes.byref(fmt), cache.ref(), which, t0, n, _ptr(out), out_dtype,
+                              _ptr(status), _stream(stream))
+    _check("kvq_dequantize", st)
+    return out
+
+
+def key_salience(fmt, q: torch.Tensor, k: torch.Tensor, order_out: torch.Tensor,
+                 order_stride_b: int, order_stride_h: int, salience_out=None, status=None,
+                 stream=None):
+    """q [B, Hq, R, D], k [B, Hkv, R, D]; order_out is a uint8 tensor whose element
+    (b, h, slot) sits at b * order_stride_b + h * order_stride_h + slot."""
+    B, Hq, R, D = q.shape
+    Hkv = k.shape[1]
+    st = lib().kvq_key_salience(ctypes.byref(fmt), _ptr(q), q.stride(0), q.stride(1), q.stride(2),
+                                _ptr(k), k.stride(0), k.stride(1), k.stride(2), B, Hq, Hkv, R,
+                                _ptr(salience_out), _ptr(order_out), order_stride_b,
+                                order_stride_h, _ptr(status), _stream(stream))
+    _check("kvq_key_salience", st)
+
+
+def decode_workspace_bytes(fmt, B, Hq, Hkv, t_quant, t_res, num_splits=0) -> int:
+    return lib().kvq_decode_workspace_bytes(ctypes.byref(fmt), B, Hq, Hkv, t_quant, t_res,
+                                            num_splits)
+
+
+def decode_attention(fmt, cache: Cache, q: torch.Tensor, t_quant: int, t_res: int, scale: float,
+                     out_dtype=F32, out=None, workspace=None, num_splits=0, status=None,
+                     stream=None):
+    """q [B, Hq, D] contiguous -> out [B, Hq, D]."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=TORCH_DTYPE[out_dtype], device=q.device)
+    need = decode_workspace_bytes(fmt, B, Hq, cache.H, t_quant, t_res, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().kvq_decode_attention(ctypes.byref(fmt), cache.ref(), _ptr(q), KVQ_DTYPE[q.dtype],
+                                    Hq, t_quant, t_res, scale, _ptr(out), out_dtype,
+                                    _ptr(workspace), workspace.numel(), num_splits, _ptr(status),
+                                    _stream(stream))
+    _check("kvq_decode_attention", st)
+    return out

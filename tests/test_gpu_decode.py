@@ -1,0 +1,176 @@
+"""GPU parity of decode attention against the float64 oracle on small seeded caches
+of every format, with sinks, residual windows, ragged tails and the degenerate
+cases (one token, raw tokens only, a split per group, split-count invariance)."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import attention as oatt
+from oracle import salience
+from oracle.formats import BF16, F16, F32, KEYS, MIXED, NUQ, VALUES
+from quantized_decode_attention_quantize_b200 import kvq
+from tests.gpu_util import Pair, dev, rel_l2, tolerance
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LUT = json.load(open(os.path.join(ROOT, "tests", "golden", "nuq3_codebook.json")))
+
+
+def fmt(**kw):
+    return synth._fmt(**kw)
+
+
+def vals(seed, shape, dt, scale=1.0, heavy=False):
+    r = np.random.default_rng(seed)
+    x = r.standard_t(4, shape) if heavy else r.standard_normal(shape)
+    return synth.to_dtype_values((x * scale).astype(np.float32), dt)
+
+
+def build(fd, B, H, Hq, tq, tr, seed=0, k_scale=1.0, luts=(None, None), mixed_q=None):
+    D, g, dt = fd["head_dim"], fd["group_tokens"], fd["src_dtype"]
+    C = max(g, -(-tq // g) * g)
+    p = Pair(fd, B, H, C, k_lut=luts[0], v_lut=luts[1])
+    K = vals(seed + 1, (B, H, tq, D), dt, k_scale, heavy=True)
+    V = vals(seed + 2, (B, H, tq, D), dt)
+    if fd["k_scheme"] == MIXED:
+        G = Hq // H
+        Q = vals(seed + 3, (B, Hq, tq, D), dt)
+        ng = C // g
+        order = np.zeros((B, H, ng, D), np.uint8)
+        for gi in range(-(-tq // g)):
+            for b in range(B):
+                for h in range(H):
+                    order[b, h, gi] = salience.key_salience(Q[b, h * G:(h + 1) * G, gi * g:(gi + 1) * g],
+                                                            K[b, h, gi * g:(gi + 1) * g])[1]
+        p.set_order(order)
+    if tq:
+        p.quantize(KEYS, K, 0, tq)
+        p.quantize(VALUES, V, 0, tq)
+    if fd["n_sink"]:
+        p.set_raw("sink_k", vals(seed + 4, (B, H, fd["n_sink"], D), dt, k_scale))
+        p.set_raw("sink_v", vals(seed + 5, (B, H, fd["n_sink"], D), dt))
+    if fd["residual_cap"]:
+        rk = np.zeros((B, H, fd["residual_cap"], D), np.float32)
+        rv = np.zeros_like(rk)
+        rk[:, :, :tr] = vals(seed + 6, (B, H, tr, D), dt, k_scale)
+        rv[:, :, :tr] = vals(seed + 7, (B, H, tr, D), dt)
+        p.set_raw("res_k", rk)
+        p.set_raw("res_v", rv)
+    return p
+
+
+def run(p, Hq, tq, tr, q_dtype, out_dtype, seed=0, num_splits=0, q=None):
+    D = p.fd["head_dim"]
+    if q is None:
+        q = vals(seed + 9, (p.B, Hq, D), q_dtype, 1.0)
+    out = kvq.decode_attention(p.fmt, p.gpu, dev(q, q_dtype), tq, tr, 1.0 / np.sqrt(D), out_dtype,
+                               num_splits=num_splits, status=p.status)
+    torch.cuda.synchronize()
+    ref = oatt.decode_attention(p.of, p.ora, q.astype(np.float64), tq, tr)
+    return out.float().cpu().numpy(), ref
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 5, 8])
+@pytest.mark.parametrize("out_dtype", [F32, BF16])
+def test_k4v2(G, out_dtype):
+    B, H, tq = 2, 2, 3 * 128 + 45
+    fd = fmt(src_dtype=BF16)
+    p = build(fd, B, H, G * H, tq, 0, seed=G)
+    out, ref = run(p, G * H, tq, 0, BF16, out_dtype, seed=G)
+    assert rel_l2(out, ref) <= tolerance(out_dtype)
+    assert p.status_bits() == 0
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_sink_and_residual(G):
+    B, H, tq, tr = 2, 2, 2 * 128 + 17, 37
+    fd = fmt(src_dtype=BF16, n_sink=1, residual_cap=128)
+    p = build(fd, B, H, G * H, tq, tr, seed=10)
+    out, ref = run(p, G * H, tq, tr, BF16, F32, seed=10)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+def test_raw_tokens_only():
+    fd = fmt(src_dtype=F16, n_sink=2, residual_cap=16)
+    p = build(fd, 1, 2, 8, 0, 9, seed=11)
+    out, ref = run(p, 8, 0, 9, F16, F32, seed=11)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+def test_single_token_returns_its_value():
+    fd = fmt(src_dtype=F16)
+    p = build(fd, 1, 2, 4, 1, 0, seed=12)
+    out, ref = run(p, 4, 1, 0, F16, F32, seed=12)
+    assert rel_l2(out, ref) <= 1e-6
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7])
+def test_split_count_invariance(splits):
+    B, H, G, tq = 1, 2, 4, 7 * 128 - 5
+    fd = fmt(src_dtype=BF16)
+    p = build(fd, B, H, G * H, tq, 0, seed=13)
+    out, ref = run(p, G * H, tq, 0, BF16, F32, seed=13, num_splits=splits)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+@pytest.mark.parametrize("dt", [F16, F32])
+@pytest.mark.parametrize("D", [32, 64, 256])
+def test_head_dims(dt, D):
+    g = 64 if D == 256 else 128
+    fd = fmt(head_dim=D, group_tokens=g, src_dtype=dt, k_bits=4, v_bits=2)
+    p = build(fd, 1, 2, 4, 2 * g + 3, 0, seed=14)
+    out, ref = run(p, 4, 2 * g + 3, 0, dt, F32, seed=14)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+def test_nuq3_outliers_rope():
+    fd = fmt(src_dtype=F16, k_scheme=NUQ, k_bits=3, k_outliers=2, v_scheme=NUQ, v_bits=3,
+             v_outliers=2, rope=1)
+    p = build(fd, 1, 3, 3, 3 * 128 + 20, 0, seed=15, k_scale=3.0, luts=(LUT["k"], LUT["v"]))
+    out, ref = run(p, 3, 3 * 128 + 20, 0, F16, F32, seed=15)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+def test_rope_at_long_positions():
+    # keys at positions past 100k: the angle t * theta_0 exceeds 1e5 rad
+    fd = fmt(src_dtype=F16, rope=1)
+    tq = 782 * 128 + 37
+    p = build(fd, 1, 1, 2, tq, 0, seed=16)
+    out, ref = run(p, 2, tq, 0, F16, F32, seed=16)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+def test_mixed_decode():
+    B, H, G = 2, 2, 5
+    fd = fmt(src_dtype=BF16, k_scheme=MIXED, k_bits=0, mixed_hi=8, mixed_mid=24)
+    p = build(fd, B, H, G * H, 2 * 128 + 60, 0, seed=17, k_scale=4.0)
+    out, ref = run(p, G * H, 2 * 128 + 60, 0, BF16, BF16, seed=17)
+    assert rel_l2(out, ref) <= 2e-3
+
+
+@pytest.mark.parametrize("scheme", ["tensor", "token", "hybrid"])
+@pytest.mark.parametrize("target", ["both", "k_only", "v_only"])
+def test_toy_int8(scheme, target):
+    # [AXES] toy as decode: 8 query rows are 8 query heads sharing one KV head
+    N = 64
+    Q, K, V = synth.toy(41, N)
+    fd = synth.toy_format(scheme, target, N)
+    p = Pair(fd, 1, 1, N)
+    p.quantize(KEYS, K[None, None], 0, N)
+    p.quantize(VALUES, V[None, None], 0, N)
+    out, ref = run(p, 8, N, 0, F32, F32, q=Q[None])
+    assert rel_l2(out, ref) <= 1e-5
+
+
+def test_nonfinite_query_flagged():
+    fd = fmt(src_dtype=F16)
+    p = build(fd, 1, 1, 2, 128, 0, seed=18)
+    q = vals(19, (1, 2, 128), F16)
+    q[0, 1, 5] = np.inf
+    kvq.decode_attention(p.fmt, p.gpu, dev(q, F16), 128, 0, 0.1, F32, status=p.status)
+    assert p.status_bits() & kvq.KVQ_DEV_NONFINITE
