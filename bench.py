@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the hot path: append-time quantization of one token group plus
+decode attention over the packed cache, on synthetic data shaped like the workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config llama3_8b]
+
+One step = kvq_quantize_keys + kvq_quantize_values of one 128-token group (the
+flush of the raw window into the packed cache) + kvq_decode_partial (split kernel)
++ kvq_decode_combine over all T tokens.  Every step is timed with CUDA events on
+the launching stream; the L2 is flushed between steps (a 512 MiB write, outside the
+events).  `value` is the effective HBM throughput of the whole step: the format's
+algorithmic bytes (codes, scales, zero-points, raw sink / residual tokens, the new
+group's source and packed output, q and out) over the step time.  One JSON line is
+printed by rank 0.  Under torchrun every rank runs its own replica (weak scaling:
+the per-GPU work is fixed), the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize GB/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="llama3_8b", choices=["llama3_8b", "llama2_7b"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---- algorithmic byte counts ---------------------------------------------------------------
+
+def fmt_bytes(cfg):
+    """Per-token / per-group byte counts of the K4V2 format (D = 128, g = 128)."""
+    D, g = cfg["D"], cfg["fmt"]["group_tokens"]
+    kb, vb = cfg["fmt"]["k_bits"], cfg["fmt"]["v_bits"]
+    raw = 2 if cfg["fmt"]["src_dtype"] != synth.F32 else 4
+    return dict(k_code=D * kb // 8, v_code=D * vb // 8, v_meta=4, k_meta_group=4 * D,
+                raw_token=2 * D * raw, g=g, D=D, raw=raw)
+
+
+def decode_kernel_bytes(cfg, tq, tr):
+    """Bytes the decode split kernel must read: packed rows, their metadata, raw
+    sink / residual tokens and the queries."""
+    f = fmt_bytes(cfg)
+    ns = cfg["fmt"]["n_sink"]
+    ngv = -(-tq // f["g"])
+    per_head = tq * (f["k_code"] + f["v_code"] + f["v_meta"]) + ngv * f["k_meta_group"] + \
+        (ns + tr) * f["raw_token"]
+    q = cfg["B"] * cfg["Hq"] * cfg["D"] * 2
+    return cfg["B"] * cfg["Hkv"] * per_head + q
+
+
+def decode_call_bytes(cfg, tq, tr):
+    return decode_kernel_bytes(cfg, tq, tr) + cfg["B"] * cfg["Hq"] * cfg["D"] * 4   # fp32 out
+
+
+def quant_bytes(cfg, n):
+    """One append of n tokens: 16-bit K and V read, codes and metadata written."""
+    f = fmt_bytes(cfg)
+    heads = cfg["B"] * cfg["Hkv"]
+    read = heads * n * f["D"] * f["raw"] * 2
+    write = heads * (n * (f["k_code"] + f["v_code"] + f["v_meta"]) + -(-n // f["g"]) * f["k_meta_group"])
+    return read + write
+
+
+# ---- clocks -----------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---- the oracle as a CPU baseline ------------------------------------------------------------
+
+class OracleSample:
+    """The float64 oracle on a bounded sample of the workload: the flush quantize of
+    one group of one KV head plus decode attention of that head's G query heads over
+    `groups` packed groups and its raw tokens.  Setup (data, cache) is not timed."""
+
+    def __init__(self, cfg, groups):
+        from oracle import cache as ocache
+        from oracle import fp
+        from oracle.formats import KEYS, VALUES, Format
+        self.cfg = cfg
+        of = Format(**cfg["fmt"])
+        g = of.group_tokens
+        self.G = cfg["Hq"] // cfg["Hkv"]
+        ns, tq_full, tr = synth.split_tokens(cfg)
+        tq = min(tq_full, groups * g)
+        T = ns + tq + tr
+        K = synth.kv_slab(cfg, 0, 0, T, "k")[None, None].astype(np.float64)
+        V = synth.kv_slab(cfg, 0, 0, T, "v")[None, None].astype(np.float64)
+        c = ocache.Cache(of, 1, 1, -(-tq // g) * g)
+        ocache.quantize(of, c, KEYS, K[:, :, ns:ns + tq], 0, tq)
+        ocache.quantize(of, c, VALUES, V[:, :, ns:ns + tq], 0, tq)
+        enc = fp.bf16_bits if of.src_dtype == synth.BF16 else fp.f16_bits
+        if ns:
+            c["sink_k"][...] = enc(K[:, :, :ns])
+            c["sink_v"][...] = enc(V[:, :, :ns])
+        if tr:
+            c["res_k"][...] = enc(K[:, :, ns + tq:])
+            c["res_v"][...] = enc(V[:, :, ns + tq:])
+        self.q = np.stack([synth.query(cfg, 0, h) for h in range(self.G)])[None].astype(np.float64)
+        self.newk, self.newv = K[:, :, ns:ns + g], V[:, :, ns:ns + g]
+        self.of, self.c, self.tq, self.tr, self.g, self.ns = of, c, tq, tr, g, ns
+        one_head = dict(cfg, B=1, Hkv=1, Hq=self.G)
+        self.nbytes = decode_call_bytes(one_head, tq, tr) + quant_bytes(one_head, g)
+
+    def run(self):
+        from oracle import cache as ocache
+        from oracle import attention as oatt
+        from oracle.formats import KEYS, VALUES
+        t0 = time.perf_counter()
+        ocache.quantize(self.of, self.c, KEYS, self.newk, 0, self.g)
+        ocache.quantize(self.of, self.c, VALUES, self.newv, 0, self.g)
+        oatt.decode_attention(self.of, self.c, self.q, self.tq, self.tr)
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return (f"oracle (numpy, float64) on one KV head of {self.cfg['name']}: quantize of one "
+                f"{self.g}-token group (K and V) + decode of its {self.G} query heads over "
+                f"{self.tq} packed rows + {self.ns + self.tr} raw tokens")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_sized(cfg, budget_s):
+    """An OracleSample whose run() takes about budget_s seconds."""
+    probe = OracleSample(cfg, 4)
+    probe.run()
+    per_group = probe.run() / 4
+    groups = int(max(1, budget_s / max(per_group, 1e-6)))
+    return OracleSample(cfg, groups)
+
+
+# ---- main --------------------------------------------------------------------------------------
+
+def setup_dist(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    cfg = synth.CONFIGS[args.config]
+    if rank != 0:
+        return
+    per_step = max(0.02, 120.0 / max(1, args.steps + args.warmup))
+    smp = oracle_sized(cfg, per_step)
+    for _ in range(args.warmup):
+        smp.run()
+    times = [smp.run() for _ in range(args.steps)]
+    sec = statistics.mean(times)
+    gbs = smp.nbytes / sec / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(cfg),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": smp.describe() + " per step"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg):
+    ns, tq, tr = synth.split_tokens(cfg)
+    f = cfg["fmt"]
+    return {"workload": f"{cfg['name']}: B={cfg['B']} Hq={cfg['Hq']} Hkv={cfg['Hkv']} D={cfg['D']} "
+                        f"T={cfg['T']} (sink {ns}, packed {tq}, residual {tr}); K{f['k_bits']} per-channel "
+                        f"g{f['group_tokens']} + V{f['v_bits']} per-token, fp16 scale/zero",
+            "B": cfg["B"], "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "D": cfg["D"], "T": cfg["T"],
+            "step": "quantize one 128-token group (K, V) + decode attention over T",
+            "l2": "flushed between steps (512 MiB write outside the timed events)",
+            "parallelism": "replicas (one independent cache per GPU)"}
+
+
+def main():
+    args = parse()
+    import torch
+    world, rank, local = setup_dist(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    from quantized_decode_attention_quantize_b200 import kvq
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[args.config]
+    fd = cfg["fmt"]
+    fmt = kvq.make_format(fd)
+    B, Hq, Hkv, D, g = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["D"], fd["group_tokens"]
+    ns, tq, tr = synth.split_tokens(cfg)
+    C = -(-tq // g) * g
+    scale = 1.0 / float(np.sqrt(D))
+
+    # ---- build the cache on the device (data drawn on the device, same recipe)
+    K = synth.device_kv(cfg, "k", device=dev, seed_offset=rank)
+    V = synth.device_kv(cfg, "v", device=dev, seed_offset=rank)
+    cache = kvq.Cache(fmt, B, Hkv, C, device=dev)
+    kvq.quantize_keys(fmt, cache, K[:, :, ns:ns + tq], 0, tq)
+    kvq.quantize_values(fmt, cache, V[:, :, ns:ns + tq], 0, tq)
+    if ns:
+        cache.array("sink_k").copy_(K[:, :, :ns].contiguous().view(-1).view(torch.uint8))
+        cache.array("sink_v").copy_(V[:, :, :ns].contiguous().view(-1).view(torch.uint8))
+    if tr:
+        cache.array("res_k").copy_(K[:, :, ns + tq:].contiguous().view(-1).view(torch.uint8))
+        cache.array("res_v").copy_(V[:, :, ns + tq:].contiguous().view(-1).view(torch.uint8))
+    # the flushed group: rewrite packed group gi_f (a full group) from its own tokens
+    gi_f = tq // g - 1
+    newk = K[:, :, ns + gi_f * g: ns + (gi_f + 1) * g].contiguous()
+    newv = V[:, :, ns + gi_f * g: ns + (gi_f + 1) * g].contiguous()
+    del K, V
+    q = synth.device_queries(cfg, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(kvq.decode_workspace_bytes(fmt, B, Hq, Hkv, tq, tr), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        kvq.quantize_keys(fmt, cache, newk, gi_f * g, g, status=status, stream=stream)
+        kvq.quantize_values(fmt, cache, newv, gi_f * g, g, status=status, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        kvq.decode_partial(fmt, cache, q, tq, tr, scale, ws, status=status, stream=stream)
+        if evs:
+            evs[2].record(stream)
+        kvq.decode_combine(fmt, B, Hq, Hkv, tq, tr, ws, out, stream=stream)
+        if evs:
+            evs[3].record(stream)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.15)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    t_quant = [e[0].elapsed_time(e[1]) for e in evs]
+    t_part = [e[1].elapsed_time(e[2]) for e in evs]
+    t_comb = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    ms_step = statistics.mean(t_step)
+    ms_part = statistics.mean(t_part)
+    ms_quant = statistics.mean(t_quant)
+    ms_comb = statistics.mean(t_comb)
+    if world > 1:
+        tt = torch.tensor([ms_step, ms_part, ms_quant, ms_comb], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step, ms_part, ms_quant, ms_comb = [float(x) for x in tt.tolist()]
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(10, args.steps // 10)
+    hk = torch.empty_like(newk, device="cpu").pin_memory()
+    hv = torch.empty_like(newv, device="cpu").pin_memory()
+    hk.copy_(newk)
+    hv.copy_(newv)
+    hq = torch.empty_like(q, device="cpu").pin_memory()
+    hq.copy_(q)
+    hout = torch.empty_like(out, device="cpu").pin_memory()
+    dk, dv, dq = torch.empty_like(newk), torch.empty_like(newv), torch.empty_like(q)
+    e2e_t = []
+    for i in range(e2e_steps + 3):
+        flush.fill_(i & 0xFF)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        kvq.quantize_keys(fmt, cache, dk, gi_f * g, g, status=status, stream=stream)
+        kvq.quantize_values(fmt, cache, dv, gi_f * g, g, status=status, stream=stream)
+        kvq.decode_attention(fmt, cache, dq, tq, tr, scale, kvq.F32, out=out, workspace=ws,
+                             status=status, stream=stream)
+        hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= 3:
+            e2e_t.append(e0.elapsed_time(e1))
+    ms_e2e = statistics.mean(e2e_t)
+    if world > 1:
+        tt = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    assert torch.isfinite(out).all()
+
+    step_bytes = decode_call_bytes(cfg, tq, tr) + quant_bytes(cfg, g)
+    kern_bytes = decode_kernel_bytes(cfg, tq, tr)
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    decode_gbs = (decode_call_bytes(cfg, tq, tr)) / ((ms_part + ms_comb) * 1e-3) / 1e9
+    quant_gbs = quant_bytes(cfg, g) / (ms_quant * 1e-3) / 1e9
+    achieved = kern_bytes / (ms_part * 1e-3) / 1e9
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        pass
+    peak = peaks.get("hbm_gbs", 6650.0)
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "decode_mma_llama3_8b.json")
+    if os.path.exists(prof):
+        try:
+            pj = json.load(open(prof))
+            if pj.get("kernel_hash") == kernel_hash():
+                traffic = pj.get("dram_bytes_per_launch")
+        except (OSError, ValueError):
+            pass
+    h2d = newk.numel() * newk.element_size() * 2 + q.numel() * q.element_size()
+    d2h = out.numel() * out.element_size()
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 tensor-core products with f32 accumulation (u4/u2 codes)",
+        "data": "synthetic (device-drawn, recipe of synth/)",
+        "config": workload_config(cfg),
+        "pct_of_8tbs": 100.0 * value / world / 8000.0,
+        "decode_gbs": decode_gbs, "quantize_gbs": quant_gbs,
+        "tokens_heads_per_s": world * B * Hq * cfg["T"] / ((ms_part + ms_comb) * 1e-3),
+        "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb},
+        "roofline": {"kernel": "decode_mma_kernel (kvq_decode_partial)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes": kern_bytes,
+                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},
+        "e2e": {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = oracle_sized(cfg, 5.0)
+        times = [smp.run() for _ in range(3)]
+        line["cpu_baseline"] = {"value": smp.nbytes / statistics.mean(times) / 1e9, "unit": "GB/s",
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": smp.describe() + ", mean of 3 runs"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def kernel_hash():
+    import hashlib
+    p = os.path.join(ROOT, "quantized_decode_attention_quantize_b200", "csrc", "decode_mma.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

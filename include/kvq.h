@@ -23,7 +23,8 @@
  *    the kernels: KVQ_DEV_NONFINITE when an input element is NaN or Inf (the inputs
  *    are rejected, as the INT8 page prescribes: the affected outputs are
  *    unspecified), KVQ_DEV_RANGE when a scale, zero-point or outlier value does not
- *    fit fp16.  The caller zeroes the word and reads it back when it wants to know.
+ *    fit fp16, KVQ_DEV_TIMEOUT when a bounded in-kernel wait expired.  The caller
+ *    zeroes the word and reads it back when it wants to know.
  *  - Layouts.  B = batch, Hkv = KV heads, Hq = query heads, G = Hq / Hkv, D = head
  *    dimension.  Query head h reads KV head h / G (contiguous GQA grouping).
  *    Every cache array is [B][Hkv][slab] with the per-(b, kv-head) slab laid out as
@@ -61,8 +62,9 @@ typedef enum kvq_status {
   KVQ_ERR_WORKSPACE = 4     /* workspace smaller than kvq_decode_workspace_bytes() */
 } kvq_status;
 
-/* Bits OR-ed into the caller's device status word. */
-enum { KVQ_DEV_NONFINITE = 1, KVQ_DEV_RANGE = 2 };
+/* Bits OR-ed into the caller's device status word.  KVQ_DEV_TIMEOUT: a bounded wait
+ * inside a kernel ran out (the kernel stopped early; its outputs are unspecified). */
+enum { KVQ_DEV_NONFINITE = 1, KVQ_DEV_RANGE = 2, KVQ_DEV_TIMEOUT = 4 };
 
 /* Element types of sources, raw tokens, queries and outputs. */
 enum { KVQ_F32 = 0, KVQ_F16 = 1, KVQ_BF16 = 2 };
@@ -266,6 +268,29 @@ kvq_status kvq_decode_attention(const kvq_format* fmt, const kvq_cache* cache,
                                 void* out, int32_t out_dtype, void* workspace,
                                 size_t workspace_bytes, int32_t num_splits,
                                 int32_t* d_status, void* stream);
+
+/* The two halves of kvq_decode_attention, for callers that time, overlap or
+ * distribute them (for instance a sequence split over several GPUs that gathers the
+ * partial states before merging them).  kvq_decode_partial runs the split kernel and
+ * leaves the partial softmax states in `workspace`; kvq_decode_combine merges them
+ * into `out`.  Both must be called with the same format, sizes and num_splits as the
+ * workspace was sized for.  Workspace layout (fp32, each part padded to 16 bytes):
+ *   m[B][Hq][S], l[B][Hq][S], o[B][Hq][S][D]   with S = kvq_decode_partial_slots();
+ * slot s holds, for one query head, the running max m (log2 domain, i.e. of
+ * scale * log2(e) * q . k), l = sum 2^(score - m) and o = sum 2^(score - m) v over
+ * its share of the tokens (m = -inf, l = 0 for an empty share). */
+int32_t kvq_decode_partial_slots(const kvq_format* fmt, int32_t batch, int32_t q_heads,
+                                 int32_t kv_heads, int64_t t_quant, int32_t t_residual,
+                                 int32_t num_splits);
+kvq_status kvq_decode_partial(const kvq_format* fmt, const kvq_cache* cache, const void* q,
+                              int32_t q_dtype, int32_t q_heads, int64_t t_quant,
+                              int32_t t_residual, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, int32_t num_splits, int32_t* d_status,
+                              void* stream);
+kvq_status kvq_decode_combine(const kvq_format* fmt, int32_t batch, int32_t q_heads,
+                              int32_t kv_heads, int64_t t_quant, int32_t t_residual,
+                              int32_t num_splits, const void* workspace, size_t workspace_bytes,
+                              void* out, int32_t out_dtype, void* stream);
 
 #ifdef __cplusplus
 }

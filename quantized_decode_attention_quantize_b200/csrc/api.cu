@@ -319,28 +319,88 @@ static kvq_status decode_args(const kvq_format* f, int32_t B, int32_t Hq, int32_
   return KVQ_OK;
 }
 
+static void plan_layout(const kvq_format* f, int32_t B, int32_t Hkv, Layout* L) {
+  std::memset(L, 0, sizeof(*L));
+  L->D = f->head_dim;
+  L->g = f->group_tokens;
+  L->B = B;
+  L->Hkv = Hkv;
+  L->n_sink = f->n_sink;
+  L->side[0].scheme = f->k_scheme;
+  L->side[0].bits = f->k_bits;
+  L->side[0].axis = f->k_axis;
+  L->side[0].nout = f->k_scheme == KVQ_NUQ ? f->k_outliers : 0;
+  L->side[1].scheme = f->v_scheme;
+  L->side[1].bits = f->v_bits;
+  L->side[1].axis = f->v_axis;
+  L->side[1].nout = f->v_scheme == KVQ_NUQ ? f->v_outliers : 0;
+  L->rope = f->rope;
+  L->src_dtype = f->src_dtype;
+}
+
 size_t kvq_decode_workspace_bytes(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,
                                   int64_t t_quant, int32_t t_res, int32_t num_splits) {
   if (decode_args(f, B, Hq, Hkv, t_quant, t_res, num_splits) != KVQ_OK) return 0;
   Layout L;
-  std::memset(&L, 0, sizeof(L));
-  L.D = f->head_dim;
-  L.g = f->group_tokens;
-  L.B = B;
-  L.Hkv = Hkv;
-  L.n_sink = f->n_sink;
-  L.side[0].scheme = f->k_scheme;
-  L.side[0].bits = f->k_bits;
-  L.side[0].axis = f->k_axis;
-  L.side[0].nout = f->k_scheme == KVQ_NUQ ? f->k_outliers : 0;
-  L.side[1].scheme = f->v_scheme;
-  L.side[1].bits = f->v_bits;
-  L.side[1].axis = f->v_axis;
-  L.side[1].nout = f->v_scheme == KVQ_NUQ ? f->v_outliers : 0;
-  L.rope = f->rope;
-  L.src_dtype = f->src_dtype;
+  plan_layout(f, B, Hkv, &L);
   DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
   return workspace_bytes(L, Hq, p);
+}
+
+int32_t kvq_decode_partial_slots(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,
+                                 int64_t t_quant, int32_t t_res, int32_t num_splits) {
+  if (decode_args(f, B, Hq, Hkv, t_quant, t_res, num_splits) != KVQ_OK) return 0;
+  Layout L;
+  plan_layout(f, B, Hkv, &L);
+  return plan_decode(L, Hq, t_quant, t_res, num_splits).S;
+}
+
+static kvq_status partial_common(const kvq_format* f, const kvq_cache* c, const void* q,
+                                 int32_t q_dtype, int32_t Hq, int64_t t_quant, int32_t t_res,
+                                 float scale, void* ws, size_t ws_bytes, int32_t num_splits,
+                                 int32_t* d_status, void* stream, Layout* L, DecodePlan* p) {
+  kvq_status s = make_layout(f, c, L);
+  if (s != KVQ_OK) return s;
+  s = decode_args(f, L->B, Hq, L->Hkv, t_quant, t_res, num_splits);
+  if (s != KVQ_OK) return s;
+  if (t_quant > L->C) return KVQ_ERR_INVALID;
+  if (!q || !aligned16(q) || !valid_dtype(q_dtype) || !(scale > 0.0f)) return KVQ_ERR_INVALID;
+  if (L->n_sink && (!L->sink[0] || !L->sink[1] || !aligned16(L->sink[0]) || !aligned16(L->sink[1])))
+    return KVQ_ERR_INVALID;
+  if (t_res && (!L->res[0] || !L->res[1] || !aligned16(L->res[0]) || !aligned16(L->res[1])))
+    return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  *p = plan_decode(*L, Hq, t_quant, t_res, num_splits);
+  if (!ws || !aligned16(ws)) return KVQ_ERR_INVALID;
+  if (ws_bytes < workspace_bytes(*L, Hq, *p)) return KVQ_ERR_WORKSPACE;
+  cudaError_t e = launch_decode_partial(*L, *p, q, q_dtype, Hq, t_quant, t_res, scale, ws, d_status,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_decode_partial(const kvq_format* f, const kvq_cache* c, const void* q,
+                              int32_t q_dtype, int32_t Hq, int64_t t_quant, int32_t t_res,
+                              float scale, void* ws, size_t ws_bytes, int32_t num_splits,
+                              int32_t* d_status, void* stream) {
+  Layout L;
+  DecodePlan p;
+  return partial_common(f, c, q, q_dtype, Hq, t_quant, t_res, scale, ws, ws_bytes, num_splits,
+                        d_status, stream, &L, &p);
+}
+
+kvq_status kvq_decode_combine(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,
+                              int64_t t_quant, int32_t t_res, int32_t num_splits, const void* ws,
+                              size_t ws_bytes, void* out, int32_t out_dtype, void* stream) {
+  kvq_status s = decode_args(f, B, Hq, Hkv, t_quant, t_res, num_splits);
+  if (s != KVQ_OK) return s;
+  if (!out || !aligned16(out) || !valid_dtype(out_dtype) || !ws || !aligned16(ws))
+    return KVQ_ERR_INVALID;
+  Layout L;
+  plan_layout(f, B, Hkv, &L);
+  DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
+  if (ws_bytes < workspace_bytes(L, Hq, p)) return KVQ_ERR_WORKSPACE;
+  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 kvq_status kvq_decode_attention(const kvq_format* f, const kvq_cache* c, const void* q,
@@ -348,25 +408,13 @@ kvq_status kvq_decode_attention(const kvq_format* f, const kvq_cache* c, const v
                                 float scale, void* out, int32_t out_dtype, void* ws,
                                 size_t ws_bytes, int32_t num_splits, int32_t* d_status,
                                 void* stream) {
+  if (!out || !aligned16(out) || !valid_dtype(out_dtype)) return KVQ_ERR_INVALID;
   Layout L;
-  kvq_status s = make_layout(f, c, &L);
+  DecodePlan p;
+  kvq_status s = partial_common(f, c, q, q_dtype, Hq, t_quant, t_res, scale, ws, ws_bytes,
+                                num_splits, d_status, stream, &L, &p);
   if (s != KVQ_OK) return s;
-  s = decode_args(f, L.B, Hq, L.Hkv, t_quant, t_res, num_splits);
-  if (s != KVQ_OK) return s;
-  if (t_quant > L.C) return KVQ_ERR_INVALID;
-  if (!q || !aligned16(q) || !out || !aligned16(out) || !valid_dtype(q_dtype) ||
-      !valid_dtype(out_dtype) || !(scale > 0.0f))
-    return KVQ_ERR_INVALID;
-  if (L.n_sink && (!L.sink[0] || !L.sink[1] || !aligned16(L.sink[0]) || !aligned16(L.sink[1])))
-    return KVQ_ERR_INVALID;
-  if (t_res && (!L.res[0] || !L.res[1] || !aligned16(L.res[0]) || !aligned16(L.res[1])))
-    return KVQ_ERR_INVALID;
-  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
-  DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
-  if (!ws || !aligned16(ws)) return KVQ_ERR_INVALID;
-  if (ws_bytes < workspace_bytes(L, Hq, p)) return KVQ_ERR_WORKSPACE;
-  cudaError_t e = launch_decode(L, p, q, q_dtype, Hq, t_quant, t_res, scale, out, out_dtype, ws,
-                                d_status, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

@@ -16,7 +16,10 @@ namespace kvq {
 
 // Fast tensor-core path (decode_mma.cu)
 bool mma_path_ok(const Layout& L, int Hq);
-int mma_ctas_per_sm();
+void plan_mma(const Layout& L, int64_t t_quant, int t_res, int max_ctas, DecodePlan& p);
+cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, const float* ws_m,
+                               const float* ws_l, const float* ws_o, void* out, int out_dtype,
+                               cudaStream_t s);
 cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
                               int Hq, int64_t t_quant, int t_res, float scale, float* ws_m,
                               float* ws_l, float* ws_o, int32_t* d_status, cudaStream_t s);
@@ -295,14 +298,19 @@ DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int 
   const bool raw = L.n_sink + t_res > 0;
   const int64_t heads = (int64_t)L.B * L.Hkv;
   p.fast = (ngv > 0 && fast_path_ok(L, Hq)) ? 1 : 0;
+  p.raw_pieces = 0;
+  if (p.fast) {
+    // persistent partition over (head, group) units; num_splits caps the CTA count
+    plan_mma(L, t_quant, t_res, num_splits, p);
+    return p;
+  }
   int sp = 0, sg = 1;
   if (ngv > 0) {
     int64_t want;
     if (num_splits > 0) {
       want = num_splits;
     } else {
-      const int sms = device_sm_count();
-      const int64_t target = p.fast ? (int64_t)sms * mma_ctas_per_sm() : (int64_t)sms * 8;
+      const int64_t target = (int64_t)device_sm_count() * 8;
       want = (target + heads - 1) / heads;
     }
     want = std::max<int64_t>(1, std::min<int64_t>(want, ngv));
@@ -322,13 +330,15 @@ size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p) {
   return align16(rows * 4) * 2 + align16(rows * L.D * 4);
 }
 
-cudaError_t launch_decode(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
-                          int64_t t_quant, int t_res, float scale, void* out, int out_dtype,
-                          void* ws, int32_t* d_status, cudaStream_t s) {
+cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
+                                  int Hq, int64_t t_quant, int t_res, float scale, void* ws,
+                                  int32_t* d_status, cudaStream_t s) {
   const size_t rows = (size_t)L.B * Hq * p.S;
   float* ws_m = reinterpret_cast<float*>(ws);
   float* ws_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align16(rows * 4));
   float* ws_o = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4));
+  if (p.fast)
+    return launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
   DecArgs a;
   a.L = L;
   a.q = q;
@@ -345,63 +355,33 @@ cudaError_t launch_decode(const Layout& L, const DecodePlan& p, const void* q, i
   a.ws_l = ws_l;
   a.ws_o = ws_o;
   a.status = d_status;
-  cudaError_t e = cudaSuccess;
-  if (p.fast) {
-    e = launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
-  } else {
-    switch (L.D) {
-      case 32: e = launch_generic<1>(a, p.S, s); break;
-      case 64: e = launch_generic<2>(a, p.S, s); break;
-      case 128: e = launch_generic<4>(a, p.S, s); break;
-      default: e = launch_generic<8>(a, p.S, s); break;
-    }
+  switch (L.D) {
+    case 32: return launch_generic<1>(a, p.S, s);
+    case 64: return launch_generic<2>(a, p.S, s);
+    case 128: return launch_generic<4>(a, p.S, s);
+    default: return launch_generic<8>(a, p.S, s);
   }
-  if (e != cudaSuccess) return e;
+}
+
+cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
+                           int out_dtype, cudaStream_t s) {
+  const size_t rows = (size_t)L.B * Hq * p.S;
+  const float* m = reinterpret_cast<const float*>(ws);
+  const float* l = reinterpret_cast<const float*>(reinterpret_cast<const char*>(ws) + align16(rows * 4));
+  const float* o = reinterpret_cast<const float*>(reinterpret_cast<const char*>(ws) + 2 * align16(rows * 4));
+  if (p.fast) return launch_combine_mma(L, p, Hq, m, l, o, out, out_dtype, s);
   CombArgs c;
   c.D = L.D;
   c.Hq = Hq;
   c.S = p.S;
-  c.m = ws_m;
-  c.l = ws_l;
-  c.o = ws_o;
+  c.m = m;
+  c.l = l;
+  c.o = o;
   c.out = out;
   c.out_dtype = out_dtype;
   dim3 grid(Hq, L.B);
   combine_kernel<<<grid, L.D < 256 ? L.D : 256, 0, s>>>(c);
   return cudaGetLastError();
-}
-
-// Generic kernel entry used by the fast path for its raw (sink + residual) slot.
-cudaError_t launch_decode_raw_generic(const Layout& L, const DecodePlan& p, const void* q,
-                                      int q_dtype, int Hq, int64_t t_quant, int t_res, float scale,
-                                      float* ws_m, float* ws_l, float* ws_o, int32_t* d_status,
-                                      cudaStream_t s) {
-  DecArgs a;
-  a.L = L;
-  a.q = q;
-  a.q_dtype = q_dtype;
-  a.Hq = Hq;
-  a.t_quant = t_quant;
-  a.t_res = t_res;
-  a.qscale = scale * kLog2e;
-  a.S = p.S;
-  a.split_groups = p.split_groups;
-  a.n_packed = 0;          // no packed splits: only CTA x = raw_slot does work
-  a.raw_slot = 0;
-  a.ws_m = ws_m;
-  a.ws_l = ws_l;
-  a.ws_o = ws_o;
-  a.status = d_status;
-  // write into slot p.raw_slot: offset the partial arrays so that split index 0 maps there
-  a.ws_m = ws_m + p.raw_slot;
-  a.ws_l = ws_l + p.raw_slot;
-  a.ws_o = ws_o + (size_t)p.raw_slot * L.D;
-  switch (L.D) {
-    case 32: return launch_generic<1>(a, 1, s);
-    case 64: return launch_generic<2>(a, 1, s);
-    case 128: return launch_generic<4>(a, 1, s);
-    default: return launch_generic<8>(a, 1, s);
-  }
 }
 
 }  // namespace kvq

@@ -52,6 +52,10 @@ kvq_status make_layout(const kvq_format* f, const kvq_cache* c, Layout* L);
 cudaError_t launch_quantize(const Layout& L, int which, const void* src, int64_t sb,
                             int64_t sh, int64_t st, int64_t t0, int64_t n,
                             int32_t* d_status, cudaStream_t s);
+bool asym_fast_ok(const Layout& L, int which);
+cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, int64_t sb,
+                                 int64_t sh, int64_t st, int64_t t0, int64_t n,
+                                 int32_t* d_status, cudaStream_t s);
 cudaError_t launch_dequantize(const Layout& L, int which, int64_t t0, int64_t n, void* out,
                               int out_dtype, int32_t* d_status, cudaStream_t s);
 cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t qsh,
@@ -61,18 +65,21 @@ cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t
 
 struct DecodePlan {
   int S;                // partial slots per query head
-  int split_groups;     // packed groups per packed split (generic path)
-  int n_packed_splits;  // splits over the packed region
-  int raw_slot;         // slot index of the raw (sink + residual) segment, -1 if none
+  int split_groups;     // generic path: packed groups per split
+  int n_packed_splits;  // generic path: splits over the packed region; fast path: groups per head
+  int raw_slot;         // generic path: slot of the raw (sink + residual) tokens, -1 if none
+  int raw_pieces;       // fast path: raw-token units per head
   int fast;             // 1 when the tensor-core K4/V2 kernel runs the packed region
   int grid_ctas;        // CTAs of the split kernel
 };
 DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int num_splits);
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p);
 bool fast_path_ok(const Layout& L, int Hq);
-cudaError_t launch_decode(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
-                          int Hq, int64_t t_quant, int t_res, float scale, void* out,
-                          int out_dtype, void* ws, int32_t* d_status, cudaStream_t s);
+cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q,
+                                  int q_dtype, int Hq, int64_t t_quant, int t_res, float scale,
+                                  void* ws, int32_t* d_status, cudaStream_t s);
+cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
+                           int out_dtype, cudaStream_t s);
 int device_sm_count();
 
 // ---------------------------------------------------------------------------

@@ -532,6 +532,7 @@ size_t quantize_smem(const Layout& L) {
 cudaError_t launch_quantize(const Layout& L, int which, const void* src, int64_t sb, int64_t sh,
                             int64_t st, int64_t t0, int64_t n, int32_t* d_status,
                             cudaStream_t s) {
+  if (asym_fast_ok(L, which)) return launch_quantize_asym(L, which, src, sb, sh, st, t0, n, d_status, s);
   QArgs a;
   a.L = L;
   a.which = which;

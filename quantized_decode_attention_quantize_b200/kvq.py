@@ -79,6 +79,10 @@ def lib():
             "kvq_decode_workspace_bytes": (SZ, [FP, I32, I32, I32, I64, I32, I32]),
             "kvq_decode_attention": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, I32,
                                            P, SZ, I32, P, P]),
+            "kvq_decode_partial_slots": (I32, [FP, I32, I32, I32, I64, I32, I32]),
+            "kvq_decode_partial": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, SZ, I32,
+                                         P, P]),
+            "kvq_decode_combine": (I32, [FP, I32, I32, I32, I64, I32, I32, P, SZ, P, I32, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -206,4 +210,26 @@ def decode_attention(fmt, cache: Cache, q: torch.Tensor, t_quant: int, t_res: in
                                     _ptr(workspace), workspace.numel(), num_splits, _ptr(status),
                                     _stream(stream))
     _check("kvq_decode_attention", st)
+    return out
+
+
+def decode_partial_slots(fmt, B, Hq, Hkv, t_quant, t_res, num_splits=0) -> int:
+    return lib().kvq_decode_partial_slots(ctypes.byref(fmt), B, Hq, Hkv, t_quant, t_res, num_splits)
+
+
+def decode_partial(fmt, cache: Cache, q: torch.Tensor, t_quant: int, t_res: int, scale: float,
+                   workspace: torch.Tensor, num_splits=0, status=None, stream=None):
+    B, Hq, D = q.shape
+    st = lib().kvq_decode_partial(ctypes.byref(fmt), cache.ref(), _ptr(q), KVQ_DTYPE[q.dtype], Hq,
+                                  t_quant, t_res, scale, _ptr(workspace), workspace.numel(),
+                                  num_splits, _ptr(status), _stream(stream))
+    _check("kvq_decode_partial", st)
+
+
+def decode_combine(fmt, B, Hq, Hkv, t_quant, t_res, workspace: torch.Tensor, out: torch.Tensor,
+                   num_splits=0, stream=None):
+    st = lib().kvq_decode_combine(ctypes.byref(fmt), B, Hq, Hkv, t_quant, t_res, num_splits,
+                                  _ptr(workspace), workspace.numel(), _ptr(out),
+                                  KVQ_DTYPE[out.dtype], _stream(stream))
+    _check("kvq_decode_combine", st)
     return out

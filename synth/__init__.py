@@ -77,10 +77,12 @@ def rng(seed, tag, *idx):
 
 
 def to_bf16_values(x32):
-    """float32 -> nearest-even bf16, returned as float32 values."""
-    u = np.ascontiguousarray(x32, np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return (u.astype(np.uint32) << 16).view(np.float32)
+    """float32 (finite, below the bf16 overflow threshold) -> nearest-even bf16,
+    returned as float32 values."""
+    u = np.array(x32, np.float32, copy=True).view(np.uint32)
+    u += np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    u &= np.uint32(0xFFFF0000)
+    return u.view(np.float32)
 
 
 def to_dtype_values(x, dtype):
@@ -94,10 +96,14 @@ def to_dtype_values(x, dtype):
 
 
 def student_t4(r, shape):
-    """Student-t with 4 degrees of freedom: N / sqrt(chi2_4 / 4)."""
+    """Student-t with 4 degrees of freedom: N / sqrt(chi2_4 / 4), chi2_4 the sum of
+    four squared standard normals."""
     n = r.standard_normal(shape, dtype=np.float32)
-    chi = r.standard_gamma(2.0, size=shape).astype(np.float32) * 2.0   # chi2 with 4 dof
-    return n / np.sqrt(chi / 4.0)
+    chi = np.zeros(shape, np.float32)
+    for _ in range(4):
+        z = r.standard_normal(shape, dtype=np.float32)
+        chi += z * z
+    return n / np.sqrt(chi * np.float32(0.25))
 
 
 def log_uniform(r, lo, hi, shape):
@@ -183,3 +189,59 @@ def random_slab(seed, shape, dtype, scale=1.0, tag="k", idx=()):
     """Plain N(0, scale^2) values in a dtype (small parity cases)."""
     r = rng(seed, tag, *idx)
     return to_dtype_values(r.standard_normal(shape, dtype=np.float32) * np.float32(scale), dtype)
+
+
+# ---- device-side generation of bulk data ------------------------------------------------
+# The same recipes drawn with torch's generator on the device, for full-size caches
+# whose every slab need not be regenerated on the host (timing runs, and the slabs a
+# full-size parity test does not sample).  Values differ from the host streams; the
+# distributions and structure are the same.
+
+def device_kv(cfg, which, T=None, B=None, H=None, device="cuda", seed_offset=0):
+    """[B, Hkv, T, D] tensor of keys or values in the source dtype, on the device."""
+    import torch
+    T = cfg["T"] if T is None else T
+    B = cfg["B"] if B is None else B
+    H = cfg["Hkv"] if H is None else H
+    D = cfg["D"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(cfg["seed"] * 1000 + TAGS[which] * 10 + seed_offset)
+    tdt = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}[cfg["fmt"]["src_dtype"]]
+    shape = (B, H, T, D)
+    name = cfg["name"]
+    cpu = torch.Generator()
+    cpu.manual_seed(cfg["seed"] * 1000 + TAGS[which] * 10 + seed_offset + 7)
+    out = torch.empty(shape, dtype=tdt, device=device)
+    for b in range(B):
+        for h in range(H):
+            if name == "llama3_8b":
+                n = torch.randn((T, D), generator=gen, device=device)
+                chi = torch.zeros((T, D), device=device)
+                for _ in range(4):
+                    z = torch.randn((T, D), generator=gen, device=device)
+                    chi += z * z
+                x = n / torch.sqrt(chi * 0.25)
+                if which == "k":
+                    ch = torch.randperm(D, generator=cpu)[: int(round(0.02 * D))]
+                    x[:, ch] *= 10.0
+            else:
+                x = torch.randn((T, D), generator=gen, device=device)
+                if which == "k":
+                    if name == "llama2_7b":
+                        ch = torch.randperm(D, generator=cpu)[:4]
+                        x[:, ch] *= 15.0
+                    elif name in ("kvquant_nuq3", "mixkvq_14b"):
+                        hi = 10.0 if name == "kvquant_nuq3" else 20.0
+                        u = torch.rand(D, generator=cpu)
+                        x *= torch.exp(np.log(0.1) + u * (np.log(hi) - np.log(0.1))).to(device)
+            out[b, h] = x.to(tdt)
+    return out
+
+
+def device_queries(cfg, B=None, Hq=None, device="cuda"):
+    """[B, Hq, D] decode queries in the query dtype, on the device."""
+    import torch
+    B = cfg["B"] if B is None else B
+    Hq = cfg["Hq"] if Hq is None else Hq
+    q = torch.tensor(queries(cfg, B, Hq), device=device)
+    return q.to({F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}[cfg["q_dtype"]])

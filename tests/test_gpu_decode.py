@@ -174,3 +174,21 @@ def test_nonfinite_query_flagged():
     q[0, 1, 5] = np.inf
     kvq.decode_attention(p.fmt, p.gpu, dev(q, F16), 128, 0, 0.1, F32, status=p.status)
     assert p.status_bits() & kvq.KVQ_DEV_NONFINITE
+
+
+@pytest.mark.parametrize("B,H,G,tq,ns,tr,splits", [
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 0),
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 1),
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 13),
+    (2, 3, 8, 5, 1, 0, 4),
+    (1, 7, 4, 9 * 128, 0, 100, 0),
+    (4, 2, 3, 3 * 128 - 7, 4, 11, 2),
+])
+def test_partition_shapes(B, H, G, tq, ns, tr, splits):
+    # the persistent partition over (head, group) units with raw-token pieces: heads
+    # spanning several CTAs, CTAs spanning several heads, tiny and ragged regions
+    fd = fmt(src_dtype=BF16, n_sink=ns, residual_cap=128)
+    p = build(fd, B, H, G * H, tq, tr, seed=40 + tq)
+    out, ref = run(p, G * H, tq, tr, BF16, F32, seed=40 + tq, num_splits=splits)
+    assert rel_l2(out, ref) <= 1e-3
+    assert p.status_bits() == 0
