@@ -292,6 +292,29 @@ kvq_status kvq_decode_combine(const kvq_format* fmt, int32_t batch, int32_t q_he
                               int32_t num_splits, const void* workspace, size_t workspace_bytes,
                               void* out, int32_t out_dtype, void* stream);
 
+/* Decode attention without a caller workspace, for callers that cannot allocate
+ * device memory at all -- for example a serving process whose allocator reserved
+ * every byte at start-up, or a plugin host that forbids allocation once running --
+ * and so can neither call cudaMalloc nor pass `workspace`.  The pages describe no
+ * such interface; it has no counterpart there.
+ *
+ * Same arguments, kernels and results as kvq_decode_attention, minus the workspace:
+ * the partial softmax states go to a fixed array of KVQ_NOALLOC_SCRATCH_BYTES inside
+ * the library (every GPU that loads the library holds it until the process exits).
+ * Nothing is allocated and nothing is freed.  Returns KVQ_ERR_WORKSPACE when the
+ * call would need more than KVQ_NOALLOC_SCRATCH_BYTES (see
+ * kvq_decode_workspace_bytes).  The first call on a device looks up the array's
+ * device address (with that device current) and keeps it for later calls; make that
+ * first call outside any stream capture.  All calls on a device share the one array
+ * and it keeps the last call's contents: calls that overlap on the GPU (on different
+ * streams, or from different host threads) race with one another. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+kvq_status kvq_decode_attention_noalloc(const kvq_format* fmt, const kvq_cache* cache,
+                                        const void* q, int32_t q_dtype, int32_t q_heads,
+                                        int64_t t_quant, int32_t t_residual, float softmax_scale,
+                                        void* out, int32_t out_dtype, int32_t num_splits,
+                                        int32_t* d_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

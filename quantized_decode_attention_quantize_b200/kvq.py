@@ -83,6 +83,8 @@ def lib():
             "kvq_decode_partial": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, SZ, I32,
                                          P, P]),
             "kvq_decode_combine": (I32, [FP, I32, I32, I32, I64, I32, I32, P, SZ, P, I32, P]),
+            "kvq_decode_attention_noalloc": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float,
+                                                   P, I32, I32, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -232,4 +234,22 @@ def decode_combine(fmt, B, Hq, Hkv, t_quant, t_res, workspace: torch.Tensor, out
                                   _ptr(workspace), workspace.numel(), _ptr(out),
                                   KVQ_DTYPE[out.dtype], _stream(stream))
     _check("kvq_decode_combine", st)
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_attention_noalloc(fmt, cache: Cache, q: torch.Tensor, t_quant: int, t_res: int,
+                             scale: float, out_dtype=F32, out=None, num_splits=0, status=None,
+                             stream=None):
+    """kvq_decode_attention_noalloc: no workspace argument (the library's own scratch)."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=TORCH_DTYPE[out_dtype], device=q.device)
+    st = lib().kvq_decode_attention_noalloc(ctypes.byref(fmt), cache.ref(), _ptr(q),
+                                            KVQ_DTYPE[q.dtype], Hq, t_quant, t_res, scale,
+                                            _ptr(out), out_dtype, num_splits, _ptr(status),
+                                            _stream(stream))
+    _check("kvq_decode_attention_noalloc", st)
     return out
