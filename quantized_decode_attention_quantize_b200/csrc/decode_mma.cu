@@ -2,19 +2,27 @@
 // per-token values (the K4V2 allocation of [K4V2]; grouping of [KVQ] "Approach"),
 // D = 128, token groups of 128, 2 <= G <= 8 query heads per KV head.
 //
-// Work.  Units are the packed token groups of every KV head plus a few pieces of
-// each head's raw (sink + residual) tokens, in head-major order.  One CTA per SM
-// takes a contiguous range of units; its twelve warps take the range's
-// units round-robin.  A warp keeps one online-softmax state per (head, unit kind)
-// and writes it to its own partial slot when it moves on; the combine kernel finds
-// the slots of a head from the same partition.  No warp ever waits for another.
+// Work.  Each KV head is a row of U items: first its raw (sink + residual) tokens in
+// items of up to 8 tokens (4 for fp32 sources), each weighted as two positions of
+// the row (the second carries no work: a raw item costs about two half groups), then
+// its packed tokens in half groups of 64.  The rows of all heads, end to end, are cut
+// into one contiguous range of positions per warp, as equal as integers allow; the
+// twelve warps of a CTA hold consecutive ranges.  Warp ranges never exceed U
+// positions, so a warp touches at most two heads.  A warp keeps one online-softmax state; when its range crosses from one
+// head into the next, the state of the first goes straight to that head's partial
+// slot 0.  At the end the warps of a CTA merge, per head, the states they hold in
+// shared memory, and the CTA writes one partial state per head into slot
+// 1 + (CTA - first CTA holding the head).  The combine kernel derives every valid
+// slot of a head from the same partition.  No warp ever waits for another warp except
+// at the one CTA barrier before the merge.
 //
-// Memory.  Every warp streams its own units through a ring of two half-group
-// stages in shared memory with 16-byte cp.async copies (all 32 lanes, coalesced): per
-// 64 tokens the key codes (4 KiB), value codes (2 KiB), value scale / zero-point
-// (256 B) and, with the first half, the group's key scale / zero-point (512 B).
-// Every byte of the format is read once; the next half group is in flight while the
-// warp computes on the current one (twelve warps per SM).
+// Memory.  Every warp streams its items through a ring of two stages in shared
+// memory with 16-byte cp.async copies (all 32 lanes, coalesced): per half group the
+// key codes (4 KiB), value codes (2 KiB), value scale / zero-point (256 B) and, when
+// the half opens the group for this warp, the group's key scale / zero-point (512 B);
+// per raw item its key and value rows.  The copy of the next item is issued before
+// the math on the current one, so every warp keeps one item in flight while it
+// computes; every byte of the format is read once.
 //
 // Math.  A 4-bit or 2-bit code masked into the low mantissa bits of an fp16 half with
 // a zero exponent field is the subnormal number c * 2^-24 * f, exact, where f = 2^p
@@ -26,15 +34,17 @@
 // and an fp16 remainder so that the key product carries ~22 bits: with G <= 4 the two
 // parts ride in the otherwise empty columns 4..7 of the same product (hi in column h,
 // remainder in column h + 4, summed with one shuffle); with G > 4 they take two
-// products.  The probabilities become the B
-// operand of the value product through an in-register 8x8 transpose (movmatrix) and
-// the value codes (pair layout) are the A operand with channels as M:
+// products.  The probabilities become the B operand of the value product through an
+// in-register 8x8 transpose (movmatrix) and the value codes (pair layout) are the A
+// operand with channels as M:
 //   A[d][t] = c[t][d] 2^-24 f_d,   B[t][h] = fp16(p[t][h] s[t])
 //   o[h][d] = 2^24 / f_d (A.B)[d][h] + sum_t p[t][h] z[t].
-// Online softmax is kept in the log2 domain.
+// Raw tokens are scored in fp32 on CUDA cores and accumulated in fp32 into the same
+// accumulator tiles (scaled by the tile's f_d / 2^24).  Online softmax is kept in the
+// log2 domain.
 //
-// Waits.  A warp only waits for its own copies (cp.async.wait_group); no warp waits for
-// another.
+// Waits.  A warp only waits for its own copies (cp.async.wait_group) and, once, at
+// the CTA barrier before the merge, which every warp reaches.
 #include <algorithm>
 #include <cstdint>
 
@@ -45,15 +55,18 @@ namespace kvq {
 namespace {
 
 constexpr int kCW = 12;                       // warps per CTA (one CTA per SM)
-constexpr int kBuffers = 2;                   // per-warp ring of half-group stages
+constexpr int kBuffers = 2;                   // per-warp ring of item stages
 constexpr int kThreads = kCW * 32;
-// a stage holds 64 tokens: key codes, value codes, value scale / zero-point, and (first
-// half only) the group's key scale / zero-point
+// a half-group stage holds 64 tokens: key codes, value codes, value scale / zero-point,
+// and (when the half opens the group for the warp) the group's key scale / zero-point
 constexpr int kHalfK = 64 * 64, kHalfV = 32 * 64, kHalfVM = 2 * 64 * 2, kHalfKM = 2 * 128 * 2;
 constexpr int kStageBytes = kHalfK + kHalfV + kHalfVM + kHalfKM;
+constexpr int kRawBytes = 2048;               // raw item: key rows, then value rows at +kRawBytes
 constexpr int kScratchBytes = 2 * 32 * 16 * 4;  // per warp: hi and lo B fragments
-constexpr int kRawPieces = 12;                // raw-token units per head (<= kCW)
+constexpr int kRecordFloats = 8 * 130;        // merge record: o[G][128], m[G], l[G]
 constexpr float kLog2e = 1.4426950408889634f;
+static_assert(2 * kRawBytes <= kStageBytes, "raw item fits a stage");
+static_assert(kRecordFloats * 4 <= kBuffers * kStageBytes, "record fits the warp's ring");
 
 struct MmaArgs {
   const uint8_t* k_codes;
@@ -65,7 +78,7 @@ struct MmaArgs {
   int64_t k_slab_bytes, v_slab_bytes;
   int64_t C;
   int ng;
-  int B, Hkv, Hq, G;
+  int Hkv, Hq, G;
   int64_t t_quant;
   int t_res, n_sink, res_cap, src_dtype;
   const void* sink_k;
@@ -75,17 +88,45 @@ struct MmaArgs {
   const void* q;
   int q_dtype;
   float qscale;
-  int ngv;        // valid groups per head
-  int rw;         // raw pieces per head
-  int uph;        // units per head (rw + ngv)
-  int64_t N;      // total units
-  int grid;
+  int nrp;        // raw positions per head (two per raw item)
+  int rt;         // raw tokens per raw item
+  int U;          // positions per head (nrp + packed halves)
+  int64_t I;      // positions in all
+  int64_t W;      // warps in all (grid * kCW)
   int S;          // partial slots per query head
   float* ws_m;
   float* ws_l;
   float* ws_o;
   int32_t* status;
 };
+
+// ---- partition of the items over the warps (shared with the combine kernel) ------------
+// Warp gw holds items [item_start(gw), item_start(gw + 1)).
+__host__ __device__ __forceinline__ int64_t item_start(int64_t gw, int64_t I, int64_t W) {
+  return gw * I / W;
+}
+// The warp holding item x.
+__host__ __device__ __forceinline__ int64_t warp_of_item(int64_t x, int64_t I, int64_t W) {
+  return ((x + 1) * W - 1) / I;
+}
+// Warps whose range ends inside head h (including empty warps placed there): the
+// first is the least gw with item_start(gw + 1) >= h U + 1, the last the greatest gw
+// with item_start(gw + 1) <= (h + 1) U.
+__host__ __device__ __forceinline__ int64_t first_ending_warp(int64_t h, int64_t U, int64_t I, int64_t W) {
+  const int64_t x = h * U + 1;
+  return (x * W + I - 1) / I - 1;
+}
+__host__ __device__ __forceinline__ int64_t last_ending_warp(int64_t h, int64_t U, int64_t I, int64_t W) {
+  const int64_t y = (h + 1) * U + 1;
+  const int64_t w = (y * W + I - 1) / I - 2;
+  return w < W - 1 ? w : W - 1;
+}
+// Head h's state that a warp carries out of h into h + 1 (slot 0) exists iff the warp
+// holding the head's last item runs past it.
+__host__ __device__ __forceinline__ bool has_crossing(int64_t h, int64_t U, int64_t I, int64_t W) {
+  const int64_t last = (h + 1) * U - 1;
+  return item_start(warp_of_item(last, I, W) + 1, I, W) > last + 1;
+}
 
 // ---- PTX helpers ------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -118,20 +159,8 @@ __device__ __forceinline__ float pow2(int e) { return __uint_as_float((uint32_t)
 // byte 1 -> byte 0 and byte 3 -> byte 2 (other bytes zero)
 __device__ __forceinline__ uint32_t odd_bytes_down(uint32_t w) { return __byte_perm(w, 0u, 0x4341u); }
 
-// ---- unit partition (shared with the combine kernel) -----------------------------
-__host__ __device__ __forceinline__ int64_t unit_start(int64_t c, int64_t N, int grid) {
-  return c * N / grid;
-}
-__host__ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t N, int grid) {
-  return (int)(((u + 1) * grid - 1) / N);
-}
-// slot of (CTA c, warp w, kind) within the head whose first CTA is c0
-__host__ __device__ __forceinline__ int slot_of(int c, int c0, int w, int kind) {
-  return ((c - c0) * kCW + w) * 2 + kind;
-}
-
-// ---- raw tokens (sink + residual) on CUDA cores ----------------------------------------
-// Four consecutive elements at element offset i (i a multiple of 4).
+// Four consecutive elements at element offset i (i a multiple of 4) of a raw row
+// (global or shared memory).
 __device__ __forceinline__ float4 load4(const void* p, int64_t i, int dtype) {
   if (dtype == KVQ_F32) return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i);
   const uint2 x = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(p) + i);
@@ -144,102 +173,15 @@ __device__ __forceinline__ float4 load4(const void* p, int64_t i, int dtype) {
                      __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u));
 }
 
-// Lane owns channels 4 lane .. 4 lane + 3; fp32, log2 domain.  Tokens go four at a
-// time: their loads are issued together, the 4 x G score reductions of a chunk are
-// independent, then one softmax update per chunk.  Writes the piece's slot.
-template <int GM>
-__device__ void raw_piece(const MmaArgs& a, int head, int piece, int slot) {
-  constexpr int kBatch = 4;
-  const int lane = threadIdx.x & 31;
-  const int b = head / a.Hkv, h = head % a.Hkv;
-  const int G = a.G;
-  const int nraw = a.n_sink + a.t_res;
-  const int r0 = piece * nraw / a.rw, r1 = (piece + 1) * nraw / a.rw;
-  float q[GM][4], o[GM][4], m[GM], l[GM];
-#pragma unroll
-  for (int hh = 0; hh < GM; ++hh) {
-    m[hh] = -INFINITY;
-    l[hh] = 0.0f;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (hh < G) x = load4(a.q, ((int64_t)b * a.Hq + h * G + hh) * 128 + 4 * lane, a.q_dtype);
-    q[hh][0] = x.x * a.qscale; q[hh][1] = x.y * a.qscale;
-    q[hh][2] = x.z * a.qscale; q[hh][3] = x.w * a.qscale;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) o[hh][k] = 0.0f;
-  }
-  auto fetch = [&](int rb, float4 (&kt)[kBatch], float4 (&vt)[kBatch]) {
-#pragma unroll
-    for (int e = 0; e < kBatch; ++e) {
-      const int r = rb + e;
-      kt[e] = vt[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < r1) {
-        const bool sink = r < a.n_sink;
-        const int64_t row = sink ? r : r - a.n_sink;
-        const int64_t rows = sink ? a.n_sink : a.res_cap;
-        const int64_t i = ((int64_t)head * rows + row) * 128 + 4 * lane;
-        kt[e] = load4(sink ? a.sink_k : a.res_k, i, a.src_dtype);
-        vt[e] = load4(sink ? a.sink_v : a.res_v, i, a.src_dtype);
-      }
-    }
-  };
-  float4 kt[kBatch], vt[kBatch];
-  for (int rb = r0; rb < r1; rb += kBatch) {
-    fetch(rb, kt, vt);
-    float sc[kBatch][GM];
-#pragma unroll
-    for (int e = 0; e < kBatch; ++e)
-#pragma unroll
-      for (int hh = 0; hh < GM; ++hh) {
-        float part = q[hh][0] * kt[e].x;
-        part = fmaf(q[hh][1], kt[e].y, part);
-        part = fmaf(q[hh][2], kt[e].z, part);
-        part = fmaf(q[hh][3], kt[e].w, part);
-        sc[e][hh] = part;
-      }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e)
-#pragma unroll
-        for (int hh = 0; hh < GM; ++hh) sc[e][hh] += __shfl_xor_sync(0xffffffffu, sc[e][hh], off);
-#pragma unroll
-    for (int hh = 0; hh < GM; ++hh) {
-      float cm = m[hh];
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e)
-        if (rb + e < r1) cm = fmaxf(cm, sc[e][hh]);
-      const float corr = ex2(m[hh] - cm);
-      l[hh] *= corr;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) o[hh][k] *= corr;
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e) {
-        const float p = rb + e < r1 ? ex2(sc[e][hh] - cm) : 0.0f;
-        l[hh] += p;
-        o[hh][0] = fmaf(p, vt[e].x, o[hh][0]);
-        o[hh][1] = fmaf(p, vt[e].y, o[hh][1]);
-        o[hh][2] = fmaf(p, vt[e].z, o[hh][2]);
-        o[hh][3] = fmaf(p, vt[e].w, o[hh][3]);
-      }
-      m[hh] = cm;
-    }
-  }
-#pragma unroll
-  for (int hh = 0; hh < GM; ++hh) {
-    if (hh < G) {
-      const int64_t sl = ((int64_t)b * a.Hq + h * G + hh) * a.S + slot;
-      *reinterpret_cast<float4*>(a.ws_o + sl * 128 + 4 * lane) = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
-      if (lane == 0) {
-        a.ws_m[sl] = m[hh];
-        a.ws_l[sl] = l[hh];
-      }
-    }
-  }
-}
-
-// ---- packed groups: per-warp state of the tensor-core path ------------------------------
+// ---- per-warp online-softmax state of the tensor-core path ------------------------------
+// Lane (g, j) holds the accumulator tiles O[cm] of the value product: rows g and g + 8
+// of tile cm are channels d0 = 16 g + 8 (cm >> 2) + 2 (cm & 3) and d0 + 1 (fields with
+// factors f = 1, 16, 1, 16 ... and 4, 64, 4, 64 ...), columns 2j, 2j + 1 are query
+// heads; m, l, W are the running max, sum and sum of p * z of heads 2j, 2j + 1 (l and
+// W summed over the lanes of a column at the end).  With DUAL (G <= 4) lanes j >= 2
+// track heads 2 (j - 2), 2 (j - 2) + 1 with zero tiles and are never written out.
 struct MmaState {
-  float O[8][4];     // O^T tiles: (channel rows of tile cm) x (heads 2j, 2j+1)
+  float O[8][4];
   float m[2], l[2], W[2];
 };
 
@@ -250,39 +192,140 @@ __device__ __forceinline__ void state_reset(MmaState& st) {
   st.l[0] = st.l[1] = st.W[0] = st.W[1] = 0.0f;
 }
 
-// Write a warp's tensor-core state for `head` into its slot.  Lane (g, j) holds heads
-// 2j, 2j + 1 (with DUAL, lanes j >= 2 hold copies of lanes j - 2 and write nothing).
+// 2^24 / f of the rows g (lo) and g + 8 (hi) of tile cm, by cm & 1
+__device__ __forceinline__ float inv_f_lo(int odd) { return odd ? 1048576.0f : 16777216.0f; }
+__device__ __forceinline__ float inv_f_hi(int odd) { return odd ? 262144.0f : 4194304.0f; }
+
+// Write a warp's state as (o[hh][128], m[hh], l[hh]) for hh < G: o of head hh at
+// o + hh * os, m and l at m + hh * ms, l + hh * ms.  Reduces l and W over the lanes of
+// a column first (the state is not usable afterwards).
 template <bool DUAL>
-__device__ void state_flush(const MmaArgs& a, MmaState& st, int head, int slot) {
+__device__ void state_emit(MmaState& st, int G, float* o, int64_t os, float* m, float* l, int64_t ms) {
   const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
-  const int b = head / a.Hkv, h = head % a.Hkv, G = a.G;
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    st.l[0] += __shfl_xor_sync(0xffffffffu, st.l[0], o);
-    st.l[1] += __shfl_xor_sync(0xffffffffu, st.l[1], o);
-    st.W[0] += __shfl_xor_sync(0xffffffffu, st.W[0], o);
-    st.W[1] += __shfl_xor_sync(0xffffffffu, st.W[1], o);
+  for (int s = 4; s < 32; s <<= 1) {
+    st.l[0] += __shfl_xor_sync(0xffffffffu, st.l[0], s);
+    st.l[1] += __shfl_xor_sync(0xffffffffu, st.l[1], s);
+    st.W[0] += __shfl_xor_sync(0xffffffffu, st.W[0], s);
+    st.W[1] += __shfl_xor_sync(0xffffffffu, st.W[1], s);
   }
-  // rows of tile cm: g -> field 2 (cm % 4) (factor 1, 16, 1, 16), g + 8 -> next field
-  // (factor 4, 64, 4, 64); 2^24 / f undoes the subnormal encoding
-  const float inv_lo[2] = {16777216.0f, 1048576.0f};   // 2^24, 2^20
-  const float inv_hi[2] = {4194304.0f, 262144.0f};     // 2^22, 2^18
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int hh = 2 * j + e;
     if (hh < G && (!DUAL || j < 2)) {
-      const int64_t sl = ((int64_t)b * a.Hq + h * G + hh) * a.S + slot;
-      float* dst = a.ws_o + sl * 128;
+      float* dst = o + hh * os;
 #pragma unroll
       for (int cm = 0; cm < 8; ++cm) {
         const int d0 = 16 * g + 8 * (cm >> 2) + 2 * (cm & 3);
-        const float v0 = fmaf(st.O[cm][e], inv_lo[cm & 1], st.W[e]);
-        const float v1 = fmaf(st.O[cm][2 + e], inv_hi[cm & 1], st.W[e]);
+        const float v0 = fmaf(st.O[cm][e], inv_f_lo(cm & 1), st.W[e]);
+        const float v1 = fmaf(st.O[cm][2 + e], inv_f_hi(cm & 1), st.W[e]);
         *reinterpret_cast<float2*>(dst + d0) = make_float2(v0, v1);
       }
       if (g == 0) {
-        a.ws_m[sl] = st.m[e];
-        a.ws_l[sl] = st.l[e];
+        m[hh * ms] = st.m[e];
+        l[hh * ms] = st.l[e];
+      }
+    }
+  }
+}
+
+// ---- raw tokens (sink + residual) staged in shared memory -------------------------------
+// nt <= 8 tokens: key rows at stg, value rows at stg + kRawBytes (source dtype).  Scores
+// in fp32 (lane: channels 4 lane .. 4 lane + 3, reduced over the warp), four tokens at
+// a time; the probabilities are accumulated into the state's tiles, each lane for its
+// own 16 channels 16 g .. 16 g + 15.
+template <bool DUAL, int GM>
+__device__ void raw_item(MmaState& st, const uint8_t* stg, int nt, int dtype,
+                         const float (&qv)[GM][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
+  const int hc = DUAL ? 2 * (j & 1) : 2 * j;           // heads hc, hc + 1 of this lane
+  const float keep = (!DUAL || j < 2) ? 1.0f : 0.0f;   // DUAL mirror lanes accumulate nothing
+  const float lkeep = g == 0 ? 1.0f : 0.0f;            // l is summed over the 8 lanes of a column
+  const int esz = dtype == KVQ_F32 ? 4 : 2;
+  const uint8_t* Kr = stg;
+  const uint8_t* Vr = stg + kRawBytes;
+#pragma unroll 1
+  for (int t = 0; t < nt; t += 4) {
+    float sc[4][GM];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float4 k = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t + e < nt) k = load4(Kr + (t + e) * 128 * esz, 4 * lane, dtype);
+#pragma unroll
+      for (int hh = 0; hh < GM; ++hh) {
+        float part = qv[hh][0] * k.x;
+        part = fmaf(qv[hh][1], k.y, part);
+        part = fmaf(qv[hh][2], k.z, part);
+        part = fmaf(qv[hh][3], k.w, part);
+        sc[e][hh] = part;
+      }
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int hh = 0; hh < GM; ++hh) sc[e][hh] += __shfl_xor_sync(0xffffffffu, sc[e][hh], s);
+    // this lane's two heads
+    float s0[4], s1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float a0 = sc[e][0], a1 = sc[e][1];
+#pragma unroll
+      for (int hh = 2; hh < GM; hh += 2) {
+        if (hc == hh) {
+          a0 = sc[e][hh];
+          a1 = sc[e][hh + 1];
+        }
+      }
+      s0[e] = t + e < nt ? a0 : -INFINITY;
+      s1[e] = t + e < nt ? a1 : -INFINITY;
+    }
+    const float mn0 = fmaxf(st.m[0], fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s0[2], s0[3])));
+    const float mn1 = fmaxf(st.m[1], fmaxf(fmaxf(s1[0], s1[1]), fmaxf(s1[2], s1[3])));
+    const float c0 = ex2(st.m[0] - mn0), c1 = ex2(st.m[1] - mn1);
+#pragma unroll
+    for (int cm = 0; cm < 8; ++cm) {
+      st.O[cm][0] *= c0;
+      st.O[cm][1] *= c1;
+      st.O[cm][2] *= c0;
+      st.O[cm][3] *= c1;
+    }
+    st.l[0] *= c0;
+    st.l[1] *= c1;
+    st.W[0] *= c0;
+    st.W[1] *= c1;
+    st.m[0] = mn0;
+    st.m[1] = mn1;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (t + e < nt) {
+        const float p0 = ex2(s0[e] - mn0), p1 = ex2(s1[e] - mn1);
+        st.l[0] = fmaf(p0, lkeep, st.l[0]);
+        st.l[1] = fmaf(p1, lkeep, st.l[1]);
+        const float q0 = p0 * keep, q1 = p1 * keep;
+        // scaled probabilities of the rows g (lo) and g + 8 (hi), even and odd tiles
+        const float a0e = q0 * (1.0f / 16777216.0f), a0o = q0 * (1.0f / 1048576.0f);
+        const float b0e = q0 * (1.0f / 4194304.0f), b0o = q0 * (1.0f / 262144.0f);
+        const float a1e = q1 * (1.0f / 16777216.0f), a1o = q1 * (1.0f / 1048576.0f);
+        const float b1e = q1 * (1.0f / 4194304.0f), b1o = q1 * (1.0f / 262144.0f);
+        const uint8_t* vrow = Vr + (t + e) * 128 * esz;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {    // channels 16 g + 4 qd .. + 3
+          const float4 v = load4(vrow, 16 * g + 4 * qd, dtype);
+          // channels 16g + 4qd + {0,1} -> tile cm = 2 qd (even: rows lo, hi), {2,3} -> cm = 2 qd + 1
+          // (cm >> 2 selects the upper 8 channels: qd >= 2)
+          const int ce = 2 * qd;   // even tile of this quad
+          const int co = ce + 1;
+          st.O[ce][0] = fmaf(a0e, v.x, st.O[ce][0]);
+          st.O[ce][1] = fmaf(a1e, v.x, st.O[ce][1]);
+          st.O[ce][2] = fmaf(b0e, v.y, st.O[ce][2]);
+          st.O[ce][3] = fmaf(b1e, v.y, st.O[ce][3]);
+          st.O[co][0] = fmaf(a0o, v.z, st.O[co][0]);
+          st.O[co][1] = fmaf(a1o, v.z, st.O[co][1]);
+          st.O[co][2] = fmaf(b0o, v.w, st.O[co][2]);
+          st.O[co][3] = fmaf(b1o, v.w, st.O[co][3]);
+        }
       }
     }
   }
@@ -546,46 +589,48 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Copy one half group (64 rows) of head `head`, group `gi` into a stage buffer: every
-// lane moves 16-byte chunks, coalesced.
-__device__ __forceinline__ void load_half(const MmaArgs& a, uint8_t* buf, int head, int gi, int hf) {
+// Copy one half group (64 rows) of head `head`, group `gi` into a stage buffer, with the
+// group's key scale / zero-point when `with_key`: every lane moves 16-byte chunks.
+__device__ __forceinline__ void load_half(const MmaArgs& a, uint8_t* buf, int64_t head, int gi, int hf,
+                                          bool with_key) {
   const int lane = threadIdx.x & 31;
   const int64_t t0 = (int64_t)gi * 128 + 64 * hf;
-  const uint8_t* kc = a.k_codes + (int64_t)head * a.k_slab_bytes + t0 * 64;
-  const uint8_t* vc = a.v_codes + (int64_t)head * a.v_slab_bytes + t0 * 32;
+  const uint8_t* kc = a.k_codes + head * a.k_slab_bytes + t0 * 64;
+  const uint8_t* vc = a.v_codes + head * a.v_slab_bytes + t0 * 32;
 #pragma unroll
   for (int e = 0; e < kHalfK / 512; ++e) cp_async16(buf + 16 * (lane + 32 * e), kc + 16 * (lane + 32 * e));
 #pragma unroll
   for (int e = 0; e < kHalfV / 512; ++e)
     cp_async16(buf + kHalfK + 16 * (lane + 32 * e), vc + 16 * (lane + 32 * e));
   if (lane < 16) {   // value scale (lanes 0..7) and zero-point (lanes 8..15), 64 rows each
-    const __half* src = (lane < 8 ? a.v_scale : a.v_zero) + (int64_t)head * a.C + t0 + 8 * (lane & 7);
+    const __half* src = (lane < 8 ? a.v_scale : a.v_zero) + head * a.C + t0 + 8 * (lane & 7);
     cp_async16(buf + kHalfK + kHalfV + 16 * lane, src);
   }
-  if (hf == 0) {     // the group's key scale (lanes 0..15) and zero-point (16..31)
-    const __half* src = (lane < 16 ? a.k_scale : a.k_zero) + ((int64_t)head * a.ng + gi) * 128 + 8 * (lane & 15);
+  if (with_key) {    // the group's key scale (lanes 0..15) and zero-point (16..31)
+    const __half* src = (lane < 16 ? a.k_scale : a.k_zero) + (head * a.ng + gi) * 128 + 8 * (lane & 15);
     cp_async16(buf + kHalfK + kHalfV + kHalfVM + 16 * lane, src);
   }
 }
 
-// Walks a warp's units (u = U0 + warp + i * kCW) without division.
-struct UnitCursor {
-  int64_t u;
-  int head, r;
-  __device__ __forceinline__ void init(int64_t u0, int uph) {
-    u = u0;
-    head = (int)(u0 / uph);
-    r = (int)(u0 % uph);
+// Copy raw item r of head `head` (its key rows, then its value rows at +kRawBytes).
+__device__ __forceinline__ void load_raw(const MmaArgs& a, uint8_t* buf, int64_t head, int r) {
+  const int lane = threadIdx.x & 31;
+  const int lg = a.src_dtype == KVQ_F32 ? 5 : 4;   // log2 of the 16-byte chunks per row
+  const int rowb = 16 << lg;                       // bytes per row
+  const int nraw = a.n_sink + a.t_res;
+  const int t0 = r * a.rt, nt = min(a.rt, nraw - t0);
+  const int per = nt << lg;
+  for (int c = lane; c < 2 * per; c += 32) {
+    const int kv = c >= per, rem = c - (kv ? per : 0);
+    const int t = rem >> lg, ch = rem & ((1 << lg) - 1);
+    const int tok = t0 + t;
+    const bool sink = tok < a.n_sink;
+    const void* arr = kv ? (sink ? a.sink_v : a.res_v) : (sink ? a.sink_k : a.res_k);
+    const int64_t row = head * (sink ? a.n_sink : a.res_cap) + (sink ? tok : tok - a.n_sink);
+    cp_async16(buf + kv * kRawBytes + t * rowb + ch * 16,
+               reinterpret_cast<const uint8_t*>(arr) + row * rowb + ch * 16);
   }
-  __device__ __forceinline__ void next(int uph) {
-    u += kCW;
-    r += kCW;
-    while (r >= uph) {
-      r -= uph;
-      ++head;
-    }
-  }
-};
+}
 
 // ---- the kernel --------------------------------------------------------------------------
 template <bool DUAL>
@@ -593,100 +638,158 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int GM = DUAL ? 4 : 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x;
-  const int64_t U0 = unit_start(c, a.N, a.grid), U1 = unit_start(c + 1, a.N, a.grid);
+  const int64_t gw = (int64_t)blockIdx.x * kCW + warp;
+  const int64_t i0 = item_start(gw, a.I, a.W), i1 = item_start(gw + 1, a.I, a.W);
+  const int U = a.U;
   uint8_t* ring = smem + (size_t)warp * (kBuffers * kStageBytes);
   uint32_t* my_scratch = reinterpret_cast<uint32_t*>(smem + (size_t)kCW * kBuffers * kStageBytes) +
                          warp * (kScratchBytes / 4);
+  int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * (kBuffers * kStageBytes + kScratchBytes));
+  const int nraw = a.n_sink + a.t_res;
 
-  // load cursor: runs kBuffers - 1 half groups ahead of the compute cursor
-  UnitCursor lc;
-  lc.init(U0 + warp, a.uph);
-  int lhf = 0;
-  auto skip_raw = [&]() {
-    while (lc.u < U1 && lc.r < a.rw) lc.next(a.uph);
-  };
-  skip_raw();
+  // load cursor: one work item ahead of the compute cursor (odd raw positions carry none)
+  int64_t lhead = i0 / U, li = i0;
+  int lr = (int)(i0 - lhead * U);
   int issued = 0;
+  auto advance_load = [&]() {
+    ++li;
+    if (++lr == U) {
+      lr = 0;
+      ++lhead;
+    }
+  };
   auto issue_next = [&]() {
-    if (lc.u < U1) {
-      load_half(a, ring + (issued % kBuffers) * kStageBytes, lc.head, lc.r - a.rw, lhf);
-      if (++lhf == 2) {
-        lhf = 0;
-        lc.next(a.uph);
-        skip_raw();
+    while (li < i1 && lr < a.nrp && (lr & 1)) advance_load();
+    if (li < i1) {
+      uint8_t* buf = ring + (issued % kBuffers) * kStageBytes;
+      if (lr < a.nrp) {
+        load_raw(a, buf, lhead, lr >> 1);
+      } else {
+        const int p = lr - a.nrp;
+        load_half(a, buf, lhead, p >> 1, p & 1, (p & 1) == 0 || li == i0);
       }
+      advance_load();
     }
     cp_async_commit();   // an empty group keeps the group count uniform
     ++issued;
   };
-#pragma unroll 1
-  for (int e = 0; e < kBuffers - 1; ++e) issue_next();
+  issue_next();
 
   MmaState st;
   state_reset(st);
   float qv[GM][4];
-  int cur_head = -1, cur_c0 = 0;
+  KeyOp ko;
+  int64_t head = i0 / U, cur_head = -1;
+  int r = (int)(i0 - head * U);
   bool qbad = false;
   int consumed = 0;
-  UnitCursor cc;
-  cc.init(U0 + warp, a.uph);
-  for (; cc.u < U1; cc.next(a.uph)) {
-    const int head = cc.head, r = cc.r;
-    if (r < a.rw) {
-      if (cur_head >= 0) {
-        state_flush<DUAL>(a, st, cur_head, slot_of(c, cur_c0, warp, 1));
-        state_reset(st);
-        cur_head = -1;
-      }
-      raw_piece<GM>(a, head, r, slot_of(c, cta_of_unit((int64_t)head * a.uph, a.N, a.grid), warp, 0));
-      continue;
-    }
+#pragma unroll 1
+  for (int64_t i = i0; i < i1; ++i) {
     if (head != cur_head) {
-      if (cur_head >= 0) {
-        state_flush<DUAL>(a, st, cur_head, slot_of(c, cur_c0, warp, 1));
+      if (cur_head >= 0) {   // the range crosses into the next head: slot 0 of this one
+        const int64_t row0 = cur_head * a.G;
+        state_emit<DUAL>(st, a.G, a.ws_o + row0 * a.S * 128, (int64_t)a.S * 128, a.ws_m + row0 * a.S,
+                         a.ws_l + row0 * a.S, a.S);
         state_reset(st);
       }
       cur_head = head;
-      cur_c0 = cta_of_unit((int64_t)head * a.uph, a.N, a.grid);
       // this head's queries, pre-scaled, for channels 4 lane .. 4 lane + 3
-      const int b = head / a.Hkv, h = head % a.Hkv;
 #pragma unroll
       for (int hh = 0; hh < GM; ++hh) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (hh < a.G) x = load4(a.q, ((int64_t)b * a.Hq + h * a.G + hh) * 128 + 4 * lane, a.q_dtype);
+        if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
         qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
         qv[hh][0] = x.x * a.qscale; qv[hh][1] = x.y * a.qscale;
         qv[hh][2] = x.z * a.qscale; qv[hh][3] = x.w * a.qscale;
       }
     }
-    const int gi = r - a.rw;
-    const int tvalid = (int)min((int64_t)128, a.t_quant - (int64_t)gi * 128);
-    KeyOp ko;
-#pragma unroll 1
-    for (int hf = 0; hf < 2; ++hf) {
-      cp_async_wait<kBuffers - 2>();
-      __syncwarp();
-      const uint8_t* stg = ring + (consumed % kBuffers) * kStageBytes;
-      if (hf == 0) {
+    if (r < a.nrp && (r & 1)) {   // second position of a raw item: no work
+      if (++r == U) {
+        r = 0;
+        ++head;
+      }
+      continue;
+    }
+    // the next item goes into the buffer consumed last time, then this one is waited
+    // for: the warp's own copy of the next item overlaps its math on this one
+    issue_next();
+    cp_async_wait<kBuffers - 1>();
+    __syncwarp();
+    const uint8_t* stg = ring + (consumed % kBuffers) * kStageBytes;
+    if (r < a.nrp) {
+      raw_item<DUAL, GM>(st, stg, min(a.rt, nraw - (r >> 1) * a.rt), a.src_dtype, qv);
+    } else {
+      const int p = r - a.nrp, gi = p >> 1, hf = p & 1;
+      if (hf == 0 || i == i0) {
         const __half* ks = reinterpret_cast<const __half*>(stg + kHalfK + kHalfV + kHalfVM);
         key_operand<DUAL, GM>(a, ks, ks + 128, my_scratch, qv, ko);
       }
-      if (tvalid > 64 * hf) mma_half<DUAL>(st, stg, ko, tvalid - 64 * hf);
-      __syncwarp();
-      ++consumed;
-      issue_next();
+      const int tvalid = (int)min((int64_t)64, a.t_quant - (int64_t)gi * 128 - 64 * hf);
+      mma_half<DUAL>(st, stg, ko, tvalid);
+    }
+    __syncwarp();
+    ++consumed;
+    if (++r == U) {
+      r = 0;
+      ++head;
     }
   }
   cp_async_wait<0>();
-  if (cur_head >= 0) state_flush<DUAL>(a, st, cur_head, slot_of(c, cur_c0, warp, 1));
+  __syncwarp();
   if (__any_sync(0xffffffffu, qbad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+
+  // ---- merge of the warps' last heads inside the CTA ----
+  // Every warp, empty ones included, belongs to the head of item i1 - 1; its record
+  // (its own ring, now idle) holds its state of that head (empty: m = -inf, l = 0, o = 0).
+  const int lh = i1 > 0 ? (int)((i1 - 1) / U) : -1;
+  float* rec = reinterpret_cast<float*>(ring);
+  if (lh >= 0) state_emit<DUAL>(st, a.G, rec, 128, rec + 8 * 128, rec + 8 * 128 + 8, 1);
+  if (lane == 0) last_head[warp] = lh;
+  __syncthreads();
+  const int G = a.G;
+  int w0 = 0;
+#pragma unroll 1
+  while (w0 < kCW) {
+    const int h = last_head[w0];
+    int w1 = w0;
+    while (w1 + 1 < kCW && last_head[w1 + 1] == h) ++w1;
+    if (h >= 0) {
+      const int64_t ca = first_ending_warp(h, U, a.I, a.W) / kCW;
+      const int slot = 1 + (int)((int64_t)blockIdx.x - ca);
+#pragma unroll 1
+      for (int idx = threadIdx.x; idx < G * 128; idx += kThreads) {
+        const int hh = idx >> 7, d = idx & 127;
+        float M = -INFINITY;
+        for (int w = w0; w <= w1; ++w) {
+          const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * (kBuffers * kStageBytes));
+          M = fmaxf(M, rw[8 * 128 + hh]);
+        }
+        float o = 0.0f, l = 0.0f;
+        for (int w = w0; w <= w1; ++w) {
+          const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * (kBuffers * kStageBytes));
+          const float mw = rw[8 * 128 + hh];
+          if (mw != -INFINITY) {
+            const float f = ex2(mw - M);
+            o = fmaf(f, rw[hh * 128 + d], o);
+            l = fmaf(f, rw[8 * 128 + 8 + hh], l);
+          }
+        }
+        const int64_t sl = ((int64_t)h * G + hh) * a.S + slot;
+        a.ws_o[sl * 128 + d] = o;
+        if (d == 0) {
+          a.ws_m[sl] = M;
+          a.ws_l[sl] = l;
+        }
+      }
+    }
+    w0 = w1 + 1;
+  }
 }
 
-// ---- combine for this path: finds the slots of a head from the partition --------------
+// ---- combine for this path: the valid slots of a head follow from the partition ---------
 struct CombArgsMma {
-  int Hkv, Hq, G, uph, rw, grid, S;
-  int64_t N;
+  int G, S;
+  int64_t rows, U, I, W;
   const float* m;
   const float* l;
   const float* o;
@@ -694,85 +797,61 @@ struct CombArgsMma {
   int out_dtype;
 };
 
+// One warp per query-head row; lane owns channels 4 lane .. 4 lane + 3.
 __global__ void __launch_bounds__(128) combine_mma_kernel(CombArgsMma a) {
-  extern __shared__ float sh[];           // [S] m, [S] weight, [S] (int) slot of valid entries
-  float* sm_m = sh;
-  float* sm_w = sh + a.S;
-  int* sm_slot = reinterpret_cast<int*>(sh + 2 * a.S);
-  __shared__ int warp_cnt[4];
-  __shared__ float red[4];
-  __shared__ float sM, sL;
-  const int hq = blockIdx.x, b = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int head = b * a.Hkv + hq / a.G;
-  const int64_t Hs = (int64_t)head * a.uph, He = Hs + a.uph;
-  const int c0 = cta_of_unit(Hs, a.N, a.grid), c1 = cta_of_unit(He - 1, a.N, a.grid);
-  const int nslots = (c1 - c0 + 1) * kCW * 2;
-  const int64_t row = (int64_t)b * a.Hq + hq;
-  // 1. compact the valid slots in slot order: slot (c, w, kind) holds data iff warp w of
-  //    CTA c owns a unit of this head and kind
-  int base = 0;
-  for (int s0 = 0; s0 < nslots; s0 += blockDim.x) {
-    const int s = s0 + threadIdx.x;
-    bool valid = false;
-    if (s < nslots) {
-      const int kind = s & 1, w = (s >> 1) % kCW, c = c0 + (s >> 1) / kCW;
-      const int64_t U0 = unit_start(c, a.N, a.grid), U1 = unit_start(c + 1, a.N, a.grid);
-      const int64_t lo0 = kind ? Hs + a.rw : Hs, hi0 = kind ? He : Hs + a.rw;
-      const int64_t lo = U0 > lo0 ? U0 : lo0, hi = U1 < hi0 ? U1 : hi0;
-      if (lo < hi) valid = lo + (((w - (lo - U0)) % kCW) + kCW) % kCW < hi;
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, valid);
-    if (lane == 0) warp_cnt[warp] = __popc(bal);
-    __syncthreads();
-    int off = base;
-    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
-    if (valid) {
-      const int idx = off + __popc(bal & ((1u << lane) - 1));
-      sm_slot[idx] = s;
-      sm_m[idx] = a.m[row * a.S + s];
-    }
-    for (int w = 0; w < 4; ++w) base += warp_cnt[w];
-    __syncthreads();
-  }
-  const int nv = base;
-  // 2. max and weights
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (row >= a.rows) return;
+  const int64_t h = row / a.G;
+  const int64_t ca = first_ending_warp(h, a.U, a.I, a.W) / kCW;
+  const int64_t cb = last_ending_warp(h, a.U, a.I, a.W) / kCW;
+  const int s_lo = has_crossing(h, a.U, a.I, a.W) ? 0 : 1;
+  const int s_hi = 1 + (int)(cb - ca);
+  const float* mrow = a.m + row * a.S;
+  const float* lrow = a.l + row * a.S;
   float M = -INFINITY;
-  for (int i = threadIdx.x; i < nv; i += blockDim.x) M = fmaxf(M, sm_m[i]);
-  M = warp_max(M);
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  if (threadIdx.x == 0) sM = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
-  M = sM;
+  for (int s = s_lo; s <= s_hi; ++s) M = fmaxf(M, mrow[s]);
   float L = 0.0f;
-  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-    const float f = sm_m[i] == -INFINITY ? 0.0f : exp2f(sm_m[i] - M);
-    sm_w[i] = f;
-    L = fmaf(a.l[row * a.S + sm_slot[i]], f, L);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = s_lo; s <= s_hi; ++s) {
+    const float ms = mrow[s];
+    if (ms == -INFINITY) continue;
+    const float f = exp2f(ms - M);
+    L = fmaf(f, lrow[s], L);
+    const float4 v = *reinterpret_cast<const float4*>(a.o + (row * a.S + s) * 128 + 4 * lane);
+    acc.x = fmaf(f, v.x, acc.x);
+    acc.y = fmaf(f, v.y, acc.y);
+    acc.z = fmaf(f, v.z, acc.z);
+    acc.w = fmaf(f, v.w, acc.w);
   }
-  L = warp_sum(L);
-  __syncthreads();
-  if (lane == 0) red[warp] = L;
-  __syncthreads();
-  if (threadIdx.x == 0) sL = (red[0] + red[1]) + (red[2] + red[3]);
-  __syncthreads();
-  const float invL = 1.0f / sL;
-  // 3. weighted sum of the partial outputs
-  const int d = threadIdx.x;
-  float o0 = 0.0f, o1 = 0.0f;
-  int i = 0;
-  for (; i + 1 < nv; i += 2) {
-    o0 = fmaf(a.o[(row * a.S + sm_slot[i]) * 128 + d], sm_w[i], o0);
-    o1 = fmaf(a.o[(row * a.S + sm_slot[i + 1]) * 128 + d], sm_w[i + 1], o1);
-  }
-  if (i < nv) o0 = fmaf(a.o[(row * a.S + sm_slot[i]) * 128 + d], sm_w[i], o0);
-  store_elem(a.out, row * 128 + d, a.out_dtype, (o0 + o1) * invL);
+  const float inv = 1.0f / L;
+  store_elem(a.out, row * 128 + 4 * lane + 0, a.out_dtype, acc.x * inv);
+  store_elem(a.out, row * 128 + 4 * lane + 1, a.out_dtype, acc.y * inv);
+  store_elem(a.out, row * 128 + 4 * lane + 2, a.out_dtype, acc.z * inv);
+  store_elem(a.out, row * 128 + 4 * lane + 3, a.out_dtype, acc.w * inv);
 }
 
-// per-warp rings of half-group stages, then per-warp scratch
+// per-warp rings of item stages, per-warp scratch, then the warps' last heads
 static_assert(kStageBytes % 128 == 0, "stage alignment");
-size_t mma_smem() { return (size_t)kCW * kBuffers * kStageBytes + (size_t)kCW * kScratchBytes; }
+size_t mma_smem() {
+  return (size_t)kCW * kBuffers * kStageBytes + (size_t)kCW * kScratchBytes + kCW * sizeof(int);
+}
+
+// Positions of a head: two per raw item of rt tokens, then one per packed half.
+struct Items {
+  int rt, nrp, nh, U;
+};
+Items head_items(const Layout& L, int64_t t_quant, int t_res) {
+  Items it;
+  it.rt = kRawBytes / (128 * (L.src_dtype == KVQ_F32 ? 4 : 2));
+  const int nraw = L.n_sink + t_res;
+  it.nrp = 2 * ((nraw + it.rt - 1) / it.rt);
+  const int64_t ngv = (t_quant + 127) / 128;
+  const int64_t rem = t_quant - (ngv - 1) * 128;
+  it.nh = (int)(2 * (ngv - 1) + (rem > 64 ? 2 : 1));
+  it.U = it.nrp + it.nh;
+  return it;
+}
 
 }  // namespace
 
@@ -785,28 +864,29 @@ bool mma_path_ok(const Layout& L, int Hq) {
          V.axis == KVQ_AXIS_TOKEN && L.rope == 0 && G >= 2 && G <= 8;
 }
 
-// Partition of the fast path: fills the plan's slot count and grid.
+// Partition of the fast path (t_quant >= 1): CTAs, slots per query head.  At least one
+// warp per head, so that no warp range is longer than a head's row of items.
 void plan_mma(const Layout& L, int64_t t_quant, int t_res, int max_ctas, DecodePlan& p) {
   const int64_t heads = (int64_t)L.B * L.Hkv;
-  const int ngv = (int)((t_quant + 127) / 128);
-  const int nraw = L.n_sink + t_res;
-  const int rw = nraw > 0 ? std::min(kRawPieces, nraw) : 0;
-  const int uph = ngv + rw;
-  const int64_t N = heads * uph;
+  const Items it = head_items(L, t_quant, t_res);
+  const int64_t I = heads * it.U;
   int64_t cap = device_sm_count();
   if (max_ctas > 0) cap = std::min<int64_t>(cap, max_ctas);
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cap, N));
-  int span = 1;
+  int64_t grid = std::min<int64_t>(cap, (I + kCW - 1) / kCW);
+  grid = std::max<int64_t>(grid, (heads + kCW - 1) / kCW);
+  grid = std::max<int64_t>(grid, 1);
+  const int64_t W = grid * kCW;
+  int64_t span = 1;
   for (int64_t h = 0; h < heads; ++h) {
-    const int c0 = cta_of_unit(h * uph, N, grid), c1 = cta_of_unit(h * uph + uph - 1, N, grid);
-    span = std::max(span, c1 - c0 + 1);
+    const int64_t ca = first_ending_warp(h, it.U, I, W) / kCW, cb = last_ending_warp(h, it.U, I, W) / kCW;
+    span = std::max(span, cb - ca + 1);
   }
-  p.S = span * kCW * 2;
-  p.grid_ctas = grid;
+  p.S = (int)(1 + span);
+  p.grid_ctas = (int)grid;
   p.raw_slot = -1;
-  p.raw_pieces = rw;
-  p.n_packed_splits = ngv;
-  p.split_groups = 1;
+  p.raw_pieces = it.nrp;
+  p.n_packed_splits = it.nh;
+  p.split_groups = it.rt;
 }
 
 cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
@@ -823,7 +903,6 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.v_slab_bytes = L.side[1].code_slab_bytes;
   a.C = L.C;
   a.ng = L.ng;
-  a.B = L.B;
   a.Hkv = L.Hkv;
   a.Hq = Hq;
   a.G = Hq / L.Hkv;
@@ -839,11 +918,11 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.q = q;
   a.q_dtype = q_dtype;
   a.qscale = scale * kLog2e;
-  a.ngv = p.n_packed_splits;
-  a.rw = p.raw_pieces;
-  a.uph = a.ngv + a.rw;
-  a.N = (int64_t)L.B * L.Hkv * a.uph;
-  a.grid = p.grid_ctas;
+  a.nrp = p.raw_pieces;
+  a.rt = p.split_groups;
+  a.U = p.raw_pieces + p.n_packed_splits;
+  a.I = (int64_t)L.B * L.Hkv * a.U;
+  a.W = (int64_t)p.grid_ctas * kCW;
   a.S = p.S;
   a.ws_m = ws_m;
   a.ws_l = ws_l;
@@ -853,7 +932,7 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   auto kern = a.G <= 4 ? decode_mma_kernel<true> : decode_mma_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, smem, s>>>(a);
+  kern<<<p.grid_ctas, kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -861,21 +940,18 @@ cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, con
                                const float* ws_l, const float* ws_o, void* out, int out_dtype,
                                cudaStream_t s) {
   CombArgsMma c;
-  c.Hkv = L.Hkv;
-  c.Hq = Hq;
   c.G = Hq / L.Hkv;
-  c.rw = p.raw_pieces;
-  c.uph = p.n_packed_splits + c.rw;
-  c.grid = p.grid_ctas;
   c.S = p.S;
-  c.N = (int64_t)L.B * L.Hkv * c.uph;
+  c.rows = (int64_t)L.B * Hq;
+  c.U = p.raw_pieces + p.n_packed_splits;
+  c.I = (int64_t)L.B * L.Hkv * c.U;
+  c.W = (int64_t)p.grid_ctas * kCW;
   c.m = ws_m;
   c.l = ws_l;
   c.o = ws_o;
   c.out = out;
   c.out_dtype = out_dtype;
-  dim3 grid(Hq, L.B);
-  combine_mma_kernel<<<grid, 128, (size_t)p.S * 3 * sizeof(float), s>>>(c);
+  combine_mma_kernel<<<(unsigned)((c.rows + 3) / 4), 128, 0, s>>>(c);
   return cudaGetLastError();
 }
 

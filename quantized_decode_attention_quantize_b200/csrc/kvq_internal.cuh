@@ -65,10 +65,10 @@ cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t
 
 struct DecodePlan {
   int S;                // partial slots per query head
-  int split_groups;     // generic path: packed groups per split
-  int n_packed_splits;  // generic path: splits over the packed region; fast path: groups per head
+  int split_groups;     // generic path: packed groups per split; fast path: tokens per raw item
+  int n_packed_splits;  // generic path: splits over the packed region; fast path: packed halves per head
   int raw_slot;         // generic path: slot of the raw (sink + residual) tokens, -1 if none
-  int raw_pieces;       // fast path: raw-token units per head
+  int raw_pieces;       // fast path: raw positions per head (two per raw item)
   int fast;             // 1 when the tensor-core K4/V2 kernel runs the packed region
   int grid_ctas;        // CTAs of the split kernel
 };

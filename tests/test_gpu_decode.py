@@ -176,19 +176,26 @@ def test_nonfinite_query_flagged():
     assert p.status_bits() & kvq.KVQ_DEV_NONFINITE
 
 
-@pytest.mark.parametrize("B,H,G,tq,ns,tr,splits", [
-    (3, 5, 2, 2 * 128 + 1, 2, 3, 0),
-    (3, 5, 2, 2 * 128 + 1, 2, 3, 1),
-    (3, 5, 2, 2 * 128 + 1, 2, 3, 13),
-    (2, 3, 8, 5, 1, 0, 4),
-    (1, 7, 4, 9 * 128, 0, 100, 0),
-    (4, 2, 3, 3 * 128 - 7, 4, 11, 2),
+@pytest.mark.parametrize("B,H,G,tq,ns,tr,splits,src", [
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 0, BF16),
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 1, BF16),
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 13, BF16),
+    (2, 3, 8, 5, 1, 0, 4, BF16),
+    (1, 7, 4, 9 * 128, 0, 100, 0, BF16),
+    (4, 2, 3, 3 * 128 - 7, 4, 11, 2, BF16),
+    (2, 3, 4, 64, 1, 13, 0, BF16),          # one half group, two raw items
+    (2, 3, 4, 65, 1, 13, 3, BF16),          # a second half with one token
+    (5, 3, 2, 7 * 128 + 64, 1, 100, 1, BF16),   # fifteen heads, one CTA asked: two
+    (2, 2, 4, 300, 1, 20, 0, F32),          # fp32 raw items of six tokens
+    (2, 2, 6, 5 * 128 + 3, 3, 0, 2, F16),
+    (16, 120, 2, 70, 1, 3, 0, BF16),        # more heads than warps on the GPU
 ])
-def test_partition_shapes(B, H, G, tq, ns, tr, splits):
-    # the persistent partition over (head, group) units with raw-token pieces: heads
-    # spanning several CTAs, CTAs spanning several heads, tiny and ragged regions
-    fd = fmt(src_dtype=BF16, n_sink=ns, residual_cap=128)
+def test_partition_shapes(B, H, G, tq, ns, tr, splits, src):
+    # the item partition: raw items and half groups cut into equal warp ranges, heads
+    # spanning several CTAs, CTAs spanning several heads, ranges that cross heads,
+    # tiny and ragged regions, more CTAs than SMs
+    fd = fmt(src_dtype=src, n_sink=ns, residual_cap=128)
     p = build(fd, B, H, G * H, tq, tr, seed=40 + tq)
-    out, ref = run(p, G * H, tq, tr, BF16, F32, seed=40 + tq, num_splits=splits)
+    out, ref = run(p, G * H, tq, tr, src, F32, seed=40 + tq, num_splits=splits)
     assert rel_l2(out, ref) <= 1e-3
     assert p.status_bits() == 0
