@@ -6,10 +6,12 @@ decode attention over the packed cache, on synthetic data shaped like the worklo
                     [--config llama3_8b]
 
 One step = kvq_quantize_keys + kvq_quantize_values of one 128-token group (the
-flush of the raw window into the packed cache) + kvq_decode_partial (split kernel)
-+ kvq_decode_combine over all T tokens.  Every step is timed with CUDA events on
-the launching stream; the L2 is flushed between steps (a 512 MiB write, outside the
-events).  `value` is the effective HBM throughput of the whole step: the format's
+flush of the raw window into the packed cache) + kvq_decode_attention over all T
+tokens (on this path one split kernel that also finishes the combine, after a memset
+of its arrival counters).  Every step is timed with CUDA events on the launching
+stream; the L2 is flushed between steps, outside the events, by a 512 MiB write and
+then a 512 MiB read of another buffer (so that no dirty line of the flush is left
+for the step to write back).  `value` is the effective HBM throughput of the whole step: the format's
 algorithmic bytes (codes, scales, zero-points, raw sink / residual tokens, the new
 group's source and packed output, q and out) over the step time.  One JSON line is
 printed by rank 0.  Under torchrun every rank runs its own replica (weak scaling:
@@ -34,6 +36,7 @@ import synth  # noqa: E402
 
 METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize GB/s"
 L2_FLUSH_BYTES = 512 << 20
+LAUNCHES_PER_STEP = 3   # asym_keys_kernel, asym_values_kernel, decode_mma_kernel
 
 
 def parse():
@@ -247,7 +250,7 @@ def workload_config(cfg):
                         f"g{f['group_tokens']} + V{f['v_bits']} per-token, fp16 scale/zero",
             "B": cfg["B"], "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "D": cfg["D"], "T": cfg["T"],
             "step": "quantize one 128-token group (K, V) + decode attention over T",
-            "l2": "flushed between steps (512 MiB write outside the timed events)",
+            "l2": "flushed between steps outside the timed events (512 MiB write, then 512 MiB read)",
             "parallelism": "replicas (one independent cache per GPU)"}
 
 
@@ -294,8 +297,13 @@ def main():
     ws = torch.empty(kvq.decode_workspace_bytes(fmt, B, Hq, Hkv, tq, tr), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        flush_r.sum()
 
     def step(evs=None):
         if evs:
@@ -304,15 +312,13 @@ def main():
         kvq.quantize_values(fmt, cache, newv, gi_f * g, g, status=status, stream=stream)
         if evs:
             evs[1].record(stream)
-        kvq.decode_partial(fmt, cache, q, tq, tr, scale, ws, status=status, stream=stream)
+        kvq.decode_attention(fmt, cache, q, tq, tr, scale, kvq.F32, out=out, workspace=ws,
+                             status=status, stream=stream)
         if evs:
             evs[2].record(stream)
-        kvq.decode_combine(fmt, B, Hq, Hkv, tq, tr, ws, out, stream=stream)
-        if evs:
-            evs[3].record(stream)
 
     for i in range(args.warmup):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         step()
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
@@ -320,7 +326,7 @@ def main():
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -328,24 +334,22 @@ def main():
     sampler.start()
     time.sleep(0.15)
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         step(evs[i])
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     t_quant = [e[0].elapsed_time(e[1]) for e in evs]
-    t_part = [e[1].elapsed_time(e[2]) for e in evs]
-    t_comb = [e[2].elapsed_time(e[3]) for e in evs]
-    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    t_dec = [e[1].elapsed_time(e[2]) for e in evs]
+    t_step = [e[0].elapsed_time(e[2]) for e in evs]
     ms_step = statistics.mean(t_step)
-    ms_part = statistics.mean(t_part)
+    ms_dec = statistics.mean(t_dec)
     ms_quant = statistics.mean(t_quant)
-    ms_comb = statistics.mean(t_comb)
     if world > 1:
-        tt = torch.tensor([ms_step, ms_part, ms_quant, ms_comb], device=dev)
+        tt = torch.tensor([ms_step, ms_dec, ms_quant], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step, ms_part, ms_quant, ms_comb = [float(x) for x in tt.tolist()]
+        ms_step, ms_dec, ms_quant = [float(x) for x in tt.tolist()]
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(10, args.steps // 10)
@@ -359,7 +363,7 @@ def main():
     dk, dv, dq = torch.empty_like(newk), torch.empty_like(newv), torch.empty_like(q)
     e2e_t = []
     for i in range(e2e_steps + 3):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -384,11 +388,11 @@ def main():
     assert torch.isfinite(out).all()
 
     step_bytes = decode_call_bytes(cfg, tq, tr) + quant_bytes(cfg, g)
-    kern_bytes = decode_kernel_bytes(cfg, tq, tr)
+    kern_bytes = decode_call_bytes(cfg, tq, tr)
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
-    decode_gbs = (decode_call_bytes(cfg, tq, tr)) / ((ms_part + ms_comb) * 1e-3) / 1e9
+    decode_gbs = kern_bytes / (ms_dec * 1e-3) / 1e9
     quant_gbs = quant_bytes(cfg, g) / (ms_quant * 1e-3) / 1e9
-    achieved = kern_bytes / (ms_part * 1e-3) / 1e9
+    achieved = decode_gbs
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -414,15 +418,16 @@ def main():
         "config": workload_config(cfg),
         "pct_of_8tbs": 100.0 * value / world / 8000.0,
         "decode_gbs": decode_gbs, "quantize_gbs": quant_gbs,
-        "tokens_heads_per_s": world * B * Hq * cfg["T"] / ((ms_part + ms_comb) * 1e-3),
-        "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb},
-        "roofline": {"kernel": "decode_mma_kernel (kvq_decode_partial)", "bound": "hbm",
+        "tokens_heads_per_s": world * B * Hq * cfg["T"] / (ms_dec * 1e-3),
+        "ms_breakdown": {"quantize": ms_quant, "decode": ms_dec},
+        "roofline": {"kernel": "decode_mma_kernel with its combine (kvq_decode_attention: counter "
+                               "memset + one split kernel)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": kern_bytes,
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},
         "e2e": {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

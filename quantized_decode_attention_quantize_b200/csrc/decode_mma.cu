@@ -98,6 +98,9 @@ struct MmaArgs {
   float* ws_l;
   float* ws_o;
   int32_t* status;
+  int* counters;  // non-null: combine in this kernel (one arrival counter per KV head, zeroed)
+  void* out;
+  int out_dtype;
 };
 
 // ---- partition of the items over the warps (shared with the combine kernel) ------------
@@ -126,6 +129,21 @@ __host__ __device__ __forceinline__ int64_t last_ending_warp(int64_t h, int64_t 
 __host__ __device__ __forceinline__ bool has_crossing(int64_t h, int64_t U, int64_t I, int64_t W) {
   const int64_t last = (h + 1) * U - 1;
   return item_start(warp_of_item(last, I, W) + 1, I, W) > last + 1;
+}
+// The valid slots of head h: s_lo (0 with a crossing state, else 1) .. s_hi, and the
+// number of CTAs that write them.
+__host__ __device__ __forceinline__ void head_slots(int64_t h, int64_t U, int64_t I, int64_t W, int cw,
+                                                    int* s_lo, int* s_hi, int* writers) {
+  const int64_t ca = first_ending_warp(h, U, I, W) / cw, cb = last_ending_warp(h, U, I, W) / cw;
+  const bool cross = has_crossing(h, U, I, W);
+  *s_lo = cross ? 0 : 1;
+  *s_hi = 1 + (int)(cb - ca);
+  int n = (int)(cb - ca + 1);
+  if (cross) {
+    const int64_t cs = warp_of_item((h + 1) * U - 1, I, W) / cw;
+    if (cs < ca || cs > cb) ++n;
+  }
+  *writers = n;
 }
 
 // ---- PTX helpers ------------------------------------------------------------------
@@ -234,9 +252,8 @@ __device__ void state_emit(MmaState& st, int G, float* o, int64_t os, float* m, 
 // in fp32 (lane: channels 4 lane .. 4 lane + 3, reduced over the warp), four tokens at
 // a time; the probabilities are accumulated into the state's tiles, each lane for its
 // own 16 channels 16 g .. 16 g + 15.
-template <bool DUAL, int GM>
-__device__ void raw_item(MmaState& st, const uint8_t* stg, int nt, int dtype,
-                         const float (&qv)[GM][4]) {
+template <bool DUAL, int GM, typename Q>
+__device__ void raw_item(MmaState& st, const uint8_t* stg, int nt, int dtype, const Q& qv) {
   const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
   const int hc = DUAL ? 2 * (j & 1) : 2 * j;           // heads hc, hc + 1 of this lane
   const float keep = (!DUAL || j < 2) ? 1.0f : 0.0f;   // DUAL mirror lanes accumulate nothing
@@ -253,10 +270,11 @@ __device__ void raw_item(MmaState& st, const uint8_t* stg, int nt, int dtype,
       if (t + e < nt) k = load4(Kr + (t + e) * 128 * esz, 4 * lane, dtype);
 #pragma unroll
       for (int hh = 0; hh < GM; ++hh) {
-        float part = qv[hh][0] * k.x;
-        part = fmaf(qv[hh][1], k.y, part);
-        part = fmaf(qv[hh][2], k.z, part);
-        part = fmaf(qv[hh][3], k.w, part);
+        const float4 q = qv.get(hh);
+        float part = q.x * k.x;
+        part = fmaf(q.y, k.y, part);
+        part = fmaf(q.z, k.z, part);
+        part = fmaf(q.w, k.w, part);
         sc[e][hh] = part;
       }
     }
@@ -337,34 +355,63 @@ struct KeyOp {
   float mult, bias0, bias1;
 };
 
+// The head's pre-scaled queries, channels 4 lane .. 4 lane + 3 of head hh: with DUAL in
+// the upper half of the warp's scratch (shared memory), otherwise in registers.
+template <bool DUAL, int GM>
+struct QVec;
+template <int GM>
+struct QVec<true, GM> {
+  float* s;   // [G][128]
+  __device__ __forceinline__ float4 get(int hh) const {
+    return *reinterpret_cast<const float4*>(s + hh * 128 + 4 * (threadIdx.x & 31));
+  }
+  __device__ __forceinline__ void set(int hh, float4 v) {
+    *reinterpret_cast<float4*>(s + hh * 128 + 4 * (threadIdx.x & 31)) = v;
+  }
+};
+template <int GM>
+struct QVec<false, GM> {
+  float v[GM][4];
+  __device__ __forceinline__ float4 get(int hh) const { return make_float4(v[hh][0], v[hh][1], v[hh][2], v[hh][3]); }
+  __device__ __forceinline__ void set(int hh, float4 x) {
+    v[hh][0] = x.x; v[hh][1] = x.y; v[hh][2] = x.z; v[hh][3] = x.w;
+  }
+};
+
 // Build the key-product B operand of a group from its per-channel scale / zero-point
 // (ks, kz in shared memory) and the head's pre-scaled queries.  DUAL: G <= 4, the
 // remainder rides in columns 4..7.
+//
+// Lane l owns channels 4 l + k (k < 4) of every head; channel 4 l + k is row
+// 2 ((l & 7) >> 1) + (k >> 1) ... of the fragments of consumer lane 4 hh + (l >> 3): k-step
+// kk = 2 ((l & 7) >> 1) + (k >> 1), register k & 1, half l & 1.  The two lanes of a pair
+// (l, l ^ 1) fill the two halves of the same four words; one shuffle gives each of them
+// two whole words (even lane: k-step kk0 = 2 ((l & 7) >> 1), odd lane: kk0 + 1), stored
+// as one 64-bit word pair.
 template <bool DUAL, int GM>
 __device__ __forceinline__ void key_operand(const MmaArgs& a, const __half* ks, const __half* kz,
-                                            uint32_t* scratch, const float (&qv)[GM][4], KeyOp& ko) {
+                                            uint32_t* scratch, const QVec<DUAL, GM>& qv, KeyOp& ko) {
   const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
   const int G = a.G;
-  // lane owns channels 4 lane .. 4 lane + 3 of every head
   const uint2 sv = *reinterpret_cast<const uint2*>(ks + 4 * lane);
   const uint2 zv = *reinterpret_cast<const uint2*>(kz + 4 * lane);
   const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
   const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
   const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zv.x));
   const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&zv.y));
-  const float s[4] = {s01.x, s01.y, s23.x, s23.y};
-  const float z[4] = {z01.x, z01.y, z23.x, z23.y};
   float av[GM][4], dz[GM];
   float amax = 0.0f;
 #pragma unroll
   for (int hh = 0; hh < GM; ++hh) {
-    dz[hh] = 0.0f;
+    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (hh < G) q = qv.get(hh);
+    av[hh][0] = q.x * s01.x;
+    av[hh][1] = q.y * s01.y;
+    av[hh][2] = q.z * s23.x;
+    av[hh][3] = q.w * s23.y;
+    dz[hh] = fmaf(q.w, z23.y, fmaf(q.z, z23.x, fmaf(q.y, z01.y, q.x * z01.x)));
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      av[hh][k] = qv[hh][k] * s[k];
-      dz[hh] = fmaf(qv[hh][k], z[k], dz[hh]);
-      amax = fmaxf(amax, fabsf(av[hh][k]));
-    }
+    for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fabsf(av[hh][k]));
   }
   amax = warp_max(amax);
   // one exponent for the group: max |a 2^(24 - e)| < 2^15
@@ -373,26 +420,32 @@ __device__ __forceinline__ void key_operand(const MmaArgs& a, const __half* ks, 
   ex = max(-100, min(127, ex));
   ko.mult = pow2(ex);
   const float sc = __uint_as_float((uint32_t)max(1, min(254, 127 + 24 - ex)) << 23);
-  const float sc16 = sc * 0.0625f;
-  // scatter into the fragment layout: channel c = 4 lane + k -> consumer lane
-  // 4 hh + lane / 8, k-step 2 ((lane & 7) / 2) + k / 2, register k & 1, half lane & 1
-  uint16_t* sh = reinterpret_cast<uint16_t*>(scratch);
-  uint16_t* sl = sh + 32 * 16 * 2;
-  const int kkbase = 2 * ((lane & 7) >> 1), half = lane & 1;
+  const float sc16 = sc * 0.0625f;   // odd k: the code sits 4 bits up (factor 16)
+  const bool odd = lane & 1;
+  const int kk0 = 2 * ((lane & 7) >> 1) + (odd ? 1 : 0);
 #pragma unroll
   for (int hh = 0; hh < GM; ++hh) {
     if (hh < G) {
-      const int dl = 4 * hh + (lane >> 3);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float x = av[hh][k] * ((k & 1) ? sc16 : sc);
-        const __half hi = __float2half_rn(x);
-        const int idx = ((dl * 8 + kkbase + (k >> 1)) * 2 + (k & 1)) * 2 + half;
-        const uint16_t lo = __half_as_ushort(__float2half_rn(x - __half2float(hi)));
-        sh[idx] = __half_as_ushort(hi);
-        if (DUAL) sh[idx + 4 * 4 * 8 * 2 * 2] = lo;   // consumer lane + 16: column hh + 4
-        else sl[idx] = lo;
-      }
+      const float x0 = av[hh][0] * sc, x1 = av[hh][1] * sc16, x2 = av[hh][2] * sc, x3 = av[hh][3] * sc16;
+      const __half2 h01 = __floats2half2_rn(x0, x1), h23 = __floats2half2_rn(x2, x3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y);
+      const __half2 l23 = __floats2half2_rn(x2 - f23.x, x3 - f23.y);
+      const uint32_t H01 = *reinterpret_cast<const uint32_t*>(&h01), H23 = *reinterpret_cast<const uint32_t*>(&h23);
+      const uint32_t L01 = *reinterpret_cast<const uint32_t*>(&l01), L23 = *reinterpret_cast<const uint32_t*>(&l23);
+      // even lane keeps k = 0, 1 and sends k = 2, 3; odd lane the reverse
+      const uint32_t rh = __shfl_xor_sync(0xffffffffu, odd ? H01 : H23, 1);
+      const uint32_t rl = __shfl_xor_sync(0xffffffffu, odd ? L01 : L23, 1);
+      const uint32_t mh = odd ? H23 : H01, ml = odd ? L23 : L01;
+      // word (kk, reg r) = (even lane's half, odd lane's half) of k = 2 (kk - kk0e) + r
+      const uint2 wh = odd ? make_uint2(__byte_perm(rh, mh, 0x5410), __byte_perm(rh, mh, 0x7632))
+                           : make_uint2(__byte_perm(mh, rh, 0x5410), __byte_perm(mh, rh, 0x7632));
+      const uint2 wl = odd ? make_uint2(__byte_perm(rl, ml, 0x5410), __byte_perm(rl, ml, 0x7632))
+                           : make_uint2(__byte_perm(ml, rl, 0x5410), __byte_perm(ml, rl, 0x7632));
+      const int dl = 4 * hh + (lane >> 3);   // consumer lane
+      *reinterpret_cast<uint2*>(scratch + dl * 16 + 2 * kk0) = wh;
+      if (DUAL) *reinterpret_cast<uint2*>(scratch + (dl + 16) * 16 + 2 * kk0) = wl;   // column hh + 4
+      else *reinterpret_cast<uint2*>(scratch + 32 * 16 + dl * 16 + 2 * kk0) = wl;
     }
   }
   // butterfly reduction of the per-head sums q~ . z over the warp
@@ -469,28 +522,33 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
   const __half* vz = vs + 64;
 
   // ---- scores of the 64 tokens (4 tiles of 16) ----
+  // all four tiles' code words first, then the k-steps tile by tile so that consecutive
+  // products go to different accumulators
   float S[4][4];
+  uint4 wlo[4], whi[4];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     S[mt][0] = S[mt][1] = S[mt][2] = S[mt][3] = 0.0f;
-    const uint4 w0 = *reinterpret_cast<const uint4*>(kc + (16 * mt + g) * 16 + 4 * j);
-    const uint4 w1 = *reinterpret_cast<const uint4*>(kc + (16 * mt + g + 8) * 16 + 4 * j);
-    const uint32_t x0[4] = {w0.x, w0.y, w0.z, w0.w};
-    const uint32_t x1[4] = {w1.x, w1.y, w1.z, w1.w};
+    wlo[mt] = *reinterpret_cast<const uint4*>(kc + (16 * mt + g) * 16 + 4 * j);
+    whi[mt] = *reinterpret_cast<const uint4*>(kc + (16 * mt + g + 8) * 16 + 4 * j);
+  }
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const uint32_t p0 = odd_bytes_down(x0[w]), p1 = odd_bytes_down(x1[w]);
-      // k-step 2w: nibbles 0 (f 1) and 1 (f 16) of each half
-      const uint32_t a00 = x0[w] & 0x000F000Fu, a01 = x1[w] & 0x000F000Fu;
-      const uint32_t a02 = x0[w] & 0x00F000F0u, a03 = x1[w] & 0x00F000F0u;
-      // k-step 2w + 1: nibbles 2 (f 1) and 3 (f 16)
-      const uint32_t a10 = p0 & 0x000F000Fu, a11 = p1 & 0x000F000Fu;
-      const uint32_t a12 = p0 & 0x00F000F0u, a13 = p1 & 0x00F000F0u;
-      mma16816(S[mt], a00, a01, a02, a03, ko.bh[2 * w][0], ko.bh[2 * w][1]);
-      mma16816(S[mt], a10, a11, a12, a13, ko.bh[2 * w + 1][0], ko.bh[2 * w + 1][1]);
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const uint32_t x0 = w == 0 ? wlo[mt].x : w == 1 ? wlo[mt].y : w == 2 ? wlo[mt].z : wlo[mt].w;
+      const uint32_t x1 = w == 0 ? whi[mt].x : w == 1 ? whi[mt].y : w == 2 ? whi[mt].z : whi[mt].w;
+      const uint32_t p0 = odd_bytes_down(x0), p1 = odd_bytes_down(x1);
+      // k-step 2w: nibbles 0 (f 1) and 1 (f 16) of each half; k-step 2w + 1: nibbles 2, 3
+      mma16816(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u,
+               ko.bh[2 * w][0], ko.bh[2 * w][1]);
+      mma16816(S[mt], p0 & 0x000F000Fu, p1 & 0x000F000Fu, p0 & 0x00F000F0u, p1 & 0x00F000F0u,
+               ko.bh[2 * w + 1][0], ko.bh[2 * w + 1][1]);
       if (!DUAL) {
-        mma16816(S[mt], a00, a01, a02, a03, ko.bl[2 * w][0], ko.bl[2 * w][1]);
-        mma16816(S[mt], a10, a11, a12, a13, ko.bl[2 * w + 1][0], ko.bl[2 * w + 1][1]);
+        mma16816(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u,
+                 ko.bl[2 * w][0], ko.bl[2 * w][1]);
+        mma16816(S[mt], p0 & 0x000F000Fu, p1 & 0x000F000Fu, p0 & 0x00F000F0u, p1 & 0x00F000F0u,
+                 ko.bl[2 * w + 1][0], ko.bl[2 * w + 1][1]);
       }
     }
   }
@@ -632,6 +690,42 @@ __device__ __forceinline__ void load_raw(const MmaArgs& a, uint8_t* buf, int64_t
   }
 }
 
+// ---- final combine of one query-head row over its valid slots -------------------------
+// Lane owns channels 4 lane .. 4 lane + 3.  Loads bypass L1: the slots were written by
+// other CTAs of the same launch when this runs inside the split kernel.
+__device__ __forceinline__ void combine_row(const float* m, const float* l, const float* o, int S,
+                                            int64_t row, int s_lo, int s_hi, int lane, void* out,
+                                            int out_dtype) {
+  const float* mrow = m + row * S;
+  const float* lrow = l + row * S;
+  float M = -INFINITY;
+  for (int s = s_lo; s <= s_hi; ++s) M = fmaxf(M, __ldcg(mrow + s));
+  float L = 0.0f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = s_lo; s <= s_hi; ++s) {
+    const float ms = __ldcg(mrow + s);
+    if (ms == -INFINITY) continue;
+    const float f = ex2(ms - M);
+    L = fmaf(f, __ldcg(lrow + s), L);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(o + (row * S + s) * 128) + lane);
+    acc.x = fmaf(f, v.x, acc.x);
+    acc.y = fmaf(f, v.y, acc.y);
+    acc.z = fmaf(f, v.z, acc.z);
+    acc.w = fmaf(f, v.w, acc.w);
+  }
+  const float inv = 1.0f / L;
+  const int64_t i = row * 128 + 4 * lane;
+  if (out_dtype == KVQ_F32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  } else {
+    store_elem(out, i + 0, out_dtype, acc.x * inv);
+    store_elem(out, i + 1, out_dtype, acc.y * inv);
+    store_elem(out, i + 2, out_dtype, acc.z * inv);
+    store_elem(out, i + 3, out_dtype, acc.w * inv);
+  }
+}
+
 // ---- the kernel --------------------------------------------------------------------------
 template <bool DUAL>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
@@ -645,6 +739,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   uint32_t* my_scratch = reinterpret_cast<uint32_t*>(smem + (size_t)kCW * kBuffers * kStageBytes) +
                          warp * (kScratchBytes / 4);
   int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * (kBuffers * kStageBytes + kScratchBytes));
+  int* cross_head = last_head + kCW;     // the head a warp left for the next one, or -1
+  int* finish = cross_head + kCW;        // [2 kCW] heads whose combine falls to this CTA
   const int nraw = a.n_sink + a.t_res;
 
   // load cursor: one work item ahead of the compute cursor (odd raw positions carry none)
@@ -677,16 +773,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
 
   MmaState st;
   state_reset(st);
-  float qv[GM][4];
+  QVec<DUAL, GM> qv;
+  if constexpr (DUAL) qv.s = reinterpret_cast<float*>(my_scratch) + 512;   // upper 2 KiB
   KeyOp ko;
   int64_t head = i0 / U, cur_head = -1;
   int r = (int)(i0 - head * U);
+  int crossed = -1;
   bool qbad = false;
   int consumed = 0;
 #pragma unroll 1
   for (int64_t i = i0; i < i1; ++i) {
     if (head != cur_head) {
       if (cur_head >= 0) {   // the range crosses into the next head: slot 0 of this one
+        crossed = (int)cur_head;
         const int64_t row0 = cur_head * a.G;
         state_emit<DUAL>(st, a.G, a.ws_o + row0 * a.S * 128, (int64_t)a.S * 128, a.ws_m + row0 * a.S,
                          a.ws_l + row0 * a.S, a.S);
@@ -699,8 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
         qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
-        qv[hh][0] = x.x * a.qscale; qv[hh][1] = x.y * a.qscale;
-        qv[hh][2] = x.z * a.qscale; qv[hh][3] = x.w * a.qscale;
+        qv.set(hh, make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale));
       }
     }
     if (r < a.nrp && (r & 1)) {   // second position of a raw item: no work
@@ -744,7 +842,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   const int lh = i1 > 0 ? (int)((i1 - 1) / U) : -1;
   float* rec = reinterpret_cast<float*>(ring);
   if (lh >= 0) state_emit<DUAL>(st, a.G, rec, 128, rec + 8 * 128, rec + 8 * 128 + 8, 1);
-  if (lane == 0) last_head[warp] = lh;
+  if (lane == 0) {
+    last_head[warp] = lh;
+    cross_head[warp] = crossed;
+  }
   __syncthreads();
   const int G = a.G;
   int w0 = 0;
@@ -784,6 +885,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
     }
     w0 = w1 + 1;
   }
+  if (!a.counters) return;
+
+  // ---- combine inside the kernel: the last CTA to write a head's slots finishes it ----
+  __threadfence();   // this CTA's slot writes are visible before its arrivals count
+  __syncthreads();
+  if (threadIdx.x < 2 * kCW) {
+    const int e = threadIdx.x;
+    const int h = e < kCW ? cross_head[e] : last_head[e - kCW];
+    bool first = h >= 0;
+    for (int k = 0; k < e && first; ++k) first = (k < kCW ? cross_head[k] : last_head[k - kCW]) != h;
+    int mine = -1;
+    if (first) {
+      int s_lo, s_hi, writers;
+      head_slots(h, U, a.I, a.W, kCW, &s_lo, &s_hi, &writers);
+      if (atomicAdd(a.counters + h, 1) == writers - 1) mine = h;
+    }
+    finish[e] = mine;
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int e = 0; e < 2 * kCW; ++e) {
+    const int h = finish[e];
+    if (h < 0) continue;
+    __threadfence();
+    if (threadIdx.x < G * 32) {
+      int s_lo, s_hi, writers;
+      head_slots(h, U, a.I, a.W, kCW, &s_lo, &s_hi, &writers);
+      combine_row(a.ws_m, a.ws_l, a.ws_o, a.S, (int64_t)h * G + (threadIdx.x >> 5), s_lo, s_hi, lane,
+                  a.out, a.out_dtype);
+    }
+  }
 }
 
 // ---- combine for this path: the valid slots of a head follow from the partition ---------
@@ -797,44 +929,21 @@ struct CombArgsMma {
   int out_dtype;
 };
 
-// One warp per query-head row; lane owns channels 4 lane .. 4 lane + 3.
+// One warp per query-head row.
 __global__ void __launch_bounds__(128) combine_mma_kernel(CombArgsMma a) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= a.rows) return;
-  const int64_t h = row / a.G;
-  const int64_t ca = first_ending_warp(h, a.U, a.I, a.W) / kCW;
-  const int64_t cb = last_ending_warp(h, a.U, a.I, a.W) / kCW;
-  const int s_lo = has_crossing(h, a.U, a.I, a.W) ? 0 : 1;
-  const int s_hi = 1 + (int)(cb - ca);
-  const float* mrow = a.m + row * a.S;
-  const float* lrow = a.l + row * a.S;
-  float M = -INFINITY;
-  for (int s = s_lo; s <= s_hi; ++s) M = fmaxf(M, mrow[s]);
-  float L = 0.0f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = s_lo; s <= s_hi; ++s) {
-    const float ms = mrow[s];
-    if (ms == -INFINITY) continue;
-    const float f = exp2f(ms - M);
-    L = fmaf(f, lrow[s], L);
-    const float4 v = *reinterpret_cast<const float4*>(a.o + (row * a.S + s) * 128 + 4 * lane);
-    acc.x = fmaf(f, v.x, acc.x);
-    acc.y = fmaf(f, v.y, acc.y);
-    acc.z = fmaf(f, v.z, acc.z);
-    acc.w = fmaf(f, v.w, acc.w);
-  }
-  const float inv = 1.0f / L;
-  store_elem(a.out, row * 128 + 4 * lane + 0, a.out_dtype, acc.x * inv);
-  store_elem(a.out, row * 128 + 4 * lane + 1, a.out_dtype, acc.y * inv);
-  store_elem(a.out, row * 128 + 4 * lane + 2, a.out_dtype, acc.z * inv);
-  store_elem(a.out, row * 128 + 4 * lane + 3, a.out_dtype, acc.w * inv);
+  int s_lo, s_hi, writers;
+  head_slots(row / a.G, a.U, a.I, a.W, kCW, &s_lo, &s_hi, &writers);
+  combine_row(a.m, a.l, a.o, a.S, row, s_lo, s_hi, lane, a.out, a.out_dtype);
 }
 
-// per-warp rings of item stages, per-warp scratch, then the warps' last heads
+// per-warp rings of item stages, per-warp scratch, then the warps' last and crossing heads
+// and the heads to finish
 static_assert(kStageBytes % 128 == 0, "stage alignment");
 size_t mma_smem() {
-  return (size_t)kCW * kBuffers * kStageBytes + (size_t)kCW * kScratchBytes + kCW * sizeof(int);
+  return (size_t)kCW * kBuffers * kStageBytes + (size_t)kCW * kScratchBytes + 4 * kCW * sizeof(int);
 }
 
 // Positions of a head: two per raw item of rt tokens, then one per packed half.
@@ -891,7 +1000,8 @@ void plan_mma(const Layout& L, int64_t t_quant, int t_res, int max_ctas, DecodeP
 
 cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
                               int64_t t_quant, int t_res, float scale, float* ws_m, float* ws_l,
-                              float* ws_o, int32_t* d_status, cudaStream_t s) {
+                              float* ws_o, int32_t* d_status, cudaStream_t s, int* counters, void* out,
+                              int out_dtype) {
   MmaArgs a;
   a.k_codes = reinterpret_cast<const uint8_t*>(L.side[0].codes);
   a.v_codes = reinterpret_cast<const uint8_t*>(L.side[1].codes);
@@ -928,6 +1038,9 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.ws_l = ws_l;
   a.ws_o = ws_o;
   a.status = d_status;
+  a.counters = counters;
+  a.out = out;
+  a.out_dtype = out_dtype;
   const size_t smem = mma_smem();
   auto kern = a.G <= 4 ? decode_mma_kernel<true> : decode_mma_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -1,8 +1,10 @@
 // Append-time quantization for the asymmetric b-bit formats (b = 2, 4, 8): keys per
 // channel over a token group, values per token ([KVQ] "Approach"; [K4V2]).  Same rules
-// as the general quantize kernel, tiled for parallelism: a key group is split into
-// blocks of 32 channels (the statistics of a channel never leave its block), values
-// into blocks of 32 tokens.  Loads are 16-byte vectors, stores are packed words.
+// as the general quantize kernel, laid out for latency: every thread issues all of its
+// 16-byte loads first, keeps its values in registers, reduces with warp shuffles and
+// packs its own codes into words, so an append of one group costs about one DRAM round
+// trip.  Keys: a CTA takes 32 channels of one group (the statistics of a channel never
+// leave it); values: a CTA takes 32 tokens.
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -11,6 +13,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCB = 32;     // channels per key block
 constexpr int kTB = 32;     // tokens per value block
+constexpr int kMaxKeyRows = 4;   // rows per thread: g <= 256 over 64 row slices
 
 struct AArgs {
   Layout L;
@@ -20,7 +23,7 @@ struct AArgs {
 };
 
 // 8 consecutive elements (16 bytes for 16-bit sources, two 16-byte loads for fp32)
-__device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, float* out, int* bad) {
+__device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, float* out) {
   if (dtype == KVQ_F32) {
     const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i);
     const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i + 4);
@@ -40,57 +43,95 @@ __device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, fl
       }
     }
   }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) *bad |= !isfinite(out[j]);
 }
 
+// 8 codes of `bits` bits packed LSB-first (bits = 2: 16 bits, 4: 32 bits; 8: two words)
+__device__ __forceinline__ uint2 pack8(const float* x, const float* s, const float* z, int bits) {
+  const int maxc = (1 << bits) - 1;
+  uint32_t lo = 0, hi = 0;
+  if (bits == 8) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) lo |= (uint32_t)asym_code(x[j], s[j], z[j], maxc) << (8 * j);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) hi |= (uint32_t)asym_code(x[4 + j], s[4 + j], z[4 + j], maxc) << (8 * j);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) lo |= (uint32_t)asym_code(x[j], s[j], z[j], maxc) << (bits * j);
+  }
+  return make_uint2(lo, hi);
+}
+
+// Keys.  Thread (warp w, lane): vector v = lane & 3 (channels cb + 8 v .. + 7) of rows
+// rs, rs + 64, ... with rs = 8 w + lane / 4.
 __global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
-  __shared__ float tile[256 * kCB];
   __shared__ float pmin[8][kCB], pmax[8][kCB];
   __shared__ float sf[kCB], zf[kCB];
   __shared__ int flags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_KEYS];
-  const int D = L.D, g = L.g, bits = S.bits, maxc = (1 << bits) - 1;
+  const int D = L.D, g = L.g, bits = S.bits;
   const int64_t ts = a.t0 + (int64_t)blockIdx.x * g;
   const int ln = (int)min((int64_t)g, a.t0 + a.n - ts);
   const int gi = (int)(ts / g);
   const int cb = blockIdx.y * kCB;
   const int head = blockIdx.z;
   const int b = head / L.Hkv, h = head % L.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int v = lane & 3, rs = warp * 8 + (lane >> 2);
   if (threadIdx.x == 0) flags = 0;
+  float x[kMaxKeyRows][8];
+  const int64_t base = (int64_t)b * a.sb + (int64_t)h * a.sh + (ts - a.t0) * a.st + cb + 8 * v;
+#pragma unroll
+  for (int k = 0; k < kMaxKeyRows; ++k) {
+    const int r = rs + 64 * k;
+    if (r < ln) load8(a.src, base + r * a.st, L.src_dtype, x[k]);
+  }
   int bad = 0;
-  // stage [ln][32] channels: 4 vectors of 8 per row
-  for (int v = threadIdx.x; v < ln * (kCB / 8); v += kThreads) {
-    const int r = v / (kCB / 8), c8 = (v % (kCB / 8)) * 8;
-    const int64_t off = (int64_t)b * a.sb + (int64_t)h * a.sh + (ts - a.t0 + r) * a.st + cb + c8;
-    load8(a.src, off, L.src_dtype, tile + r * kCB + c8, &bad);
+  float mn[8], mx[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    mn[c] = INFINITY;
+    mx[c] = -INFINITY;
   }
-  __syncthreads();
-  if (bad) atomicOr(&flags, 1);
-  // per-channel min / max: 8 row slices per channel
-  {
-    const int c = threadIdx.x % kCB, slice = threadIdx.x / kCB;
-    float mn = INFINITY, mx = -INFINITY;
-    for (int r = slice; r < ln; r += 8) {
-      const float x = tile[r * kCB + c];
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+#pragma unroll
+  for (int k = 0; k < kMaxKeyRows; ++k) {
+    if (rs + 64 * k < ln) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        bad |= !isfinite(x[k][c]);
+        mn[c] = fminf(mn[c], x[k][c]);
+        mx[c] = fmaxf(mx[c], x[k][c]);
+      }
     }
-    pmin[slice][c] = mn;
-    pmax[slice][c] = mx;
   }
+  // over the 8 row slices of the warp (lanes with equal v)
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      mn[c] = fminf(mn[c], __shfl_xor_sync(0xffffffffu, mn[c], o));
+      mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], o));
+    }
+  __syncthreads();   // flags initialised
+  if (lane < 4) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      pmin[warp][8 * v + c] = mn[c];
+      pmax[warp][8 * v + c] = mx[c];
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&flags, 1);
   __syncthreads();
   if (threadIdx.x < kCB) {
     const int c = threadIdx.x;
-    float mn = pmin[0][c], mx = pmax[0][c];
+    float m0 = pmin[0][c], m1 = pmax[0][c];
 #pragma unroll
     for (int k = 1; k < 8; ++k) {
-      mn = fminf(mn, pmin[k][c]);
-      mx = fmaxf(mx, pmax[k][c]);
+      m0 = fminf(m0, pmin[k][c]);
+      m1 = fmaxf(m1, pmax[k][c]);
     }
     __half s, z;
-    if (!asym_params(mn, mx, bits, &s, &z)) atomicOr(&flags, 2);
+    if (!asym_params(m0, m1, bits, &s, &z)) atomicOr(&flags, 2);
     const int64_t mi = ((int64_t)head * L.ng + gi) * D + cb + c;
     reinterpret_cast<__half*>(S.scale)[mi] = s;
     reinterpret_cast<__half*>(S.zero)[mi] = z;
@@ -98,26 +139,28 @@ __global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
     zf[c] = __half2float(z);
   }
   __syncthreads();
-  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
-  if (bits == 8) {
-    for (int v = threadIdx.x; v < ln * (kCB / 4); v += kThreads) {
-      const int r = v / (kCB / 4), c4 = (v % (kCB / 4)) * 4;
-      uint32_t w = 0;
+  float s8[8], z8[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) w |= (uint32_t)asym_code(tile[r * kCB + c4 + j], sf[c4 + j], zf[c4 + j], maxc) << (8 * j);
-      *reinterpret_cast<uint32_t*>(codes + (ts + r) * D + cb + c4) = w;
-    }
-  } else {
-    const int per = 32 / bits, wpb = kCB / per, W = D / per;   // words per row-block, per row
-    uint32_t* dst = reinterpret_cast<uint32_t*>(codes) + ts * W + cb / per;
-    for (int v = threadIdx.x; v < ln * wpb; v += kThreads) {
-      const int r = v / wpb, w = v % wpb;
-      uint32_t word = 0;
-      for (int j = 0; j < per; ++j) {
-        const int c = w * per + j;
-        word |= (uint32_t)asym_code(tile[r * kCB + c], sf[c], zf[c], maxc) << (bits * j);
-      }
-      dst[r * W + w] = word;
+  for (int c = 0; c < 8; ++c) {
+    s8[c] = sf[8 * v + c];
+    z8[c] = zf[8 * v + c];
+  }
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
+  const int rowb = D * bits / 8;   // bytes per code row
+#pragma unroll
+  for (int k = 0; k < kMaxKeyRows; ++k) {
+    const int r = rs + 64 * k;
+    const bool ok = r < ln;
+    uint2 w = make_uint2(0u, 0u);
+    if (ok) w = pack8(x[k], s8, z8, bits);
+    uint8_t* row = codes + (ts + r) * rowb;
+    if (bits == 8) {
+      if (ok) *reinterpret_cast<uint2*>(row + cb + 8 * v) = w;
+    } else if (bits == 4) {
+      if (ok) *reinterpret_cast<uint32_t*>(row + (cb + 8 * v) / 2) = w.x;
+    } else {   // 2-bit: 16 channels per word, this lane's 8 are its low (v even) or high half
+      const uint32_t other = __shfl_xor_sync(0xffffffffu, w.x, 1);
+      if (ok && (v & 1) == 0) *reinterpret_cast<uint32_t*>(row + (cb + 8 * v) / 4) = w.x | (other << 16);
     }
   }
   __syncthreads();
@@ -125,74 +168,123 @@ __global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
     flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
 }
 
+// Values.  A warp takes 4 consecutive tokens of the block; lane (sub, vl) holds vector
+// vl (channels 8 vl .. 8 vl + 7) of one token, sub = lane / nvec, nvec = D / 8 lanes per
+// token, so a pass covers 32 / nvec tokens and a warp ceil(4 nvec / 32) passes.
 __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
-  extern __shared__ __align__(16) uint8_t vsm[];   // [kTB][D] codes
+  constexpr int kPass = 4;   // at most 4 passes (D = 256)
   __shared__ int flags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_VALUES];
-  const int D = L.D, bits = S.bits, maxc = (1 << bits) - 1;
+  const int D = L.D, bits = S.bits;
   const int64_t tb = a.t0 + (int64_t)blockIdx.x * kTB;
   const int nt = (int)min((int64_t)kTB, a.t0 + a.n - tb);
   const int head = blockIdx.y;
   const int b = head / L.Hkv, h = head % L.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nvec = D / 8, rpp = 32 / nvec, sub = lane / nvec, vl = lane % nvec;
+  const int passes = (4 + rpp - 1) / rpp;
   if (threadIdx.x == 0) flags = 0;
-  __syncthreads();
+  float x[kPass][8];
+  const int64_t base = (int64_t)b * a.sb + (int64_t)h * a.sh + (tb - a.t0) * a.st + 8 * vl;
+#pragma unroll
+  for (int p = 0; p < kPass; ++p) {
+    const int t = warp * 4 + p * rpp + sub;   // token within the block
+    if (p < passes && p * rpp + sub < 4 && t < nt) load8(a.src, base + t * a.st, L.src_dtype, x[p]);
+  }
+  __syncthreads();   // flags initialised
   int bad = 0, rbad = 0;
-  // one warp per token row: lane owns D / 32 consecutive channels (multiple of 8 when
-  // D >= 256, else handled by the 8-wide loads of 32 / (D / 8) lanes)
-  for (int r = warp; r < nt; r += kThreads / 32) {
-    const int64_t off = (int64_t)b * a.sb + (int64_t)h * a.sh + (tb - a.t0 + r) * a.st;
-    float x[8];
-    const int nvec = D / 8;                  // 8-wide vectors per row (4..32)
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
+  uint32_t half_prev = 0;   // 2- and 4-bit, one token per pass: the even token's half words
+  uint32_t half_prev2 = 0;
+#pragma unroll
+  for (int p = 0; p < kPass; ++p) {
+    if (p >= passes) break;
+    const int tl = p * rpp + sub;        // token within the warp's 4
+    const int t = warp * 4 + tl;
+    const bool ok = tl < 4 && t < nt;
     float mn = INFINITY, mx = -INFINITY;
-    if (lane < nvec) {
-      load8(a.src, off + 8 * lane, L.src_dtype, x, &bad);
+    if (ok) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        mn = fminf(mn, x[j]);
-        mx = fmaxf(mx, x[j]);
+        bad |= !isfinite(x[p][j]);
+        mn = fminf(mn, x[p][j]);
+        mx = fmaxf(mx, x[p][j]);
       }
     }
-    mn = warp_min(mn);
-    mx = warp_max(mx);
+    for (int o = 1; o < nvec; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
     __half s, z;
-    const bool ok = asym_params(mn, mx, bits, &s, &z);
-    if (lane == 0) {
-      rbad |= !ok;
-      reinterpret_cast<__half*>(S.scale)[(int64_t)head * L.C + tb + r] = s;
-      reinterpret_cast<__half*>(S.zero)[(int64_t)head * L.C + tb + r] = z;
+    const bool good = asym_params(mn, mx, bits, &s, &z);
+    if (ok && vl == 0) {
+      rbad |= !good;
+      reinterpret_cast<__half*>(S.scale)[(int64_t)head * L.C + tb + t] = s;
+      reinterpret_cast<__half*>(S.zero)[(int64_t)head * L.C + tb + t] = z;
     }
-    if (lane < nvec) {
-      const float sfv = __half2float(s), zfv = __half2float(z);
-      uint32_t lo = 0, hi = 0;
+    float s8[8], z8[8];
+    const float sv = __half2float(s), zv = __half2float(z);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) lo |= (uint32_t)asym_code(x[j], sfv, zfv, maxc) << (8 * j);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) hi |= (uint32_t)asym_code(x[4 + j], sfv, zfv, maxc) << (8 * j);
-      *reinterpret_cast<uint2*>(vsm + r * D + 8 * lane) = make_uint2(lo, hi);
+    for (int j = 0; j < 8; ++j) {
+      s8[j] = sv;
+      z8[j] = zv;
+    }
+    uint2 w = make_uint2(0u, 0u);
+    if (ok) w = pack8(x[p], s8, z8, bits);
+    if (bits == 8) {
+      if (ok) *reinterpret_cast<uint2*>(codes + (tb + t) * D + 8 * vl) = w;
+      continue;
+    }
+    // pair layout: word j of pair u holds 16 / bits channels of token 2u (low 16 bits)
+    // and token 2u + 1 (high 16 bits); this lane's 8 channels are one half word (2-bit)
+    // or two (4-bit: channels 8 vl .. + 3 and + 4 .. + 7)
+    const uint32_t h0 = w.x & 0xffffu;
+    const uint32_t h1 = bits == 2 ? 0u : (w.x >> 16);
+    uint32_t o0, o1;
+    bool even;
+    if (rpp >= 2) {   // partner token in lane ^ nvec of the same pass
+      o0 = __shfl_xor_sync(0xffffffffu, h0, nvec);
+      o1 = __shfl_xor_sync(0xffffffffu, h1, nvec);
+      even = (sub & 1) == 0;
+    } else {          // one token per pass: partner in the neighbouring pass of this lane
+      o0 = half_prev;
+      o1 = half_prev2;
+      even = (p & 1) == 0;
+      half_prev = h0;
+      half_prev2 = h1;
+    }
+    const int64_t u = (tb + t) / 2;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(codes) + u * (D * bits / 16);
+    const bool last_odd = (t + 1 == nt) && even;   // a lone last token: high half zero
+    if (rpp >= 2) {
+      if (ok && even) {
+        const uint32_t hi0 = last_odd ? 0u : o0, hi1 = last_odd ? 0u : o1;
+        if (bits == 2) dst[vl] = h0 | (hi0 << 16);
+        else {
+          dst[2 * vl] = h0 | (hi0 << 16);
+          dst[2 * vl + 1] = h1 | (hi1 << 16);
+        }
+      }
+    } else {
+      // store at the odd pass (or at an even pass whose token is the block's last)
+      if (ok && !even) {
+        if (bits == 2) dst[vl] = o0 | (h0 << 16);
+        else {
+          dst[2 * vl] = o0 | (h0 << 16);
+          dst[2 * vl + 1] = o1 | (h1 << 16);
+        }
+      } else if (ok && last_odd) {
+        if (bits == 2) dst[vl] = h0;
+        else {
+          dst[2 * vl] = h0;
+          dst[2 * vl + 1] = h1;
+        }
+      }
     }
   }
-  if (bad) atomicOr(&flags, 1);
-  if (rbad) atomicOr(&flags, 2);
-  __syncthreads();
-  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
-  if (bits == 8) {
-    for (int v = threadIdx.x; v < nt * D / 16; v += kThreads)
-      reinterpret_cast<uint4*>(codes + tb * D)[v] = reinterpret_cast<const uint4*>(vsm)[v];
-  } else {
-    // pair layout: word w of pair u holds (16 / b) channels of token 2u (low half) and 2u + 1
-    const int per = 16 / bits, WP = D / per, P = (nt + 1) / 2;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(codes) + (tb / 2) * WP;
-    for (int v = threadIdx.x; v < P * WP; v += kThreads) {
-      const int u = v / WP, w = v % WP;
-      uint32_t lo = 0, hi = 0;
-      for (int j = 0; j < per; ++j) lo |= (uint32_t)vsm[(2 * u) * D + w * per + j] << (bits * j);
-      if (2 * u + 1 < nt)
-        for (int j = 0; j < per; ++j) hi |= (uint32_t)vsm[(2 * u + 1) * D + w * per + j] << (bits * j);
-      dst[v] = lo | (hi << 16);
-    }
-  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&flags, 1);
+  if (__any_sync(0xffffffffu, rbad) && lane == 0) atomicOr(&flags, 2);
   __syncthreads();
   if (threadIdx.x == 0 && flags)
     flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
@@ -203,7 +295,7 @@ __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
 bool asym_fast_ok(const Layout& L, int which) {
   const Side& S = L.side[which];
   if (S.scheme != KVQ_ASYM) return false;
-  if (which == KVQ_KEYS) return S.axis == KVQ_AXIS_CHANNEL && L.g <= 256 && L.D % kCB == 0;
+  if (which == KVQ_KEYS) return S.axis == KVQ_AXIS_CHANNEL && L.g <= 64 * kMaxKeyRows && L.D % kCB == 0;
   return S.axis == KVQ_AXIS_TOKEN && L.D >= 32 && L.D <= 256;
 }
 
@@ -223,7 +315,7 @@ cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, in
     asym_keys_kernel<<<grid, kThreads, 0, s>>>(a);
   } else {
     dim3 grid((unsigned)((n + kTB - 1) / kTB), L.B * L.Hkv);
-    asym_values_kernel<<<grid, kThreads, (size_t)kTB * L.D, s>>>(a);
+    asym_values_kernel<<<grid, kThreads, 0, s>>>(a);
   }
   return cudaGetLastError();
 }

@@ -199,3 +199,28 @@ def test_partition_shapes(B, H, G, tq, ns, tr, splits, src):
     out, ref = run(p, G * H, tq, tr, src, F32, seed=40 + tq, num_splits=splits)
     assert rel_l2(out, ref) <= 1e-3
     assert p.status_bits() == 0
+
+
+@pytest.mark.parametrize("B,H,G,tq,ns,tr,splits", [
+    (8, 8, 4, 32 * 128 - 1, 1, 128, 0),
+    (3, 5, 2, 2 * 128 + 1, 2, 3, 13),
+    (5, 3, 8, 7 * 128 + 64, 1, 100, 1),
+])
+def test_combine_in_split_kernel_matches_two_launches(B, H, G, tq, ns, tr, splits):
+    # decode_attention finishes the combine inside the split kernel on this path; the
+    # separate partial + combine launches must give the same bits
+    fd = fmt(src_dtype=BF16, n_sink=ns, residual_cap=128)
+    p = build(fd, B, H, G * H, tq, tr, seed=90 + G)
+    q = dev(vals(91, (B, G * H, 128), BF16), BF16)
+    scale = 1.0 / np.sqrt(128.0)
+    one = kvq.decode_attention(p.fmt, p.gpu, q, tq, tr, scale, F32, num_splits=splits, status=p.status)
+    ws = torch.empty(kvq.decode_workspace_bytes(p.fmt, B, G * H, H, tq, tr, splits), dtype=torch.uint8,
+                     device="cuda")
+    kvq.decode_partial(p.fmt, p.gpu, q, tq, tr, scale, ws, num_splits=splits, status=p.status)
+    two = torch.empty_like(one)
+    kvq.decode_combine(p.fmt, B, G * H, H, tq, tr, ws, two, num_splits=splits)
+    torch.cuda.synchronize()
+    assert torch.equal(one, two)
+    ref = oatt.decode_attention(p.of, p.ora, q.float().cpu().numpy().astype(np.float64), tq, tr)
+    assert rel_l2(one.cpu().numpy(), ref) <= 1e-3
+    assert p.status_bits() == 0
