@@ -6,10 +6,9 @@ decode attention over the packed cache, on synthetic data shaped like the worklo
                     [--config llama3_8b]
 
 One step = kvq_quantize_keys + kvq_quantize_values of one 128-token group (the
-flush of the raw window into the packed cache) + kvq_decode_attention over all T
-tokens (on this path one split kernel that also finishes the combine, after a memset
-of its arrival counters).  Every step is timed with CUDA events on the launching
-stream; the L2 is flushed between steps, outside the events, by a 512 MiB write and
+flush of the raw window into the packed cache) + kvq_decode_partial (split kernel)
++ kvq_decode_combine over all T tokens.  Every step is timed with CUDA events on the
+launching stream; the L2 is flushed between steps, outside the events, by a 512 MiB write and
 then a 512 MiB read of another buffer (so that no dirty line of the flush is left
 for the step to write back).  `value` is the effective HBM throughput of the whole step: the format's
 algorithmic bytes (codes, scales, zero-points, raw sink / residual tokens, the new
@@ -36,7 +35,7 @@ import synth  # noqa: E402
 
 METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize GB/s"
 L2_FLUSH_BYTES = 512 << 20
-LAUNCHES_PER_STEP = 3   # asym_keys_kernel, asym_values_kernel, decode_mma_kernel
+LAUNCHES_PER_STEP = 4   # asym_keys_kernel, asym_values_kernel, decode_mma_kernel, combine_mma_kernel
 
 
 def parse():
@@ -312,10 +311,12 @@ def main():
         kvq.quantize_values(fmt, cache, newv, gi_f * g, g, status=status, stream=stream)
         if evs:
             evs[1].record(stream)
-        kvq.decode_attention(fmt, cache, q, tq, tr, scale, kvq.F32, out=out, workspace=ws,
-                             status=status, stream=stream)
+        kvq.decode_partial(fmt, cache, q, tq, tr, scale, ws, status=status, stream=stream)
         if evs:
             evs[2].record(stream)
+        kvq.decode_combine(fmt, B, Hq, Hkv, tq, tr, ws, out, stream=stream)
+        if evs:
+            evs[3].record(stream)
 
     for i in range(args.warmup):
         flush_l2(i)
@@ -326,7 +327,7 @@ def main():
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -341,15 +342,17 @@ def main():
     if world > 1:
         dist.barrier()
     t_quant = [e[0].elapsed_time(e[1]) for e in evs]
-    t_dec = [e[1].elapsed_time(e[2]) for e in evs]
-    t_step = [e[0].elapsed_time(e[2]) for e in evs]
+    t_part = [e[1].elapsed_time(e[2]) for e in evs]
+    t_comb = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
     ms_step = statistics.mean(t_step)
-    ms_dec = statistics.mean(t_dec)
+    ms_part = statistics.mean(t_part)
+    ms_comb = statistics.mean(t_comb)
     ms_quant = statistics.mean(t_quant)
     if world > 1:
-        tt = torch.tensor([ms_step, ms_dec, ms_quant], device=dev)
+        tt = torch.tensor([ms_step, ms_part, ms_comb, ms_quant], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step, ms_dec, ms_quant = [float(x) for x in tt.tolist()]
+        ms_step, ms_part, ms_comb, ms_quant = [float(x) for x in tt.tolist()]
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(10, args.steps // 10)
@@ -388,11 +391,11 @@ def main():
     assert torch.isfinite(out).all()
 
     step_bytes = decode_call_bytes(cfg, tq, tr) + quant_bytes(cfg, g)
-    kern_bytes = decode_call_bytes(cfg, tq, tr)
+    kern_bytes = decode_kernel_bytes(cfg, tq, tr)
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
-    decode_gbs = kern_bytes / (ms_dec * 1e-3) / 1e9
+    decode_gbs = decode_call_bytes(cfg, tq, tr) / ((ms_part + ms_comb) * 1e-3) / 1e9
     quant_gbs = quant_bytes(cfg, g) / (ms_quant * 1e-3) / 1e9
-    achieved = decode_gbs
+    achieved = kern_bytes / (ms_part * 1e-3) / 1e9
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -418,10 +421,9 @@ def main():
         "config": workload_config(cfg),
         "pct_of_8tbs": 100.0 * value / world / 8000.0,
         "decode_gbs": decode_gbs, "quantize_gbs": quant_gbs,
-        "tokens_heads_per_s": world * B * Hq * cfg["T"] / (ms_dec * 1e-3),
-        "ms_breakdown": {"quantize": ms_quant, "decode": ms_dec},
-        "roofline": {"kernel": "decode_mma_kernel with its combine (kvq_decode_attention: counter "
-                               "memset + one split kernel)", "bound": "hbm",
+        "tokens_heads_per_s": world * B * Hq * cfg["T"] / ((ms_part + ms_comb) * 1e-3),
+        "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb},
+        "roofline": {"kernel": "decode_mma_kernel (kvq_decode_partial)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": kern_bytes,
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},

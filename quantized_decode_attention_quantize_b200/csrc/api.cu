@@ -358,8 +358,7 @@ int32_t kvq_decode_partial_slots(const kvq_format* f, int32_t B, int32_t Hq, int
 static kvq_status partial_common(const kvq_format* f, const kvq_cache* c, const void* q,
                                  int32_t q_dtype, int32_t Hq, int64_t t_quant, int32_t t_res,
                                  float scale, void* ws, size_t ws_bytes, int32_t num_splits,
-                                 int32_t* d_status, void* stream, Layout* L, DecodePlan* p,
-                                 void* out = nullptr, int32_t out_dtype = 0, int* combined = nullptr) {
+                                 int32_t* d_status, void* stream, Layout* L, DecodePlan* p) {
   kvq_status s = make_layout(f, c, L);
   if (s != KVQ_OK) return s;
   s = decode_args(f, L->B, Hq, L->Hkv, t_quant, t_res, num_splits);
@@ -375,8 +374,7 @@ static kvq_status partial_common(const kvq_format* f, const kvq_cache* c, const 
   if (!ws || !aligned16(ws)) return KVQ_ERR_INVALID;
   if (ws_bytes < workspace_bytes(*L, Hq, *p)) return KVQ_ERR_WORKSPACE;
   cudaError_t e = launch_decode_partial(*L, *p, q, q_dtype, Hq, t_quant, t_res, scale, ws, d_status,
-                                        reinterpret_cast<cudaStream_t>(stream), out, out_dtype,
-                                        combined);
+                                        reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -413,10 +411,9 @@ kvq_status kvq_decode_attention(const kvq_format* f, const kvq_cache* c, const v
   if (!out || !aligned16(out) || !valid_dtype(out_dtype)) return KVQ_ERR_INVALID;
   Layout L;
   DecodePlan p;
-  int combined = 0;
   kvq_status s = partial_common(f, c, q, q_dtype, Hq, t_quant, t_res, scale, ws, ws_bytes,
-                                num_splits, d_status, stream, &L, &p, out, out_dtype, &combined);
-  if (s != KVQ_OK || combined) return s;
+                                num_splits, d_status, stream, &L, &p);
+  if (s != KVQ_OK) return s;
   cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }

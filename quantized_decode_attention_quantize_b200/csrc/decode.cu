@@ -22,8 +22,7 @@ cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, con
                                cudaStream_t s);
 cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
                               int Hq, int64_t t_quant, int t_res, float scale, float* ws_m,
-                              float* ws_l, float* ws_o, int32_t* d_status, cudaStream_t s,
-                              int* counters, void* out, int out_dtype);
+                              float* ws_l, float* ws_o, int32_t* d_status, cudaStream_t s);
 
 namespace {
 
@@ -326,35 +325,21 @@ DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int 
   return p;
 }
 
-// m [rows], l [rows], o [rows][D] (rows = B * Hq * S), then, on the tensor-core path,
-// one arrival counter per KV head for the combine inside the split kernel.
+// m [rows], l [rows], o [rows][D] (rows = B * Hq * S).
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p) {
   const size_t rows = (size_t)L.B * Hq * p.S;
-  const size_t counters = p.fast ? align16((size_t)L.B * L.Hkv * 4) : 0;
-  return align16(rows * 4) * 2 + align16(rows * L.D * 4) + counters;
+  return align16(rows * 4) * 2 + align16(rows * L.D * 4);
 }
 
 cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
                                   int Hq, int64_t t_quant, int t_res, float scale, void* ws,
-                                  int32_t* d_status, cudaStream_t s, void* out, int out_dtype,
-                                  int* combined) {
+                                  int32_t* d_status, cudaStream_t s) {
   const size_t rows = (size_t)L.B * Hq * p.S;
   float* ws_m = reinterpret_cast<float*>(ws);
   float* ws_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align16(rows * 4));
   float* ws_o = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4));
-  if (combined) *combined = 0;
-  if (p.fast) {
-    int* counters = nullptr;
-    if (out) {   // combine in the split kernel: arrival counters start at zero
-      counters = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4) +
-                                        align16(rows * L.D * 4));
-      cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)L.B * L.Hkv * 4, s);
-      if (e != cudaSuccess) return e;
-      if (combined) *combined = 1;
-    }
-    return launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s,
-                             counters, out, out_dtype);
-  }
+  if (p.fast)
+    return launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
   DecArgs a;
   a.L = L;
   a.q = q;

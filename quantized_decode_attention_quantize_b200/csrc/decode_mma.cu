@@ -98,9 +98,6 @@ struct MmaArgs {
   float* ws_l;
   float* ws_o;
   int32_t* status;
-  int* counters;  // non-null: combine in this kernel (one arrival counter per KV head, zeroed)
-  void* out;
-  int out_dtype;
 };
 
 // ---- partition of the items over the warps (shared with the combine kernel) ------------
@@ -130,20 +127,12 @@ __host__ __device__ __forceinline__ bool has_crossing(int64_t h, int64_t U, int6
   const int64_t last = (h + 1) * U - 1;
   return item_start(warp_of_item(last, I, W) + 1, I, W) > last + 1;
 }
-// The valid slots of head h: s_lo (0 with a crossing state, else 1) .. s_hi, and the
-// number of CTAs that write them.
+// The valid slots of head h: s_lo (0 with a crossing state, else 1) .. s_hi.
 __host__ __device__ __forceinline__ void head_slots(int64_t h, int64_t U, int64_t I, int64_t W, int cw,
-                                                    int* s_lo, int* s_hi, int* writers) {
+                                                    int* s_lo, int* s_hi) {
   const int64_t ca = first_ending_warp(h, U, I, W) / cw, cb = last_ending_warp(h, U, I, W) / cw;
-  const bool cross = has_crossing(h, U, I, W);
-  *s_lo = cross ? 0 : 1;
+  *s_lo = has_crossing(h, U, I, W) ? 0 : 1;
   *s_hi = 1 + (int)(cb - ca);
-  int n = (int)(cb - ca + 1);
-  if (cross) {
-    const int64_t cs = warp_of_item((h + 1) * U - 1, I, W) / cw;
-    if (cs < ca || cs > cb) ++n;
-  }
-  *writers = n;
 }
 
 // ---- PTX helpers ------------------------------------------------------------------
@@ -691,8 +680,7 @@ __device__ __forceinline__ void load_raw(const MmaArgs& a, uint8_t* buf, int64_t
 }
 
 // ---- final combine of one query-head row over its valid slots -------------------------
-// Lane owns channels 4 lane .. 4 lane + 3.  Loads bypass L1: the slots were written by
-// other CTAs of the same launch when this runs inside the split kernel.
+// Lane owns channels 4 lane .. 4 lane + 3.
 __device__ __forceinline__ void combine_row(const float* m, const float* l, const float* o, int S,
                                             int64_t row, int s_lo, int s_hi, int lane, void* out,
                                             int out_dtype) {
@@ -739,8 +727,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   uint32_t* my_scratch = reinterpret_cast<uint32_t*>(smem + (size_t)kCW * kBuffers * kStageBytes) +
                          warp * (kScratchBytes / 4);
   int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * (kBuffers * kStageBytes + kScratchBytes));
-  int* cross_head = last_head + kCW;     // the head a warp left for the next one, or -1
-  int* finish = cross_head + kCW;        // [2 kCW] heads whose combine falls to this CTA
   const int nraw = a.n_sink + a.t_res;
 
   // load cursor: one work item ahead of the compute cursor (odd raw positions carry none)
@@ -769,7 +755,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
     cp_async_commit();   // an empty group keeps the group count uniform
     ++issued;
   };
-  issue_next();
+#pragma unroll 1
+  for (int e = 0; e < kBuffers - 1; ++e) issue_next();
 
   MmaState st;
   state_reset(st);
@@ -778,14 +765,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   KeyOp ko;
   int64_t head = i0 / U, cur_head = -1;
   int r = (int)(i0 - head * U);
-  int crossed = -1;
   bool qbad = false;
   int consumed = 0;
 #pragma unroll 1
   for (int64_t i = i0; i < i1; ++i) {
     if (head != cur_head) {
       if (cur_head >= 0) {   // the range crosses into the next head: slot 0 of this one
-        crossed = (int)cur_head;
         const int64_t row0 = cur_head * a.G;
         state_emit<DUAL>(st, a.G, a.ws_o + row0 * a.S * 128, (int64_t)a.S * 128, a.ws_m + row0 * a.S,
                          a.ws_l + row0 * a.S, a.S);
@@ -842,10 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   const int lh = i1 > 0 ? (int)((i1 - 1) / U) : -1;
   float* rec = reinterpret_cast<float*>(ring);
   if (lh >= 0) state_emit<DUAL>(st, a.G, rec, 128, rec + 8 * 128, rec + 8 * 128 + 8, 1);
-  if (lane == 0) {
-    last_head[warp] = lh;
-    cross_head[warp] = crossed;
-  }
+  if (lane == 0) last_head[warp] = lh;
   __syncthreads();
   const int G = a.G;
   int w0 = 0;
@@ -885,37 +867,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
     }
     w0 = w1 + 1;
   }
-  if (!a.counters) return;
-
-  // ---- combine inside the kernel: the last CTA to write a head's slots finishes it ----
-  __threadfence();   // this CTA's slot writes are visible before its arrivals count
-  __syncthreads();
-  if (threadIdx.x < 2 * kCW) {
-    const int e = threadIdx.x;
-    const int h = e < kCW ? cross_head[e] : last_head[e - kCW];
-    bool first = h >= 0;
-    for (int k = 0; k < e && first; ++k) first = (k < kCW ? cross_head[k] : last_head[k - kCW]) != h;
-    int mine = -1;
-    if (first) {
-      int s_lo, s_hi, writers;
-      head_slots(h, U, a.I, a.W, kCW, &s_lo, &s_hi, &writers);
-      if (atomicAdd(a.counters + h, 1) == writers - 1) mine = h;
-    }
-    finish[e] = mine;
-  }
-  __syncthreads();
-#pragma unroll 1
-  for (int e = 0; e < 2 * kCW; ++e) {
-    const int h = finish[e];
-    if (h < 0) continue;
-    __threadfence();
-    if (threadIdx.x < G * 32) {
-      int s_lo, s_hi, writers;
-      head_slots(h, U, a.I, a.W, kCW, &s_lo, &s_hi, &writers);
-      combine_row(a.ws_m, a.ws_l, a.ws_o, a.S, (int64_t)h * G + (threadIdx.x >> 5), s_lo, s_hi, lane,
-                  a.out, a.out_dtype);
-    }
-  }
 }
 
 // ---- combine for this path: the valid slots of a head follow from the partition ---------
@@ -934,16 +885,15 @@ __global__ void __launch_bounds__(128) combine_mma_kernel(CombArgsMma a) {
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= a.rows) return;
-  int s_lo, s_hi, writers;
-  head_slots(row / a.G, a.U, a.I, a.W, kCW, &s_lo, &s_hi, &writers);
+  int s_lo, s_hi;
+  head_slots(row / a.G, a.U, a.I, a.W, kCW, &s_lo, &s_hi);
   combine_row(a.m, a.l, a.o, a.S, row, s_lo, s_hi, lane, a.out, a.out_dtype);
 }
 
-// per-warp rings of item stages, per-warp scratch, then the warps' last and crossing heads
-// and the heads to finish
+// per-warp rings of item stages, per-warp scratch, then the warps' last heads
 static_assert(kStageBytes % 128 == 0, "stage alignment");
 size_t mma_smem() {
-  return (size_t)kCW * kBuffers * kStageBytes + (size_t)kCW * kScratchBytes + 4 * kCW * sizeof(int);
+  return (size_t)kCW * kBuffers * kStageBytes + (size_t)kCW * kScratchBytes + kCW * sizeof(int);
 }
 
 // Positions of a head: two per raw item of rt tokens, then one per packed half.
@@ -1000,8 +950,7 @@ void plan_mma(const Layout& L, int64_t t_quant, int t_res, int max_ctas, DecodeP
 
 cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
                               int64_t t_quant, int t_res, float scale, float* ws_m, float* ws_l,
-                              float* ws_o, int32_t* d_status, cudaStream_t s, int* counters, void* out,
-                              int out_dtype) {
+                              float* ws_o, int32_t* d_status, cudaStream_t s) {
   MmaArgs a;
   a.k_codes = reinterpret_cast<const uint8_t*>(L.side[0].codes);
   a.v_codes = reinterpret_cast<const uint8_t*>(L.side[1].codes);
@@ -1038,9 +987,6 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.ws_l = ws_l;
   a.ws_o = ws_o;
   a.status = d_status;
-  a.counters = counters;
-  a.out = out;
-  a.out_dtype = out_dtype;
   const size_t smem = mma_smem();
   auto kern = a.G <= 4 ? decode_mma_kernel<true> : decode_mma_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

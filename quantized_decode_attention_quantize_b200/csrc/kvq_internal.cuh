@@ -75,13 +75,9 @@ struct DecodePlan {
 DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int num_splits);
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p);
 bool fast_path_ok(const Layout& L, int Hq);
-// With `out` non-null and the tensor-core path planned, the split kernel also finishes
-// the combine (the last CTA of each head writes its rows of `out`); returns with
-// *combined = 1 then.  Otherwise only the partial states are written.
 cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q,
                                   int q_dtype, int Hq, int64_t t_quant, int t_res, float scale,
-                                  void* ws, int32_t* d_status, cudaStream_t s, void* out = nullptr,
-                                  int out_dtype = 0, int* combined = nullptr);
+                                  void* ws, int32_t* d_status, cudaStream_t s);
 cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
                            int out_dtype, cudaStream_t s);
 int device_sm_count();

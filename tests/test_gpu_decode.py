@@ -206,9 +206,8 @@ def test_partition_shapes(B, H, G, tq, ns, tr, splits, src):
     (3, 5, 2, 2 * 128 + 1, 2, 3, 13),
     (5, 3, 8, 7 * 128 + 64, 1, 100, 1),
 ])
-def test_combine_in_split_kernel_matches_two_launches(B, H, G, tq, ns, tr, splits):
-    # decode_attention finishes the combine inside the split kernel on this path; the
-    # separate partial + combine launches must give the same bits
+def test_decode_attention_matches_partial_then_combine(B, H, G, tq, ns, tr, splits):
+    # the one-call entry point and the separate partial + combine calls give the same bits
     fd = fmt(src_dtype=BF16, n_sink=ns, residual_cap=128)
     p = build(fd, B, H, G * H, tq, tr, seed=90 + G)
     q = dev(vals(91, (B, G * H, 128), BF16), BF16)
