@@ -218,6 +218,19 @@ def setup_dist(args):
     return world, rank, local
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over the process group (any backend: the
+    tensor lives on `device`, CPU for gloo); identity without a group of size > 1."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def run_reference(args, world, rank):
     cfg = synth.CONFIGS[args.config]
     if rank != 0:
@@ -349,10 +362,7 @@ def main():
     ms_part = statistics.mean(t_part)
     ms_comb = statistics.mean(t_comb)
     ms_quant = statistics.mean(t_quant)
-    if world > 1:
-        tt = torch.tensor([ms_step, ms_part, ms_comb, ms_quant], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step, ms_part, ms_comb, ms_quant = [float(x) for x in tt.tolist()]
+    ms_step, ms_part, ms_comb, ms_quant = max_over_ranks([ms_step, ms_part, ms_comb, ms_quant], dev)
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(10, args.steps // 10)
@@ -382,11 +392,7 @@ def main():
         e1.synchronize()
         if i >= 3:
             e2e_t.append(e0.elapsed_time(e1))
-    ms_e2e = statistics.mean(e2e_t)
-    if world > 1:
-        tt = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
+    ms_e2e = max_over_ranks([statistics.mean(e2e_t)], dev)[0]
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     assert torch.isfinite(out).all()
 
