@@ -80,6 +80,53 @@ __device__ __forceinline__ void consume_token(WarpState<NC, GM>& st, int G, cons
   }
 }
 
+// Process up to kBatch tokens at once (ok[e] marks the valid ones): the score
+// reductions of all tokens and heads run together, then one softmax update per head.
+constexpr int kBatch = 4;
+template <int NC, int GM>
+__device__ __forceinline__ void consume_batch(WarpState<NC, GM>& st, int G, const float (&kh)[kBatch][NC],
+                                              const float (&vh)[kBatch][NC], const bool (&ok)[kBatch]) {
+  float sc[kBatch][GM];
+#pragma unroll
+  for (int e = 0; e < kBatch; ++e)
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh) {
+      float part = 0.0f;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) part = fmaf(st.q[hh][j], kh[e][j], part);
+      sc[e][hh] = part;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e)
+#pragma unroll
+      for (int hh = 0; hh < GM; ++hh) sc[e][hh] += __shfl_xor_sync(0xffffffffu, sc[e][hh], o);
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    if (hh < G) {
+      float mn = st.m[hh];
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e)
+        if (ok[e]) mn = fmaxf(mn, sc[e][hh]);
+      const float corr = exp2f(st.m[hh] - mn);   // 0 when m = -inf
+      st.l[hh] *= corr;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) st.o[hh][j] *= corr;
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e) {
+        if (ok[e]) {
+          const float p = exp2f(sc[e][hh] - mn);
+          st.l[hh] += p;
+#pragma unroll
+          for (int j = 0; j < NC; ++j) st.o[hh][j] = fmaf(p, vh[e][j], st.o[hh][j]);
+        }
+      }
+      st.m[hh] = mn;
+    }
+  }
+}
+
 // Rotate-half RoPE of the lane's key channels at absolute position pos: channel pairs
 // (c, c + D/2) are both owned by the lane (j and j + NC/2).
 template <int NC>
@@ -92,6 +139,23 @@ __device__ __forceinline__ void rope(float* kh, const double* theta, int64_t pos
     const float x1 = kh[j], x2 = kh[j + NC / 2];
     kh[j] = x1 * c - x2 * s;
     kh[j + NC / 2] = x2 * c + x1 * s;
+  }
+}
+
+// The same rotation from a running (cos, sin) per channel pair, which then advances by
+// the per-step rotation (cst, snt): exact anchors in fp64 at every group, fp32 steps
+// within it.
+template <int NC>
+__device__ __forceinline__ void rope_step(float* kh, float* cs, float* sn, const float* cst,
+                                          const float* snt) {
+#pragma unroll
+  for (int j = 0; j < NC / 2; ++j) {
+    const float x1 = kh[j], x2 = kh[j + NC / 2];
+    kh[j] = x1 * cs[j] - x2 * sn[j];
+    kh[j + NC / 2] = x2 * cs[j] + x1 * sn[j];
+    const float c2 = cs[j] * cst[j] - sn[j] * snt[j];
+    sn[j] = sn[j] * cst[j] + cs[j] * snt[j];
+    cs[j] = c2;
   }
 }
 
@@ -138,6 +202,26 @@ __global__ void __launch_bounds__(kWarps * 32) decode_generic_kernel(DecArgs a) 
     const int64_t g1 = min(ngv, g0 + a.split_groups);
     const Side& SK = L.side[0];
     const Side& SV = L.side[1];
+    // fast element paths: keys per channel (ASYM b < 8, NUQ), values per token (ASYM b < 8, NUQ)
+    const bool k_fast = (SK.scheme == KVQ_ASYM && SK.bits < 8 && SK.axis == KVQ_AXIS_CHANNEL) ||
+                        (SK.scheme == KVQ_NUQ && SK.axis == KVQ_AXIS_CHANNEL);
+    const bool v_fast = (SV.scheme == KVQ_ASYM && SV.bits < 8 && SV.axis == KVQ_AXIS_TOKEN) ||
+                        (SV.scheme == KVQ_NUQ && SV.axis == KVQ_AXIS_TOKEN);
+    // nuq codebooks: lane i holds entry i & 7
+    const float klut = SK.scheme == KVQ_NUQ ? __half2float(SK.lut[lane & 7]) : 0.0f;
+    const float vlut = SV.scheme == KVQ_NUQ ? __half2float(SV.lut[lane & 7]) : 0.0f;
+    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(SK.codes) + sl * SK.code_slab_bytes;
+    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(SV.codes) + sl * SV.code_slab_bytes;
+    float cst[NC / 2 > 0 ? NC / 2 : 1], snt[NC / 2 > 0 ? NC / 2 : 1];
+    if (L.rope) {
+#pragma unroll
+      for (int j = 0; j < NC / 2; ++j) {
+        double sn, cs;
+        sincos((double)kWarps * theta[j], &sn, &cs);
+        cst[j] = (float)cs;
+        snt[j] = (float)sn;
+      }
+    }
     for (int64_t gi = g0; gi < g1; ++gi) {
       if (SK.scheme == KVQ_MIXED) {
         __syncthreads();
@@ -145,37 +229,101 @@ __global__ void __launch_bounds__(kWarps * 32) decode_generic_kernel(DecArgs a) 
         __syncthreads();
       }
       const int64_t tb = gi * L.g, te = min(a.t_quant, tb + L.g);
-      for (int64_t t = tb + warp; t < te; t += kWarps) {
+      // this group's per-channel key metadata for the lane's channels
+      float ks[NC], kz[NC];
+      if (k_fast) {
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
-          const int c = lane + 32 * j;
-          kh[j] = SK.scheme == KVQ_MIXED ? mixed_slot_value(L, sl, t, inv[c]) : deq_dense(L, 0, sl, t, c);
-          vh[j] = deq_dense(L, 1, sl, t, c);
+          const int64_t mi = (sl * L.ng + gi) * D + lane + 32 * j;
+          ks[j] = meta_f16(SK.scale, mi);
+          kz[j] = meta_f16(SK.zero, mi);
         }
-        if (SK.nout > 0) {
-          const int rr = (int)(t - tb);
-          const int32_t* rp = L.k_out_rowptr + (sl * L.ng + gi) * (L.g + 1);
-          const int64_t e0 = (sl * L.ng + gi) * (int64_t)D * SK.nout;
-          for (int e = rp[rr]; e < rp[rr + 1]; ++e) {
-            const int c = L.k_out_col[e0 + e];
-            const float v = __half2float(L.k_out_val[e0 + e]);
+      }
+      // RoPE anchor at this warp's first token of the group
+      float cs[NC / 2 > 0 ? NC / 2 : 1], sn[NC / 2 > 0 ? NC / 2 : 1];
+      if (L.rope) {
 #pragma unroll
-            for (int j = 0; j < NC; ++j)
-              if (c == lane + 32 * j) kh[j] = v;
-          }
+        for (int j = 0; j < NC / 2; ++j) {
+          double s2, c2;
+          sincos((double)(L.n_sink + tb + warp) * theta[j], &s2, &c2);
+          cs[j] = (float)c2;
+          sn[j] = (float)s2;
         }
-        if (SV.nout > 0) {
-          for (int e = 0; e < SV.nout; ++e) {
-            const int64_t idx = (sl * L.C + t) * SV.nout + e;
-            const int c = L.v_out_col[idx];
-            const float v = __half2float(L.v_out_val[idx]);
+      }
+      for (int64_t t0 = tb + warp; t0 < te; t0 += kWarps * kBatch) {
+        float kb[kBatch][NC], vb[kBatch][NC];
+        bool ok[kBatch];
 #pragma unroll
-            for (int j = 0; j < NC; ++j)
-              if (c == lane + 32 * j) vh[j] = v;
+        for (int e = 0; e < kBatch; ++e) {
+          const int64_t t = t0 + (int64_t)e * kWarps;
+          ok[e] = t < te;
+          const int64_t tt = ok[e] ? t : tb;   // a valid row for the loads of unused slots
+#pragma unroll
+          for (int j = 0; j < NC; ++j) {
+            const int c = lane + 32 * j;
+            float kv;
+            if (k_fast) {
+              uint32_t code;
+              if (SK.scheme == KVQ_NUQ) {
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(kbase) + tt * (3 * D / 32);
+                code = ((w[c / 16] >> (2 * (c % 16))) & 3u) | (((w[D / 16 + c / 32] >> (c % 32)) & 1u) << 2);
+                kv = __fmaf_rn(__shfl_sync(0xffffffffu, klut, (int)code), ks[j], kz[j]);
+              } else {
+                const int b = SK.bits, per = 32 / b;
+                const uint32_t w = reinterpret_cast<const uint32_t*>(kbase)[tt * (D / per) + c / per];
+                code = (w >> (b * (c % per))) & ((1u << b) - 1);
+                kv = __fmaf_rn((float)code, ks[j], kz[j]);
+              }
+            } else {
+              kv = SK.scheme == KVQ_MIXED ? mixed_slot_value(L, sl, tt, inv[c]) : deq_dense(L, 0, sl, tt, c);
+            }
+            kb[e][j] = kv;
           }
+          if (v_fast) {
+            const float vs = meta_f16(SV.scale, sl * L.C + tt), vz = meta_f16(SV.zero, sl * L.C + tt);
+#pragma unroll
+            for (int j = 0; j < NC; ++j) {
+              const int c = lane + 32 * j;
+              if (SV.scheme == KVQ_NUQ) {
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(vbase) + tt * (3 * D / 32);
+                const uint32_t code = ((w[c / 16] >> (2 * (c % 16))) & 3u) | (((w[D / 16 + c / 32] >> (c % 32)) & 1u) << 2);
+                vb[e][j] = __fmaf_rn(__shfl_sync(0xffffffffu, vlut, (int)code), vs, vz);
+              } else {
+                const int b = SV.bits, per = 16 / b;
+                const uint32_t w = reinterpret_cast<const uint32_t*>(vbase)[(tt >> 1) * (D / per) + c / per];
+                const uint32_t code = (w >> (16 * (int)(tt & 1) + b * (c % per))) & ((1u << b) - 1);
+                vb[e][j] = __fmaf_rn((float)code, vs, vz);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < NC; ++j) vb[e][j] = deq_dense(L, 1, sl, tt, lane + 32 * j);
+          }
+          if (SK.nout > 0 && ok[e]) {
+            const int rr = (int)(t - tb);
+            const int32_t* rp = L.k_out_rowptr + (sl * L.ng + gi) * (L.g + 1);
+            const int64_t e0 = (sl * L.ng + gi) * (int64_t)D * SK.nout;
+            for (int x = rp[rr]; x < rp[rr + 1]; ++x) {
+              const int c = L.k_out_col[e0 + x];
+              const float v = __half2float(L.k_out_val[e0 + x]);
+#pragma unroll
+              for (int j = 0; j < NC; ++j)
+                if (c == lane + 32 * j) kb[e][j] = v;
+            }
+          }
+          if (SV.nout > 0 && ok[e]) {
+            for (int x = 0; x < SV.nout; ++x) {
+              const int64_t idx = (sl * L.C + t) * SV.nout + x;
+              const int c = L.v_out_col[idx];
+              const float v = __half2float(L.v_out_val[idx]);
+#pragma unroll
+              for (int j = 0; j < NC; ++j)
+                if (c == lane + 32 * j) vb[e][j] = v;
+            }
+          }
+          if (L.rope) rope_step<NC>(kb[e], cs, sn, cst, snt);
         }
-        if (L.rope) rope<NC>(kh, theta, L.n_sink + t);
-        consume_token<NC, GM>(st, G, kh, vh);
+        consume_batch<NC, GM>(st, G, kb, vb, ok);
       }
     }
   } else if (split == a.raw_slot) {

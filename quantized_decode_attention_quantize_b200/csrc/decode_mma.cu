@@ -1,6 +1,6 @@
 // Tensor-core split-KV decode over a packed cache of 4-bit per-channel keys and 2-bit
 // per-token values (the K4V2 allocation of [K4V2]; grouping of [KVQ] "Approach"),
-// D = 128, token groups of 128, 2 <= G <= 8 query heads per KV head.
+// D = 128, token groups of 128, 1 <= G <= 8 query heads per KV head.
 //
 // Work.  Each KV head is a row of U items: first its raw (sink + residual) tokens in
 // items of up to 8 tokens (4 for fp32 sources), each weighted as two positions of
@@ -920,7 +920,7 @@ bool mma_path_ok(const Layout& L, int Hq) {
   const int G = Hq / L.Hkv;
   return L.D == 128 && L.g == 128 && K.scheme == KVQ_ASYM && K.bits == 4 &&
          K.axis == KVQ_AXIS_CHANNEL && V.scheme == KVQ_ASYM && V.bits == 2 &&
-         V.axis == KVQ_AXIS_TOKEN && L.rope == 0 && G >= 2 && G <= 8;
+         V.axis == KVQ_AXIS_TOKEN && L.rope == 0 && G >= 1 && G <= 8;
 }
 
 // Partition of the fast path (t_quant >= 1): CTAs, slots per query head.  At least one

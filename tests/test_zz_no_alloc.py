@@ -38,9 +38,9 @@ def test_noalloc_matches_workspace_entry_point(G, src, out_dtype):
 
 def test_noalloc_rejects_oversized_requests():
     # a workspace need above the scratch size is refused before anything runs
-    fd = fmt(src_dtype=BF16)
+    fd = fmt(src_dtype=BF16, rope=1)        # the generic path: 64 splits per head as asked
     f = kvq.make_format(fd)
-    B, Hq, Hkv, tq = 64, 64, 64, 131072     # one query head per KV head, 64 splits each
+    B, Hq, Hkv, tq = 64, 64, 64, 131072
     need = kvq.decode_workspace_bytes(f, B, Hq, Hkv, tq, 0, 64)
     assert need > kvq.NOALLOC_SCRATCH_BYTES
     cache = kvq.kvq_cache(batch=B, kv_heads=Hkv, capacity=tq)
