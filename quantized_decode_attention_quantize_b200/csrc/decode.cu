@@ -24,6 +24,12 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
                               int Hq, int64_t t_quant, int t_res, float scale, float* ws_m,
                               float* ws_l, float* ws_o, int32_t* d_status, cudaStream_t s);
 
+// CUDA-core path with four consecutive channels per lane (decode_cc.cu)
+bool cc_path_ok(const Layout& L, int Hq);
+cudaError_t launch_decode_cc(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
+                             int64_t t_quant, int t_res, float scale, float* ws_m, float* ws_l,
+                             float* ws_o, int32_t* d_status, cudaStream_t s);
+
 namespace {
 
 constexpr int kWarps = 4;
@@ -488,6 +494,8 @@ cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const vo
   float* ws_o = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4));
   if (p.fast)
     return launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
+  if (cc_path_ok(L, Hq))
+    return launch_decode_cc(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
   DecArgs a;
   a.L = L;
   a.q = q;

@@ -1,0 +1,444 @@
+// Split-KV decode on CUDA cores for D = 128 packed formats that the tensor-core kernel
+// does not take: nuq3 keys and values with sparse outliers and RoPE on the keys
+// ([KVQ] "Approach", "Dense-and-Sparse"), MixKVQ salience-ordered keys ([MIX] Fig. 4),
+// asymmetric 2/4-bit keys with RoPE, G <= 8 query heads per KV head.
+//
+// Same work split, partial states and combine as the generic kernel (split = a run of
+// token groups of one KV head, or the raw sink + residual tokens; four warps, token t
+// to warp t mod 4).  What differs is the lane layout: lane l owns the four consecutive
+// channels 4 l .. 4 l + 3, so one 32-bit word of a packed row holds all of its codes,
+// one load per plane and token; the group's per-channel key scale / zero-point sit in
+// registers.  MIXED keys are walked in storage-slot order (lane l: slots 4 l .. 4 l + 3)
+// against the query gathered into slot order once per group.  RoPE pairs (c, c + 64)
+// live in lanes l and l ^ 16 and meet through one shuffle; the rotation is anchored
+// exactly (fp64) at each group and advanced in fp32 from token to token.  Scores of
+// four tokens are reduced together, then one softmax update per head.
+#include <cmath>
+
+#include "decode_common.cuh"
+
+namespace kvq {
+
+namespace {
+
+constexpr int kW = 4;        // warps per CTA
+constexpr int kB = 4;        // tokens per batch
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kRS = 132;     // merge record stride (floats): o[128], m, l, padding to 16 bytes
+
+struct CcArgs {
+  Layout L;
+  const void* q;
+  int q_dtype, Hq;
+  int64_t t_quant;
+  int t_res;
+  float qscale;
+  int S, split_groups, n_packed, raw_slot;
+  float* ws_m;
+  float* ws_l;
+  float* ws_o;
+  int32_t* status;
+};
+
+// Four consecutive elements of a raw row (16-bit or fp32 source).
+__device__ __forceinline__ float4 ld4(const void* p, int64_t i, int dtype) {
+  if (dtype == KVQ_F32) return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i);
+  const uint2 x = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(p) + i);
+  if (dtype == KVQ_F16) {
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  }
+  return make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u),
+                     __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u));
+}
+
+// Rotate-half RoPE of the lane's four channels: lanes l < 16 hold x1 of pairs
+// i = 4 l + j, lanes l + 16 the partner x2.
+__device__ __forceinline__ void rope4(float* x, const float* cs, const float* sn, int lane) {
+  const bool first = lane < 16;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float other = __shfl_xor_sync(0xffffffffu, x[j], 16);
+    x[j] = first ? fmaf(x[j], cs[j], -other * sn[j]) : fmaf(x[j], cs[j], other * sn[j]);
+  }
+}
+
+// nuq3 codes of channels 4 l .. 4 l + 3 of a row (2-bit plane then 1-bit plane).
+__device__ __forceinline__ void nuq_codes(const uint32_t* row, int lane, uint32_t* code) {
+  const uint32_t w2 = row[lane >> 2] >> (8 * (lane & 3));
+  const uint32_t w1 = row[8 + (lane >> 3)] >> (4 * (lane & 7));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) code[j] = ((w2 >> (2 * j)) & 3u) | (((w1 >> j) & 1u) << 2);
+}
+
+template <int GM>
+__global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
+  extern __shared__ __align__(16) float smem[];
+  const Layout& L = a.L;
+  constexpr int D = 128;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = a.Hq / L.Hkv;
+  const int64_t sl = (int64_t)b * L.Hkv + h;
+  const Side& SK = L.side[0];
+  const Side& SV = L.side[1];
+  const bool mixed = SK.scheme == KVQ_MIXED;
+  float* qsm = smem;                                  // [GM][128] pre-scaled queries (MIXED)
+  uint8_t* order = reinterpret_cast<uint8_t*>(smem + GM * D);   // [128] slot -> channel (MIXED)
+  float* wst = smem + GM * D + 32;                    // [kW][G][kRS] merge records
+
+  float q[GM][4], o[GM][4], m[GM], l[GM];
+  int bad = 0;
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    m[hh] = -INFINITY;
+    l[hh] = 0.0f;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (hh < G) {
+      x = ld4(a.q, ((int64_t)b * a.Hq + h * G + hh) * D + 4 * lane, a.q_dtype);
+      bad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+    }
+    q[hh][0] = x.x * a.qscale; q[hh][1] = x.y * a.qscale;
+    q[hh][2] = x.z * a.qscale; q[hh][3] = x.w * a.qscale;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[hh][j] = 0.0f;
+    if (mixed && warp == 0)
+      *reinterpret_cast<float4*>(qsm + hh * D + 4 * lane) = make_float4(q[hh][0], q[hh][1], q[hh][2], q[hh][3]);
+  }
+  // RoPE frequencies of this lane's pairs i = 4 (l & 15) + j
+  double theta[4];
+  if (L.rope) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) theta[j] = pow((double)L.rope_base, -2.0 * (double)(4 * (lane & 15) + j) / (double)D);
+  }
+
+  auto consume = [&](const float (&kb)[kB][4], const float (&vb)[kB][4], const float (&qk)[GM][4],
+                     const bool (&ok)[kB]) {
+    float sc[kB][GM];
+#pragma unroll
+    for (int e = 0; e < kB; ++e)
+#pragma unroll
+      for (int hh = 0; hh < GM; ++hh) {
+        float part = qk[hh][0] * kb[e][0];
+        part = fmaf(qk[hh][1], kb[e][1], part);
+        part = fmaf(qk[hh][2], kb[e][2], part);
+        part = fmaf(qk[hh][3], kb[e][3], part);
+        sc[e][hh] = part;
+      }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1)
+#pragma unroll
+      for (int e = 0; e < kB; ++e)
+#pragma unroll
+        for (int hh = 0; hh < GM; ++hh) sc[e][hh] += __shfl_xor_sync(0xffffffffu, sc[e][hh], s);
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh) {
+      if (hh < G) {
+        float mn = m[hh];
+#pragma unroll
+        for (int e = 0; e < kB; ++e)
+          if (ok[e]) mn = fmaxf(mn, sc[e][hh]);
+        const float corr = exp2f(m[hh] - mn);
+        l[hh] *= corr;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[hh][j] *= corr;
+#pragma unroll
+        for (int e = 0; e < kB; ++e) {
+          if (ok[e]) {
+            const float p = exp2f(sc[e][hh] - mn);
+            l[hh] += p;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[hh][j] = fmaf(p, vb[e][j], o[hh][j]);
+          }
+        }
+        m[hh] = mn;
+      }
+    }
+  };
+
+  if (split < a.n_packed) {
+    if (mixed) __syncthreads();   // qsm written
+    const int64_t ngv = (a.t_quant + L.g - 1) / L.g;
+    const int64_t g0 = (int64_t)split * a.split_groups;
+    const int64_t g1 = min(ngv, g0 + a.split_groups);
+    const float klut = SK.scheme == KVQ_NUQ ? __half2float(SK.lut[lane & 7]) : 0.0f;
+    const float vlut = SV.scheme == KVQ_NUQ ? __half2float(SV.lut[lane & 7]) : 0.0f;
+    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(SK.codes) + sl * SK.code_slab_bytes;
+    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(SV.codes) + sl * SV.code_slab_bytes;
+    const int hi = L.mixed_hi, mid = L.mixed_mid, lo = L.mixed_lo;
+    float cst[4], snt[4];
+    if (L.rope) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        double sn2, cs2;
+        sincos((double)kW * theta[j], &sn2, &cs2);
+        cst[j] = (float)cs2;
+        snt[j] = (float)sn2;
+      }
+    }
+    for (int64_t gi = g0; gi < g1; ++gi) {
+      const int64_t tb = gi * L.g, te = min(a.t_quant, tb + L.g);
+      // group metadata of the lane's channels (slots for MIXED) and, for MIXED, the
+      // query in slot order
+      float ks[4] = {0.f, 0.f, 0.f, 0.f}, kz[4] = {0.f, 0.f, 0.f, 0.f};
+      float qk[GM][4];
+#pragma unroll
+      for (int hh = 0; hh < GM; ++hh)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qk[hh][j] = q[hh][j];
+      if (mixed) {
+        __syncthreads();
+        if (threadIdx.x < D) order[threadIdx.x] = L.k_order[(sl * L.ng + gi) * D + threadIdx.x];
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int slot = 4 * lane + j;
+          const int ch = order[slot];
+#pragma unroll
+          for (int hh = 0; hh < GM; ++hh) qk[hh][j] = qsm[hh * D + ch];
+          if (slot >= hi) {
+            const int64_t mi = (sl * L.ng + gi) * (D - hi) + (slot - hi);
+            ks[j] = meta_f16(SK.scale, mi);
+            kz[j] = meta_f16(SK.zero, mi);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t mi = (sl * L.ng + gi) * D + 4 * lane + j;
+          ks[j] = meta_f16(SK.scale, mi);
+          kz[j] = meta_f16(SK.zero, mi);
+        }
+      }
+      float cs[4], sn[4];
+      if (L.rope) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          double s2, c2;
+          sincos((double)(L.n_sink + tb + warp) * theta[j], &s2, &c2);
+          cs[j] = (float)c2;
+          sn[j] = (float)s2;
+        }
+      }
+      const uint8_t* gbase = mixed ? reinterpret_cast<const uint8_t*>(SK.codes) +
+                                         (sl * L.ng + gi) * (int64_t)L.mixed_group_bytes
+                                   : nullptr;
+      for (int64_t t0 = tb + warp; t0 < te; t0 += kW * kB) {
+        float kb[kB][4], vb[kB][4];
+        bool ok[kB];
+#pragma unroll
+        for (int e = 0; e < kB; ++e) {
+          const int64_t t = t0 + (int64_t)e * kW;
+          ok[e] = t < te;
+          const int64_t tt = ok[e] ? t : tb;
+          // keys
+          if (mixed) {
+            const int r = (int)(tt - tb);
+            const int s0 = 4 * lane;
+            if (s0 < hi) {
+              // raw 16-bit slots (MIXED sources are fp16 or bf16)
+              const float4 f = ld4(gbase, (int64_t)r * hi + s0, L.src_dtype);
+              kb[e][0] = f.x; kb[e][1] = f.y; kb[e][2] = f.z; kb[e][3] = f.w;
+            } else if (s0 < hi + mid) {
+              const int e0 = s0 - hi;
+              const uint32_t w = reinterpret_cast<const uint32_t*>(gbase + (int64_t)L.g * hi * 2)[r * (mid / 8) + e0 / 8] >>
+                                 (4 * (e0 % 8));
+#pragma unroll
+              for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (4 * j)) & 15u), ks[j], kz[j]);
+            } else {
+              const int e0 = s0 - hi - mid;
+              const uint32_t w =
+                  reinterpret_cast<const uint32_t*>(gbase + (int64_t)L.g * hi * 2 + (int64_t)L.g * mid / 2)[r * (lo / 16) + e0 / 16] >>
+                  (2 * (e0 % 16));
+#pragma unroll
+              for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (2 * j)) & 3u), ks[j], kz[j]);
+            }
+          } else if (SK.scheme == KVQ_NUQ) {
+            uint32_t code[4];
+            nuq_codes(reinterpret_cast<const uint32_t*>(kbase) + tt * 12, lane, code);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn(__shfl_sync(0xffffffffu, klut, (int)code[j]), ks[j], kz[j]);
+          } else {   // ASYM 2 / 4 bits, row layout
+            const int bb = SK.bits;
+            const int bitoff = 4 * lane * bb;
+            const uint32_t w = reinterpret_cast<const uint32_t*>(kbase)[tt * (D * bb / 32) + bitoff / 32] >> (bitoff % 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (bb * j)) & ((1u << bb) - 1)), ks[j], kz[j]);
+          }
+          // values (per token)
+          const float vs = meta_f16(SV.scale, sl * L.C + tt), vz = meta_f16(SV.zero, sl * L.C + tt);
+          if (SV.scheme == KVQ_NUQ) {
+            uint32_t code[4];
+            nuq_codes(reinterpret_cast<const uint32_t*>(vbase) + tt * 12, lane, code);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) vb[e][j] = __fmaf_rn(__shfl_sync(0xffffffffu, vlut, (int)code[j]), vs, vz);
+          } else {   // ASYM 2 / 4 bits, pair layout
+            const int bb = SV.bits, per = 16 / bb;
+            const int c0 = 4 * lane;
+            const uint32_t w = reinterpret_cast<const uint32_t*>(vbase)[(tt >> 1) * (D / per) + c0 / per] >>
+                               (16 * (int)(tt & 1) + bb * (c0 % per));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) vb[e][j] = __fmaf_rn((float)((w >> (bb * j)) & ((1u << bb) - 1)), vs, vz);
+          }
+          // sparse outliers overwrite (before RoPE)
+          if (SK.nout > 0 && ok[e]) {
+            const int rr = (int)(t - tb);
+            const int32_t* rp = L.k_out_rowptr + (sl * L.ng + gi) * (L.g + 1);
+            const int64_t e0 = (sl * L.ng + gi) * (int64_t)D * SK.nout;
+            const int x0 = rp[rr], x1 = rp[rr + 1];
+            for (int x = x0; x < x1; ++x) {
+              const int c = L.k_out_col[e0 + x];
+              const float v = __half2float(L.k_out_val[e0 + x]);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (c == 4 * lane + j) kb[e][j] = v;
+            }
+          }
+          if (SV.nout > 0 && ok[e]) {
+            for (int x = 0; x < SV.nout; ++x) {
+              const int64_t idx = (sl * L.C + t) * SV.nout + x;
+              const int c = L.v_out_col[idx];
+              const float v = __half2float(L.v_out_val[idx]);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (c == 4 * lane + j) vb[e][j] = v;
+            }
+          }
+          if (L.rope) {
+            rope4(kb[e], cs, sn, lane);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float c2 = cs[j] * cst[j] - sn[j] * snt[j];
+              sn[j] = sn[j] * cst[j] + cs[j] * snt[j];
+              cs[j] = c2;
+            }
+          }
+        }
+        consume(kb, vb, qk, ok);
+      }
+    }
+  } else if (split == a.raw_slot) {
+    const int nraw = L.n_sink + a.t_res;
+    for (int r0 = warp; r0 < nraw; r0 += kW * kB) {
+      float kb[kB][4], vb[kB][4];
+      bool ok[kB];
+#pragma unroll
+      for (int e = 0; e < kB; ++e) {
+        const int r = r0 + e * kW;
+        ok[e] = r < nraw;
+        const int rr = ok[e] ? r : r0;
+        const bool sink = rr < L.n_sink;
+        const int64_t row = sink ? rr : rr - L.n_sink;
+        const int64_t rows = sink ? L.n_sink : L.res_cap;
+        const int64_t i = (sl * rows + row) * D + 4 * lane;
+        const float4 kf = ld4(sink ? L.sink[0] : L.res[0], i, L.src_dtype);
+        const float4 vf = ld4(sink ? L.sink[1] : L.res[1], i, L.src_dtype);
+        kb[e][0] = kf.x; kb[e][1] = kf.y; kb[e][2] = kf.z; kb[e][3] = kf.w;
+        vb[e][0] = vf.x; vb[e][1] = vf.y; vb[e][2] = vf.z; vb[e][3] = vf.w;
+        if (L.rope) {
+          const int64_t pos = sink ? rr : L.n_sink + a.t_quant + row;
+          float cs[4], sn[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            double s2, c2;
+            sincos((double)pos * theta[j], &s2, &c2);
+            cs[j] = (float)c2;
+            sn[j] = (float)s2;
+          }
+          rope4(kb[e], cs, sn, lane);
+        }
+      }
+      consume(kb, vb, q, ok);
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+
+  // merge the warps' states and write this split's partial state
+  float* mine = wst + (size_t)warp * G * kRS;
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    if (hh < G) {
+      *reinterpret_cast<float4*>(mine + hh * kRS + 4 * lane) = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+      if (lane == 0) {
+        mine[hh * kRS + D] = m[hh];
+        mine[hh * kRS + D + 1] = l[hh];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int hh = i / D, d = i % D;
+    float M = -INFINITY;
+    for (int w = 0; w < kW; ++w) M = fmaxf(M, wst[((size_t)w * G + hh) * kRS + D]);
+    float lsum = 0.0f, osum = 0.0f;
+    for (int w = 0; w < kW; ++w) {
+      const float* pw = wst + ((size_t)w * G + hh) * kRS;
+      const float f = pw[D] == -INFINITY ? 0.0f : exp2f(pw[D] - M);
+      lsum = fmaf(pw[D + 1], f, lsum);
+      osum = fmaf(pw[d], f, osum);
+    }
+    const int64_t slot = ((int64_t)b * a.Hq + h * G + hh) * a.S + split;
+    a.ws_o[slot * D + d] = osum;
+    if (d == 0) {
+      a.ws_m[slot] = M;
+      a.ws_l[slot] = lsum;
+    }
+  }
+}
+
+template <int GM>
+cudaError_t launch_cc_g(const CcArgs& a, int grid_x, cudaStream_t s) {
+  const int G = a.Hq / a.L.Hkv;
+  // queries (GM x 128), slot order (128 B), merge records; the records are 16-byte aligned
+  const size_t smem = ((size_t)GM * 128 + 32 + (size_t)kW * G * kRS) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(decode_cc_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(grid_x, a.L.Hkv, a.L.B);
+  decode_cc_kernel<GM><<<grid, kW * 32, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool cc_path_ok(const Layout& L, int Hq) {
+  const Side& K = L.side[0];
+  const Side& V = L.side[1];
+  const int G = Hq / L.Hkv;
+  if (L.D != 128 || G < 1 || G > 8) return false;
+  const bool k_ok = (K.scheme == KVQ_NUQ && K.axis == KVQ_AXIS_CHANNEL) ||
+                    (K.scheme == KVQ_ASYM && K.axis == KVQ_AXIS_CHANNEL && (K.bits == 2 || K.bits == 4)) ||
+                    (K.scheme == KVQ_MIXED && !L.rope);
+  const bool v_ok = (V.scheme == KVQ_NUQ && V.axis == KVQ_AXIS_TOKEN) ||
+                    (V.scheme == KVQ_ASYM && V.axis == KVQ_AXIS_TOKEN && (V.bits == 2 || V.bits == 4));
+  return k_ok && v_ok;
+}
+
+cudaError_t launch_decode_cc(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
+                             int64_t t_quant, int t_res, float scale, float* ws_m, float* ws_l,
+                             float* ws_o, int32_t* d_status, cudaStream_t s) {
+  CcArgs a;
+  a.L = L;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.Hq = Hq;
+  a.t_quant = t_quant;
+  a.t_res = t_res;
+  a.qscale = scale * kLog2e;
+  a.S = p.S;
+  a.split_groups = p.split_groups;
+  a.n_packed = p.n_packed_splits;
+  a.raw_slot = p.raw_slot;
+  a.ws_m = ws_m;
+  a.ws_l = ws_l;
+  a.ws_o = ws_o;
+  a.status = d_status;
+  const int G = Hq / L.Hkv;
+  if (G <= 1) return launch_cc_g<1>(a, p.S, s);
+  if (G <= 2) return launch_cc_g<2>(a, p.S, s);
+  if (G <= 4) return launch_cc_g<4>(a, p.S, s);
+  return launch_cc_g<8>(a, p.S, s);
+}
+
+}  // namespace kvq

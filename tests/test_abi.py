@@ -137,7 +137,7 @@ def test_host_validation_rejects_before_launch():
 
 
 def test_workspace_bytes_with_explicit_splits():
-    f = _fmt()
+    f = _fmt(k_bits=8)   # 8-bit keys: the generic split-per-group-run path
     # slots: 4 packed splits, no raw tokens -> B*Hq*4 * (2 + D) floats (16-byte padded)
     n = kvq.decode_workspace_bytes(f, 1, 32, 32, 4096, 0, 4)
     rows = 32 * 4
