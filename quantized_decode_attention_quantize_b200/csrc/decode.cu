@@ -139,9 +139,8 @@ template <int NC>
 __device__ __forceinline__ void rope(float* kh, const double* theta, int64_t pos) {
 #pragma unroll
   for (int j = 0; j < NC / 2; ++j) {
-    double sn, cs;
-    sincos((double)pos * theta[j], &sn, &cs);
-    const float c = (float)cs, s = (float)sn;
+    float s, c;
+    angle_sincos((double)pos, theta[j], &s, &c);
     const float x1 = kh[j], x2 = kh[j + NC / 2];
     kh[j] = x1 * c - x2 * s;
     kh[j + NC / 2] = x2 * c + x1 * s;
@@ -222,10 +221,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_generic_kernel(DecArgs a) 
     if (L.rope) {
 #pragma unroll
       for (int j = 0; j < NC / 2; ++j) {
-        double sn, cs;
-        sincos((double)kWarps * theta[j], &sn, &cs);
-        cst[j] = (float)cs;
-        snt[j] = (float)sn;
+        angle_sincos((double)kWarps, theta[j], &snt[j], &cst[j]);
       }
     }
     for (int64_t gi = g0; gi < g1; ++gi) {
@@ -250,10 +246,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_generic_kernel(DecArgs a) 
       if (L.rope) {
 #pragma unroll
         for (int j = 0; j < NC / 2; ++j) {
-          double s2, c2;
-          sincos((double)(L.n_sink + tb + warp) * theta[j], &s2, &c2);
-          cs[j] = (float)c2;
-          sn[j] = (float)s2;
+          angle_sincos((double)(L.n_sink + tb + warp), theta[j], &sn[j], &cs[j]);
         }
       }
       for (int64_t t0 = tb + warp; t0 < te; t0 += kWarps * kBatch) {

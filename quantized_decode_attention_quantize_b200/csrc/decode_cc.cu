@@ -26,7 +26,19 @@ constexpr int kB = 4;        // tokens per batch
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRS = 132;     // merge record stride (floats): o[128], m, l, padding to 16 bytes
 
+// Byte offsets of the regions of a chunk stage (32 tokens of one group, with the
+// group's metadata), each 16-byte aligned; computed on the host for the layout.
+struct CcStage {
+  int k, k_mid, k_lo;       // key rows (MIXED: raw, 4-bit and 2-bit planes)
+  int v, vs, vz;            // value rows, value scale / zero-point
+  int voc, vov;             // value outliers: columns, values
+  int ks, kz, ord;          // group key scale / zero-point, MIXED slot order
+  int rp, kc, kv;           // key outliers: 33 row pointers, the group's columns and values
+  int bytes;
+};
+
 struct CcArgs {
+  CcStage st;
   Layout L;
   const void* q;
   int q_dtype, Hq;
@@ -72,8 +84,24 @@ __device__ __forceinline__ void nuq_codes(const uint32_t* row, int lane, uint32_
   for (int j = 0; j < 4; ++j) code[j] = ((w2 >> (2 * j)) & 3u) | (((w1 >> j) & 1u) << 2);
 }
 
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// bytes (a multiple of 16) from src to dst, all lanes of the warp
+__device__ __forceinline__ void cp_range(uint8_t* dst, const void* src, int bytes, int lane) {
+  for (int o = 16 * lane; o < bytes; o += 512) cp16(dst + o, reinterpret_cast<const uint8_t*>(src) + o);
+}
+
 template <int GM>
-__global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
+__global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcArgs a) {
   extern __shared__ __align__(16) float smem[];
   const Layout& L = a.L;
   constexpr int D = 128;
@@ -84,9 +112,10 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
   const Side& SK = L.side[0];
   const Side& SV = L.side[1];
   const bool mixed = SK.scheme == KVQ_MIXED;
-  float* qsm = smem;                                  // [GM][128] pre-scaled queries (MIXED)
-  uint8_t* order = reinterpret_cast<uint8_t*>(smem + GM * D);   // [128] slot -> channel (MIXED)
-  float* wst = smem + GM * D + 32;                    // [kW][G][kRS] merge records
+  const CcStage& SG = a.st;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(smem) + (size_t)warp * 2 * SG.bytes;   // [kW][2] stages
+  float* qsm = smem + (size_t)kW * 2 * SG.bytes / 4;  // [GM][128] pre-scaled queries (MIXED)
+  float* wst = qsm + GM * D;                          // [kW][G][kRS] merge records
 
   float q[GM][4], o[GM][4], m[GM], l[GM];
   int bad = 0;
@@ -113,9 +142,16 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
     for (int j = 0; j < 4; ++j) theta[j] = pow((double)L.rope_base, -2.0 * (double)(4 * (lane & 15) + j) / (double)D);
   }
 
+  // Scores of kB tokens x GM heads: value i = e GM + hh, N = kB GM values (a power of two
+  // <= 32).  A reduce-scatter over the warp (each level halves the values a lane keeps)
+  // leaves lane l with the full score of value l >> (5 - log2 N); the softmax of a head
+  // over the batch then takes two shuffle levels, and every lane gets each probability by
+  // one broadcast for the value accumulation.
   auto consume = [&](const float (&kb)[kB][4], const float (&vb)[kB][4], const float (&qk)[GM][4],
                      const bool (&ok)[kB]) {
-    float sc[kB][GM];
+    constexpr int N = kB * GM;
+    constexpr int LN = N == 4 ? 2 : N == 8 ? 3 : N == 16 ? 4 : 5;
+    float v[N];
 #pragma unroll
     for (int e = 0; e < kB; ++e)
 #pragma unroll
@@ -124,33 +160,54 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
         part = fmaf(qk[hh][1], kb[e][1], part);
         part = fmaf(qk[hh][2], kb[e][2], part);
         part = fmaf(qk[hh][3], kb[e][3], part);
-        sc[e][hh] = part;
+        v[e * GM + hh] = part;
       }
+    // reduce-scatter: level with offset o = 16, 8, ... keeps the half selected by that lane bit
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1)
+    for (int lev = 0; lev < LN; ++lev) {
+      const int off = 16 >> lev;
+      const int half = N >> (lev + 1);
+      const bool upper = lane & off;
 #pragma unroll
-      for (int e = 0; e < kB; ++e)
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? v[i] : v[i + half];
+        const float keep = upper ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+    }
 #pragma unroll
-        for (int hh = 0; hh < GM; ++hh) sc[e][hh] += __shfl_xor_sync(0xffffffffu, sc[e][hh], s);
+    for (int off = 16 >> LN; off > 0; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    const int idx = lane >> (5 - LN);
+    const int my_e = idx / GM, my_h = idx % GM;
+    const bool my_ok = ok[0] && (my_e == 0) || ok[1] && (my_e == 1) || ok[2] && (my_e == 2) || ok[3] && (my_e == 3);
+    const float s_mine = my_ok ? v[0] : -INFINITY;
+    // batch max of my head over the tokens (lane bits 4 and 3 carry the token)
+    float bm = fmaxf(s_mine, __shfl_xor_sync(0xffffffffu, s_mine, 16));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+    float mh_old = m[0];
+#pragma unroll
+    for (int hh = 1; hh < GM; ++hh)
+      if (my_h == hh) mh_old = m[hh];
+    const float mnew = fmaxf(mh_old, bm);
+    const float p_mine = my_ok ? exp2f(s_mine - mnew) : 0.0f;
+    float psum = p_mine + __shfl_xor_sync(0xffffffffu, p_mine, 16);
+    psum += __shfl_xor_sync(0xffffffffu, psum, 8);
+    const float corr_mine = exp2f(mh_old - mnew);   // 0 when m = -inf
 #pragma unroll
     for (int hh = 0; hh < GM; ++hh) {
+      const int src = hh << (5 - LN);   // lane of (token 0, head hh)
+      const float corr = __shfl_sync(0xffffffffu, corr_mine, src);
+      const float mn = __shfl_sync(0xffffffffu, mnew, src);
+      const float ps = __shfl_sync(0xffffffffu, psum, src);
       if (hh < G) {
-        float mn = m[hh];
-#pragma unroll
-        for (int e = 0; e < kB; ++e)
-          if (ok[e]) mn = fmaxf(mn, sc[e][hh]);
-        const float corr = exp2f(m[hh] - mn);
-        l[hh] *= corr;
+        l[hh] = fmaf(l[hh], corr, ps);
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[hh][j] *= corr;
 #pragma unroll
         for (int e = 0; e < kB; ++e) {
-          if (ok[e]) {
-            const float p = exp2f(sc[e][hh] - mn);
-            l[hh] += p;
+          const float p = __shfl_sync(0xffffffffu, p_mine, (e * GM + hh) << (5 - LN));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) o[hh][j] = fmaf(p, vb[e][j], o[hh][j]);
-          }
+          for (int j = 0; j < 4; ++j) o[hh][j] = fmaf(p, vb[e][j], o[hh][j]);
         }
         m[hh] = mn;
       }
@@ -162,134 +219,167 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
     const int64_t ngv = (a.t_quant + L.g - 1) / L.g;
     const int64_t g0 = (int64_t)split * a.split_groups;
     const int64_t g1 = min(ngv, g0 + a.split_groups);
+    const int cpg = L.g / 32;                         // chunks per group
+    const int64_t nchunk = (g1 - g0) * cpg;
     const float klut = SK.scheme == KVQ_NUQ ? __half2float(SK.lut[lane & 7]) : 0.0f;
     const float vlut = SV.scheme == KVQ_NUQ ? __half2float(SV.lut[lane & 7]) : 0.0f;
-    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(SK.codes) + sl * SK.code_slab_bytes;
-    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(SV.codes) + sl * SV.code_slab_bytes;
     const int hi = L.mixed_hi, mid = L.mixed_mid, lo = L.mixed_lo;
+    const int krow = SK.code_row_bytes, vrow = SV.code_row_bytes;
+    const int nmeta = mixed ? D - hi : D;
     float cst[4], snt[4];
     if (L.rope) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        double sn2, cs2;
-        sincos((double)kW * theta[j], &sn2, &cs2);
-        cst[j] = (float)cs2;
-        snt[j] = (float)sn2;
+        angle_sincos(1.0, theta[j], &snt[j], &cst[j]);   // one position
       }
     }
-    for (int64_t gi = g0; gi < g1; ++gi) {
-      const int64_t tb = gi * L.g, te = min(a.t_quant, tb + L.g);
-      // group metadata of the lane's channels (slots for MIXED) and, for MIXED, the
-      // query in slot order
+    // the warp's chunks: k = warp, warp + kW, ...; a chunk past t_quant is skipped
+    auto chunk_t0 = [&](int64_t k) { return (g0 + k / cpg) * L.g + 32 * (k % cpg); };
+    int64_t lk = warp;   // load cursor
+    int issued = 0;
+    auto issue_next = [&]() {
+      while (lk < nchunk && chunk_t0(lk) >= a.t_quant) lk += kW;
+      if (lk < nchunk) {
+        uint8_t* st = ring + (issued & 1) * SG.bytes;
+        const int64_t gi = g0 + lk / cpg, sub = lk % cpg, t0 = chunk_t0(lk);
+        const int64_t grp = sl * L.ng + gi;
+        if (mixed) {
+          const uint8_t* gb = reinterpret_cast<const uint8_t*>(SK.codes) + grp * (int64_t)L.mixed_group_bytes;
+          cp_range(st + SG.k, gb + sub * 32 * hi * 2, 32 * hi * 2, lane);
+          cp_range(st + SG.k_mid, gb + (int64_t)L.g * hi * 2 + sub * 32 * mid / 2, 32 * mid / 2, lane);
+          cp_range(st + SG.k_lo, gb + (int64_t)L.g * hi * 2 + (int64_t)L.g * mid / 2 + sub * 32 * lo / 4, 32 * lo / 4, lane);
+          cp_range(st + SG.ord, L.k_order + grp * D, D, lane);
+        } else {
+          cp_range(st + SG.k, reinterpret_cast<const uint8_t*>(SK.codes) + sl * SK.code_slab_bytes + t0 * krow,
+                   32 * krow, lane);
+        }
+        cp_range(st + SG.ks, reinterpret_cast<const __half*>(SK.scale) + grp * nmeta, nmeta * 2, lane);
+        cp_range(st + SG.kz, reinterpret_cast<const __half*>(SK.zero) + grp * nmeta, nmeta * 2, lane);
+        cp_range(st + SG.v, reinterpret_cast<const uint8_t*>(SV.codes) + sl * SV.code_slab_bytes + t0 * vrow,
+                 32 * vrow, lane);
+        cp_range(st + SG.vs, reinterpret_cast<const __half*>(SV.scale) + sl * L.C + t0, 64, lane);
+        cp_range(st + SG.vz, reinterpret_cast<const __half*>(SV.zero) + sl * L.C + t0, 64, lane);
+        if (SV.nout > 0) {
+          cp_range(st + SG.voc, L.v_out_col + (sl * L.C + t0) * SV.nout, 32 * SV.nout, lane);
+          cp_range(st + SG.vov, L.v_out_val + (sl * L.C + t0) * SV.nout, 64 * SV.nout, lane);
+        }
+        if (SK.nout > 0) {
+          const int32_t* rp = L.k_out_rowptr + grp * (L.g + 1) + 32 * sub;
+          cp4(st + SG.rp + 4 * lane, rp + lane);
+          if (lane == 0) cp4(st + SG.rp + 128, rp + 32);
+          cp_range(st + SG.kc, L.k_out_col + grp * D * SK.nout, D * SK.nout, lane);
+          cp_range(st + SG.kv, L.k_out_val + grp * D * SK.nout, D * SK.nout * 2, lane);
+        }
+        lk += kW;
+      }
+      cp_commit();
+      ++issued;
+    };
+    issue_next();
+    int consumed = 0;
+    for (int64_t k = warp; k < nchunk; k += kW) {
+      const int64_t t0 = chunk_t0(k);
+      if (t0 >= a.t_quant) continue;
+      issue_next();
+      cp_wait<1>();
+      __syncwarp();
+      const uint8_t* st = ring + (consumed & 1) * SG.bytes;
+      const int nt = (int)min((int64_t)32, a.t_quant - t0);
+      // group metadata of the lane's channels (slots for MIXED); MIXED: query in slot order
       float ks[4] = {0.f, 0.f, 0.f, 0.f}, kz[4] = {0.f, 0.f, 0.f, 0.f};
       float qk[GM][4];
 #pragma unroll
       for (int hh = 0; hh < GM; ++hh)
 #pragma unroll
         for (int j = 0; j < 4; ++j) qk[hh][j] = q[hh][j];
+      const __half* kss = reinterpret_cast<const __half*>(st + SG.ks);
+      const __half* kzs = reinterpret_cast<const __half*>(st + SG.kz);
       if (mixed) {
-        __syncthreads();
-        if (threadIdx.x < D) order[threadIdx.x] = L.k_order[(sl * L.ng + gi) * D + threadIdx.x];
-        __syncthreads();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int slot = 4 * lane + j;
-          const int ch = order[slot];
+          const int ch = st[SG.ord + slot];
 #pragma unroll
           for (int hh = 0; hh < GM; ++hh) qk[hh][j] = qsm[hh * D + ch];
           if (slot >= hi) {
-            const int64_t mi = (sl * L.ng + gi) * (D - hi) + (slot - hi);
-            ks[j] = meta_f16(SK.scale, mi);
-            kz[j] = meta_f16(SK.zero, mi);
+            ks[j] = __half2float(kss[slot - hi]);
+            kz[j] = __half2float(kzs[slot - hi]);
           }
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int64_t mi = (sl * L.ng + gi) * D + 4 * lane + j;
-          ks[j] = meta_f16(SK.scale, mi);
-          kz[j] = meta_f16(SK.zero, mi);
+          ks[j] = __half2float(kss[4 * lane + j]);
+          kz[j] = __half2float(kzs[4 * lane + j]);
         }
       }
       float cs[4], sn[4];
       if (L.rope) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          double s2, c2;
-          sincos((double)(L.n_sink + tb + warp) * theta[j], &s2, &c2);
-          cs[j] = (float)c2;
-          sn[j] = (float)s2;
+          angle_sincos((double)(L.n_sink + t0), theta[j], &sn[j], &cs[j]);
         }
       }
-      const uint8_t* gbase = mixed ? reinterpret_cast<const uint8_t*>(SK.codes) +
-                                         (sl * L.ng + gi) * (int64_t)L.mixed_group_bytes
-                                   : nullptr;
-      for (int64_t t0 = tb + warp; t0 < te; t0 += kW * kB) {
+      for (int r0 = 0; r0 < nt; r0 += kB) {
         float kb[kB][4], vb[kB][4];
         bool ok[kB];
 #pragma unroll
         for (int e = 0; e < kB; ++e) {
-          const int64_t t = t0 + (int64_t)e * kW;
-          ok[e] = t < te;
-          const int64_t tt = ok[e] ? t : tb;
+          const int r = r0 + e;
+          ok[e] = r < nt;
+          const int rr = ok[e] ? r : 0;
           // keys
           if (mixed) {
-            const int r = (int)(tt - tb);
             const int s0 = 4 * lane;
             if (s0 < hi) {
-              // raw 16-bit slots (MIXED sources are fp16 or bf16)
-              const float4 f = ld4(gbase, (int64_t)r * hi + s0, L.src_dtype);
+              const float4 f = ld4(st + SG.k, rr * hi + s0, L.src_dtype);
               kb[e][0] = f.x; kb[e][1] = f.y; kb[e][2] = f.z; kb[e][3] = f.w;
             } else if (s0 < hi + mid) {
               const int e0 = s0 - hi;
-              const uint32_t w = reinterpret_cast<const uint32_t*>(gbase + (int64_t)L.g * hi * 2)[r * (mid / 8) + e0 / 8] >>
-                                 (4 * (e0 % 8));
+              const uint32_t w = reinterpret_cast<const uint32_t*>(st + SG.k_mid)[rr * (mid / 8) + e0 / 8] >> (4 * (e0 % 8));
 #pragma unroll
               for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (4 * j)) & 15u), ks[j], kz[j]);
             } else {
               const int e0 = s0 - hi - mid;
-              const uint32_t w =
-                  reinterpret_cast<const uint32_t*>(gbase + (int64_t)L.g * hi * 2 + (int64_t)L.g * mid / 2)[r * (lo / 16) + e0 / 16] >>
-                  (2 * (e0 % 16));
+              const uint32_t w = reinterpret_cast<const uint32_t*>(st + SG.k_lo)[rr * (lo / 16) + e0 / 16] >> (2 * (e0 % 16));
 #pragma unroll
               for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (2 * j)) & 3u), ks[j], kz[j]);
             }
           } else if (SK.scheme == KVQ_NUQ) {
             uint32_t code[4];
-            nuq_codes(reinterpret_cast<const uint32_t*>(kbase) + tt * 12, lane, code);
+            nuq_codes(reinterpret_cast<const uint32_t*>(st + SG.k + rr * krow), lane, code);
 #pragma unroll
             for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn(__shfl_sync(0xffffffffu, klut, (int)code[j]), ks[j], kz[j]);
           } else {   // ASYM 2 / 4 bits, row layout
             const int bb = SK.bits;
             const int bitoff = 4 * lane * bb;
-            const uint32_t w = reinterpret_cast<const uint32_t*>(kbase)[tt * (D * bb / 32) + bitoff / 32] >> (bitoff % 32);
+            const uint32_t w = reinterpret_cast<const uint32_t*>(st + SG.k + rr * krow)[bitoff / 32] >> (bitoff % 32);
 #pragma unroll
             for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (bb * j)) & ((1u << bb) - 1)), ks[j], kz[j]);
           }
-          // values (per token)
-          const float vs = meta_f16(SV.scale, sl * L.C + tt), vz = meta_f16(SV.zero, sl * L.C + tt);
+          // values
+          const float vs = __half2float(reinterpret_cast<const __half*>(st + SG.vs)[rr]);
+          const float vz = __half2float(reinterpret_cast<const __half*>(st + SG.vz)[rr]);
           if (SV.scheme == KVQ_NUQ) {
             uint32_t code[4];
-            nuq_codes(reinterpret_cast<const uint32_t*>(vbase) + tt * 12, lane, code);
+            nuq_codes(reinterpret_cast<const uint32_t*>(st + SG.v + rr * vrow), lane, code);
 #pragma unroll
             for (int j = 0; j < 4; ++j) vb[e][j] = __fmaf_rn(__shfl_sync(0xffffffffu, vlut, (int)code[j]), vs, vz);
-          } else {   // ASYM 2 / 4 bits, pair layout
+          } else {   // ASYM 2 / 4 bits, pair layout (t0 even)
             const int bb = SV.bits, per = 16 / bb;
             const int c0 = 4 * lane;
-            const uint32_t w = reinterpret_cast<const uint32_t*>(vbase)[(tt >> 1) * (D / per) + c0 / per] >>
-                               (16 * (int)(tt & 1) + bb * (c0 % per));
+            const uint32_t w = reinterpret_cast<const uint32_t*>(st + SG.v)[(rr >> 1) * (D / per) + c0 / per] >>
+                               (16 * (rr & 1) + bb * (c0 % per));
 #pragma unroll
             for (int j = 0; j < 4; ++j) vb[e][j] = __fmaf_rn((float)((w >> (bb * j)) & ((1u << bb) - 1)), vs, vz);
           }
           // sparse outliers overwrite (before RoPE)
           if (SK.nout > 0 && ok[e]) {
-            const int rr = (int)(t - tb);
-            const int32_t* rp = L.k_out_rowptr + (sl * L.ng + gi) * (L.g + 1);
-            const int64_t e0 = (sl * L.ng + gi) * (int64_t)D * SK.nout;
+            const int32_t* rp = reinterpret_cast<const int32_t*>(st + SG.rp);
             const int x0 = rp[rr], x1 = rp[rr + 1];
             for (int x = x0; x < x1; ++x) {
-              const int c = L.k_out_col[e0 + x];
-              const float v = __half2float(L.k_out_val[e0 + x]);
+              const int c = st[SG.kc + x];
+              const float v = __half2float(reinterpret_cast<const __half*>(st + SG.kv)[x]);
 #pragma unroll
               for (int j = 0; j < 4; ++j)
                 if (c == 4 * lane + j) kb[e][j] = v;
@@ -297,9 +387,8 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
           }
           if (SV.nout > 0 && ok[e]) {
             for (int x = 0; x < SV.nout; ++x) {
-              const int64_t idx = (sl * L.C + t) * SV.nout + x;
-              const int c = L.v_out_col[idx];
-              const float v = __half2float(L.v_out_val[idx]);
+              const int c = st[SG.voc + rr * SV.nout + x];
+              const float v = __half2float(reinterpret_cast<const __half*>(st + SG.vov)[rr * SV.nout + x]);
 #pragma unroll
               for (int j = 0; j < 4; ++j)
                 if (c == 4 * lane + j) vb[e][j] = v;
@@ -317,7 +406,11 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
         }
         consume(kb, vb, qk, ok);
       }
+      __syncwarp();
+      ++consumed;
     }
+    cp_wait<0>();
+    __syncwarp();
   } else if (split == a.raw_slot) {
     const int nraw = L.n_sink + a.t_res;
     for (int r0 = warp; r0 < nraw; r0 += kW * kB) {
@@ -341,10 +434,7 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
           float cs[4], sn[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            double s2, c2;
-            sincos((double)pos * theta[j], &s2, &c2);
-            cs[j] = (float)c2;
-            sn[j] = (float)s2;
+            angle_sincos((double)pos, theta[j], &sn[j], &cs[j]);
           }
           rope4(kb[e], cs, sn, lane);
         }
@@ -390,8 +480,8 @@ __global__ void __launch_bounds__(kW * 32) decode_cc_kernel(CcArgs a) {
 template <int GM>
 cudaError_t launch_cc_g(const CcArgs& a, int grid_x, cudaStream_t s) {
   const int G = a.Hq / a.L.Hkv;
-  // queries (GM x 128), slot order (128 B), merge records; the records are 16-byte aligned
-  const size_t smem = ((size_t)GM * 128 + 32 + (size_t)kW * G * kRS) * sizeof(float);
+  // stage rings, queries (GM x 128), merge records; every part 16-byte aligned
+  const size_t smem = (size_t)kW * 2 * a.st.bytes + ((size_t)GM * 128 + (size_t)kW * G * kRS) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(decode_cc_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -402,11 +492,48 @@ cudaError_t launch_cc_g(const CcArgs& a, int grid_x, cudaStream_t s) {
 
 }  // namespace
 
+constexpr int kStageMax = 8192;
+
+int up16(int x) { return (x + 15) & ~15; }
+
+CcStage stage_layout(const Layout& L) {
+  const Side& K = L.side[0];
+  const Side& V = L.side[1];
+  const bool mixed = K.scheme == KVQ_MIXED;
+  CcStage g;
+  int o = 0;
+  g.k = o;
+  if (mixed) {
+    g.k_mid = g.k + 32 * L.mixed_hi * 2;
+    g.k_lo = g.k_mid + 32 * L.mixed_mid / 2;
+    o = g.k_lo + 32 * L.mixed_lo / 4;
+  } else {
+    g.k_mid = g.k_lo = 0;
+    o += 32 * K.code_row_bytes;
+  }
+  o = up16(o);
+  g.v = o;  o = up16(o + 32 * V.code_row_bytes);
+  g.vs = o; o += 64;
+  g.vz = o; o += 64;
+  g.voc = o; o = up16(o + 32 * V.nout);
+  g.vov = o; o = up16(o + 64 * V.nout);
+  const int nmeta = mixed ? L.D - L.mixed_hi : L.D;
+  g.ks = o; o = up16(o + nmeta * 2);
+  g.kz = o; o = up16(o + nmeta * 2);
+  g.ord = o; o += mixed ? L.D : 0;
+  g.rp = o; o += K.nout > 0 ? 144 : 0;
+  g.kc = o; o = up16(o + L.D * K.nout);
+  g.kv = o; o = up16(o + L.D * K.nout * 2);
+  g.bytes = o;
+  return g;
+}
+
 bool cc_path_ok(const Layout& L, int Hq) {
   const Side& K = L.side[0];
   const Side& V = L.side[1];
   const int G = Hq / L.Hkv;
-  if (L.D != 128 || G < 1 || G > 8) return false;
+  if (L.D != 128 || G < 1 || G > 8 || L.g % 32) return false;
+  if (stage_layout(L).bytes > kStageMax) return false;
   const bool k_ok = (K.scheme == KVQ_NUQ && K.axis == KVQ_AXIS_CHANNEL) ||
                     (K.scheme == KVQ_ASYM && K.axis == KVQ_AXIS_CHANNEL && (K.bits == 2 || K.bits == 4)) ||
                     (K.scheme == KVQ_MIXED && !L.rope);
@@ -419,6 +546,7 @@ cudaError_t launch_decode_cc(const Layout& L, const DecodePlan& p, const void* q
                              int64_t t_quant, int t_res, float scale, float* ws_m, float* ws_l,
                              float* ws_o, int32_t* d_status, cudaStream_t s) {
   CcArgs a;
+  a.st = stage_layout(L);
   a.L = L;
   a.q = q;
   a.q_dtype = q_dtype;

@@ -10,6 +10,20 @@
 
 namespace kvq {
 
+// sin and cos of the RoPE angle pos * theta (radians, up to ~1e5 at long context): the
+// angle is first reduced modulo 2 pi in double (one fused multiply-add with the double
+// nearest to 2 pi; error ~1e-11 rad at 131k tokens), so that the library sincos works on
+// |r| <= pi.
+__device__ __forceinline__ void angle_sincos(double pos, double theta, float* s, float* c) {
+  const double two_pi = 6.283185307179586;
+  const double x = pos * theta;
+  const double r = fma(-rint(x * (1.0 / two_pi)), two_pi, x);
+  double sd, cd;
+  sincos(r, &sd, &cd);
+  *s = (float)sd;
+  *c = (float)cd;
+}
+
 __device__ __forceinline__ float meta_f16(const void* p, int64_t i) {
   return __half2float(reinterpret_cast<const __half*>(p)[i]);
 }
