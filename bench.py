@@ -35,7 +35,26 @@ import synth  # noqa: E402
 
 METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize GB/s"
 L2_FLUSH_BYTES = 512 << 20
-LAUNCHES_PER_STEP = 4   # asym_keys_kernel, asym_values_kernel, decode_mma_kernel, combine_mma_kernel
+LAUNCHES_PER_STEP = 4   # quantize keys, quantize values, split kernel, combine (+ salience for MIXED)
+PATH_DTYPE = {
+    "decode_mma_kernel": "f16 tensor-core products with f32 accumulation (u4/u2 codes)",
+    "decode_cc_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
+    "decode_generic_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
+}
+
+
+def decode_path(cfg):
+    """The split kernel the library plans for this workload (same rules as its planner)."""
+    f = cfg["fmt"]
+    G = cfg["Hq"] // cfg["Hkv"]
+    if is_k4v2(cfg) and f["head_dim"] == 128 and f["group_tokens"] == 128 and 1 <= G <= 8:
+        return "decode_mma_kernel"
+    k_ok = (f["k_scheme"] == synth.NUQ) or (f["k_scheme"] == synth.ASYM and f["k_bits"] in (2, 4)) or \
+        (f["k_scheme"] == synth.MIXED and not f["rope"])
+    v_ok = (f["v_scheme"] == synth.NUQ) or (f["v_scheme"] == synth.ASYM and f["v_bits"] in (2, 4))
+    if f["head_dim"] == 128 and G <= 8 and f["group_tokens"] % 32 == 0 and k_ok and v_ok:
+        return "decode_cc_kernel"
+    return "decode_generic_kernel"
 
 
 def parse():
@@ -44,7 +63,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="llama3_8b", choices=["llama3_8b", "llama2_7b"])
+    ap.add_argument("--config", default="llama3_8b",
+                    choices=["llama3_8b", "llama2_7b", "kvquant_nuq3", "mixkvq_14b"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -74,6 +94,25 @@ def decode_kernel_bytes(cfg, tq, tr):
 
 def decode_call_bytes(cfg, tq, tr):
     return decode_kernel_bytes(cfg, tq, tr) + cfg["B"] * cfg["Hq"] * cfg["D"] * 4   # fp32 out
+
+
+K4V2 = dict(k_scheme=synth.ASYM, k_bits=4, k_axis=synth.CHANNEL, v_scheme=synth.ASYM, v_bits=2,
+            v_axis=synth.TOKEN, k_outliers=0, v_outliers=0, rope=0)
+
+
+def is_k4v2(cfg):
+    return all(cfg["fmt"][k] == v for k, v in K4V2.items())
+
+
+def cache_read_bytes(cache, cfg, tq, tr):
+    """Algorithmic decode bytes of any format: every cache array the decode reads (codes,
+    metadata, slot order, outliers: sized for the packed capacity, i.e. t_quant rounded up
+    to whole groups; raw sink / residual tokens: the ones in use), plus q and the fp32 out."""
+    raw = {"sink_k", "sink_v", "res_k", "res_v"}
+    n = sum(t.numel() for name, t in cache.tensors.items() if name not in raw | {"k_lut", "v_lut"})
+    esz = 4 if cfg["fmt"]["src_dtype"] == synth.F32 else 2
+    n += cfg["B"] * cfg["Hkv"] * (cfg["fmt"]["n_sink"] + tr) * 2 * cfg["D"] * esz
+    return n + cfg["B"] * cfg["Hq"] * cfg["D"] * (2 + 4)
 
 
 def quant_bytes(cfg, n):
@@ -154,7 +193,13 @@ class OracleSample:
         T = ns + tq + tr
         K = synth.kv_slab(cfg, 0, 0, T, "k")[None, None].astype(np.float64)
         V = synth.kv_slab(cfg, 0, 0, T, "v")[None, None].astype(np.float64)
-        c = ocache.Cache(of, 1, 1, -(-tq // g) * g)
+        luts = (None, None)
+        if of.k_scheme == synth.NUQ:
+            cb = json.load(open(os.path.join(ROOT, "tests", "golden", "nuq3_codebook.json")))
+            luts = (cb["k"], cb["v"])
+        c = ocache.Cache(of, 1, 1, -(-tq // g) * g, k_lut=luts[0], v_lut=luts[1])
+        if of.k_scheme == synth.MIXED:   # a valid slot order (salience is not timed here)
+            c["k_order"][...] = np.arange(of.head_dim, dtype=np.uint8)
         ocache.quantize(of, c, KEYS, K[:, :, ns:ns + tq], 0, tq)
         ocache.quantize(of, c, VALUES, V[:, :, ns:ns + tq], 0, tq)
         enc = fp.bf16_bits if of.src_dtype == synth.BF16 else fp.f16_bits
@@ -168,7 +213,14 @@ class OracleSample:
         self.newk, self.newv = K[:, :, ns:ns + g], V[:, :, ns:ns + g]
         self.of, self.c, self.tq, self.tr, self.g, self.ns = of, c, tq, tr, g, ns
         one_head = dict(cfg, B=1, Hkv=1, Hq=self.G)
-        self.nbytes = decode_call_bytes(one_head, tq, tr) + quant_bytes(one_head, g)
+        if is_k4v2(cfg):
+            self.nbytes = decode_call_bytes(one_head, tq, tr) + quant_bytes(one_head, g)
+        else:   # the packed arrays it reads, its raw tokens, q and out, one group's input
+            packed = sum(a.nbytes for n, a in c.arrays.items()
+                         if n not in ("sink_k", "sink_v", "res_k", "res_v", "k_lut", "v_lut"))
+            esz = 4 if of.src_dtype == synth.F32 else 2
+            self.nbytes = packed + (ns + tr) * 2 * of.head_dim * esz + self.G * of.head_dim * 6 + \
+                2 * g * of.head_dim * esz
 
     def run(self):
         from oracle import cache as ocache
@@ -257,11 +309,22 @@ def run_reference(args, world, rank):
 def workload_config(cfg):
     ns, tq, tr = synth.split_tokens(cfg)
     f = cfg["fmt"]
+    names = {synth.NONE: "raw", synth.SYM8: "INT8 sym", synth.ASYM: "asym", synth.NUQ: "nuq", synth.MIXED: "mixed"}
+    kdesc = (f"mixed {f['mixed_hi']} raw / {f['mixed_mid']} 4-bit / rest 2-bit by salience"
+             if f["k_scheme"] == synth.MIXED else f"{names[f['k_scheme']]}{f['k_bits']} per-channel")
+    extra = []
+    if f["k_outliers"] or f["v_outliers"]:
+        extra.append(f"top-{max(f['k_outliers'], f['v_outliers'])} fp16 outliers per vector")
+    if f["rope"]:
+        extra.append(f"RoPE base {f['rope_base']:g} on keys")
+    n_app = cfg.get("append", f["group_tokens"])
     return {"workload": f"{cfg['name']}: B={cfg['B']} Hq={cfg['Hq']} Hkv={cfg['Hkv']} D={cfg['D']} "
-                        f"T={cfg['T']} (sink {ns}, packed {tq}, residual {tr}); K{f['k_bits']} per-channel "
-                        f"g{f['group_tokens']} + V{f['v_bits']} per-token, fp16 scale/zero",
+                        f"T={cfg['T']} (sink {ns}, packed {tq}, residual {tr}); K {kdesc} "
+                        f"g{f['group_tokens']} + V {names[f['v_scheme']]}{f['v_bits']} per-token"
+                        + ("; " + ", ".join(extra) if extra else ""),
             "B": cfg["B"], "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "D": cfg["D"], "T": cfg["T"],
-            "step": "quantize one 128-token group (K, V) + decode attention over T",
+            "step": f"append of {n_app} tokens (quantize K, V" +
+                    (", salience" if f["k_scheme"] == synth.MIXED else "") + ") + decode attention over T",
             "l2": "flushed between steps outside the timed events (512 MiB write, then 512 MiB read)",
             "parallelism": "replicas (one independent cache per GPU)"}
 
@@ -290,7 +353,23 @@ def main():
     # ---- build the cache on the device (data drawn on the device, same recipe)
     K = synth.device_kv(cfg, "k", device=dev, seed_offset=rank)
     V = synth.device_kv(cfg, "v", device=dev, seed_offset=rank)
-    cache = kvq.Cache(fmt, B, Hkv, C, device=dev)
+    luts = (None, None)
+    if fd["k_scheme"] == synth.NUQ:
+        cb = json.load(open(os.path.join(ROOT, "tests", "golden", "nuq3_codebook.json")))
+        luts = (cb["k"], cb["v"])
+    cache = kvq.Cache(fmt, B, Hkv, C, device=dev, k_lut=luts[0], v_lut=luts[1])
+    mixed = fd["k_scheme"] == synth.MIXED
+    qwin = None
+    if mixed:   # salience windows: query rows at every packed position (device-drawn)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(cfg["seed"] * 1000 + 44 + rank)
+        mu = torch.exp(torch.empty((1, Hq, 1, D), device=dev).uniform_(np.log(0.1), np.log(5.0), generator=gen))
+        qwin = (torch.randn((B, Hq, tq, D), device=dev, generator=gen) * mu).to(K.dtype)
+        order = cache.array("k_order")
+        for gi in range(-(-tq // g)):
+            t0, ln = gi * g, min(g, tq - gi * g)
+            kvq.key_salience(fmt, qwin[:, :, t0:t0 + ln], K[:, :, ns + t0:ns + t0 + ln], order[gi * D:],
+                             Hkv * (C // g) * D, (C // g) * D)
     kvq.quantize_keys(fmt, cache, K[:, :, ns:ns + tq], 0, tq)
     kvq.quantize_values(fmt, cache, V[:, :, ns:ns + tq], 0, tq)
     if ns:
@@ -299,11 +378,15 @@ def main():
     if tr:
         cache.array("res_k").copy_(K[:, :, ns + tq:].contiguous().view(-1).view(torch.uint8))
         cache.array("res_v").copy_(V[:, :, ns + tq:].contiguous().view(-1).view(torch.uint8))
-    # the flushed group: rewrite packed group gi_f (a full group) from its own tokens
-    gi_f = tq // g - 1
-    newk = K[:, :, ns + gi_f * g: ns + (gi_f + 1) * g].contiguous()
-    newv = V[:, :, ns + gi_f * g: ns + (gi_f + 1) * g].contiguous()
-    del K, V
+    # the append: rewrite the last n_app packed tokens (whole groups) from their own
+    # values -- one group (the flush of the residual window), or the workload's append
+    n_app = cfg.get("append", g)
+    a0 = (tq // g) * g - n_app
+    gi_f = a0 // g
+    newk = K[:, :, ns + a0: ns + a0 + n_app].contiguous()
+    newv = V[:, :, ns + a0: ns + a0 + n_app].contiguous()
+    neww = qwin[:, :, a0:a0 + n_app].contiguous() if mixed else None
+    del K, V, qwin
     q = synth.device_queries(cfg, device=dev)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
     ws = torch.empty(kvq.decode_workspace_bytes(fmt, B, Hq, Hkv, tq, tr), dtype=torch.uint8, device=dev)
@@ -317,11 +400,21 @@ def main():
         flush.fill_(i & 0xFF)
         flush_r.sum()
 
+    order = cache.array("k_order") if mixed else None
+
+    def append(k_src, v_src, w_src):
+        if mixed:
+            for j in range(n_app // g):
+                kvq.key_salience(fmt, w_src[:, :, j * g:(j + 1) * g], k_src[:, :, j * g:(j + 1) * g],
+                                 order[(gi_f + j) * D:], Hkv * (C // g) * D, (C // g) * D,
+                                 status=status, stream=stream)
+        kvq.quantize_keys(fmt, cache, k_src, a0, n_app, status=status, stream=stream)
+        kvq.quantize_values(fmt, cache, v_src, a0, n_app, status=status, stream=stream)
+
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        kvq.quantize_keys(fmt, cache, newk, gi_f * g, g, status=status, stream=stream)
-        kvq.quantize_values(fmt, cache, newv, gi_f * g, g, status=status, stream=stream)
+        append(newk, newv, neww)
         if evs:
             evs[1].record(stream)
         kvq.decode_partial(fmt, cache, q, tq, tr, scale, ws, status=status, stream=stream)
@@ -374,6 +467,11 @@ def main():
     hq.copy_(q)
     hout = torch.empty_like(out, device="cpu").pin_memory()
     dk, dv, dq = torch.empty_like(newk), torch.empty_like(newv), torch.empty_like(q)
+    hw = dw = None
+    if mixed:
+        hw = torch.empty_like(neww, device="cpu").pin_memory()
+        hw.copy_(neww)
+        dw = torch.empty_like(neww)
     e2e_t = []
     for i in range(e2e_steps + 3):
         flush_l2(i)
@@ -383,8 +481,9 @@ def main():
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         dq.copy_(hq, non_blocking=True)
-        kvq.quantize_keys(fmt, cache, dk, gi_f * g, g, status=status, stream=stream)
-        kvq.quantize_values(fmt, cache, dv, gi_f * g, g, status=status, stream=stream)
+        if mixed:
+            dw.copy_(hw, non_blocking=True)
+        append(dk, dv, dw)
         kvq.decode_attention(fmt, cache, dq, tq, tr, scale, kvq.F32, out=out, workspace=ws,
                              status=status, stream=stream)
         hout.copy_(out, non_blocking=True)
@@ -396,11 +495,24 @@ def main():
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     assert torch.isfinite(out).all()
 
-    step_bytes = decode_call_bytes(cfg, tq, tr) + quant_bytes(cfg, g)
-    kern_bytes = decode_kernel_bytes(cfg, tq, tr)
+    path = decode_path(cfg)
+    if is_k4v2(cfg):
+        call_bytes = decode_call_bytes(cfg, tq, tr)
+        kern_bytes = decode_kernel_bytes(cfg, tq, tr)
+        q_bytes = quant_bytes(cfg, n_app)
+    else:
+        call_bytes = cache_read_bytes(cache, cfg, tq, tr)
+        kern_bytes = call_bytes - B * Hq * D * 4
+        esz = 4 if fd["src_dtype"] == synth.F32 else 2
+        packed = sum(t.numel() for name, t in cache.tensors.items()
+                     if name not in ("sink_k", "sink_v", "res_k", "res_v", "k_lut", "v_lut"))
+        q_bytes = B * Hkv * n_app * D * esz * 2 + packed * n_app // C
+        if mixed:
+            q_bytes += B * Hq * n_app * D * esz
+    step_bytes = call_bytes + q_bytes
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
-    decode_gbs = decode_call_bytes(cfg, tq, tr) / ((ms_part + ms_comb) * 1e-3) / 1e9
-    quant_gbs = quant_bytes(cfg, g) / (ms_quant * 1e-3) / 1e9
+    decode_gbs = call_bytes / ((ms_part + ms_comb) * 1e-3) / 1e9
+    quant_gbs = q_bytes / (ms_quant * 1e-3) / 1e9
     achieved = kern_bytes / (ms_part * 1e-3) / 1e9
     peaks = {}
     try:
@@ -418,26 +530,30 @@ def main():
         except (OSError, ValueError):
             pass
     h2d = newk.numel() * newk.element_size() * 2 + q.numel() * q.element_size()
+    if mixed:
+        h2d += neww.numel() * neww.element_size()
     d2h = out.numel() * out.element_size()
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16 tensor-core products with f32 accumulation (u4/u2 codes)",
+        "vs_baseline": None, "dtype": PATH_DTYPE[path],
         "data": "synthetic (device-drawn, recipe of synth/)",
         "config": workload_config(cfg),
         "pct_of_8tbs": 100.0 * value / world / 8000.0,
         "decode_gbs": decode_gbs, "quantize_gbs": quant_gbs,
         "tokens_heads_per_s": world * B * Hq * cfg["T"] / ((ms_part + ms_comb) * 1e-3),
         "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb},
-        "roofline": {"kernel": "decode_mma_kernel (kvq_decode_partial)", "bound": "hbm",
+        "roofline": {"kernel": f"{path} (kvq_decode_partial)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": kern_bytes,
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},
         "e2e": {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (n_app // g if mixed else 0)) * args.steps,
         "clocks": clocks,
     }
+    if path != "decode_mma_kernel":
+        line["roofline"]["traffic"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = oracle_sized(cfg, 5.0)
         times = [smp.run() for _ in range(3)]
