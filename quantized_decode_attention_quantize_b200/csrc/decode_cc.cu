@@ -100,7 +100,10 @@ __device__ __forceinline__ void cp_range(uint8_t* dst, const void* src, int byte
   for (int o = 16 * lane; o < bytes; o += 512) cp16(dst + o, reinterpret_cast<const uint8_t*>(src) + o);
 }
 
-template <int GM>
+// KF: key format (kNuq, kAsym, kMixed); VF: value format (kNuq, kAsym); ROPE on keys.
+constexpr int kNuq = 0, kAsym = 1, kMixed = 2;
+
+template <int GM, int KF, int VF, bool ROPE>
 __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcArgs a) {
   extern __shared__ __align__(16) float smem[];
   const Layout& L = a.L;
@@ -111,7 +114,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
   const int64_t sl = (int64_t)b * L.Hkv + h;
   const Side& SK = L.side[0];
   const Side& SV = L.side[1];
-  const bool mixed = SK.scheme == KVQ_MIXED;
+  constexpr bool mixed = KF == kMixed;
   const CcStage& SG = a.st;
   uint8_t* ring = reinterpret_cast<uint8_t*>(smem) + (size_t)warp * 2 * SG.bytes;   // [kW][2] stages
   float* qsm = smem + (size_t)kW * 2 * SG.bytes / 4;  // [GM][128] pre-scaled queries (MIXED)
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
   }
   // RoPE frequencies of this lane's pairs i = 4 (l & 15) + j
   double theta[4];
-  if (L.rope) {
+  if (ROPE) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) theta[j] = pow((double)L.rope_base, -2.0 * (double)(4 * (lane & 15) + j) / (double)D);
   }
@@ -221,13 +224,13 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
     const int64_t g1 = min(ngv, g0 + a.split_groups);
     const int cpg = L.g / 32;                         // chunks per group
     const int64_t nchunk = (g1 - g0) * cpg;
-    const float klut = SK.scheme == KVQ_NUQ ? __half2float(SK.lut[lane & 7]) : 0.0f;
-    const float vlut = SV.scheme == KVQ_NUQ ? __half2float(SV.lut[lane & 7]) : 0.0f;
+    const float klut = KF == kNuq ? __half2float(SK.lut[lane & 7]) : 0.0f;
+    const float vlut = VF == kNuq ? __half2float(SV.lut[lane & 7]) : 0.0f;
     const int hi = L.mixed_hi, mid = L.mixed_mid, lo = L.mixed_lo;
     const int krow = SK.code_row_bytes, vrow = SV.code_row_bytes;
     const int nmeta = mixed ? D - hi : D;
     float cst[4], snt[4];
-    if (L.rope) {
+    if (ROPE) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         angle_sincos(1.0, theta[j], &snt[j], &cst[j]);   // one position
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
         uint8_t* st = ring + (issued & 1) * SG.bytes;
         const int64_t gi = g0 + lk / cpg, sub = lk % cpg, t0 = chunk_t0(lk);
         const int64_t grp = sl * L.ng + gi;
-        if (mixed) {
+        if constexpr (mixed) {
           const uint8_t* gb = reinterpret_cast<const uint8_t*>(SK.codes) + grp * (int64_t)L.mixed_group_bytes;
           cp_range(st + SG.k, gb + sub * 32 * hi * 2, 32 * hi * 2, lane);
           cp_range(st + SG.k_mid, gb + (int64_t)L.g * hi * 2 + sub * 32 * mid / 2, 32 * mid / 2, lane);
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
         for (int j = 0; j < 4; ++j) qk[hh][j] = q[hh][j];
       const __half* kss = reinterpret_cast<const __half*>(st + SG.ks);
       const __half* kzs = reinterpret_cast<const __half*>(st + SG.kz);
-      if (mixed) {
+      if constexpr (mixed) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int slot = 4 * lane + j;
@@ -314,7 +317,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
         }
       }
       float cs[4], sn[4];
-      if (L.rope) {
+      if (ROPE) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           angle_sincos((double)(L.n_sink + t0), theta[j], &sn[j], &cs[j]);
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
           ok[e] = r < nt;
           const int rr = ok[e] ? r : 0;
           // keys
-          if (mixed) {
+          if constexpr (mixed) {
             const int s0 = 4 * lane;
             if (s0 < hi) {
               const float4 f = ld4(st + SG.k, rr * hi + s0, L.src_dtype);
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
 #pragma unroll
               for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (2 * j)) & 3u), ks[j], kz[j]);
             }
-          } else if (SK.scheme == KVQ_NUQ) {
+          } else if constexpr (KF == kNuq) {
             uint32_t code[4];
             nuq_codes(reinterpret_cast<const uint32_t*>(st + SG.k + rr * krow), lane, code);
 #pragma unroll
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
           // values
           const float vs = __half2float(reinterpret_cast<const __half*>(st + SG.vs)[rr]);
           const float vz = __half2float(reinterpret_cast<const __half*>(st + SG.vz)[rr]);
-          if (SV.scheme == KVQ_NUQ) {
+          if constexpr (VF == kNuq) {
             uint32_t code[4];
             nuq_codes(reinterpret_cast<const uint32_t*>(st + SG.v + rr * vrow), lane, code);
 #pragma unroll
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
                 if (c == 4 * lane + j) vb[e][j] = v;
             }
           }
-          if (L.rope) {
+          if (ROPE) {
             rope4(kb[e], cs, sn, lane);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
         const float4 vf = ld4(sink ? L.sink[1] : L.res[1], i, L.src_dtype);
         kb[e][0] = kf.x; kb[e][1] = kf.y; kb[e][2] = kf.z; kb[e][3] = kf.w;
         vb[e][0] = vf.x; vb[e][1] = vf.y; vb[e][2] = vf.z; vb[e][3] = vf.w;
-        if (L.rope) {
+        if (ROPE) {
           const int64_t pos = sink ? rr : L.n_sink + a.t_quant + row;
           float cs[4], sn[4];
 #pragma unroll
@@ -477,17 +480,37 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
   }
 }
 
-template <int GM>
-cudaError_t launch_cc_g(const CcArgs& a, int grid_x, cudaStream_t s) {
+template <int GM, int KF, int VF, bool ROPE>
+cudaError_t launch_cc_k(const CcArgs& a, int grid_x, cudaStream_t s) {
   const int G = a.Hq / a.L.Hkv;
   // stage rings, queries (GM x 128), merge records; every part 16-byte aligned
   const size_t smem = (size_t)kW * 2 * a.st.bytes + ((size_t)GM * 128 + (size_t)kW * G * kRS) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(decode_cc_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  auto kern = decode_cc_kernel<GM, KF, VF, ROPE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(grid_x, a.L.Hkv, a.L.B);
-  decode_cc_kernel<GM><<<grid, kW * 32, smem, s>>>(a);
+  kern<<<grid, kW * 32, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+template <int GM, int KF>
+cudaError_t launch_cc_v(const CcArgs& a, int grid_x, cudaStream_t s) {
+  const bool vnuq = a.L.side[1].scheme == KVQ_NUQ;
+  if constexpr (KF == kMixed) {   // MIXED keys take no RoPE
+    return vnuq ? launch_cc_k<GM, KF, kNuq, false>(a, grid_x, s) : launch_cc_k<GM, KF, kAsym, false>(a, grid_x, s);
+  } else {
+    if (a.L.rope)
+      return vnuq ? launch_cc_k<GM, KF, kNuq, true>(a, grid_x, s) : launch_cc_k<GM, KF, kAsym, true>(a, grid_x, s);
+    return vnuq ? launch_cc_k<GM, KF, kNuq, false>(a, grid_x, s) : launch_cc_k<GM, KF, kAsym, false>(a, grid_x, s);
+  }
+}
+
+template <int GM>
+cudaError_t launch_cc_g(const CcArgs& a, int grid_x, cudaStream_t s) {
+  const int ks = a.L.side[0].scheme;
+  if (ks == KVQ_NUQ) return launch_cc_v<GM, kNuq>(a, grid_x, s);
+  if (ks == KVQ_MIXED) return launch_cc_v<GM, kMixed>(a, grid_x, s);
+  return launch_cc_v<GM, kAsym>(a, grid_x, s);
 }
 
 }  // namespace
