@@ -5,8 +5,8 @@ decode attention over the packed cache, on synthetic data shaped like the worklo
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config llama3_8b]
 
-One step = kvq_quantize_keys + kvq_quantize_values of one 128-token group (the
-flush of the raw window into the packed cache) + kvq_decode_partial (split kernel)
+One step = kvq_quantize_kv (keys and values) of one 128-token group (the flush of
+the raw window into the packed cache) + kvq_decode_partial (split kernel)
 + kvq_decode_combine over all T tokens.  Every step is timed with CUDA events on the
 launching stream; the L2 is flushed between steps, outside the events, by a 512 MiB write and
 then a 512 MiB read of another buffer (so that no dirty line of the flush is left
@@ -35,7 +35,7 @@ import synth  # noqa: E402
 
 METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize GB/s"
 L2_FLUSH_BYTES = 512 << 20
-LAUNCHES_PER_STEP = 4   # quantize keys, quantize values, split kernel, combine (+ salience for MIXED)
+LAUNCHES_PER_STEP = 3   # quantize K+V (one launch on the K4/V2 path), split kernel, combine
 PATH_DTYPE = {
     "decode_mma_kernel": "f16 tensor-core products with f32 accumulation (u4/u2 codes)",
     "decode_cc_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
@@ -408,8 +408,7 @@ def main():
                 kvq.key_salience(fmt, w_src[:, :, j * g:(j + 1) * g], k_src[:, :, j * g:(j + 1) * g],
                                  order[(gi_f + j) * D:], Hkv * (C // g) * D, (C // g) * D,
                                  status=status, stream=stream)
-        kvq.quantize_keys(fmt, cache, k_src, a0, n_app, status=status, stream=stream)
-        kvq.quantize_values(fmt, cache, v_src, a0, n_app, status=status, stream=stream)
+        kvq.quantize_kv(fmt, cache, k_src, v_src, a0, n_app, status=status, stream=stream)
 
     def step(evs=None):
         if evs:
@@ -549,7 +548,8 @@ def main():
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},
         "e2e": {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (LAUNCHES_PER_STEP + (n_app // g if mixed else 0)) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (0 if is_k4v2(cfg) else 1) + (n_app // g if mixed else 0))
+        * args.steps,
         "clocks": clocks,
     }
     if path != "decode_mma_kernel":

@@ -221,6 +221,16 @@ kvq_status kvq_quantize_values(const kvq_format* fmt, const kvq_cache* cache,
                                int64_t stride_t, int64_t t0, int64_t n,
                                int32_t* d_status, void* stream);
 
+/* Keys and values of one append: the same as kvq_quantize_keys(k_src) followed by
+ * kvq_quantize_values(v_src) on the same stream, both sources with the same strides,
+ * and bit for bit the same cache contents.  When both sides use the asymmetric
+ * per-channel / per-token kernels (the K4/V2 decode format among them) it is one
+ * launch instead of two. */
+kvq_status kvq_quantize_kv(const kvq_format* fmt, const kvq_cache* cache, const void* k_src,
+                           const void* v_src, int64_t stride_b, int64_t stride_h,
+                           int64_t stride_t, int64_t t0, int64_t n, int32_t* d_status,
+                           void* stream);
+
 /* Reconstruct packed rows [t0, t0 + n) of keys or values (which = KVQ_KEYS/VALUES)
  * into `out` (device, [B][Hkv][n][D] contiguous, out_dtype).  fp32 output is the exact
  * x^ of the scheme; fp16 / bf16 output is that fp32 value rounded to nearest-even.

@@ -266,6 +266,29 @@ kvq_status kvq_quantize_values(const kvq_format* f, const kvq_cache* c, const vo
   return quantize_common(KVQ_VALUES, f, c, src, sb, sh, st, t0, n, d_status, stream);
 }
 
+kvq_status kvq_quantize_kv(const kvq_format* f, const kvq_cache* c, const void* k_src,
+                           const void* v_src, int64_t sb, int64_t sh, int64_t st, int64_t t0,
+                           int64_t n, int32_t* d_status, void* stream) {
+  Layout L;
+  kvq_status s = make_layout(f, c, &L);
+  if (s != KVQ_OK) return s;
+  if (n < 0 || t0 < 0 || t0 % L.g || t0 + n > L.C) return KVQ_ERR_INVALID;
+  if (n == 0) return KVQ_OK;
+  if (!k_src || !v_src || !aligned16(k_src) || !aligned16(v_src)) return KVQ_ERR_INVALID;
+  const int64_t eb = dtype_bytes(L.src_dtype);
+  if (st < L.D || sb < 0 || sh < 0) return KVQ_ERR_INVALID;
+  if ((st * eb) % 16 || (sh * eb) % 16 || (sb * eb) % 16) return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  if (asym_fast_ok(L, KVQ_KEYS) && asym_fast_ok(L, KVQ_VALUES)) {
+    cudaError_t e = launch_quantize_asym_kv(L, k_src, v_src, sb, sh, st, t0, n, d_status,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  }
+  s = quantize_common(KVQ_KEYS, f, c, k_src, sb, sh, st, t0, n, d_status, stream);
+  if (s != KVQ_OK) return s;
+  return quantize_common(KVQ_VALUES, f, c, v_src, sb, sh, st, t0, n, d_status, stream);
+}
+
 kvq_status kvq_dequantize(const kvq_format* f, const kvq_cache* c, int32_t which, int64_t t0,
                           int64_t n, void* out, int32_t out_dtype, int32_t* d_status,
                           void* stream) {

@@ -316,6 +316,32 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
           kz[j] = __half2float(kzs[4 * lane + j]);
         }
       }
+      // MIXED: the lane's plane (raw 16-bit, 4-bit or 2-bit slots), its word offset in a row,
+      // the row stride, and the first code's shift
+      int m_base = 0, m_stride = 0, m_shift = 0, m_bw = 0;
+      uint32_t m_mask = 0u;
+      bool m_raw = false;
+      if constexpr (mixed) {
+        const int s0 = 4 * lane;
+        if (s0 < hi) {
+          m_raw = true;   // m_bw = 0: the code formula is not used (and shifts stay < 32)
+          m_base = SG.k + 2 * s0;
+          m_stride = 2 * hi;
+        } else if (s0 < hi + mid) {
+          const int e0 = s0 - hi;
+          m_base = SG.k_mid + 4 * (e0 / 8);
+          m_stride = mid / 2;
+          m_shift = 4 * (e0 % 8);
+          m_bw = 4;
+        } else {
+          const int e0 = s0 - hi - mid;
+          m_base = SG.k_lo + 4 * (e0 / 16);
+          m_stride = lo / 4;
+          m_shift = 2 * (e0 % 16);
+          m_bw = 2;
+        }
+        m_mask = m_raw ? 0u : (1u << m_bw) - 1u;
+      }
       float cs[4], sn[4];
       if (ROPE) {
 #pragma unroll
@@ -333,20 +359,18 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
           const int rr = ok[e] ? r : 0;
           // keys
           if constexpr (mixed) {
-            const int s0 = 4 * lane;
-            if (s0 < hi) {
-              const float4 f = ld4(st + SG.k, rr * hi + s0, L.src_dtype);
-              kb[e][0] = f.x; kb[e][1] = f.y; kb[e][2] = f.z; kb[e][3] = f.w;
-            } else if (s0 < hi + mid) {
-              const int e0 = s0 - hi;
-              const uint32_t w = reinterpret_cast<const uint32_t*>(st + SG.k_mid)[rr * (mid / 8) + e0 / 8] >> (4 * (e0 % 8));
+            // one word (two for raw slots) at the lane's plane position; no divergent paths
+            const uint8_t* wp = st + m_base + rr * m_stride;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wp);
+            uint32_t w1 = 0u;
+            if (m_raw) w1 = *reinterpret_cast<const uint32_t*>(wp + 4);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (4 * j)) & 15u), ks[j], kz[j]);
-            } else {
-              const int e0 = s0 - hi - mid;
-              const uint32_t w = reinterpret_cast<const uint32_t*>(st + SG.k_lo)[rr * (lo / 16) + e0 / 16] >> (2 * (e0 % 16));
-#pragma unroll
-              for (int j = 0; j < 4; ++j) kb[e][j] = __fmaf_rn((float)((w >> (2 * j)) & 3u), ks[j], kz[j]);
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t hbits = ((j < 2 ? w0 : w1) >> (16 * (j & 1))) & 0xffffu;
+              const float raw = L.src_dtype == KVQ_F16 ? half_bits_to_float((uint16_t)hbits)
+                                                       : __uint_as_float(hbits << 16);
+              const float dq = __fmaf_rn((float)((w0 >> (m_shift + m_bw * j)) & m_mask), ks[j], kz[j]);
+              kb[e][j] = m_raw ? raw : dq;
             }
           } else if constexpr (KF == kNuq) {
             uint32_t code[4];
@@ -388,7 +412,18 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
                 if (c == 4 * lane + j) kb[e][j] = v;
             }
           }
-          if (SV.nout > 0 && ok[e]) {
+          if (SV.nout == 2 && ok[e]) {   // both entries in two loads
+            const uint32_t cols = *reinterpret_cast<const uint16_t*>(st + SG.voc + rr * 2);
+            const uint32_t vals = *reinterpret_cast<const uint32_t*>(st + SG.vov + rr * 4);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int c = (int)((cols >> (8 * x)) & 0xffu);
+              const float v = half_bits_to_float((uint16_t)(vals >> (16 * x)));
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (c == 4 * lane + j) vb[e][j] = v;
+            }
+          } else if (SV.nout > 0 && ok[e]) {
             for (int x = 0; x < SV.nout; ++x) {
               const int c = st[SG.voc + rr * SV.nout + x];
               const float v = __half2float(reinterpret_cast<const __half*>(st + SG.vov)[rr * SV.nout + x]);

@@ -56,6 +56,9 @@ bool asym_fast_ok(const Layout& L, int which);
 cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, int64_t sb,
                                  int64_t sh, int64_t st, int64_t t0, int64_t n,
                                  int32_t* d_status, cudaStream_t s);
+cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const void* vsrc, int64_t sb,
+                                    int64_t sh, int64_t st, int64_t t0, int64_t n, int32_t* d_status,
+                                    cudaStream_t s);
 cudaError_t launch_dequantize(const Layout& L, int which, int64_t t0, int64_t n, void* out,
                               int out_dtype, int32_t* d_status, cudaStream_t s);
 cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t qsh,

@@ -63,18 +63,18 @@ __device__ __forceinline__ uint2 pack8(const float* x, const float* s, const flo
 
 // Keys.  Thread (warp w, lane): vector v = lane & 3 (channels cb + 8 v .. + 7) of rows
 // rs, rs + 64, ... with rs = 8 w + lane / 4.
-__global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
+__device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, int bz) {
   __shared__ float pmin[8][kCB], pmax[8][kCB];
   __shared__ float sf[kCB], zf[kCB];
   __shared__ int flags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_KEYS];
   const int D = L.D, g = L.g, bits = S.bits;
-  const int64_t ts = a.t0 + (int64_t)blockIdx.x * g;
+  const int64_t ts = a.t0 + (int64_t)bx * g;
   const int ln = (int)min((int64_t)g, a.t0 + a.n - ts);
   const int gi = (int)(ts / g);
-  const int cb = blockIdx.y * kCB;
-  const int head = blockIdx.z;
+  const int cb = by * kCB;
+  const int head = bz;
   const int b = head / L.Hkv, h = head % L.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int v = lane & 3, rs = warp * 8 + (lane >> 2);
@@ -171,15 +171,16 @@ __global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
 // Values.  A warp takes 4 consecutive tokens of the block; lane (sub, vl) holds vector
 // vl (channels 8 vl .. 8 vl + 7) of one token, sub = lane / nvec, nvec = D / 8 lanes per
 // token, so a pass covers 32 / nvec tokens and a warp ceil(4 nvec / 32) passes.
-__global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
+__device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by) {
   constexpr int kPass = 4;   // at most 4 passes (D = 256)
-  __shared__ int flags;
+  __shared__ int vflags;
+  int& flags = vflags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_VALUES];
   const int D = L.D, bits = S.bits;
-  const int64_t tb = a.t0 + (int64_t)blockIdx.x * kTB;
+  const int64_t tb = a.t0 + (int64_t)bx * kTB;
   const int nt = (int)min((int64_t)kTB, a.t0 + a.n - tb);
-  const int head = blockIdx.y;
+  const int head = by;
   const int b = head / L.Hkv, h = head % L.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nvec = D / 8, rpp = 32 / nvec, sub = lane / nvec, vl = lane % nvec;
@@ -290,6 +291,27 @@ __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
     flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
 }
 
+__global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
+  asym_keys_block(a, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+__global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
+  asym_values_block(a, blockIdx.x, blockIdx.y);
+}
+
+// Keys and values of one append in one launch: blocks [0, nk) are key blocks
+// (group, channel block, head), the rest value blocks (token block, head).
+__global__ void __launch_bounds__(kThreads) asym_kv_kernel(AArgs ak, AArgs av, int kgx, int kgy, int nk,
+                                                           int vgx) {
+  const int b = blockIdx.x;
+  if (b < nk) {
+    asym_keys_block(ak, b % kgx, (b / kgx) % kgy, b / (kgx * kgy));
+  } else {
+    const int v = b - nk;
+    asym_values_block(av, v % vgx, v / vgx);
+  }
+}
+
 }  // namespace
 
 bool asym_fast_ok(const Layout& L, int which) {
@@ -317,6 +339,31 @@ cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, in
     dim3 grid((unsigned)((n + kTB - 1) / kTB), L.B * L.Hkv);
     asym_values_kernel<<<grid, kThreads, 0, s>>>(a);
   }
+  return cudaGetLastError();
+}
+
+}  // namespace kvq
+
+namespace kvq {
+
+cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const void* vsrc, int64_t sb,
+                                    int64_t sh, int64_t st, int64_t t0, int64_t n, int32_t* d_status,
+                                    cudaStream_t s) {
+  AArgs ak, av;
+  ak.L = av.L = L;
+  ak.src = ksrc;
+  av.src = vsrc;
+  ak.sb = av.sb = sb;
+  ak.sh = av.sh = sh;
+  ak.st = av.st = st;
+  ak.t0 = av.t0 = t0;
+  ak.n = av.n = n;
+  ak.status = av.status = d_status;
+  const int kgx = (int)((n + L.g - 1) / L.g), kgy = L.D / kCB, heads = L.B * L.Hkv;
+  const int vgx = (int)((n + kTB - 1) / kTB);
+  const int64_t nk = (int64_t)kgx * kgy * heads, nv = (int64_t)vgx * heads;
+  if (nk + nv > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  asym_kv_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, kgy, (int)nk, vgx);
   return cudaGetLastError();
 }
 

@@ -73,6 +73,7 @@ def lib():
             "kvq_cache_array_bytes": (SZ, [FP, I32, I32, I64, I32]),
             "kvq_quantize_keys": (I32, [FP, CP, P, I64, I64, I64, I64, I64, P, P]),
             "kvq_quantize_values": (I32, [FP, CP, P, I64, I64, I64, I64, I64, P, P]),
+            "kvq_quantize_kv": (I32, [FP, CP, P, P, I64, I64, I64, I64, I64, P, P]),
             "kvq_dequantize": (I32, [FP, CP, I32, I64, I64, P, I32, P, P]),
             "kvq_key_salience": (I32, [FP, P, I64, I64, I64, P, I64, I64, I64, I32, I32, I32, I32,
                                        P, P, I64, I64, P, P]),
@@ -165,6 +166,17 @@ def quantize_values(fmt, cache: Cache, src: torch.Tensor, t0: int, n: int, statu
                                    src.stride(1), src.stride(2), t0, n, _ptr(status),
                                    _stream(stream))
     _check("kvq_quantize_values", st)
+
+
+def quantize_kv(fmt, cache: Cache, k_src: torch.Tensor, v_src: torch.Tensor, t0: int, n: int,
+                status=None, stream=None):
+    """Keys and values of one append (same strides), one launch where the kernels allow."""
+    if k_src.stride() != v_src.stride():
+        raise ValueError("k_src and v_src must have the same strides")
+    st = lib().kvq_quantize_kv(ctypes.byref(fmt), cache.ref(), _ptr(k_src), _ptr(v_src),
+                               k_src.stride(0), k_src.stride(1), k_src.stride(2), t0, n,
+                               _ptr(status), _stream(stream))
+    _check("kvq_quantize_kv", st)
 
 
 def dequantize(fmt, cache: Cache, which: int, t0: int, n: int, out_dtype=F32, out=None,

@@ -13,7 +13,8 @@ from oracle.cache import dequantize as odeq
 from oracle.formats import (ASYM, BF16, CHANNEL, F16, F32, KEYS, MIXED, NONE, NUQ, SYM8,
                             TENSOR, TOKEN, VALUES)
 from quantized_decode_attention_quantize_b200 import kvq
-from tests.gpu_util import Pair
+from oracle import cache as ocache
+from tests.gpu_util import Pair, dev
 
 pytestmark = pytest.mark.gpu
 
@@ -205,3 +206,31 @@ def test_none_scheme_copies_raw():
     p.quantize(KEYS, K[None, None], 0, N)
     p.quantize(VALUES, V[None, None], 0, N)
     p.assert_arrays_equal()
+
+
+@pytest.mark.parametrize("fd", [
+    dict(src_dtype=BF16),                                              # K4/V2: one fused launch
+    dict(src_dtype=F16, k_bits=2, v_bits=4),
+    dict(src_dtype=BF16, k_scheme=NUQ, k_bits=3, k_outliers=2, v_scheme=NUQ, v_bits=3, v_outliers=2),
+])
+def test_quantize_kv_matches_separate_calls_and_oracle(fd):
+    # kvq_quantize_kv = kvq_quantize_keys then kvq_quantize_values, bit for bit
+    B, H, D, g = 2, 3, 128, 128
+    n = 2 * g + 40
+    f = fmt(**fd)
+    luts = (LUT["k"], LUT["v"]) if fd.get("k_scheme") == NUQ else (None, None)
+    p = Pair(f, B, H, 3 * g, k_lut=luts[0], v_lut=luts[1])
+    K = values(21, (B, H, n, D), fd["src_dtype"])
+    V = values(22, (B, H, n, D), fd["src_dtype"])
+    kd, vd = dev(K, fd["src_dtype"]), dev(V, fd["src_dtype"])
+    kvq.quantize_kv(p.fmt, p.gpu, kd, vd, 0, n, status=p.status)
+    ocache.quantize(p.of, p.ora, KEYS, K.astype(np.float64), 0, n)
+    ocache.quantize(p.of, p.ora, VALUES, V.astype(np.float64), 0, n)
+    p.assert_arrays_equal()
+    assert p.status_bits() == 0
+    other = kvq.Cache(p.fmt, B, H, 3 * g, k_lut=luts[0], v_lut=luts[1])
+    kvq.quantize_keys(p.fmt, other, kd, 0, n)
+    kvq.quantize_values(p.fmt, other, vd, 0, n)
+    torch.cuda.synchronize()
+    for name, t in other.tensors.items():
+        assert torch.equal(t, p.gpu.array(name)), name
