@@ -264,13 +264,17 @@ __device__ void do_nuq(const QArgs& a, const QSmem& sm, int ln, int64_t ts, int 
   __syncthreads();
   int range_bad = 0;
   if (a.which == KVQ_KEYS) {
-    for (int c = threadIdx.x; c < D; c += blockDim.x) {
-      // top-k |x| of the column, ties to the lower row (rows are scanned upward, so a
-      // later row displaces an entry only with a strictly larger magnitude)
+    // Two threads per channel (adjacent lanes): the even one scans rows [0, h), the odd one
+    // rows [h, ln), h = ceil(ln / 2).  Each keeps its own top-k |x| (ties to the lower row:
+    // a later row displaces an entry only with a strictly larger magnitude); the global
+    // top-k is the top-k of the 2k candidates, rows of the even thread first on ties.
+    const int half = threadIdx.x & 1, h2 = (ln + 1) / 2;
+    const int r_lo = half ? h2 : 0, r_hi = half ? ln : h2;
+    for (int c = threadIdx.x >> 1; c < D; c += blockDim.x >> 1) {
       float ba[8];
       int bi[8];
       int cnt = 0;
-      for (int r = 0; r < ln; ++r) {
+      for (int r = r_lo; r < r_hi; ++r) {
         const float v = fabsf(sm.tile[r * D + c]);
         int pos = cnt;
         while (pos > 0 && v > ba[pos - 1]) --pos;
@@ -285,8 +289,43 @@ __device__ void do_nuq(const QArgs& a, const QSmem& sm, int ln, int64_t ts, int 
           if (cnt < k) ++cnt;
         }
       }
+      // merge with the partner's list: candidates of the even thread first
+      const int pcnt = __shfl_xor_sync(0xffffffffu, cnt, 1);
+      float ca[16];
+      int ci[16];
+      int n_c = 0;
+      for (int j = 0; j < 8; ++j) {
+        const float pv = __shfl_xor_sync(0xffffffffu, j < cnt ? ba[j] : 0.0f, 1);
+        const int pi = __shfl_xor_sync(0xffffffffu, j < cnt ? bi[j] : 0, 1);
+        if (half == 0 && j < cnt) { ca[n_c] = ba[j]; ci[n_c] = bi[j]; ++n_c; }
+        if (half == 1 && j < pcnt) { ca[n_c] = pv; ci[n_c] = pi; ++n_c; }
+      }
+      for (int j = 0; j < 8; ++j) {
+        const float pv = __shfl_xor_sync(0xffffffffu, j < cnt ? ba[j] : 0.0f, 1);
+        const int pi = __shfl_xor_sync(0xffffffffu, j < cnt ? bi[j] : 0, 1);
+        if (half == 0 && j < pcnt) { ca[n_c] = pv; ci[n_c] = pi; ++n_c; }
+        if (half == 1 && j < cnt) { ca[n_c] = ba[j]; ci[n_c] = bi[j]; ++n_c; }
+      }
+      // top-k of the candidates in order (candidates of lower rows come first, so a
+      // strict comparison keeps the lower row on ties)
+      cnt = 0;
+      for (int x = 0; x < n_c; ++x) {
+        const float v = ca[x];
+        int pos = cnt;
+        while (pos > 0 && v > ba[pos - 1]) --pos;
+        if (pos < k) {
+          const int last = cnt < k ? cnt : k - 1;
+          for (int j = last; j > pos; --j) {
+            ba[j] = ba[j - 1];
+            bi[j] = bi[j - 1];
+          }
+          ba[pos] = v;
+          bi[pos] = ci[x];
+          if (cnt < k) ++cnt;
+        }
+      }
       float mn = INFINITY, mx = -INFINITY;
-      for (int r = 0; r < ln; ++r) {
+      for (int r = r_lo; r < r_hi; ++r) {
         bool out = false;
         for (int j = 0; j < cnt; ++j) out |= (bi[j] == r);
         if (!out) {
@@ -295,29 +334,47 @@ __device__ void do_nuq(const QArgs& a, const QSmem& sm, int ln, int64_t ts, int 
           mx = fmaxf(mx, x);
         }
       }
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       if (!(mn <= mx)) mn = mx = 0.0f;
-      for (int j = 0; j < cnt; ++j) atomicOr(&sm.omask[bi[j] * mw + c / 32], 1u << (c % 32));
       __half s, z;
-      range_bad |= !nuq_params(mn, mx, &s, &z);
-      hs[(sl * L.ng + gi) * D + c] = s;
-      hz[(sl * L.ng + gi) * D + c] = z;
+      const bool ok = nuq_params(mn, mx, &s, &z);
+      if (half == 0) {
+        for (int j = 0; j < cnt; ++j) atomicOr(&sm.omask[bi[j] * mw + c / 32], 1u << (c % 32));
+        range_bad |= !ok;
+        hs[(sl * L.ng + gi) * D + c] = s;
+        hz[(sl * L.ng + gi) * D + c] = z;
+      }
       const float sf = __half2float(s), zf = __half2float(z);
-      for (int r = 0; r < ln; ++r) {
+      for (int r = r_lo; r < r_hi; ++r) {
         const float x = fminf(fmaxf(sm.tile[r * D + c], mn), mx);
         sm.codes[r * D + c] = (uint8_t)nuq_code(x, sf, zf, sm.mids);
       }
     }
     __syncthreads();
     if (k > 0) {
-      // CSR by token row: counts, exclusive scan, then entries in channel order
-      if (threadIdx.x == 0) {
-        int acc = 0;
-        sm.rowptr[0] = 0;
-        for (int r = 0; r < g; ++r) {
-          if (r < ln)
-            for (int w = 0; w < mw; ++w) acc += __popc(sm.omask[r * mw + w]);
-          sm.rowptr[r + 1] = acc;
+      // CSR by token row: per-row counts, a block-wide exclusive scan, then each row's
+      // entries in channel order
+      int* cnt_scan = sm.rowptr;   // [g + 1]
+      {
+        const int r = threadIdx.x;   // g <= blockDim.x
+        int cr = 0;
+        if (r < ln)
+          for (int w = 0; w < mw; ++w) cr += __popc(sm.omask[r * mw + w]);
+        // inclusive scan within the warp, then across warps
+        int incl = cr;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
         }
+        __shared__ int wsum[kThreads / 32];
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; ++w) base += wsum[w];
+        if (r < g) cnt_scan[r + 1] = base + incl;
+        if (r == 0) cnt_scan[0] = 0;
       }
       __syncthreads();
       int32_t* rp = L.k_out_rowptr + (sl * L.ng + gi) * (g + 1);
