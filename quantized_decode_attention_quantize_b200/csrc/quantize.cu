@@ -405,28 +405,37 @@ __device__ void do_nuq(const QArgs& a, const QSmem& sm, int ln, int64_t ts, int 
       if (vbad) atomicOr(sm.flag, 2);
     }
   } else {
-    for (int r = warp; r < ln; r += nw) {
-      const float* row = sm.tile + r * D;
-      uint32_t chosen = 0;           // bit j: channel lane + 32 j chosen
+    // Value rows: each half warp takes one row (lanes 16 h .. 16 h + 15, channels
+    // (lane & 15) + 16 j), so a warp works on two rows with one instruction stream and
+    // every reduction is four shuffle levels.
+    const int hl = lane & 15, hw = lane >> 4;
+    const int nj = D / 16;
+    const int rows_per_pass = 2 * nw;
+    const int passes = (ln + rows_per_pass - 1) / rows_per_pass;
+    for (int pass = 0; pass < passes; ++pass) {
+      const int r = pass * rows_per_pass + 2 * warp + hw;
+      const bool live = r < ln;
+      const float* row = sm.tile + (live ? r : 0) * D;
+      uint32_t chosen = 0;           // bit j: channel hl + 16 j chosen
       int sel[8];
       for (int e = 0; e < k; ++e) {
         float ba = -1.0f;
         int bc = 1 << 30;
-        for (int j = 0; j * 32 < D; ++j) {
-          const int c = lane + 32 * j;
+        for (int j = 0; j < nj; ++j) {
+          const int c = hl + 16 * j;
           if (!(chosen & (1u << j))) {
             const float v = fabsf(row[c]);
             if (v > ba) { ba = v; bc = c; }
           }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+        for (int o = 8; o > 0; o >>= 1) {
           const float oa = __shfl_xor_sync(0xffffffffu, ba, o);
           const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
           if (oa > ba || (oa == ba && oc < bc)) { ba = oa; bc = oc; }
         }
         sel[e] = bc;
-        if ((bc & 31) == lane) chosen |= 1u << (bc >> 5);
+        if ((bc & 15) == hl) chosen |= 1u << (bc >> 4);
       }
       // ascending channel order
       for (int i = 1; i < k; ++i) {
@@ -436,36 +445,41 @@ __device__ void do_nuq(const QArgs& a, const QSmem& sm, int ln, int64_t ts, int 
         sel[j] = v;
       }
       float mn = INFINITY, mx = -INFINITY;
-      for (int j = 0; j * 32 < D; ++j) {
+      for (int j = 0; j < nj; ++j) {
         if (!(chosen & (1u << j))) {
-          const float x = row[lane + 32 * j];
+          const float x = row[hl + 16 * j];
           mn = fminf(mn, x);
           mx = fmaxf(mx, x);
         }
       }
-      mn = warp_min(mn);
-      mx = warp_max(mx);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
       if (!(mn <= mx)) mn = mx = 0.0f;
       __half s, z;
       const bool ok = nuq_params(mn, mx, &s, &z);
       const float sf = __half2float(s), zf = __half2float(z);
-      for (int j = 0; j * 32 < D; ++j) {
-        const int c = lane + 32 * j;
-        const float x = fminf(fmaxf(row[c], mn), mx);
-        sm.codes[r * D + c] = (uint8_t)nuq_code(x, sf, zf, sm.mids);
-      }
-      if (lane == 0) {
-        range_bad |= !ok;
-        hs[sl * L.C + ts + r] = s;
-        hz[sl * L.C + ts + r] = z;
-      }
-      if (lane < k) {
-        int c = sel[0];
-        for (int e = 1; e < k; ++e) if (lane == e) c = sel[e];
-        const __half hv = __float2half_rn(row[c]);
-        range_bad |= !isfinite(__half2float(hv));
-        L.v_out_col[(sl * L.C + ts + r) * k + lane] = (uint8_t)c;
-        L.v_out_val[(sl * L.C + ts + r) * k + lane] = hv;
+      if (live) {
+        for (int j = 0; j < nj; ++j) {
+          const int c = hl + 16 * j;
+          const float x = fminf(fmaxf(row[c], mn), mx);
+          sm.codes[r * D + c] = (uint8_t)nuq_code(x, sf, zf, sm.mids);
+        }
+        if (hl == 0) {
+          range_bad |= !ok;
+          hs[sl * L.C + ts + r] = s;
+          hz[sl * L.C + ts + r] = z;
+        }
+        if (hl < k) {
+          int c = sel[0];
+          for (int e = 1; e < k; ++e) if (hl == e) c = sel[e];
+          const __half hv = __float2half_rn(row[c]);
+          range_bad |= !isfinite(__half2float(hv));
+          L.v_out_col[(sl * L.C + ts + r) * k + hl] = (uint8_t)c;
+          L.v_out_val[(sl * L.C + ts + r) * k + hl] = hv;
+        }
       }
     }
   }
