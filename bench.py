@@ -372,6 +372,21 @@ def main():
                              Hkv * (C // g) * D, (C // g) * D)
     kvq.quantize_keys(fmt, cache, K[:, :, ns:ns + tq], 0, tq)
     kvq.quantize_values(fmt, cache, V[:, :, ns:ns + tq], 0, tq)
+    # full-cache quantize rate (keys + values of all packed tokens in one call, timed
+    # again after the build above)
+    fq_ms = []
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kvq.quantize_kv(fmt, cache, K[:, :, ns:ns + tq], V[:, :, ns:ns + tq], 0, tq)
+        e1.record()
+        e1.synchronize()
+        fq_ms.append(e0.elapsed_time(e1))
+    fq_read = 2 * B * Hkv * tq * D * K.element_size()
+    fq_written = sum(t.numel() for name, t in cache.tensors.items()
+                     if name not in ("sink_k", "sink_v", "res_k", "res_v", "k_lut", "v_lut"))
+    full_quant = {"ms": min(fq_ms), "gbs": (fq_read + fq_written) / (min(fq_ms) * 1e-3) / 1e9,
+                  "bytes": fq_read + fq_written, "tokens": tq}
     if ns:
         cache.array("sink_k").copy_(K[:, :, :ns].contiguous().view(-1).view(torch.uint8))
         cache.array("sink_v").copy_(V[:, :, :ns].contiguous().view(-1).view(torch.uint8))
@@ -542,6 +557,7 @@ def main():
         "decode_gbs": decode_gbs, "quantize_gbs": quant_gbs,
         "tokens_heads_per_s": world * B * Hq * cfg["T"] / ((ms_part + ms_comb) * 1e-3),
         "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb},
+        "full_cache_quantize": full_quant,
         "roofline": {"kernel": f"{path} (kvq_decode_partial)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": kern_bytes,

@@ -1,9 +1,10 @@
 // MixKVQ key-channel salience ([MIX] Figure 3: A = I * S; Figure 4: recomputed over
 // each window of R buffered tokens).
 //
-// One CTA per (kv head, batch), one thread per channel d.  I_d sums |Q[d]| over the
-// G query heads of the group and the R window rows in fp64, head-major then row, and
-// divides by G * R; S_d is the fp64 range of K[:, d]; A_d = I_d * S_d.  The rank of a
+// One CTA per (kv head, batch), one thread per channel d.  The window rows are staged
+// through shared memory in chunks of 64 rows with coalesced (16-byte where the strides
+// allow) loads by all threads.  I_d sums |Q[d]| over the G query heads of the group and
+// the R window rows in fp64, head-major then row, and divides by G * R; S_d is the fp64 range of K[:, d]; A_d = I_d * S_d.  The rank of a
 // channel is the number of channels with a larger A (or an equal A and a lower
 // index), so order[rank] = d sorts by descending salience with ties to the lower
 // channel.  Every fp64 step is a single IEEE operation, so the result is the same
@@ -23,35 +24,73 @@ struct SalArgs {
   uint8_t* order;
   int64_t osb, osh;
   int32_t* status;
+  int q_vec, k_vec;   // 16-byte staging loads allowed (aligned base and strides)
 };
 
+constexpr int kRC = 64;   // window rows per staged chunk
+
+// Rows [r0, r0 + nr) of a [R][D] window (element offsets base + r * rstride + c) into
+// buf[r - r0][c], by all D threads of the CTA.
+__device__ __forceinline__ void stage_rows(uint8_t* buf, const void* src, int64_t base, int64_t rstride,
+                                           int r0, int nr, int D, int esz, bool vec) {
+  const uint8_t* s8 = reinterpret_cast<const uint8_t*>(src);
+  if (vec) {
+    const int vpr = D * esz / 16;
+    for (int v = threadIdx.x; v < nr * vpr; v += blockDim.x) {
+      const int row = v / vpr, cv = v - row * vpr;
+      *reinterpret_cast<uint4*>(buf + (size_t)row * D * esz + cv * 16) =
+          *reinterpret_cast<const uint4*>(s8 + (base + (int64_t)(r0 + row) * rstride) * esz + cv * 16);
+    }
+  } else {
+    for (int i = threadIdx.x; i < nr * D; i += blockDim.x) {
+      const int row = i / D, c = i - row * D;
+      const uint8_t* from = s8 + (base + (int64_t)(r0 + row) * rstride + c) * esz;
+      uint8_t* to = buf + (size_t)i * esz;
+      for (int e = 0; e < esz; ++e) to[e] = from[e];
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
+  extern __shared__ __align__(16) uint8_t sbuf[];   // [kRC][D] source elements
   __shared__ double A[256];
   __shared__ int bad;
   const int d = threadIdx.x;
   const int h = blockIdx.x, b = blockIdx.y;
   const int G = a.Hq / a.Hkv;
+  const int D = a.D;
+  const int esz = a.dtype == KVQ_F32 ? 4 : 2;
   if (d == 0) bad = 0;
-  __syncthreads();
   double acc = 0.0;
   int nonfinite = 0;
   for (int hh = 0; hh < G; ++hh) {
-    const int64_t qb = (int64_t)b * a.qsb + (int64_t)(h * G + hh) * a.qsh + d;
-#pragma unroll 8
-    for (int r = 0; r < a.R; ++r) {
-      const float x = load_elem(a.q, qb + (int64_t)r * a.qst, a.dtype);
-      nonfinite |= !isfinite(x);
-      acc = __dadd_rn(acc, fabs((double)x));
+    const int64_t qb = (int64_t)b * a.qsb + (int64_t)(h * G + hh) * a.qsh;
+    for (int r0 = 0; r0 < a.R; r0 += kRC) {
+      const int nr = min(kRC, a.R - r0);
+      __syncthreads();
+      stage_rows(sbuf, a.q, qb, a.qst, r0, nr, D, esz, a.q_vec);
+      __syncthreads();
+      for (int r = 0; r < nr; ++r) {
+        const float x = load_elem(sbuf, (int64_t)r * D + d, a.dtype);
+        nonfinite |= !isfinite(x);
+        acc = __dadd_rn(acc, fabs((double)x));
+      }
     }
   }
   const double intensity = __ddiv_rn(acc, (double)G * (double)a.R);
-  const int64_t kb = (int64_t)b * a.ksb + (int64_t)h * a.ksh + d;
+  const int64_t kb = (int64_t)b * a.ksb + (int64_t)h * a.ksh;
   float mn = INFINITY, mx = -INFINITY;
-  for (int r = 0; r < a.R; ++r) {
-    const float x = load_elem(a.k, kb + (int64_t)r * a.kst, a.dtype);
-    nonfinite |= !isfinite(x);
-    mn = fminf(mn, x);
-    mx = fmaxf(mx, x);
+  for (int r0 = 0; r0 < a.R; r0 += kRC) {
+    const int nr = min(kRC, a.R - r0);
+    __syncthreads();
+    stage_rows(sbuf, a.k, kb, a.kst, r0, nr, D, esz, a.k_vec);
+    __syncthreads();
+    for (int r = 0; r < nr; ++r) {
+      const float x = load_elem(sbuf, (int64_t)r * D + d, a.dtype);
+      nonfinite |= !isfinite(x);
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
   }
   const double range = __dsub_rn((double)mx, (double)mn);
   const double sal = __dmul_rn(intensity, range);
@@ -94,8 +133,18 @@ cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t
   a.osb = osb;
   a.osh = osh;
   a.status = d_status;
+  const int esz = L.src_dtype == KVQ_F32 ? 4 : 2;
+  auto vec_ok = [&](const void* p, int64_t s1, int64_t s2, int64_t s3) {
+    return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && (s1 * esz) % 16 == 0 && (s2 * esz) % 16 == 0 &&
+           (s3 * esz) % 16 == 0 && (L.D * esz) % 16 == 0;
+  };
+  a.q_vec = vec_ok(q, qsb, qsh, qst);
+  a.k_vec = vec_ok(k, ksb, ksh, kst);
+  const size_t smem = (size_t)kRC * L.D * esz;
+  cudaError_t e = cudaFuncSetAttribute(salience_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(Hkv, B);
-  salience_kernel<<<grid, L.D, 0, s>>>(a);
+  salience_kernel<<<grid, L.D, smem, s>>>(a);
   return cudaGetLastError();
 }
 
