@@ -57,7 +57,7 @@ extern "C" {
 typedef enum kvq_status {
   KVQ_OK = 0,
   KVQ_ERR_INVALID = 1,      /* bad argument: null, misaligned, out of range, shape mismatch */
-  KVQ_ERR_UNSUPPORTED = 2,  /* well-formed request this build does not implement */
+  KVQ_ERR_UNSUPPORTED = 2,  /* well-formed request this library does not implement */
   KVQ_ERR_CUDA = 3,         /* a CUDA call or a kernel launch failed */
   KVQ_ERR_WORKSPACE = 4     /* workspace smaller than kvq_decode_workspace_bytes() */
 } kvq_status;

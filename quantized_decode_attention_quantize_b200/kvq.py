@@ -62,7 +62,7 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} not built; run __graft_entry__.build()")
+            raise RuntimeError(f"{LIB_PATH} not built; run python -m quantized_decode_attention_quantize_b200.build")
         L = ctypes.CDLL(LIB_PATH)
         P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         FP, CP = ctypes.POINTER(kvq_format), ctypes.POINTER(kvq_cache)
