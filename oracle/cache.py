@@ -3,7 +3,9 @@
 Arrays have the exact element types and shapes of the device arrays (fp16 values as
 their uint16 encodings), so a test compares them byte for byte.  Operations follow
 the library's entry points: `quantize(fmt, cache, which, src, t0, n)` appends whole
-token groups, `dequantize(fmt, cache, which, t0, n)` reconstructs fp32 values.
+token groups, `dequantize(fmt, cache, which, t0, n)` reconstructs fp32 values.  With
+`k_rotate` the keys are quantized in the Walsh-Hadamard basis (oracle.rotate) and
+reconstructed back into the original one.
 
 Per-group rules come from oracle.quant, packing from oracle.pack; the grouping is
 that of [AXES] "What rows and columns mean" (tensor / token / channel) and of
@@ -13,7 +15,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import fp, pack, quant
+from . import fp, pack, quant, rotate
 from .formats import (ASYM, BF16, CHANNEL, F16, F32, KEYS, MIXED, NONE, NUQ, SYM8,
                       TENSOR, TOKEN, VALUES, Format, side)
 
@@ -133,6 +135,9 @@ def quantize(fmt: Format, cache: Cache, which: int, src, t0: int, n: int):
     """Quantize src [B, H, n, D] (exact source values, float64) into rows [t0, t0+n)."""
     src = np.asarray(src, np.float64)
     quant.check_finite(src)
+    if which == KEYS and fmt.k_rotate:
+        # [K4V2] "Rotation Integration": keys are rotated before their statistics
+        src = rotate.wht_f32(src)
     B, H = cache.B, cache.H
     assert src.shape[:3] == (B, H, n)
     scheme, bits, axis, nout = side(fmt, which)
@@ -290,6 +295,14 @@ def dequantize(fmt: Format, cache: Cache, which: int, t0: int, n: int, b=None, h
 
 
 def _deq_slab(fmt, cache, which, b, h, t0, n):
+    out = _deq_slab_stored(fmt, cache, which, b, h, t0, n)
+    if which == KEYS and fmt.k_rotate and n > 0:
+        # the stored basis is rotated; the normalised transform is its own inverse
+        out = rotate.wht_f32(out)
+    return out
+
+
+def _deq_slab_stored(fmt, cache, which, b, h, t0, n):
     A = cache.arrays
     D, g = fmt.head_dim, fmt.group_tokens
     scheme, bits, axis, nout = side(fmt, which)

@@ -46,6 +46,7 @@ class Format:
     residual_cap: int = 0
     rope: int = 0
     rope_base: float = 10000.0
+    k_rotate: int = 0     # keys rotated by the normalised Walsh-Hadamard transform (oracle.rotate)
 
     def as_dict(self):
         return asdict(self)

@@ -42,7 +42,7 @@ def _fmt(**kw):
                 k_scheme=ASYM, k_bits=4, k_axis=CHANNEL, k_outliers=0,
                 v_scheme=ASYM, v_bits=2, v_axis=TOKEN, v_outliers=0,
                 mixed_hi=0, mixed_mid=0, n_sink=0, residual_cap=0,
-                rope=0, rope_base=10000.0)
+                rope=0, rope_base=10000.0, k_rotate=0)
     base.update(kw)
     return base
 
@@ -53,6 +53,10 @@ CONFIGS = {
     "llama3_8b": dict(name="llama3_8b", B=8, Hq=32, Hkv=8, D=128, T=32768, seed=7,
                       q_dtype=BF16,
                       fmt=_fmt(src_dtype=BF16, n_sink=1, residual_cap=128)),
+    # the Llama-3-8B workload with key-only Walsh-Hadamard rotation (same data recipe)
+    "llama3_8b_wht": dict(name="llama3_8b_wht", recipe="llama3_8b", B=8, Hq=32, Hkv=8, D=128,
+                          T=32768, seed=7, q_dtype=BF16,
+                          fmt=_fmt(src_dtype=BF16, n_sink=1, residual_cap=128, k_rotate=1)),
     "kvquant_nuq3": dict(name="kvquant_nuq3", B=1, Hq=32, Hkv=32, D=128, T=131072, seed=7,
                          q_dtype=F16,
                          fmt=_fmt(src_dtype=F16, k_scheme=NUQ, k_bits=3, k_outliers=2,
@@ -114,7 +118,7 @@ def kv_slab(cfg, b, h, T=None, which="k"):
     """Keys or values of one (b, kv-head) slab: float32 values [T, D] in src dtype."""
     T = cfg["T"] if T is None else T
     D = cfg["D"]
-    name = cfg["name"]
+    name = cfg.get("recipe", cfg["name"])
     seed = cfg["seed"]
     dt = cfg["fmt"]["src_dtype"]
     r = rng(seed, which, b, h)
@@ -146,7 +150,7 @@ def query(cfg, b, hq):
     """Decode query of one query head: float32 values [D] in q dtype."""
     r = rng(cfg["seed"], "q", b, hq)
     q = r.standard_normal(cfg["D"], dtype=np.float32)
-    if cfg["name"] == "mixkvq_14b":
+    if cfg.get("recipe", cfg["name"]) == "mixkvq_14b":
         q *= log_uniform(rng(cfg["seed"], "qchan", b, hq), 0.1, 5.0, (cfg["D"],))
     return to_dtype_values(q, cfg["q_dtype"])
 
@@ -208,7 +212,7 @@ def device_kv(cfg, which, T=None, B=None, H=None, device="cuda", seed_offset=0):
     gen.manual_seed(cfg["seed"] * 1000 + TAGS[which] * 10 + seed_offset)
     tdt = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}[cfg["fmt"]["src_dtype"]]
     shape = (B, H, T, D)
-    name = cfg["name"]
+    name = cfg.get("recipe", cfg["name"])
     cpu = torch.Generator()
     cpu.manual_seed(cfg["seed"] * 1000 + TAGS[which] * 10 + seed_offset + 7)
     out = torch.empty(shape, dtype=tdt, device=device)
