@@ -64,7 +64,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="llama3_8b",
-                    choices=["llama3_8b", "llama2_7b", "kvquant_nuq3", "mixkvq_14b"])
+                    choices=["llama3_8b", "llama2_7b", "kvquant_nuq3", "mixkvq_14b", "llama3_8b_wht"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -102,6 +102,12 @@ K4V2 = dict(k_scheme=synth.ASYM, k_bits=4, k_axis=synth.CHANNEL, v_scheme=synth.
 
 def is_k4v2(cfg):
     return all(cfg["fmt"][k] == v for k, v in K4V2.items())
+
+
+def fused_kv(cfg):
+    """kvq_quantize_kv is one launch for K4/V2 without key rotation (rotated keys need whole
+    rows and take the general quantize kernel)."""
+    return is_k4v2(cfg) and not cfg["fmt"].get("k_rotate", 0)
 
 
 def cache_read_bytes(cache, cfg, tq, tr):
@@ -312,6 +318,8 @@ def workload_config(cfg):
     names = {synth.NONE: "raw", synth.SYM8: "INT8 sym", synth.ASYM: "asym", synth.NUQ: "nuq", synth.MIXED: "mixed"}
     kdesc = (f"mixed {f['mixed_hi']} raw / {f['mixed_mid']} 4-bit / rest 2-bit by salience"
              if f["k_scheme"] == synth.MIXED else f"{names[f['k_scheme']]}{f['k_bits']} per-channel")
+    if f.get("k_rotate"):
+        kdesc += " after a Walsh-Hadamard rotation of each key"
     extra = []
     if f["k_outliers"] or f["v_outliers"]:
         extra.append(f"top-{max(f['k_outliers'], f['v_outliers'])} fp16 outliers per vector")
@@ -539,7 +547,7 @@ def main():
     if os.path.exists(prof):
         try:
             pj = json.load(open(prof))
-            if pj.get("kernel_hash") == kernel_hash():
+            if pj.get("kernel_hash") == kernel_hash() and cfg["name"] == pj.get("config", "llama3_8b"):
                 traffic = pj.get("dram_bytes_per_launch")
         except (OSError, ValueError):
             pass
@@ -564,7 +572,7 @@ def main():
                      "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},
         "e2e": {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (LAUNCHES_PER_STEP + (0 if is_k4v2(cfg) else 1) + (n_app // g if mixed else 0))
+        "gpu_launches": (LAUNCHES_PER_STEP + (0 if fused_kv(cfg) else 1) + (n_app // g if mixed else 0))
         * args.steps,
         "clocks": clocks,
     }

@@ -39,7 +39,10 @@
  *  [MIX]    "MixKVQ: Query-Aware Mixed-Precision KV Cache Quantization for
  *           Long-Context Reasoning", Figures 3 and 4.
  *  [K4V2]   "Quantize What Counts: More for Keys, Less for Values", Technical
- *           Summary ("Key Contributions", "Results").
+ *           Summary ("Key Contributions", "Results", "Rotation Integration").
+ *  [TQ]     "Statistical Inference and Quality Measures of KV Cache Quantisations
+ *           Inspired by TurboQuant", Technical Summary (the KQV scheme's
+ *           Walsh-Hadamard transform, "Fat-Tail Robustness").
  */
 #ifndef KVQ_H_
 #define KVQ_H_
@@ -125,6 +128,17 @@ typedef struct kvq_format {
                             its absolute position ([KVQ] "Approach")                      */
   float rope_base;       /* RoPE base (10000); rotate-half pairs (i, i + D/2),
                             theta_i = base^(-2i/D)                                       */
+  int32_t k_rotate;      /* 1: key-only rotation ([K4V2] "Rotation Integration", [TQ]):
+                            every key row x is replaced, before its statistics, by
+                            y = H_D x / sqrt(D), the orthonormal Sylvester-ordered
+                            Walsh-Hadamard transform, evaluated in fp32 as the butterfly
+                            over strides 1, 2, ..., D/2 (pair (i, i+h) -> (a+b, a-b),
+                            each rounded) and one product with fl32(1/sqrt(D)).  Codes,
+                            metadata and outliers then live in the rotated basis;
+                            kvq_dequantize maps keys back with the same transform (its
+                            own inverse) and decode rotates the query instead, since
+                            q'.y = q.x.  Raw sink and residual keys stay unrotated.
+                            Keys of scheme SYM8, ASYM or NUQ, without rope.            */
 } kvq_format;
 
 /* Cache arrays.  Per (b, kv-head) slab, with capacity C tokens (a multiple of g),

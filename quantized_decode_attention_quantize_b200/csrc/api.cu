@@ -1,5 +1,6 @@
 // Host layer of the C ABI: argument validation, array sizes, layout derivation and
 // kernel dispatch.  No allocation, no synchronisation, no global state.
+#include <cmath>
 #include <cstring>
 
 #include "kvq_internal.cuh"
@@ -116,6 +117,10 @@ kvq_status kvq_format_check(const kvq_format* f) {
   if (f->rope != 0 && f->rope != 1) return KVQ_ERR_INVALID;
   if (f->rope && !(f->rope_base > 1.0f)) return KVQ_ERR_INVALID;
   if (f->rope && D < 64) return KVQ_ERR_UNSUPPORTED;
+  if (f->k_rotate != 0 && f->k_rotate != 1) return KVQ_ERR_INVALID;
+  if (f->k_rotate && (f->rope || (f->k_scheme != KVQ_SYM8 && f->k_scheme != KVQ_ASYM &&
+                                  f->k_scheme != KVQ_NUQ)))
+    return KVQ_ERR_UNSUPPORTED;
   kvq_status a = check_side(f, KVQ_KEYS);
   if (a == KVQ_ERR_INVALID) return a;
   kvq_status b = check_side(f, KVQ_VALUES);
@@ -178,6 +183,8 @@ kvq_status make_layout(const kvq_format* f, const kvq_cache* c, Layout* L) {
   L->res_cap = f->residual_cap;
   L->rope = f->rope;
   L->rope_base = f->rope_base;
+  L->k_rotate = f->k_rotate;
+  L->rot_scale = (float)(1.0 / std::sqrt((double)f->head_dim));
   L->mixed_hi = f->mixed_hi;
   L->mixed_mid = f->mixed_mid;
   L->mixed_lo = f->head_dim - f->mixed_hi - f->mixed_mid;

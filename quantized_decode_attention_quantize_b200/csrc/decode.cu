@@ -11,6 +11,7 @@
 #include <cmath>
 
 #include "decode_common.cuh"
+#include "wht.cuh"
 
 namespace kvq {
 
@@ -192,6 +193,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_generic_kernel(DecArgs a) 
       }
       st.q[hh][j] = x * a.qscale;
     }
+    // packed keys of a rotating format are in the Walsh-Hadamard basis: so is the query
+    if (L.k_rotate && split < a.n_packed) wht_strided<NC>(st.q[hh], lane, L.rot_scale);
   }
   double theta[NC / 2 > 0 ? NC / 2 : 1];
   if (L.rope) {

@@ -16,6 +16,7 @@
 #include <cmath>
 
 #include "decode_common.cuh"
+#include "wht.cuh"
 
 namespace kvq {
 
@@ -131,8 +132,15 @@ __global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_cc_kernel(CcA
       x = ld4(a.q, ((int64_t)b * a.Hq + h * G + hh) * D + 4 * lane, a.q_dtype);
       bad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
     }
-    q[hh][0] = x.x * a.qscale; q[hh][1] = x.y * a.qscale;
-    q[hh][2] = x.z * a.qscale; q[hh][3] = x.w * a.qscale;
+    float sc = a.qscale;
+    if (L.k_rotate && split < a.n_packed) {   // packed keys in the Walsh-Hadamard basis
+      float v[4] = {x.x, x.y, x.z, x.w};
+      wht128_quad_unscaled(v, lane);
+      x = make_float4(v[0], v[1], v[2], v[3]);
+      sc *= L.rot_scale;
+    }
+    q[hh][0] = x.x * sc; q[hh][1] = x.y * sc;
+    q[hh][2] = x.z * sc; q[hh][3] = x.w * sc;
 #pragma unroll
     for (int j = 0; j < 4; ++j) o[hh][j] = 0.0f;
     if (mixed && warp == 0)

@@ -49,6 +49,7 @@
 #include <cstdint>
 
 #include "kvq_internal.cuh"
+#include "wht.cuh"
 
 namespace kvq {
 
@@ -88,6 +89,8 @@ struct MmaArgs {
   const void* q;
   int q_dtype;
   float qscale;
+  int k_rotate;   // packed keys in the Walsh-Hadamard basis: their queries are rotated
+  float rot_scale;
   int nrp;        // raw positions per head (two per raw item)
   int rt;         // raw tokens per raw item
   int U;          // positions per head (nrp + packed halves)
@@ -765,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   KeyOp ko;
   int64_t head = i0 / U, cur_head = -1;
   int r = (int)(i0 - head * U);
-  bool qbad = false;
+  bool qbad = false, qload = true, qrot = false;
   int consumed = 0;
 #pragma unroll 1
   for (int64_t i = i0; i < i1; ++i) {
@@ -777,14 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
         state_reset(st);
       }
       cur_head = head;
-      // this head's queries, pre-scaled, for channels 4 lane .. 4 lane + 3
-#pragma unroll
-      for (int hh = 0; hh < GM; ++hh) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
-        qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
-        qv.set(hh, make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale));
-      }
+      qload = true;
     }
     if (r < a.nrp && (r & 1)) {   // second position of a raw item: no work
       if (++r == U) {
@@ -792,6 +788,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
         ++head;
       }
       continue;
+    }
+    // this head's queries, pre-scaled, for channels 4 lane .. 4 lane + 3; raw tokens use
+    // them as given, packed keys of a rotating format in the rotated basis (a head's raw
+    // items come before its packed ones, so a warp switches at most once per head)
+    const bool want_rot = a.k_rotate && r >= a.nrp;
+    if (qload || want_rot != qrot) {
+#pragma unroll
+      for (int hh = 0; hh < GM; ++hh) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
+        qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+        float sc = a.qscale;
+        if (want_rot) {
+          float v[4] = {x.x, x.y, x.z, x.w};
+          wht128_quad_unscaled(v, lane);
+          x = make_float4(v[0], v[1], v[2], v[3]);
+          sc *= a.rot_scale;
+        }
+        qv.set(hh, make_float4(x.x * sc, x.y * sc, x.z * sc, x.w * sc));
+      }
+      qload = false;
+      qrot = want_rot;
     }
     // the next item goes into the buffer consumed last time, then this one is waited
     // for: the warp's own copy of the next item overlaps its math on this one
@@ -977,6 +995,8 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.q = q;
   a.q_dtype = q_dtype;
   a.qscale = scale * kLog2e;
+  a.k_rotate = L.k_rotate;
+  a.rot_scale = L.rot_scale;
   a.nrp = p.raw_pieces;
   a.rt = p.split_groups;
   a.U = p.raw_pieces + p.n_packed_splits;

@@ -2,9 +2,11 @@
 //
 // One CTA per (32-token chunk, kv head, batch): the dense values are written into a
 // shared-memory tile (MIXED keys scatter slot -> channel through the group's order),
-// the chunk's sparse outliers overwrite their positions, and the tile is stored
+// the chunk's sparse outliers overwrite their positions, keys of a rotating format are
+// transformed back to the original basis, and the tile is stored
 // coalesced in the output dtype (fp32 exact, 16-bit by round-to-nearest-even).
 #include "decode_common.cuh"
+#include "wht.cuh"
 
 namespace kvq {
 namespace {
@@ -59,6 +61,10 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DqArgs a) {
         }
       }
     }
+    __syncthreads();
+  }
+  if (a.which == KVQ_KEYS && L.k_rotate) {   // back from the rotated basis (own inverse)
+    wht_tile_rows(tile, nt, D, L.rot_scale);
     __syncthreads();
   }
   const int64_t obase = (sl * a.n + (tb - a.t0)) * D;

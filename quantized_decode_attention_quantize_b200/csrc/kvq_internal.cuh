@@ -32,6 +32,8 @@ struct Layout {
   int ng;                    // C / g
   int n_sink, res_cap, rope;
   float rope_base;
+  int k_rotate;              // keys stored in the Walsh-Hadamard basis
+  float rot_scale;           // fl32(1 / sqrt(D))
   int mixed_hi, mixed_mid, mixed_lo, mixed_group_bytes;
   Side side[2];
   uint8_t* k_order;

@@ -1,7 +1,8 @@
 // Append-time quantization of K / V token groups into the packed cache.
 //
 // One CTA per (token group, kv head, batch).  The group's n <= g rows of D source
-// values are staged in shared memory as fp32 (128-bit coalesced loads), the group
+// values are staged in shared memory as fp32 (128-bit coalesced loads; key rows of a
+// rotating format are then Walsh-Hadamard transformed in place), the group
 // statistics are reduced (per-channel min/max or absmax by column threads, per-token
 // by warp shuffles), metadata are rounded as the format states, and codes are
 // encoded and packed into 32-bit words that are stored coalesced.
@@ -11,6 +12,7 @@
 // with per-vector dense-and-sparse outliers); [MIX] Figure 3 (salience tiers);
 // [K4V2] (more bits for keys than values).
 #include "kvq_internal.cuh"
+#include "wht.cuh"
 
 namespace kvq {
 namespace {
@@ -571,6 +573,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(QArgs a) {
   const int gi = (int)(ts / g);
   load_tile(a, ln, ts - a.t0, sm.tile, sm.flag);
   __syncthreads();
+  if (a.which == KVQ_KEYS && L.k_rotate) {   // statistics and codes in the rotated basis
+    wht_tile_rows(sm.tile, ln, D, L.rot_scale);
+    __syncthreads();
+  }
   const Side& S = L.side[a.which];
   switch (S.scheme) {
     case KVQ_NONE: {

@@ -317,7 +317,8 @@ __global__ void __launch_bounds__(kThreads) asym_kv_kernel(AArgs ak, AArgs av, i
 bool asym_fast_ok(const Layout& L, int which) {
   const Side& S = L.side[which];
   if (S.scheme != KVQ_ASYM) return false;
-  if (which == KVQ_KEYS) return S.axis == KVQ_AXIS_CHANNEL && L.g <= 64 * kMaxKeyRows && L.D % kCB == 0;
+  if (which == KVQ_KEYS)   // a rotating format needs whole rows: the general kernel
+    return !L.k_rotate && S.axis == KVQ_AXIS_CHANNEL && L.g <= 64 * kMaxKeyRows && L.D % kCB == 0;
   return S.axis == KVQ_AXIS_TOKEN && L.D >= 32 && L.D <= 256;
 }
 

@@ -40,7 +40,8 @@ class kvq_format(ctypes.Structure):
         "head_dim", "group_tokens", "src_dtype",
         "k_scheme", "k_bits", "k_axis", "k_outliers",
         "v_scheme", "v_bits", "v_axis", "v_outliers",
-        "mixed_hi", "mixed_mid", "n_sink", "residual_cap", "rope")] + [("rope_base", ctypes.c_float)]
+        "mixed_hi", "mixed_mid", "n_sink", "residual_cap", "rope")] + [("rope_base", ctypes.c_float),
+                                                                ("k_rotate", ctypes.c_int32)]
 
 
 class kvq_cache(ctypes.Structure):
@@ -116,7 +117,7 @@ def _stream(stream):
 def make_format(d: dict) -> kvq_format:
     f = kvq_format()
     for name, _ in kvq_format._fields_:
-        setattr(f, name, d[name])
+        setattr(f, name, d.get(name, 0) if name == "k_rotate" else d[name])
     return f
 
 

@@ -79,6 +79,13 @@ def _fmt(**kw):
     (dict(k_scheme=kvq.NUQ, k_bits=3, k_outliers=9), kvq.KVQ_ERR_INVALID),
     (dict(rope=1, rope_base=0.5), kvq.KVQ_ERR_INVALID),
     (dict(head_dim=32, group_tokens=64, rope=1), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(k_rotate=2), kvq.KVQ_ERR_INVALID),
+    (dict(k_rotate=1, rope=1), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(k_rotate=1, k_scheme=kvq.MIXED, mixed_hi=8, mixed_mid=24), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(k_rotate=1, k_scheme=kvq.NONE, k_bits=0), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(k_rotate=1), kvq.KVQ_OK),
+    (dict(k_rotate=1, k_scheme=kvq.NUQ, k_bits=3, k_outliers=2), kvq.KVQ_OK),
+    (dict(k_rotate=1, k_scheme=kvq.SYM8, k_bits=8, k_axis=kvq.TOKEN), kvq.KVQ_OK),
     (dict(), kvq.KVQ_OK),
 ])
 def test_format_check(kw, want):
