@@ -717,8 +717,15 @@ __device__ __forceinline__ void combine_row(const float* m, const float* l, cons
   }
 }
 
+// Four query channels 4 lane .. 4 lane + 3 taken into the Walsh-Hadamard basis of the keys.
+__device__ __forceinline__ float4 rotate_q(float4 x, int lane, float c) {
+  float v[4] = {x.x, x.y, x.z, x.w};
+  wht128_quad_unscaled(v, lane);
+  return make_float4(v[0] * c, v[1] * c, v[2] * c, v[3] * c);
+}
+
 // ---- the kernel --------------------------------------------------------------------------
-template <bool DUAL>
+template <bool DUAL, bool ROT>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int GM = DUAL ? 4 : 8;
@@ -768,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   KeyOp ko;
   int64_t head = i0 / U, cur_head = -1;
   int r = (int)(i0 - head * U);
-  bool qbad = false, qload = true, qrot = false;
+  bool qbad = false, qrot = false;
   int consumed = 0;
 #pragma unroll 1
   for (int64_t i = i0; i < i1; ++i) {
@@ -780,7 +787,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
         state_reset(st);
       }
       cur_head = head;
-      qload = true;
+      if constexpr (ROT) qrot = r >= a.nrp;
+      // this head's queries, pre-scaled, for channels 4 lane .. 4 lane + 3 (as given for
+      // raw tokens; in the Walsh-Hadamard basis for the packed keys of a rotating format)
+#pragma unroll
+      for (int hh = 0; hh < GM; ++hh) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
+        qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+        if constexpr (ROT) {
+          if (qrot) x = rotate_q(x, lane, a.rot_scale);
+        }
+        qv.set(hh, make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale));
+      }
     }
     if (r < a.nrp && (r & 1)) {   // second position of a raw item: no work
       if (++r == U) {
@@ -789,27 +808,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
       }
       continue;
     }
-    // this head's queries, pre-scaled, for channels 4 lane .. 4 lane + 3; raw tokens use
-    // them as given, packed keys of a rotating format in the rotated basis (a head's raw
-    // items come before its packed ones, so a warp switches at most once per head)
-    const bool want_rot = a.k_rotate && r >= a.nrp;
-    if (qload || want_rot != qrot) {
+    if constexpr (ROT) {   // a head's raw items come first: at most one switch per head
+      if (r >= a.nrp && !qrot) {
+        qrot = true;
 #pragma unroll
-      for (int hh = 0; hh < GM; ++hh) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
-        qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
-        float sc = a.qscale;
-        if (want_rot) {
-          float v[4] = {x.x, x.y, x.z, x.w};
-          wht128_quad_unscaled(v, lane);
-          x = make_float4(v[0], v[1], v[2], v[3]);
-          sc *= a.rot_scale;
+        for (int hh = 0; hh < GM; ++hh) {
+          float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (hh < a.G) x = load4(a.q, (head * a.G + hh) * 128 + 4 * lane, a.q_dtype);
+          x = rotate_q(x, lane, a.rot_scale);
+          qv.set(hh, make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale));
         }
-        qv.set(hh, make_float4(x.x * sc, x.y * sc, x.z * sc, x.w * sc));
       }
-      qload = false;
-      qrot = want_rot;
     }
     // the next item goes into the buffer consumed last time, then this one is waited
     // for: the warp's own copy of the next item overlaps its math on this one
@@ -1008,7 +1017,8 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.ws_o = ws_o;
   a.status = d_status;
   const size_t smem = mma_smem();
-  auto kern = a.G <= 4 ? decode_mma_kernel<true> : decode_mma_kernel<false>;
+  auto kern = a.G <= 4 ? (a.k_rotate ? decode_mma_kernel<true, true> : decode_mma_kernel<true, false>)
+                       : (a.k_rotate ? decode_mma_kernel<false, true> : decode_mma_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<p.grid_ctas, kThreads, smem, s>>>(a);

@@ -6,6 +6,7 @@
 // trip.  Keys: a CTA takes 32 channels of one group (the statistics of a channel never
 // leave it); values: a CTA takes 32 tokens.
 #include "kvq_internal.cuh"
+#include "wht.cuh"
 
 namespace kvq {
 namespace {
@@ -291,6 +292,154 @@ __device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by
     flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
 }
 
+// Keys of a rotating format (D = 128, g <= 128): a CTA takes one whole group, since the
+// Walsh-Hadamard transform mixes all channels of a row.  Warp w holds rows w, w + 8, ...
+// (16 at most); lane l holds channels 4 l .. 4 l + 3 of each, loaded as one 8-byte (16-bit
+// source) or 16-byte (fp32) vector.  Rows are transformed in registers (strides 1, 2 in
+// the lane, 4 .. 64 across lanes, then the product with fl32(1/sqrt(D))), the per-channel
+// min / max go through shared memory across the 8 warps, and the codes of four channels
+// are packed by the lane and merged with its neighbours' by shuffles into row words.
+constexpr int kRotRows = 16;
+__device__ __forceinline__ void asym_keys_rot_block(const AArgs& a, int bx, int head) {
+  __shared__ float pmin[8][128], pmax[8][128];
+  __shared__ float sf[128], zf[128];
+  __shared__ int flags;
+  const Layout& L = a.L;
+  const Side& S = L.side[KVQ_KEYS];
+  const int g = L.g, bits = S.bits;
+  const int64_t ts = a.t0 + (int64_t)bx * g;
+  const int ln = (int)min((int64_t)g, a.t0 + a.n - ts);
+  const int gi = (int)(ts / g);
+  const int b = head / L.Hkv, h = head % L.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) flags = 0;
+  float x[kRotRows][4];
+  const int64_t base = (int64_t)b * a.sb + (int64_t)h * a.sh + (ts - a.t0) * a.st + 4 * lane;
+#pragma unroll
+  for (int k = 0; k < kRotRows; ++k) {
+    const int r = warp + 8 * k;
+    if (r < ln) {
+      const int64_t i = base + r * a.st;
+      if (L.src_dtype == KVQ_F32) {
+        const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.src) + i);
+        x[k][0] = v.x; x[k][1] = v.y; x[k][2] = v.z; x[k][3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.src) + i);
+        const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (L.src_dtype == KVQ_F16) {
+            x[k][2 * j] = half_bits_to_float((uint16_t)(w[j] & 0xffffu));
+            x[k][2 * j + 1] = half_bits_to_float((uint16_t)(w[j] >> 16));
+          } else {
+            x[k][2 * j] = __uint_as_float(w[j] << 16);
+            x[k][2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+          }
+        }
+      }
+    } else {
+      x[k][0] = x[k][1] = x[k][2] = x[k][3] = 0.0f;
+    }
+  }
+  int bad = 0;
+  float mn[4], mx[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    mn[j] = INFINITY;
+    mx[j] = -INFINITY;
+  }
+#pragma unroll
+  for (int k = 0; k < kRotRows; ++k) {
+    if (warp + 8 * k < ln) {   // warp-uniform: the shuffles of the transform see all lanes
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bad |= !isfinite(x[k][j]);
+      wht128_quad_unscaled(x[k], lane);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[k][j] = __fmul_rn(x[k][j], L.rot_scale);
+        mn[j] = fminf(mn[j], x[k][j]);
+        mx[j] = fmaxf(mx[j], x[k][j]);
+      }
+    }
+  }
+  __syncthreads();   // flags initialised
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    pmin[warp][4 * lane + j] = mn[j];
+    pmax[warp][4 * lane + j] = mx[j];
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&flags, 1);
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    const int c = threadIdx.x;
+    float m0 = pmin[0][c], m1 = pmax[0][c];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) {
+      m0 = fminf(m0, pmin[w][c]);
+      m1 = fmaxf(m1, pmax[w][c]);
+    }
+    __half sh, zh;
+    if (!asym_params(m0, m1, bits, &sh, &zh)) atomicOr(&flags, 2);
+    const int64_t mi = ((int64_t)head * L.ng + gi) * 128 + c;
+    reinterpret_cast<__half*>(S.scale)[mi] = sh;
+    reinterpret_cast<__half*>(S.zero)[mi] = zh;
+    sf[c] = __half2float(sh);
+    zf[c] = __half2float(zh);
+  }
+  __syncthreads();
+  float s4[4], z4[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    s4[j] = sf[4 * lane + j];
+    z4[j] = zf[4 * lane + j];
+  }
+  const int maxc = (1 << bits) - 1;
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
+  const int rowb = 128 * bits / 8;
+#pragma unroll
+  for (int k = 0; k < kRotRows; ++k) {
+    const int r = warp + 8 * k;
+    if (r < ln) {   // warp-uniform
+      uint32_t v = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v |= (uint32_t)asym_code(x[k][j], s4[j], z4[j], maxc) << (bits * j);
+      uint8_t* row = codes + (ts + r) * rowb;
+      if (bits == 8) {
+        *reinterpret_cast<uint32_t*>(row + 4 * lane) = v;
+      } else if (bits == 4) {   // word lane / 2: this lane's 16 bits at 16 (lane & 1)
+        v <<= 16 * (lane & 1);
+        v |= __shfl_xor_sync(0xffffffffu, v, 1);
+        if ((lane & 1) == 0) reinterpret_cast<uint32_t*>(row)[lane >> 1] = v;
+      } else {                  // 2-bit: word lane / 4, this lane's 8 bits at 8 (lane & 3)
+        v <<= 8 * (lane & 3);
+        v |= __shfl_xor_sync(0xffffffffu, v, 1);
+        v |= __shfl_xor_sync(0xffffffffu, v, 2);
+        if ((lane & 3) == 0) reinterpret_cast<uint32_t*>(row)[lane >> 2] = v;
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && flags)
+    flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
+}
+
+__global__ void __launch_bounds__(kThreads) asym_keys_rot_kernel(AArgs a) {
+  asym_keys_rot_block(a, blockIdx.x, blockIdx.y);
+}
+
+// A rotating format's append in one launch: blocks [0, nk) take one key group each
+// (group, head), the rest are value blocks.
+__global__ void __launch_bounds__(kThreads) asym_kv_rot_kernel(AArgs ak, AArgs av, int kgx, int nk,
+                                                               int vgx) {
+  const int b = blockIdx.x;
+  if (b < nk) {
+    asym_keys_rot_block(ak, b % kgx, b / kgx);
+  } else {
+    const int v = b - nk;
+    asym_values_block(av, v % vgx, v / vgx);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
   asym_keys_block(a, blockIdx.x, blockIdx.y, blockIdx.z);
 }
@@ -317,8 +466,11 @@ __global__ void __launch_bounds__(kThreads) asym_kv_kernel(AArgs ak, AArgs av, i
 bool asym_fast_ok(const Layout& L, int which) {
   const Side& S = L.side[which];
   if (S.scheme != KVQ_ASYM) return false;
-  if (which == KVQ_KEYS)   // a rotating format needs whole rows: the general kernel
-    return !L.k_rotate && S.axis == KVQ_AXIS_CHANNEL && L.g <= 64 * kMaxKeyRows && L.D % kCB == 0;
+  if (which == KVQ_KEYS) {
+    if (S.axis != KVQ_AXIS_CHANNEL) return false;
+    if (L.k_rotate) return L.D == 128 && L.g <= 8 * kRotRows;   // whole rows per CTA
+    return L.g <= 64 * kMaxKeyRows && L.D % kCB == 0;
+  }
   return S.axis == KVQ_AXIS_TOKEN && L.D >= 32 && L.D <= 256;
 }
 
@@ -333,7 +485,10 @@ cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, in
   a.t0 = t0;
   a.n = n;
   a.status = d_status;
-  if (which == KVQ_KEYS) {
+  if (which == KVQ_KEYS && L.k_rotate) {
+    dim3 grid((unsigned)((n + L.g - 1) / L.g), L.B * L.Hkv);
+    asym_keys_rot_kernel<<<grid, kThreads, 0, s>>>(a);
+  } else if (which == KVQ_KEYS) {
     dim3 grid((unsigned)((n + L.g - 1) / L.g), L.D / kCB, L.B * L.Hkv);
     asym_keys_kernel<<<grid, kThreads, 0, s>>>(a);
   } else {
@@ -360,11 +515,14 @@ cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const voi
   ak.t0 = av.t0 = t0;
   ak.n = av.n = n;
   ak.status = av.status = d_status;
-  const int kgx = (int)((n + L.g - 1) / L.g), kgy = L.D / kCB, heads = L.B * L.Hkv;
+  const int kgx = (int)((n + L.g - 1) / L.g), kgy = L.k_rotate ? 1 : L.D / kCB, heads = L.B * L.Hkv;
   const int vgx = (int)((n + kTB - 1) / kTB);
   const int64_t nk = (int64_t)kgx * kgy * heads, nv = (int64_t)vgx * heads;
   if (nk + nv > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  asym_kv_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, kgy, (int)nk, vgx);
+  if (L.k_rotate)
+    asym_kv_rot_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, (int)nk, vgx);
+  else
+    asym_kv_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, kgy, (int)nk, vgx);
   return cudaGetLastError();
 }
 

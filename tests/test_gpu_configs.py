@@ -32,6 +32,7 @@ CASES = [
     ("llama3_8b", [(0, 0), (3, 5), (7, 7)]),
     ("mixkvq_14b", [(0, 0), (15, 7)]),
     ("kvquant_nuq3", [(0, 17)]),
+    ("llama3_8b_wht", [(0, 0), (7, 7)]),
 ]
 
 

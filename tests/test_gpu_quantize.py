@@ -212,6 +212,8 @@ def test_none_scheme_copies_raw():
     dict(src_dtype=BF16),                                              # K4/V2: one fused launch
     dict(src_dtype=F16, k_bits=2, v_bits=4),
     dict(src_dtype=BF16, k_scheme=NUQ, k_bits=3, k_outliers=2, v_scheme=NUQ, v_bits=3, v_outliers=2),
+    dict(src_dtype=BF16, k_rotate=1),                                  # rotated keys: fused launch
+    dict(src_dtype=F32, k_bits=8, k_rotate=1),
 ])
 def test_quantize_kv_matches_separate_calls_and_oracle(fd):
     # kvq_quantize_kv = kvq_quantize_keys then kvq_quantize_values, bit for bit

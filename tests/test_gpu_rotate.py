@@ -43,6 +43,19 @@ def test_rotated_keys_quantize_and_dequantize(dt, kw):
     deq_check(p, VALUES, 0, n)
 
 
+@pytest.mark.parametrize("g,kb", [(16, 4), (64, 2), (112, 8)])
+def test_rotated_keys_group_sizes_and_partial_rewrite(g, kb):
+    # the whole-group register kernel at g < 128, a partial last group, then its rewrite
+    B, H, D = 2, 2, 128
+    p = Pair(synth._fmt(head_dim=D, group_tokens=g, src_dtype=BF16, k_bits=kb, k_rotate=1), B, H, 4 * g)
+    K = values(7, (B, H, 4 * g, D), BF16, 2.0, outlier_cols=3)
+    p.quantize(KEYS, K[:, :, :g + 5], 0, g + 5)
+    p.assert_arrays_equal()
+    p.quantize(KEYS, K[:, :, g:3 * g + 1], g, 2 * g + 1)
+    p.assert_arrays_equal()
+    deq_check(p, KEYS, 0, 3 * g + 1)
+
+
 @pytest.mark.parametrize("D,g", [(32, 16), (64, 48), (256, 128)])
 def test_rotated_keys_other_head_dims(D, g):
     B, H, n = 1, 2, 5 * g - 3
