@@ -105,9 +105,9 @@ def is_k4v2(cfg):
 
 
 def fused_kv(cfg):
-    """kvq_quantize_kv is one launch for K4/V2 without key rotation (rotated keys need whole
-    rows and take the general quantize kernel)."""
-    return is_k4v2(cfg) and not cfg["fmt"].get("k_rotate", 0)
+    """kvq_quantize_kv is one launch for K4/V2 (with rotated keys too, at D = 128, g <= 128)."""
+    f = cfg["fmt"]
+    return is_k4v2(cfg) and (not f.get("k_rotate", 0) or (f["head_dim"] == 128 and f["group_tokens"] <= 128))
 
 
 def cache_read_bytes(cache, cfg, tq, tr):
