@@ -37,7 +37,7 @@ METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize 
 L2_FLUSH_BYTES = 512 << 20
 LAUNCHES_PER_STEP = 3   # quantize K+V (one launch on the K4/V2 path), split kernel, combine
 PATH_DTYPE = {
-    "decode_mma_kernel": "f16 tensor-core products with f32 accumulation (u4/u2 codes)",
+    "decode_mma_kernel": "f16 tensor-core products with f32 accumulation (u4/u2 codes; bf16 raw key slots)",
     "decode_cc_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
     "decode_generic_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
 }
@@ -47,7 +47,9 @@ def decode_path(cfg):
     """The split kernel the library plans for this workload (same rules as its planner)."""
     f = cfg["fmt"]
     G = cfg["Hq"] // cfg["Hkv"]
-    if is_k4v2(cfg) and f["head_dim"] == 128 and f["group_tokens"] == 128 and 1 <= G <= 8:
+    mix = f["k_scheme"] == synth.MIXED and f["mixed_hi"] == 8 and f["mixed_mid"] == 24 and \
+        f["src_dtype"] == synth.BF16 and f["v_scheme"] == synth.ASYM and f["v_bits"] == 2 and not f["rope"]
+    if (is_k4v2(cfg) or mix) and f["head_dim"] == 128 and f["group_tokens"] == 128 and 1 <= G <= 8:
         return "decode_mma_kernel"
     k_ok = (f["k_scheme"] == synth.NUQ) or (f["k_scheme"] == synth.ASYM and f["k_bits"] in (2, 4)) or \
         (f["k_scheme"] == synth.MIXED and not f["rope"])

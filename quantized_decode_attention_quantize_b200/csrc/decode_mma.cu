@@ -66,6 +66,12 @@ constexpr int kRawBytes = 2048;               // raw item: key rows, then value 
 constexpr int kScratchBytes = 2 * 32 * 16 * 4;  // per warp: hi and lo B fragments
 constexpr int kRecordFloats = 8 * 130;        // merge record: o[G][128], m[G], l[G]
 constexpr float kLog2e = 1.4426950408889634f;
+// MIXED keys (8 raw bf16 / 24 4-bit / 96 2-bit slots per token) in the key region of a
+// half stage: raw plane [64][8] bf16, 4-bit plane [64][3] words, 2-bit plane [64][6]
+// words, then the group's slot order [128]; slot scale / zero-point [120] each in the
+// key-metadata region (zero-points at +256 bytes).
+constexpr int kMixRaw = 0, kMixMid = 64 * 16, kMixLo = kMixMid + 64 * 12, kMixOrd = kMixLo + 64 * 24;
+static_assert(kMixOrd + 128 <= kHalfK, "mixed key planes fit the key region");
 static_assert(2 * kRawBytes <= kStageBytes, "raw item fits a stage");
 static_assert(kRecordFloats * 4 <= kBuffers * kStageBytes, "record fits the warp's ring");
 
@@ -86,6 +92,8 @@ struct MmaArgs {
   const void* sink_v;
   const void* res_k;
   const void* res_v;
+  const uint8_t* k_order;   // MIXED keys: slot -> channel per group
+  int64_t k_group_bytes;    // MIXED keys: bytes of one group's three planes
   const void* q;
   int q_dtype;
   float qscale;
@@ -146,6 +154,14 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
                                          uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816_bf16(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -342,10 +358,15 @@ __device__ void raw_item(MmaState& st, const uint8_t* stg, int nt, int dtype, co
 }
 
 // The key-product B operand of one group (per lane), its exponent and bias.
-struct KeyOp {
-  uint32_t bh[8][2], bl[8][2];
+// The key-product B operand of a group: k-steps of high (bh) and, without DUAL, low (bl)
+// fp16 parts; MIXED adds two k-steps for the 4-bit slots and one bf16 k-step for the raw
+// slots (eight 2-bit k-steps, two 4-bit, one raw).
+template <bool MIX>
+struct KeyOpT {
+  uint32_t bh[MIX ? 11 : 8][2], bl[MIX ? 11 : 8][2];
   float mult, bias0, bias1;
 };
+using KeyOp = KeyOpT<false>;
 
 // The head's pre-scaled queries, channels 4 lane .. 4 lane + 3 of head hh: with DUAL in
 // the upper half of the warp's scratch (shared memory), otherwise in registers.
@@ -502,10 +523,210 @@ __device__ __forceinline__ void key_operand(const MmaArgs& a, const __half* ks, 
   __syncwarp();
 }
 
+// Per-head sums dz[hh] over the warp, delivered as the biases of the lane's columns
+// (heads 2j, 2j + 1; with DUAL heads 2 (j & 1), 2 (j & 1) + 1).
+template <bool DUAL, int GM>
+__device__ __forceinline__ void head_sums(const float (&dz)[GM], float* b0, float* b1) {
+  const int lane = threadIdx.x & 31, j = lane & 3;
+  const int h0 = DUAL ? 2 * (j & 1) : 2 * j, h1 = h0 + 1;
+  const bool u4 = lane & 16, u3 = lane & 8, u2 = lane & 4;
+  if constexpr (GM == 4) {
+    float v2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float send = u4 ? dz[k] : dz[k + 2];
+      const float keep = u4 ? dz[k + 2] : dz[k];
+      v2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float v3 = (u3 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, u3 ? v2[0] : v2[1], 8);
+    v3 += __shfl_xor_sync(0xffffffffu, v3, 4);
+    v3 += __shfl_xor_sync(0xffffffffu, v3, 2);
+    v3 += __shfl_xor_sync(0xffffffffu, v3, 1);
+    *b0 = __shfl_sync(0xffffffffu, v3, 16 * ((h0 >> 1) & 1) + 8 * (h0 & 1));
+    *b1 = __shfl_sync(0xffffffffu, v3, 16 * ((h1 >> 1) & 1) + 8 * (h1 & 1));
+  } else {
+    float v2[4], v3[2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float send = u4 ? dz[k] : dz[k + 4];
+      const float keep = u4 ? dz[k + 4] : dz[k];
+      v2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float send = u3 ? v2[k] : v2[k + 2];
+      const float keep = u3 ? v2[k + 2] : v2[k];
+      v3[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float v4 = (u2 ? v3[1] : v3[0]) + __shfl_xor_sync(0xffffffffu, u2 ? v3[0] : v3[1], 4);
+    v4 += __shfl_xor_sync(0xffffffffu, v4, 2);
+    v4 += __shfl_xor_sync(0xffffffffu, v4, 1);
+    *b0 = __shfl_sync(0xffffffffu, v4, ((h0 >> 2) & 1) * 16 + ((h0 >> 1) & 1) * 8 + (h0 & 1) * 4);
+    *b1 = __shfl_sync(0xffffffffu, v4, ((h1 >> 2) & 1) * 16 + ((h1 >> 1) & 1) * 8 + (h1 & 1) * 4);
+  }
+}
+
+__device__ __forceinline__ void split_half2(float x0, float x1, uint32_t* hi, uint32_t* lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - f.x, x1 - f.y);
+  *hi = *reinterpret_cast<const uint32_t*>(&h);
+  *lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+__device__ __forceinline__ void split_bf162(float x0, float x1, uint32_t* hi, uint32_t* lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 f = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - f.x, x1 - f.y);
+  *hi = *reinterpret_cast<const uint32_t*>(&h);
+  *lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// MIXED keys ([MIX] Figure 3 tiers: 8 raw, 24 4-bit, 96 2-bit slots in salience order).
+// The score of token t is sum_s B[s] A[t][s] over slots: A holds the codes as fp16
+// subnormals in place (2-bit field f of a word: factor 4^f; 4-bit nibble: 1 or 16) and
+// the raw slots as bf16; B[s] = q[order[s]] s_s 2^(24 - e) / factor for coded slots and
+// q[order[s]] for raw ones; sum_s q[order[s]] z_s is the bias.  Lane (g, j) builds its
+// own fragments (head g, or with DUAL the low part of head g - 4 for g >= 4) from the
+// slot products that the warp first writes to its scratch in slot order.
+//
+// k-steps of lane j: 2-bit slots, k-step 4 sg + qq: word w = 4 sg + j of the 2-bit
+// plane (none when w >= 6), registers 2 qq and 2 qq + 1 of the word, register r being
+// (r < 4 ? x : odd_bytes_down(x)) & (0x00030003 << 2 (r & 3)), whose low / high halves
+// hold slots (r < 4 ? 0 : 4) + (r & 3) and that + 8 of the word; 4-bit slots, k-step
+// 8 + qq: word j of the 4-bit plane (none for j = 3), registers 2 qq, 2 qq + 1, register r
+// being (r < 2 ? x : odd(x)) & (r even ? 0x000F000F : 0x00F000F0) with slots r, r + 4;
+// raw slots, k-step 10 (bf16): word j of the raw plane = slots 2 j, 2 j + 1, the upper
+// eight k-columns empty.
+template <bool DUAL, int GM>
+__device__ __forceinline__ void key_operand_mixed(const MmaArgs& a, const uint8_t* stage, uint32_t* scratch,
+                                                  const QVec<DUAL, GM>& qv, KeyOpT<true>& ko) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
+  const int G = a.G;
+  const uint8_t* ord = stage + kMixOrd;
+  const __half* ks = reinterpret_cast<const __half*>(stage + kHalfK + kHalfV + kHalfVM);
+  const __half* kz = ks + 128;
+  float* av = reinterpret_cast<float*>(scratch);   // [GM][128] slot products, slot order
+  int ch[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ch[i] = ord[4 * lane + i] & 127;   // a channel of the head
+  float qs[GM][4];
+  if constexpr (DUAL) {
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qs[hh][i] = qv.s[hh * 128 + ch[i]];
+  } else {   // the queries live in registers by channel: go through the scratch once
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh) *reinterpret_cast<float4*>(av + hh * 128 + 4 * lane) = qv.get(hh);
+    __syncwarp();
+#pragma unroll
+    for (int hh = 0; hh < GM; ++hh)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qs[hh][i] = av[hh * 128 + ch[i]];
+    __syncwarp();
+  }
+  float sv[4], zv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int sl = 4 * lane + i;
+    sv[i] = sl >= 8 ? __half2float(ks[sl - 8]) : 0.0f;
+    zv[i] = sl >= 8 ? __half2float(kz[sl - 8]) : 0.0f;
+  }
+  float dz[GM];
+  float amax = 0.0f;
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh) {
+    dz[hh] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float x = qs[hh][i] * sv[i];
+      dz[hh] = fmaf(qs[hh][i], zv[i], dz[hh]);
+      amax = fmaxf(amax, fabsf(x));
+      if (lane >= 2) qs[hh][i] = x;   // lanes 0, 1 hold the raw slots 0..7: keep q
+    }
+  }
+  amax = warp_max(amax);
+  int ex = 0;
+  if (amax > 0.0f) ex = (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 + 10;
+  ex = max(-100, min(127, ex));
+  ko.mult = pow2(ex);
+  const float sc = lane >= 2 ? __uint_as_float((uint32_t)max(1, min(254, 127 + 24 - ex)) << 23) : 1.0f;
+#pragma unroll
+  for (int hh = 0; hh < GM; ++hh)
+    *reinterpret_cast<float4*>(av + hh * 128 + 4 * lane) =
+        make_float4(qs[hh][0] * sc, qs[hh][1] * sc, qs[hh][2] * sc, qs[hh][3] * sc);
+  head_sums<DUAL, GM>(dz, &ko.bias0, &ko.bias1);
+  __syncwarp();
+  const int hd = DUAL ? (g & 3) : g;
+  const bool live = hd < G;
+  const bool low_lane = DUAL && g >= 4;   // columns 4..7 carry the low parts
+  const float* ah = av + (live ? hd : 0) * 128;
+  auto put = [&](int k, float v0, float v1, float v2, float v3) {
+    uint32_t h0, l0, h1, l1;
+    split_half2(v0, v1, &h0, &l0);
+    split_half2(v2, v3, &h1, &l1);
+    if (DUAL) {
+      ko.bh[k][0] = low_lane ? l0 : h0;
+      ko.bh[k][1] = low_lane ? l1 : h1;
+    } else {
+      ko.bh[k][0] = h0; ko.bh[k][1] = h1;
+      ko.bl[k][0] = l0; ko.bl[k][1] = l1;
+    }
+  };
+  // 2-bit slots 32 + 16 w + p
+#pragma unroll
+  for (int sg = 0; sg < 2; ++sg) {
+    const int w = 4 * sg + j;
+    const bool ok = live && w < 6;
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = 2 * qq + e, f = r & 3;
+        const int p = (r < 4 ? 0 : 4) + f;
+        const float inv = f == 0 ? 1.0f : f == 1 ? 0.25f : f == 2 ? 0.0625f : 0.015625f;
+        v[2 * e] = ok ? ah[32 + 16 * w + p] * inv : 0.0f;
+        v[2 * e + 1] = ok ? ah[32 + 16 * w + p + 8] * inv : 0.0f;
+      }
+      put(4 * sg + qq, v[0], v[1], v[2], v[3]);
+    }
+  }
+  // 4-bit slots 8 + 8 w + p
+  {
+    const bool ok = live && j < 3;
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = 2 * qq + e;
+        const float inv = (r & 1) ? 0.0625f : 1.0f;
+        v[2 * e] = ok ? ah[8 + 8 * j + r] * inv : 0.0f;
+        v[2 * e + 1] = ok ? ah[8 + 8 * j + r + 4] * inv : 0.0f;
+      }
+      put(8 + qq, v[0], v[1], v[2], v[3]);
+    }
+  }
+  // raw slots 2 j, 2 j + 1 (bf16)
+  {
+    uint32_t h0, l0;
+    split_bf162(live ? ah[2 * j] : 0.0f, live ? ah[2 * j + 1] : 0.0f, &h0, &l0);
+    if (DUAL) {
+      ko.bh[10][0] = low_lane ? l0 : h0;
+      ko.bh[10][1] = 0u;
+    } else {
+      ko.bh[10][0] = h0; ko.bh[10][1] = 0u;
+      ko.bl[10][0] = l0; ko.bl[10][1] = 0u;
+    }
+  }
+  __syncwarp();
+}
+
 // 64 tokens (one half of a group) held in a ring stage: key codes [64][16] words,
 // value codes [32 pairs][16] words, value scale / zero-point [64] each.
-template <bool DUAL>
-__device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, const KeyOp& ko,
+template <bool DUAL, bool MIX>
+__device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, const KeyOpT<MIX>& ko,
                                          int tvalid) {
   const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
   const uint32_t* kc = reinterpret_cast<const uint32_t*>(stage);
@@ -517,6 +738,55 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
   // all four tiles' code words first, then the k-steps tile by tile so that consecutive
   // products go to different accumulators
   float S[4][4];
+  float Sr[MIX ? 4 : 1][4];   // MIXED: raw-slot products, already in score units
+  if constexpr (MIX) {
+    // per tile: the 2-bit words 4 sg + j, the 4-bit word j and the raw word j of rows
+    // g and g + 8 (k-step layout in key_operand_mixed)
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      S[mt][0] = S[mt][1] = S[mt][2] = S[mt][3] = 0.0f;
+      Sr[mt][0] = Sr[mt][1] = Sr[mt][2] = Sr[mt][3] = 0.0f;
+      const int r0 = 16 * mt + g, r1 = r0 + 8;
+#pragma unroll
+      for (int sg = 0; sg < 2; ++sg) {
+        const int w = 4 * sg + j;
+        uint32_t x0 = 0u, x1 = 0u;
+        if (w < 6) {
+          x0 = *reinterpret_cast<const uint32_t*>(stage + kMixLo + r0 * 24 + 4 * w);
+          x1 = *reinterpret_cast<const uint32_t*>(stage + kMixLo + r1 * 24 + 4 * w);
+        }
+        const uint32_t y0 = odd_bytes_down(x0), y1 = odd_bytes_down(x1);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint32_t s0 = qq < 2 ? x0 : y0, s1 = qq < 2 ? x1 : y1;
+          const uint32_t ma = 0x00030003u << (2 * ((2 * qq) & 3)), mb = 0x00030003u << (2 * ((2 * qq + 1) & 3));
+          mma16816(S[mt], s0 & ma, s1 & ma, s0 & mb, s1 & mb, ko.bh[4 * sg + qq][0], ko.bh[4 * sg + qq][1]);
+          if (!DUAL)
+            mma16816(S[mt], s0 & ma, s1 & ma, s0 & mb, s1 & mb, ko.bl[4 * sg + qq][0], ko.bl[4 * sg + qq][1]);
+        }
+      }
+      {
+        uint32_t x0 = 0u, x1 = 0u;
+        if (j < 3) {
+          x0 = *reinterpret_cast<const uint32_t*>(stage + kMixMid + r0 * 12 + 4 * j);
+          x1 = *reinterpret_cast<const uint32_t*>(stage + kMixMid + r1 * 12 + 4 * j);
+        }
+        const uint32_t y0 = odd_bytes_down(x0), y1 = odd_bytes_down(x1);
+        mma16816(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u, ko.bh[8][0], ko.bh[8][1]);
+        mma16816(S[mt], y0 & 0x000F000Fu, y1 & 0x000F000Fu, y0 & 0x00F000F0u, y1 & 0x00F000F0u, ko.bh[9][0], ko.bh[9][1]);
+        if (!DUAL) {
+          mma16816(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u, ko.bl[8][0], ko.bl[8][1]);
+          mma16816(S[mt], y0 & 0x000F000Fu, y1 & 0x000F000Fu, y0 & 0x00F000F0u, y1 & 0x00F000F0u, ko.bl[9][0], ko.bl[9][1]);
+        }
+      }
+      {
+        const uint32_t x0 = *reinterpret_cast<const uint32_t*>(stage + kMixRaw + r0 * 16 + 4 * j);
+        const uint32_t x1 = *reinterpret_cast<const uint32_t*>(stage + kMixRaw + r1 * 16 + 4 * j);
+        mma16816_bf16(Sr[mt], x0, x1, 0u, 0u, ko.bh[10][0], ko.bh[10][1]);
+        if (!DUAL) mma16816_bf16(Sr[mt], x0, x1, 0u, 0u, ko.bl[10][0], ko.bl[10][1]);
+      }
+    }
+  } else {
   uint4 wlo[4], whi[4];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
@@ -544,12 +814,16 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
       }
     }
   }
+  }
   // ---- online softmax (log2 domain) ----
   if (DUAL) {   // add the remainder columns (lane j ^ 2) to the high-part columns
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) S[mt][e] += __shfl_xor_sync(0xffffffffu, S[mt][e], 2);
+      for (int e = 0; e < 4; ++e) {
+        S[mt][e] += __shfl_xor_sync(0xffffffffu, S[mt][e], 2);
+        if constexpr (MIX) Sr[mt][e] += __shfl_xor_sync(0xffffffffu, Sr[mt][e], 2);
+      }
   }
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
@@ -557,6 +831,10 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
     S[mt][1] = fmaf(S[mt][1], ko.mult, ko.bias1);
     S[mt][2] = fmaf(S[mt][2], ko.mult, ko.bias0);
     S[mt][3] = fmaf(S[mt][3], ko.mult, ko.bias1);
+    if constexpr (MIX) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) S[mt][e] += Sr[mt][e];
+    }
   }
   const bool partial = tvalid < 64;
   if (partial) {
@@ -641,14 +919,27 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 // Copy one half group (64 rows) of head `head`, group `gi` into a stage buffer, with the
 // group's key scale / zero-point when `with_key`: every lane moves 16-byte chunks.
+template <bool MIX>
 __device__ __forceinline__ void load_half(const MmaArgs& a, uint8_t* buf, int64_t head, int gi, int hf,
                                           bool with_key) {
   const int lane = threadIdx.x & 31;
   const int64_t t0 = (int64_t)gi * 128 + 64 * hf;
-  const uint8_t* kc = a.k_codes + head * a.k_slab_bytes + t0 * 64;
   const uint8_t* vc = a.v_codes + head * a.v_slab_bytes + t0 * 32;
+  if constexpr (MIX) {
+    // the group's planes: raw [128][8] 16-bit (2048 B), 4-bit [128][3] words (1536 B),
+    // 2-bit [128][6] words; this half's rows of each
+    const uint8_t* gb = a.k_codes + head * a.k_slab_bytes + (int64_t)gi * a.k_group_bytes;
 #pragma unroll
-  for (int e = 0; e < kHalfK / 512; ++e) cp_async16(buf + 16 * (lane + 32 * e), kc + 16 * (lane + 32 * e));
+    for (int e = 0; e < 2; ++e) cp_async16(buf + kMixRaw + 16 * (lane + 32 * e), gb + 1024 * hf + 16 * (lane + 32 * e));
+    for (int c = lane; c < 48; c += 32) cp_async16(buf + kMixMid + 16 * c, gb + 2048 + 768 * hf + 16 * c);
+#pragma unroll
+    for (int e = 0; e < 3; ++e)
+      cp_async16(buf + kMixLo + 16 * (lane + 32 * e), gb + 3584 + 1536 * hf + 16 * (lane + 32 * e));
+  } else {
+    const uint8_t* kc = a.k_codes + head * a.k_slab_bytes + t0 * 64;
+#pragma unroll
+    for (int e = 0; e < kHalfK / 512; ++e) cp_async16(buf + 16 * (lane + 32 * e), kc + 16 * (lane + 32 * e));
+  }
 #pragma unroll
   for (int e = 0; e < kHalfV / 512; ++e)
     cp_async16(buf + kHalfK + 16 * (lane + 32 * e), vc + 16 * (lane + 32 * e));
@@ -656,9 +947,18 @@ __device__ __forceinline__ void load_half(const MmaArgs& a, uint8_t* buf, int64_
     const __half* src = (lane < 8 ? a.v_scale : a.v_zero) + head * a.C + t0 + 8 * (lane & 7);
     cp_async16(buf + kHalfK + kHalfV + 16 * lane, src);
   }
-  if (with_key) {    // the group's key scale (lanes 0..15) and zero-point (16..31)
-    const __half* src = (lane < 16 ? a.k_scale : a.k_zero) + (head * a.ng + gi) * 128 + 8 * (lane & 15);
-    cp_async16(buf + kHalfK + kHalfV + kHalfVM + 16 * lane, src);
+  if (with_key) {
+    if constexpr (MIX) {   // slot order into the key region; 120 scales (lanes 0..14), zero-points (16..30)
+      const int64_t grp = head * a.ng + gi;
+      if (lane < 8) cp_async16(buf + kMixOrd + 16 * lane, a.k_order + grp * 128 + 16 * lane);
+      if ((lane & 15) < 15) {
+        const __half* src = (lane < 16 ? a.k_scale : a.k_zero) + grp * 120 + 8 * (lane & 15);
+        cp_async16(buf + kHalfK + kHalfV + kHalfVM + 16 * lane, src);
+      }
+    } else {   // the group's key scale (lanes 0..15) and zero-point (16..31)
+      const __half* src = (lane < 16 ? a.k_scale : a.k_zero) + (head * a.ng + gi) * 128 + 8 * (lane & 15);
+      cp_async16(buf + kHalfK + kHalfV + kHalfVM + 16 * lane, src);
+    }
   }
 }
 
@@ -725,7 +1025,7 @@ __device__ __forceinline__ float4 rotate_q(float4 x, int lane, float c) {
 }
 
 // ---- the kernel --------------------------------------------------------------------------
-template <bool DUAL, bool ROT>
+template <bool DUAL, bool ROT, bool MIX>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int GM = DUAL ? 4 : 8;
@@ -758,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
         load_raw(a, buf, lhead, lr >> 1);
       } else {
         const int p = lr - a.nrp;
-        load_half(a, buf, lhead, p >> 1, p & 1, (p & 1) == 0 || li == i0);
+        load_half<MIX>(a, buf, lhead, p >> 1, p & 1, (p & 1) == 0 || li == i0);
       }
       advance_load();
     }
@@ -772,7 +1072,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   state_reset(st);
   QVec<DUAL, GM> qv;
   if constexpr (DUAL) qv.s = reinterpret_cast<float*>(my_scratch) + 512;   // upper 2 KiB
-  KeyOp ko;
+  KeyOpT<MIX> ko;
   int64_t head = i0 / U, cur_head = -1;
   int r = (int)(i0 - head * U);
   bool qbad = false, qrot = false;
@@ -832,10 +1132,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
       const int p = r - a.nrp, gi = p >> 1, hf = p & 1;
       if (hf == 0 || i == i0) {
         const __half* ks = reinterpret_cast<const __half*>(stg + kHalfK + kHalfV + kHalfVM);
-        key_operand<DUAL, GM>(a, ks, ks + 128, my_scratch, qv, ko);
+        if constexpr (MIX) key_operand_mixed<DUAL, GM>(a, stg, my_scratch, qv, ko);
+        else key_operand<DUAL, GM>(a, ks, ks + 128, my_scratch, qv, ko);
       }
       const int tvalid = (int)min((int64_t)64, a.t_quant - (int64_t)gi * 128 - 64 * hf);
-      mma_half<DUAL>(st, stg, ko, tvalid);
+      mma_half<DUAL, MIX>(st, stg, ko, tvalid);
     }
     __syncwarp();
     ++consumed;
@@ -945,8 +1246,11 @@ bool mma_path_ok(const Layout& L, int Hq) {
   const Side& K = L.side[0];
   const Side& V = L.side[1];
   const int G = Hq / L.Hkv;
-  return L.D == 128 && L.g == 128 && K.scheme == KVQ_ASYM && K.bits == 4 &&
-         K.axis == KVQ_AXIS_CHANNEL && V.scheme == KVQ_ASYM && V.bits == 2 &&
+  const bool k4 = K.scheme == KVQ_ASYM && K.bits == 4 && K.axis == KVQ_AXIS_CHANNEL;
+  // MIXED keys with the [MIX] Figure 3 tiers (8 raw bf16, 24 4-bit, 96 2-bit slots)
+  const bool mix = K.scheme == KVQ_MIXED && L.mixed_hi == 8 && L.mixed_mid == 24 &&
+                   L.src_dtype == KVQ_BF16;
+  return L.D == 128 && L.g == 128 && (k4 || mix) && V.scheme == KVQ_ASYM && V.bits == 2 &&
          V.axis == KVQ_AXIS_TOKEN && L.rope == 0 && G >= 1 && G <= 8;
 }
 
@@ -1001,6 +1305,8 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.sink_v = L.sink[1];
   a.res_k = L.res[0];
   a.res_v = L.res[1];
+  a.k_order = L.k_order;
+  a.k_group_bytes = L.mixed_group_bytes;
   a.q = q;
   a.q_dtype = q_dtype;
   a.qscale = scale * kLog2e;
@@ -1017,8 +1323,10 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.ws_o = ws_o;
   a.status = d_status;
   const size_t smem = mma_smem();
-  auto kern = a.G <= 4 ? (a.k_rotate ? decode_mma_kernel<true, true> : decode_mma_kernel<true, false>)
-                       : (a.k_rotate ? decode_mma_kernel<false, true> : decode_mma_kernel<false, false>);
+  const bool mix = L.side[0].scheme == KVQ_MIXED;
+  auto kern = mix ? (a.G <= 4 ? decode_mma_kernel<true, false, true> : decode_mma_kernel<false, false, true>)
+            : a.G <= 4 ? (a.k_rotate ? decode_mma_kernel<true, true, false> : decode_mma_kernel<true, false, false>)
+                       : (a.k_rotate ? decode_mma_kernel<false, true, false> : decode_mma_kernel<false, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<p.grid_ctas, kThreads, smem, s>>>(a);

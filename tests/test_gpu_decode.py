@@ -153,6 +153,40 @@ def test_mixed_decode():
     assert rel_l2(out, ref) <= 2e-3
 
 
+@pytest.mark.parametrize("G", [1, 2, 4, 5, 8])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_mixed_decode_tensor_core_path(G, splits):
+    # the [MIX] Figure 3 tiers on tensor cores: 2-bit and 4-bit slots as fp16 subnormals,
+    # raw bf16 slots in their own bf16 product, slot order per group; sink, residual
+    # window, a ragged last group
+    B, H, tq, tr = 2, 3, 3 * 128 + 45, 29
+    fd = fmt(src_dtype=BF16, k_scheme=MIXED, k_bits=0, mixed_hi=8, mixed_mid=24, n_sink=1,
+             residual_cap=64)
+    p = build(fd, B, H, G * H, tq, tr, seed=110 + G, k_scale=4.0)
+    out, ref = run(p, G * H, tq, tr, BF16, F32, seed=110 + G, num_splits=splits)
+    assert rel_l2(out, ref) <= 1e-3
+    assert p.status_bits() == 0
+
+
+@pytest.mark.parametrize("kw", [dict(mixed_hi=16, mixed_mid=16), dict(src_dtype=F16)])
+def test_mixed_decode_cuda_core_path(kw):
+    # tiers other than 8 / 24 / 96, and fp16 sources, take the CUDA-core kernel
+    B, H, G, tq = 2, 2, 4, 2 * 128 + 60
+    fd = fmt(**dict(dict(src_dtype=BF16, k_scheme=MIXED, k_bits=0, mixed_hi=8, mixed_mid=24), **kw))
+    p = build(fd, B, H, G * H, tq, 0, seed=18, k_scale=4.0)
+    out, ref = run(p, G * H, tq, 0, fd["src_dtype"], F32, seed=18)
+    assert rel_l2(out, ref) <= 1e-3
+
+
+def test_mixed_decode_heavy_raw_slots():
+    # raw slots carrying most of the score: keys x 40 on a few channels of every group
+    B, H, G, tq = 1, 2, 4, 2 * 128
+    fd = fmt(src_dtype=BF16, k_scheme=MIXED, k_bits=0, mixed_hi=8, mixed_mid=24)
+    p = build(fd, B, H, G * H, tq, 0, seed=19, k_scale=40.0)
+    out, ref = run(p, G * H, tq, 0, BF16, F32, seed=19)
+    assert rel_l2(out, ref) <= 1e-3
+
+
 @pytest.mark.parametrize("scheme", ["tensor", "token", "hybrid"])
 @pytest.mark.parametrize("target", ["both", "k_only", "v_only"])
 def test_toy_int8(scheme, target):
