@@ -366,6 +366,11 @@ static void plan_layout(const kvq_format* f, int32_t B, int32_t Hkv, Layout* L) 
   L->side[1].nout = f->v_scheme == KVQ_NUQ ? f->v_outliers : 0;
   L->rope = f->rope;
   L->src_dtype = f->src_dtype;
+  // every format field the decode planner reads (the tiers select the MIXED kernel)
+  L->mixed_hi = f->mixed_hi;
+  L->mixed_mid = f->mixed_mid;
+  L->mixed_lo = f->head_dim - f->mixed_hi - f->mixed_mid;
+  L->k_rotate = f->k_rotate;
 }
 
 size_t kvq_decode_workspace_bytes(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,

@@ -88,6 +88,29 @@ SHAPES = [
 ]
 
 
+MIXED_SHAPES = [
+    # MixKVQ tiers (8 / 24 / 96) on bf16: the tensor-core plan too
+    (16, 8, 5, 16384, 0, 0, 0, synth.BF16),
+    (1, 2, 5, 4096, 0, 0, 1, synth.BF16),
+    (2, 3, 4, 3 * 128 + 45, 1, 29, 3, synth.BF16),
+]
+
+
+@pytest.mark.parametrize("B,Hkv,G,tq,ns,tr,splits,src", MIXED_SHAPES)
+def test_mixed_tiers_plan_like_k4v2(B, Hkv, G, tq, ns, tr, splits, src):
+    # every host planning helper sees the tiers: the slot count, the workspace of the
+    # split kernel and the combine agree with the tensor-core partition
+    fd = synth._fmt(src_dtype=src, k_scheme=synth.MIXED, k_bits=0, mixed_hi=8, mixed_mid=24,
+                    n_sink=ns, residual_cap=max(tr, 1))
+    f = kvq.make_format(fd)
+    U = positions_per_head(tq, ns + tr, 2)
+    want = model(B * Hkv, U, splits)
+    assert kvq.decode_partial_slots(f, B, G * Hkv, Hkv, tq, tr, splits) == want
+    rows = B * G * Hkv * want
+    assert kvq.decode_workspace_bytes(f, B, G * Hkv, Hkv, tq, tr, splits) == \
+        2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4
+
+
 @pytest.mark.parametrize("B,Hkv,G,tq,ns,tr,splits,src", SHAPES)
 def test_planned_slots_match_the_partition_model(B, Hkv, G, tq, ns, tr, splits, src):
     fd = synth._fmt(src_dtype=src, n_sink=ns, residual_cap=max(tr, 1))
