@@ -2,8 +2,8 @@
 // each window of R buffered tokens).
 //
 // One CTA per (kv head, batch), one thread per channel d.  The window rows are staged
-// through shared memory in chunks of 64 rows with coalesced (16-byte where the strides
-// allow) loads by all threads.  I_d sums |Q[d]| over the G query heads of the group and
+// through shared memory in chunks of 64 rows, double-buffered with asynchronous 16-byte
+// copies (element copies where the strides do not allow them) by all threads.  I_d sums |Q[d]| over the G query heads of the group and
 // the R window rows in fp64, head-major then row, and divides by G * R; S_d is the fp64 range of K[:, d]; A_d = I_d * S_d.  The rank of a
 // channel is the number of channels with a larger A (or an equal A and a lower
 // index), so order[rank] = d sorts by descending salience with ties to the lower
@@ -29,8 +29,15 @@ struct SalArgs {
 
 constexpr int kRC = 64;   // window rows per staged chunk
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
 // Rows [r0, r0 + nr) of a [R][D] window (element offsets base + r * rstride + c) into
-// buf[r - r0][c], by all D threads of the CTA.
+// buf[r - r0][c], by all D threads of the CTA: asynchronous 16-byte copies when the
+// base and strides allow (completed by the caller's wait), element copies otherwise.
 __device__ __forceinline__ void stage_rows(uint8_t* buf, const void* src, int64_t base, int64_t rstride,
                                            int r0, int nr, int D, int esz, bool vec) {
   const uint8_t* s8 = reinterpret_cast<const uint8_t*>(src);
@@ -38,8 +45,7 @@ __device__ __forceinline__ void stage_rows(uint8_t* buf, const void* src, int64_
     const int vpr = D * esz / 16;
     for (int v = threadIdx.x; v < nr * vpr; v += blockDim.x) {
       const int row = v / vpr, cv = v - row * vpr;
-      *reinterpret_cast<uint4*>(buf + (size_t)row * D * esz + cv * 16) =
-          *reinterpret_cast<const uint4*>(s8 + (base + (int64_t)(r0 + row) * rstride) * esz + cv * 16);
+      cp_async16(buf + (size_t)row * D * esz + cv * 16, s8 + (base + (int64_t)(r0 + row) * rstride) * esz + cv * 16);
     }
   } else {
     for (int i = threadIdx.x; i < nr * D; i += blockDim.x) {
@@ -51,8 +57,11 @@ __device__ __forceinline__ void stage_rows(uint8_t* buf, const void* src, int64_
   }
 }
 
+// The window as one sequence of chunks: query rows of head 0, 1, ..., G - 1 (R rows each,
+// kRC at a time), then the key rows.  Two staging buffers: chunk c + 1 is in flight while
+// chunk c is summed, so the fp64 chain of each channel overlaps the loads.
 __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
-  extern __shared__ __align__(16) uint8_t sbuf[];   // [kRC][D] source elements
+  extern __shared__ __align__(16) uint8_t sbuf[];   // [2][kRC][D] source elements
   __shared__ double A[256];
   __shared__ int bad;
   const int d = threadIdx.x;
@@ -60,38 +69,54 @@ __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
   const int G = a.Hq / a.Hkv;
   const int D = a.D;
   const int esz = a.dtype == KVQ_F32 ? 4 : 2;
+  const size_t bufb = (size_t)kRC * D * esz;
+  const int cpw = (a.R + kRC - 1) / kRC;            // chunks per window
+  const int nq = G * cpw, n = nq + cpw;
+  const int64_t kb = (int64_t)b * a.ksb + (int64_t)h * a.ksh;
+  auto issue = [&](int c) {
+    if (c < n) {
+      uint8_t* buf = sbuf + (c & 1) * bufb;
+      const int w = c < nq ? c % cpw : c - nq;
+      const int r0 = w * kRC, nr = min(kRC, a.R - r0);
+      if (c < nq) {
+        const int64_t qb = (int64_t)b * a.qsb + (int64_t)(h * G + c / cpw) * a.qsh;
+        stage_rows(buf, a.q, qb, a.qst, r0, nr, D, esz, a.q_vec);
+      } else {
+        stage_rows(buf, a.k, kb, a.kst, r0, nr, D, esz, a.k_vec);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
   if (d == 0) bad = 0;
   double acc = 0.0;
+  float mn = INFINITY, mx = -INFINITY;
   int nonfinite = 0;
-  for (int hh = 0; hh < G; ++hh) {
-    const int64_t qb = (int64_t)b * a.qsb + (int64_t)(h * G + hh) * a.qsh;
-    for (int r0 = 0; r0 < a.R; r0 += kRC) {
-      const int nr = min(kRC, a.R - r0);
-      __syncthreads();
-      stage_rows(sbuf, a.q, qb, a.qst, r0, nr, D, esz, a.q_vec);
-      __syncthreads();
+  issue(0);
+  for (int c = 0; c < n; ++c) {
+    issue(c + 1);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();   // chunk c staged by every thread
+    const uint8_t* buf = sbuf + (c & 1) * bufb;
+    const int w = c < nq ? c % cpw : c - nq;
+    const int nr = min(kRC, a.R - w * kRC);
+    if (c < nq) {      // head-major, then row: the order of the plain definition
       for (int r = 0; r < nr; ++r) {
-        const float x = load_elem(sbuf, (int64_t)r * D + d, a.dtype);
+        const float x = load_elem(buf, (int64_t)r * D + d, a.dtype);
         nonfinite |= !isfinite(x);
         acc = __dadd_rn(acc, fabs((double)x));
       }
+    } else {
+      for (int r = 0; r < nr; ++r) {
+        const float x = load_elem(buf, (int64_t)r * D + d, a.dtype);
+        nonfinite |= !isfinite(x);
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+      }
     }
+    __syncthreads();   // before chunk c + 2 overwrites this buffer
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   const double intensity = __ddiv_rn(acc, (double)G * (double)a.R);
-  const int64_t kb = (int64_t)b * a.ksb + (int64_t)h * a.ksh;
-  float mn = INFINITY, mx = -INFINITY;
-  for (int r0 = 0; r0 < a.R; r0 += kRC) {
-    const int nr = min(kRC, a.R - r0);
-    __syncthreads();
-    stage_rows(sbuf, a.k, kb, a.kst, r0, nr, D, esz, a.k_vec);
-    __syncthreads();
-    for (int r = 0; r < nr; ++r) {
-      const float x = load_elem(sbuf, (int64_t)r * D + d, a.dtype);
-      nonfinite |= !isfinite(x);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
-    }
-  }
   const double range = __dsub_rn((double)mx, (double)mn);
   const double sal = __dmul_rn(intensity, range);
   A[d] = sal;
@@ -140,7 +165,7 @@ cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t
   };
   a.q_vec = vec_ok(q, qsb, qsh, qst);
   a.k_vec = vec_ok(k, ksb, ksh, kst);
-  const size_t smem = (size_t)kRC * L.D * esz;
+  const size_t smem = 2 * (size_t)kRC * L.D * esz;
   cudaError_t e = cudaFuncSetAttribute(salience_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(Hkv, B);
