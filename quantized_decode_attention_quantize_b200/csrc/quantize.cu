@@ -515,6 +515,7 @@ __device__ void do_mixed(const QArgs& a, const QSmem& sm, int ln, int64_t ts, in
     const int c = ord[j];
     const int bits = j < hi + mid ? 4 : 2;
     float mn = sm.tile[c], mx = mn;
+#pragma unroll 8
     for (int r = 1; r < ln; ++r) {
       const float x = sm.tile[r * D + c];
       mn = fminf(mn, x);

@@ -60,6 +60,16 @@ __device__ __forceinline__ void stage_rows(uint8_t* buf, const void* src, int64_
 // The window as one sequence of chunks: query rows of head 0, 1, ..., G - 1 (R rows each,
 // kRC at a time), then the key rows.  Two staging buffers: chunk c + 1 is in flight while
 // chunk c is summed, so the fp64 chain of each channel overlaps the loads.
+// One staged element as fp32 (exact), for source dtype DT.
+template <int DT>
+__device__ __forceinline__ float staged(const uint8_t* buf, int i) {
+  if constexpr (DT == KVQ_F32) return reinterpret_cast<const float*>(buf)[i];
+  const uint16_t h = reinterpret_cast<const uint16_t*>(buf)[i];
+  if constexpr (DT == KVQ_F16) return half_bits_to_float(h);
+  return __uint_as_float((uint32_t)h << 16);
+}
+
+template <int DT>
 __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
   extern __shared__ __align__(16) uint8_t sbuf[];   // [2][kRC][D] source elements
   __shared__ double A[256];
@@ -68,7 +78,7 @@ __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int G = a.Hq / a.Hkv;
   const int D = a.D;
-  const int esz = a.dtype == KVQ_F32 ? 4 : 2;
+  constexpr int esz = DT == KVQ_F32 ? 4 : 2;
   const size_t bufb = (size_t)kRC * D * esz;
   const int cpw = (a.R + kRC - 1) / kRC;            // chunks per window
   const int nq = G * cpw, n = nq + cpw;
@@ -100,15 +110,14 @@ __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
     const int w = c < nq ? c % cpw : c - nq;
     const int nr = min(kRC, a.R - w * kRC);
     if (c < nq) {      // head-major, then row: the order of the plain definition
-      for (int r = 0; r < nr; ++r) {
-        const float x = load_elem(buf, (int64_t)r * D + d, a.dtype);
-        nonfinite |= !isfinite(x);
-        acc = __dadd_rn(acc, fabs((double)x));
-      }
+      // (a NaN or an infinity among the |Q| carries through to acc, checked at the end)
+#pragma unroll 16
+      for (int r = 0; r < nr; ++r) acc = __dadd_rn(acc, (double)fabsf(staged<DT>(buf, r * D + d)));
     } else {
+#pragma unroll 16
       for (int r = 0; r < nr; ++r) {
-        const float x = load_elem(buf, (int64_t)r * D + d, a.dtype);
-        nonfinite |= !isfinite(x);
+        const float x = staged<DT>(buf, r * D + d);
+        nonfinite |= !(fabsf(x) <= 3.402823466e38f);   // NaN and +-inf
         mn = fminf(mn, x);
         mx = fmaxf(mx, x);
       }
@@ -116,6 +125,7 @@ __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
     __syncthreads();   // before chunk c + 2 overwrites this buffer
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+  nonfinite |= !isfinite(acc);
   const double intensity = __ddiv_rn(acc, (double)G * (double)a.R);
   const double range = __dsub_rn((double)mx, (double)mn);
   const double sal = __dmul_rn(intensity, range);
@@ -123,6 +133,7 @@ __global__ void __launch_bounds__(256) salience_kernel(SalArgs a) {
   if (nonfinite) atomicOr(&bad, 1);
   __syncthreads();
   int rank = 0;
+#pragma unroll 16
   for (int e = 0; e < a.D; ++e) {
     const double v = A[e];
     rank += (v > sal || (v == sal && e < d)) ? 1 : 0;
@@ -166,10 +177,12 @@ cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t
   a.q_vec = vec_ok(q, qsb, qsh, qst);
   a.k_vec = vec_ok(k, ksb, ksh, kst);
   const size_t smem = 2 * (size_t)kRC * L.D * esz;
-  cudaError_t e = cudaFuncSetAttribute(salience_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = L.src_dtype == KVQ_F32 ? salience_kernel<KVQ_F32>
+             : L.src_dtype == KVQ_F16 ? salience_kernel<KVQ_F16> : salience_kernel<KVQ_BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(Hkv, B);
-  salience_kernel<<<grid, L.D, smem, s>>>(a);
+  kern<<<grid, L.D, smem, s>>>(a);
   return cudaGetLastError();
 }
 
