@@ -499,12 +499,29 @@ __device__ void do_mixed(const QArgs& a, const QSmem& sm, int ln, int64_t ts, in
   uint8_t* ord = sm.codes;  // [D] slot -> channel
   for (int j = threadIdx.x; j < D; j += blockDim.x) ord[j] = L.k_order[(sl * L.ng + gi) * D + j];
   __syncthreads();
+  // permute every staged row into slot order once (a warp per row: gather, then write
+  // back), so that the statistics and the codes below read slots contiguously
+  {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int per = D / 32;   // slots per lane
+    for (int r = warp; r < ln; r += nw) {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (e < per) v[e] = sm.tile[r * D + ord[per * lane + e]];
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (e < per) sm.tile[r * D + per * lane + e] = v[e];
+    }
+  }
+  __syncthreads();
   uint8_t* gbase = reinterpret_cast<uint8_t*>(S.codes) + (sl * L.ng + gi) * (int64_t)L.mixed_group_bytes;
   // raw plane [g][hi]
   uint16_t* raw = reinterpret_cast<uint16_t*>(gbase);
   for (int i = threadIdx.x; i < ln * hi; i += blockDim.x) {
     const int r = i / hi, j = i % hi;
-    const float v = sm.tile[r * D + ord[j]];
+    const float v = sm.tile[r * D + j];
     raw[r * hi + j] = L.src_dtype == KVQ_F16 ? __half_as_ushort(__float2half_rn(v))
                                              : (uint16_t)(__float_as_uint(v) >> 16);
   }
@@ -512,12 +529,11 @@ __device__ void do_mixed(const QArgs& a, const QSmem& sm, int ln, int64_t ts, in
   __half* hz = reinterpret_cast<__half*>(S.zero) + (sl * L.ng + gi) * (D - hi);
   int range_bad = 0;
   for (int j = hi + threadIdx.x; j < D; j += blockDim.x) {
-    const int c = ord[j];
     const int bits = j < hi + mid ? 4 : 2;
-    float mn = sm.tile[c], mx = mn;
+    float mn = sm.tile[j], mx = mn;
 #pragma unroll 8
     for (int r = 1; r < ln; ++r) {
-      const float x = sm.tile[r * D + c];
+      const float x = sm.tile[r * D + j];
       mn = fminf(mn, x);
       mx = fmaxf(mx, x);
     }
@@ -535,18 +551,21 @@ __device__ void do_mixed(const QArgs& a, const QSmem& sm, int ln, int64_t ts, in
   const int Wm = mid / 8, Wl = lo / 16;
   for (int i = threadIdx.x; i < ln * (Wm + Wl); i += blockDim.x) {
     const int r = i / (Wm + Wl), w = i % (Wm + Wl);
+    const float* row = sm.tile + r * D;
     uint32_t word = 0;
     if (w < Wm) {
+#pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int j = hi + w * 8 + e;
-        word |= (uint32_t)asym_code(sm.tile[r * D + ord[j]], sm.sf[j], sm.zf[j], 15) << (4 * e);
+        word |= (uint32_t)asym_code(row[j], sm.sf[j], sm.zf[j], 15) << (4 * e);
       }
       midp[r * Wm + w] = word;
     } else {
       const int w2 = w - Wm;
+#pragma unroll
       for (int e = 0; e < 16; ++e) {
         const int j = hi + mid + w2 * 16 + e;
-        word |= (uint32_t)asym_code(sm.tile[r * D + ord[j]], sm.sf[j], sm.zf[j], 3) << (2 * e);
+        word |= (uint32_t)asym_code(row[j], sm.sf[j], sm.zf[j], 3) << (2 * e);
       }
       lop[r * Wl + w2] = word;
     }
