@@ -549,6 +549,41 @@ __device__ void do_mixed(const QArgs& a, const QSmem& sm, int ln, int64_t ts, in
   uint32_t* midp = reinterpret_cast<uint32_t*>(gbase + g * hi * 2);
   uint32_t* lop = reinterpret_cast<uint32_t*>(gbase + g * hi * 2 + g * mid / 2);
   const int Wm = mid / 8, Wl = lo / 16;
+  if (D == 128) {
+    // a warp per row, lane l on slots 4 l .. 4 l + 3 (one float4 of the slot-ordered row;
+    // tier boundaries are multiples of 8 slots, so a lane sits in one tier): 4-bit words
+    // join the halves of lanes l, l ^ 1, 2-bit words the bytes of four lanes
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int s0 = 4 * lane;
+    const bool is_mid = s0 >= hi && s0 < hi + mid, is_lo = s0 >= hi + mid;
+    float sf4[4], zf4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sf4[e] = s0 >= hi ? sm.sf[s0 + e] : 0.0f;
+      zf4[e] = s0 >= hi ? sm.zf[s0 + e] : 0.0f;
+    }
+    for (int r = warp; r < ln; r += nw) {
+      const float4 x4 = *reinterpret_cast<const float4*>(sm.tile + r * D + s0);
+      const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+      uint32_t v4 = 0, v2 = 0;
+      if (s0 >= hi) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = asym_code(xs[e], sf4[e], zf4[e], is_mid ? 15 : 3);
+          v4 |= (uint32_t)c << (4 * e);
+          v2 |= (uint32_t)c << (2 * e);
+        }
+      }
+      v4 <<= 16 * (lane & 1);
+      v4 |= __shfl_xor_sync(0xffffffffu, v4, 1);
+      v2 <<= 8 * (lane & 3);
+      v2 |= __shfl_xor_sync(0xffffffffu, v2, 1);
+      v2 |= __shfl_xor_sync(0xffffffffu, v2, 2);
+      if (is_mid && (lane & 1) == 0) midp[r * Wm + (s0 - hi) / 8] = v4;
+      if (is_lo && (lane & 3) == 0) lop[r * Wl + (s0 - hi - mid) / 16] = v2;
+    }
+    return;
+  }
   for (int i = threadIdx.x; i < ln * (Wm + Wl); i += blockDim.x) {
     const int r = i / (Wm + Wl), w = i % (Wm + Wl);
     const float* row = sm.tile + r * D;
