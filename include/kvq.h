@@ -316,6 +316,29 @@ kvq_status kvq_decode_combine(const kvq_format* fmt, int32_t batch, int32_t q_he
                               int32_t num_splits, const void* workspace, size_t workspace_bytes,
                               void* out, int32_t out_dtype, void* stream);
 
+/* Sequence split ([KVQ] "Approach": contexts spread over several GPUs).  Each part of a
+ * context (a disjoint set of tokens: its own cache with its own sink / packed / residual
+ * tokens, typically one per GPU) runs kvq_decode_partial as usual and then this combine,
+ * which writes out[B][Hq][D] fp32 and lse[B][Hq] fp32, the natural log of the part's
+ * softmax denominator: lse = log sum_t exp(softmax_scale * q . k_t).  Arguments and
+ * errors otherwise as kvq_decode_combine (out and lse device, 16-byte aligned). */
+kvq_status kvq_decode_combine_lse(const kvq_format* fmt, int32_t batch, int32_t q_heads,
+                                  int32_t kv_heads, int64_t t_quant, int32_t t_residual,
+                                  int32_t num_splits, const void* workspace,
+                                  size_t workspace_bytes, float* out, float* lse, void* stream);
+
+/* Merge of n_parts such results, gathered into outs[n_parts][rows][head_dim] and
+ * lses[n_parts][rows] (device fp32, 16-byte aligned; rows = B * Hq): for every row,
+ * out = sum_r w_r outs[r] / sum_r w_r with w_r = exp(lses[r] - max_r lses[r]); a part
+ * with lse = -inf (no tokens) has weight 0.  out is written in out_dtype; lse_out
+ * (nullable) receives the merged log-denominator.  The gather itself (one all-gather
+ * of (head_dim + 1) * 4 bytes per query row and part) belongs to the caller's
+ * collective library.  KVQ_ERR_INVALID for n_parts outside [1, 4096], rows outside
+ * [1, 2^31], an unsupported head_dim, or bad pointers. */
+kvq_status kvq_merge_states(int32_t n_parts, int64_t rows, int32_t head_dim, const float* outs,
+                            const float* lses, void* out, int32_t out_dtype, float* lse_out,
+                            void* stream);
+
 /* Decode attention without a caller workspace, for callers that cannot allocate
  * device memory at all -- for example a serving process whose allocator reserved
  * every byte at start-up, or a plugin host that forbids allocation once running --

@@ -48,6 +48,26 @@ def attention(q, K, V, scale):
     return (p @ np.asarray(V, np.float64)) / p.sum(axis=-1, keepdims=True)
 
 
+def attention_lse(q, K, V, scale):
+    """(out [G, D], lse [G]) of stable softmax attention, lse = log sum_t exp(scale q.k_t)."""
+    q = np.asarray(q, np.float64)
+    s = (q @ np.asarray(K, np.float64).T) * scale
+    mx = s.max(axis=-1, keepdims=True)
+    p = np.exp(s - mx)
+    den = p.sum(axis=-1, keepdims=True)
+    return (p @ np.asarray(V, np.float64)) / den, (mx + np.log(den))[..., 0]
+
+
+def merge_parts(outs, lses):
+    """Attention over disjoint token sets from each set's (out, lse): the softmax weights of
+    the union split into per-set weights exp(lse_r - lse), lse = log sum_r exp(lse_r)."""
+    outs = np.asarray(outs, np.float64)
+    lses = np.asarray(lses, np.float64)
+    m = lses.max(axis=0)
+    w = np.exp(lses - m)
+    return (w[..., None] * outs).sum(axis=0) / w.sum(axis=0)[..., None], m + np.log(w.sum(axis=0))
+
+
 def kv_slab(fmt, cache, b, h, t_quant, t_res):
     """(K [T, D], V [T, D]) float64 of one KV head: sink, packed rows, residual."""
     A = cache.arrays

@@ -434,7 +434,34 @@ kvq_status kvq_decode_combine(const kvq_format* f, int32_t B, int32_t Hq, int32_
   plan_layout(f, B, Hkv, &L);
   DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
   if (ws_bytes < workspace_bytes(L, Hq, p)) return KVQ_ERR_WORKSPACE;
-  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_decode_combine_lse(const kvq_format* f, int32_t B, int32_t Hq, int32_t Hkv,
+                                  int64_t t_quant, int32_t t_res, int32_t num_splits, const void* ws,
+                                  size_t ws_bytes, float* out, float* lse, void* stream) {
+  kvq_status s = decode_args(f, B, Hq, Hkv, t_quant, t_res, num_splits);
+  if (s != KVQ_OK) return s;
+  if (!out || !aligned16(out) || !lse || !aligned16(lse) || !ws || !aligned16(ws)) return KVQ_ERR_INVALID;
+  Layout L;
+  plan_layout(f, B, Hkv, &L);
+  DecodePlan p = plan_decode(L, Hq, t_quant, t_res, num_splits);
+  if (ws_bytes < workspace_bytes(L, Hq, p)) return KVQ_ERR_WORKSPACE;
+  cudaError_t e = launch_combine(L, Hq, p, ws, out, KVQ_F32, lse, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_merge_states(int32_t n_parts, int64_t rows, int32_t head_dim, const float* outs,
+                            const float* lses, void* out, int32_t out_dtype, float* lse_out,
+                            void* stream) {
+  if (n_parts < 1 || n_parts > 4096 || rows < 1 || rows > ((int64_t)1 << 31)) return KVQ_ERR_INVALID;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128 && head_dim != 256) return KVQ_ERR_INVALID;
+  if (!outs || !aligned16(outs) || !lses || !aligned16(lses) || !out || !aligned16(out) ||
+      !valid_dtype(out_dtype) || (lse_out && !aligned16(lse_out)))
+    return KVQ_ERR_INVALID;
+  cudaError_t e = launch_merge_states(n_parts, rows, head_dim, outs, lses, out, out_dtype, lse_out,
+                                      reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -449,7 +476,7 @@ kvq_status kvq_decode_attention(const kvq_format* f, const kvq_cache* c, const v
   kvq_status s = partial_common(f, c, q, q_dtype, Hq, t_quant, t_res, scale, ws, ws_bytes,
                                 num_splits, d_status, stream, &L, &p);
   if (s != KVQ_OK) return s;
-  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

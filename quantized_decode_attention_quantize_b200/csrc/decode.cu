@@ -20,7 +20,7 @@ bool mma_path_ok(const Layout& L, int Hq);
 void plan_mma(const Layout& L, int64_t t_quant, int t_res, int max_ctas, DecodePlan& p);
 cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, const float* ws_m,
                                const float* ws_l, const float* ws_o, void* out, int out_dtype,
-                               cudaStream_t s);
+                               float* lse, cudaStream_t s);
 cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
                               int Hq, int64_t t_quant, int t_res, float scale, float* ws_m,
                               float* ws_l, float* ws_o, int32_t* d_status, cudaStream_t s);
@@ -390,6 +390,7 @@ struct CombArgs {
   const float* o;
   void* out;
   int out_dtype;
+  float* lse;   // nullable
 };
 
 __global__ void __launch_bounds__(256) combine_kernel(CombArgs a) {
@@ -407,6 +408,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombArgs a) {
       o = fmaf(a.o[(row * a.S + s) * a.D + d], f, o);
     }
     store_elem(a.out, row * a.D + d, a.out_dtype, o / L);
+    if (a.lse && d == 0) a.lse[row] = (M + log2f(L)) * 0.6931471805599453f;   // natural log
   }
 }
 
@@ -517,12 +519,12 @@ cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const vo
 }
 
 cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
-                           int out_dtype, cudaStream_t s) {
+                           int out_dtype, float* lse, cudaStream_t s) {
   const size_t rows = (size_t)L.B * Hq * p.S;
   const float* m = reinterpret_cast<const float*>(ws);
   const float* l = reinterpret_cast<const float*>(reinterpret_cast<const char*>(ws) + align16(rows * 4));
   const float* o = reinterpret_cast<const float*>(reinterpret_cast<const char*>(ws) + 2 * align16(rows * 4));
-  if (p.fast) return launch_combine_mma(L, p, Hq, m, l, o, out, out_dtype, s);
+  if (p.fast) return launch_combine_mma(L, p, Hq, m, l, o, out, out_dtype, lse, s);
   CombArgs c;
   c.D = L.D;
   c.Hq = Hq;
@@ -532,6 +534,7 @@ cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const v
   c.o = o;
   c.out = out;
   c.out_dtype = out_dtype;
+  c.lse = lse;
   dim3 grid(Hq, L.B);
   combine_kernel<<<grid, L.D < 256 ? L.D : 256, 0, s>>>(c);
   return cudaGetLastError();

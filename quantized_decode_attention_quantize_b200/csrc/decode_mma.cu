@@ -986,7 +986,7 @@ __device__ __forceinline__ void load_raw(const MmaArgs& a, uint8_t* buf, int64_t
 // Lane owns channels 4 lane .. 4 lane + 3.
 __device__ __forceinline__ void combine_row(const float* m, const float* l, const float* o, int S,
                                             int64_t row, int s_lo, int s_hi, int lane, void* out,
-                                            int out_dtype) {
+                                            int out_dtype, float* lse) {
   const float* mrow = m + row * S;
   const float* lrow = l + row * S;
   float M = -INFINITY;
@@ -1006,6 +1006,8 @@ __device__ __forceinline__ void combine_row(const float* m, const float* l, cons
   }
   const float inv = 1.0f / L;
   const int64_t i = row * 128 + 4 * lane;
+  // natural log of the row's softmax denominator (scores were kept as log2 units)
+  if (lse && lane == 0) lse[row] = (M + __log2f(L)) * 0.6931471805599453f;
   if (out_dtype == KVQ_F32) {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
@@ -1206,6 +1208,7 @@ struct CombArgsMma {
   const float* o;
   void* out;
   int out_dtype;
+  float* lse;   // nullable
 };
 
 // One warp per query-head row.
@@ -1215,7 +1218,7 @@ __global__ void __launch_bounds__(128) combine_mma_kernel(CombArgsMma a) {
   if (row >= a.rows) return;
   int s_lo, s_hi;
   head_slots(row / a.G, a.U, a.I, a.W, kCW, &s_lo, &s_hi);
-  combine_row(a.m, a.l, a.o, a.S, row, s_lo, s_hi, lane, a.out, a.out_dtype);
+  combine_row(a.m, a.l, a.o, a.S, row, s_lo, s_hi, lane, a.out, a.out_dtype, a.lse);
 }
 
 // per-warp rings of item stages, per-warp scratch, then the warps' last heads
@@ -1335,7 +1338,7 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
 
 cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, const float* ws_m,
                                const float* ws_l, const float* ws_o, void* out, int out_dtype,
-                               cudaStream_t s) {
+                               float* lse, cudaStream_t s) {
   CombArgsMma c;
   c.G = Hq / L.Hkv;
   c.S = p.S;
@@ -1348,6 +1351,7 @@ cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, con
   c.o = ws_o;
   c.out = out;
   c.out_dtype = out_dtype;
+  c.lse = lse;
   combine_mma_kernel<<<(unsigned)((c.rows + 3) / 4), 128, 0, s>>>(c);
   return cudaGetLastError();
 }

@@ -84,7 +84,11 @@ cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const vo
                                   int q_dtype, int Hq, int64_t t_quant, int t_res, float scale,
                                   void* ws, int32_t* d_status, cudaStream_t s);
 cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
-                           int out_dtype, cudaStream_t s);
+                           int out_dtype, float* lse, cudaStream_t s);
+// out = sum_r w_r out_r / sum_r w_r with w_r = exp(lse_r - max_r lse_r) over n parts
+// (outs [n][rows][D] fp32, lses [n][rows] fp32).
+cudaError_t launch_merge_states(int n, int64_t rows, int D, const float* outs, const float* lses,
+                                void* out, int out_dtype, float* lse_out, cudaStream_t s);
 int device_sm_count();
 
 // ---------------------------------------------------------------------------

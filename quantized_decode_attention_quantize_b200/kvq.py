@@ -85,6 +85,8 @@ def lib():
             "kvq_decode_partial": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, SZ, I32,
                                          P, P]),
             "kvq_decode_combine": (I32, [FP, I32, I32, I32, I64, I32, I32, P, SZ, P, I32, P]),
+            "kvq_decode_combine_lse": (I32, [FP, I32, I32, I32, I64, I32, I32, P, SZ, P, P, P]),
+            "kvq_merge_states": (I32, [I32, I64, I32, P, P, P, I32, P, P]),
             "kvq_decode_attention_noalloc": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float,
                                                    P, I32, I32, P, P]),
         }
@@ -247,6 +249,29 @@ def decode_combine(fmt, B, Hq, Hkv, t_quant, t_res, workspace: torch.Tensor, out
                                   _ptr(workspace), workspace.numel(), _ptr(out),
                                   KVQ_DTYPE[out.dtype], _stream(stream))
     _check("kvq_decode_combine", st)
+    return out
+
+
+def decode_combine_lse(fmt, B, Hq, Hkv, t_quant, t_res, workspace: torch.Tensor, out: torch.Tensor,
+                       lse: torch.Tensor, num_splits=0, stream=None):
+    """kvq_decode_combine_lse: out [B, Hq, D] fp32 and lse [B, Hq] fp32 of one part."""
+    st = lib().kvq_decode_combine_lse(ctypes.byref(fmt), B, Hq, Hkv, t_quant, t_res, num_splits,
+                                      _ptr(workspace), workspace.numel(), _ptr(out), _ptr(lse),
+                                      _stream(stream))
+    _check("kvq_decode_combine_lse", st)
+    return out, lse
+
+
+def merge_states(outs: torch.Tensor, lses: torch.Tensor, out_dtype=F32, out=None, lse_out=None,
+                 stream=None):
+    """kvq_merge_states: outs [n, rows..., D] fp32, lses [n, rows...] fp32 -> out [rows..., D]."""
+    n, D = outs.shape[0], outs.shape[-1]
+    rows = lses[0].numel()
+    if out is None:
+        out = torch.empty(outs.shape[1:], dtype=TORCH_DTYPE[out_dtype], device=outs.device)
+    st = lib().kvq_merge_states(n, rows, D, _ptr(outs), _ptr(lses), _ptr(out), KVQ_DTYPE[out.dtype],
+                                _ptr(lse_out), _stream(stream))
+    _check("kvq_merge_states", st)
     return out
 
 

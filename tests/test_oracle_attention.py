@@ -95,3 +95,25 @@ def test_rope_identities():
 def test_rel_l2():
     assert attention.rel_l2([3.0, 4.0], [3.0, 4.0]) == 0.0
     assert abs(attention.rel_l2([3.0, 4.0], [0.0, 5.0]) - math.sqrt(10) / 5) < 1e-15
+
+
+def test_merge_of_disjoint_parts_is_attention_over_the_union():
+    # the softmax over a union of token sets splits into per-set weights exp(lse_r - lse)
+    from oracle.attention import attention_lse, merge_parts
+    rng = np.random.default_rng(17)
+    q = rng.standard_normal((4, 32)) * 2.0
+    K = rng.standard_normal((50, 32))
+    V = rng.standard_normal((50, 32))
+    whole, lse = attention_lse(q, K, V, 0.3)
+    np.testing.assert_allclose(whole, attention.attention(q, K, V, 0.3), rtol=1e-13, atol=1e-14)
+    # lse by brute force
+    brute = np.array([np.log(sum(np.exp(0.3 * float(q[g] @ K[t])) for t in range(50))) for g in range(4)])
+    np.testing.assert_allclose(lse, brute, rtol=1e-13)
+    cuts = [0, 7, 30, 31, 50]
+    parts = [attention_lse(q, K[a:b], V[a:b], 0.3) for a, b in zip(cuts, cuts[1:])]
+    merged, mlse = merge_parts([p[0] for p in parts], [p[1] for p in parts])
+    np.testing.assert_allclose(merged, whole, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(mlse, lse, rtol=1e-13)
+    # one part is the identity
+    one, one_lse = merge_parts([whole], [lse])
+    np.testing.assert_allclose(one, whole, rtol=1e-15)
