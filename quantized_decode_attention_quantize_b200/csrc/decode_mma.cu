@@ -585,7 +585,7 @@ __device__ __forceinline__ void split_bf162(float x0, float x1, uint32_t* hi, ui
 // The score of token t is sum_s B[s] A[t][s] over slots: A holds the codes as fp16
 // subnormals in place (2-bit field f of a word: factor 4^f; 4-bit nibble: 1 or 16) and
 // the raw slots as bf16; B[s] = q[order[s]] s_s 2^(24 - e) / factor for coded slots and
-// q[order[s]] for raw ones; sum_s q[order[s]] z_s is the bias.  Lane (g, j) builds its
+// q[order[s]] 2^-e for raw ones; sum_s q[order[s]] z_s is the bias.  Lane (g, j) builds its
 // own fragments (head g, or with DUAL the low part of head g - 4 for g >= 4) from the
 // slot products that the warp first writes to its scratch in slot order.
 //
@@ -650,7 +650,10 @@ __device__ __forceinline__ void key_operand_mixed(const MmaArgs& a, const uint8_
   if (amax > 0.0f) ex = (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 + 10;
   ex = max(-100, min(127, ex));
   ko.mult = pow2(ex);
-  const float sc = lane >= 2 ? __uint_as_float((uint32_t)max(1, min(254, 127 + 24 - ex)) << 23) : 1.0f;
+  // coded slots: 2^(24 - ex) (the codes enter as c 2^-24); raw slots: 2^-ex, so that after
+  // the accumulator is scaled by 2^ex both give q . k (powers of two: exact)
+  const float sc = lane >= 2 ? __uint_as_float((uint32_t)max(1, min(254, 127 + 24 - ex)) << 23)
+                             : __uint_as_float((uint32_t)max(1, min(254, 127 - ex)) << 23);
 #pragma unroll
   for (int hh = 0; hh < GM; ++hh)
     *reinterpret_cast<float4*>(av + hh * 128 + 4 * lane) =
@@ -738,14 +741,12 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
   // all four tiles' code words first, then the k-steps tile by tile so that consecutive
   // products go to different accumulators
   float S[4][4];
-  float Sr[MIX ? 4 : 1][4];   // MIXED: raw-slot products, already in score units
   if constexpr (MIX) {
     // per tile: the 2-bit words 4 sg + j, the 4-bit word j and the raw word j of rows
     // g and g + 8 (k-step layout in key_operand_mixed)
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
       S[mt][0] = S[mt][1] = S[mt][2] = S[mt][3] = 0.0f;
-      Sr[mt][0] = Sr[mt][1] = Sr[mt][2] = Sr[mt][3] = 0.0f;
       const int r0 = 16 * mt + g, r1 = r0 + 8;
 #pragma unroll
       for (int sg = 0; sg < 2; ++sg) {
@@ -782,8 +783,8 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
       {
         const uint32_t x0 = *reinterpret_cast<const uint32_t*>(stage + kMixRaw + r0 * 16 + 4 * j);
         const uint32_t x1 = *reinterpret_cast<const uint32_t*>(stage + kMixRaw + r1 * 16 + 4 * j);
-        mma16816_bf16(Sr[mt], x0, x1, 0u, 0u, ko.bh[10][0], ko.bh[10][1]);
-        if (!DUAL) mma16816_bf16(Sr[mt], x0, x1, 0u, 0u, ko.bl[10][0], ko.bl[10][1]);
+        mma16816_bf16(S[mt], x0, x1, 0u, 0u, ko.bh[10][0], ko.bh[10][1]);
+        if (!DUAL) mma16816_bf16(S[mt], x0, x1, 0u, 0u, ko.bl[10][0], ko.bl[10][1]);
       }
     }
   } else {
@@ -820,10 +821,7 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        S[mt][e] += __shfl_xor_sync(0xffffffffu, S[mt][e], 2);
-        if constexpr (MIX) Sr[mt][e] += __shfl_xor_sync(0xffffffffu, Sr[mt][e], 2);
-      }
+      for (int e = 0; e < 4; ++e) S[mt][e] += __shfl_xor_sync(0xffffffffu, S[mt][e], 2);
   }
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
@@ -831,10 +829,6 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
     S[mt][1] = fmaf(S[mt][1], ko.mult, ko.bias1);
     S[mt][2] = fmaf(S[mt][2], ko.mult, ko.bias0);
     S[mt][3] = fmaf(S[mt][3], ko.mult, ko.bias1);
-    if constexpr (MIX) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) S[mt][e] += Sr[mt][e];
-    }
   }
   const bool partial = tvalid < 64;
   if (partial) {
