@@ -149,3 +149,27 @@ def test_workspace_bytes_with_explicit_splits():
     n = kvq.decode_workspace_bytes(f, 1, 32, 32, 4096, 0, 4)
     rows = 32 * 4
     assert n == 2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4
+
+
+def test_sequence_split_entry_points_validate_on_the_host():
+    # nothing is launched: every call below fails validation before touching memory
+    L = kvq.lib()
+    f = _fmt()
+    ws = ctypes.c_void_p(0x400000)
+    out = ctypes.c_void_p(0x200000)
+    lse = ctypes.c_void_p(0x500000)
+    # combine_lse: missing or misaligned lse, too small a workspace
+    assert L.kvq_decode_combine_lse(ctypes.byref(f), 1, 4, 1, 256, 0, 0, ws, 1 << 20, out, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_decode_combine_lse(ctypes.byref(f), 1, 4, 1, 256, 0, 0, ws, 1 << 20, out,
+                                    ctypes.c_void_p(0x500004), None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_decode_combine_lse(ctypes.byref(f), 1, 4, 1, 256, 0, 0, ws, 4, out, lse, None) == kvq.KVQ_ERR_WORKSPACE
+    # merge: part count, rows, head dim, dtype, alignment
+    outs = ctypes.c_void_p(0x600000)
+    lses = ctypes.c_void_p(0x700000)
+    assert L.kvq_merge_states(0, 8, 128, outs, lses, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_merge_states(5000, 8, 128, outs, lses, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_merge_states(2, 0, 128, outs, lses, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_merge_states(2, 8, 96, outs, lses, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_merge_states(2, 8, 128, outs, lses, out, 9, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_merge_states(2, 8, 128, ctypes.c_void_p(0x600008), lses, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_merge_states(2, 8, 128, outs, None, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
