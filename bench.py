@@ -37,7 +37,7 @@ METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize 
 L2_FLUSH_BYTES = 512 << 20
 LAUNCHES_PER_STEP = 3   # quantize K+V (one launch on the K4/V2 path), split kernel, combine
 PATH_DTYPE = {
-    "decode_mma_kernel": "f16 tensor-core products with f32 accumulation (u4/u2 codes; bf16 raw key slots)",
+    "decode_mma_kernel": "f16 tensor-core operands (codes as exact f16 subnormals), f32 accumulation",
     "decode_cc_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
     "decode_generic_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
 }
@@ -560,7 +560,9 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": PATH_DTYPE[path],
+        "vs_baseline": None,
+        "dtype": PATH_DTYPE[path] + ("; raw key slots bf16" if fd["k_scheme"] == synth.MIXED and
+                                     path == "decode_mma_kernel" else ""),
         "data": "synthetic (device-drawn, recipe of synth/)",
         "config": workload_config(cfg),
         "pct_of_8tbs": 100.0 * value / world / 8000.0,
