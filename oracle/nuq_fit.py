@@ -8,8 +8,11 @@ normalized per vector to [-1, 1] by the vector's midpoint and half-range (the
 NormalFloat convention the page says KVQuant builds on), with the vector's outliers
 left out, then rounded to fp16 and sorted.
 
-Parity unpinned: the page gives no centroid values.  The fit only produces an input
-(the codebook) that both the library and the oracle then take as given.
+Pinned (tests/test_oracle_nuq_fit.py): Lloyd recovers eight point masses, gives equal
+cells on a uniform grid and the brute-force best split for k = 2; the normalization maps
+the dense range onto [-1, 1] without the outliers.  Parity unpinned: the centroid values
+for real data (the page gives none).  The fit only produces an input (the codebook)
+that both the library and the oracle then take as given.
 """
 from __future__ import annotations
 
