@@ -16,7 +16,12 @@ t: pairs (i, i + D/2), theta_i = base^(-2i/D), the rotate-half convention.
 Pinned by tests/test_oracle_attention.py (T = 1 returns v_0, q = 0 returns the mean
 of v, equal keys return the mean, shift invariance, a pure-Python brute force on
 tiny shapes, RoPE identities: norm preservation, identity at t = 0, dependence of
-q_m . k_n on n - m only).
+q_m . k_n on n - m only; the log-sum-exp by brute force, and the merge of disjoint
+token sets equal to the attention over their union).
+
+attention_lse / merge_parts state the sequence split ([KVQ] "Approach": contexts spread
+over GPUs): each set of tokens gives its output and lse = log sum_t exp(scale q . k_t),
+and the union's softmax weights split into exp(lse_r - lse) per set.
 """
 from __future__ import annotations
 
