@@ -1,0 +1,125 @@
+"""KQV: scalar MSE codes for the keys, scalar codes plus a 1-bit QJL sketch of the
+residual for the values, both after a Walsh-Hadamard rotation.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  The library does not implement
+this scheme yet; these definitions are the reference its kernels will be held to.
+
+[TQ] "Statistical Inference and Quality Measures of KV Cache Quantisations Inspired by
+TurboQuant", Technical Summary: "Theoretical Framework" (a coordinate of a uniformly
+random unit vector in d dimensions is Beta((d-1)/2, (d-1)/2)-distributed on [-1, 1]),
+"Quantization Schemes" (KQV: rotation of K and V; K by n-bit scalar MSE codes; V by
+(n-1)-bit scalar MSE codes and a 1-bit QJL sketch) and "Key Contributions" (the sketch
+is unbiased; its inner-product variance is pi/2 ||r||^2 / d).
+
+Readings (the page names the pieces, not their constants):
+  * "n bits" is a per-coordinate budget: K n bits a coordinate, V n - 1 bits and one
+    sketch bit;
+  * the scalar MSE quantizer is the Lloyd-Max quantizer of that Beta marginal, applied to
+    the rotated vector divided by its norm; the norm is kept in float64 here;
+  * the sketch of a residual r is s = sign(S r) in {-1, +1}^m (sign(0) = +1) with the
+    norm ||r|| kept, S an m x d matrix of independent N(0, 1) entries that is an input
+    (the method's random numbers are drawn outside and passed in); m = d;
+  * the estimators are <q, r> ~ sqrt(pi/2) / m ||r|| <S q, s> and
+    r ~ sqrt(pi/2) / m ||r|| S^T s (both unbiased over S);
+  * the rotation is the orthonormal Sylvester Walsh-Hadamard matrix in float64.
+
+Pins (tests/test_oracle_kqv.py): at d = 3 the marginal is uniform and Lloyd-Max is the
+uniform quantizer; the 1-bit centroid is E|x| in closed form at every d; for large d the
+scaled centroids approach the Gaussian Lloyd-Max table; the sketch's mean and variance
+match the closed forms by Monte Carlo over seeded S.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import scipy.linalg
+
+
+def marginal_pdf(x, d):
+    """Density of one coordinate of a uniformly random unit vector in R^d, on [-1, 1]:
+    (1 - x^2)^((d - 3) / 2) / B(1/2, (d - 1)/2)."""
+    x = np.asarray(x, np.float64)
+    logc = math.lgamma(d / 2.0) - math.lgamma(0.5) - math.lgamma((d - 1) / 2.0)
+    inside = np.abs(x) < 1.0
+    xi = np.where(inside, x, 0.0)
+    return np.where(inside, np.exp(logc + (d - 3) / 2.0 * np.log1p(-xi * xi)), 0.0)
+
+
+def lloyd_max(bits, d, iters=300, grid=400001):
+    """Lloyd-Max centroids (2^bits, ascending) of the marginal at dimension d: thresholds at
+    midpoints, centroids at the conditional means, by midpoint quadrature on a uniform grid
+    over [-L, L], L = min(1, 14 / sqrt(d)) (the mass beyond 14 standard deviations is below
+    1e-40)."""
+    k = 1 << bits
+    L = min(1.0, 14.0 / math.sqrt(d))
+    x = (np.arange(grid) + 0.5) / grid * 2.0 * L - L
+    w = marginal_pdf(x, d)
+    w = w / w.sum()
+    cdf = np.cumsum(w)
+    c = np.interp((np.arange(k) + 0.5) / k, cdf, x)
+    for _ in range(iters):
+        t = (c[:-1] + c[1:]) / 2.0
+        lab = np.searchsorted(t, x, side="left")
+        mass = np.bincount(lab, weights=w, minlength=k)
+        mom = np.bincount(lab, weights=w * x, minlength=k)
+        c = np.where(mass > 0, mom / np.maximum(mass, 1e-300), c)
+    return np.sort(c)
+
+
+def rotation(d):
+    """The orthonormal Walsh-Hadamard matrix H_d / sqrt(d) (symmetric, its own inverse)."""
+    return scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)
+
+
+def scalar_encode(y, cb):
+    """Codes of y / ||y|| against the centroids cb (nearest, a midpoint going low), and ||y||."""
+    y = np.asarray(y, np.float64)
+    nrm = float(np.linalg.norm(y))
+    u = y / nrm if nrm > 0 else np.zeros_like(y)
+    mids = (cb[:-1] + cb[1:]) / 2.0
+    return np.searchsorted(mids, u, side="left"), nrm
+
+
+def scalar_decode(codes, nrm, cb):
+    return nrm * np.asarray(cb)[codes]
+
+
+def qjl_sketch(r, S):
+    """(signs of S r in {-1, +1}, ||r||)."""
+    p = np.asarray(S, np.float64) @ np.asarray(r, np.float64)
+    return np.where(p >= 0.0, 1.0, -1.0), float(np.linalg.norm(r))
+
+
+def qjl_inner(q, signs, rnorm, S):
+    """Unbiased estimate of <q, r> from the sketch of r."""
+    m = S.shape[0]
+    return math.sqrt(math.pi / 2.0) / m * rnorm * float((np.asarray(S) @ np.asarray(q, np.float64)) @ signs)
+
+
+def qjl_vector(signs, rnorm, S):
+    """Unbiased estimate of r itself from its sketch."""
+    m = S.shape[0]
+    return math.sqrt(math.pi / 2.0) / m * rnorm * (np.asarray(S).T @ signs)
+
+
+def kqv_key(k, bits, cb=None):
+    """Reconstruction of a key row under KQV: rotate, n-bit scalar codes, back."""
+    d = k.shape[-1]
+    R = rotation(d)
+    cb = lloyd_max(bits, d) if cb is None else cb
+    codes, nrm = scalar_encode(R @ k, cb)
+    return R @ scalar_decode(codes, nrm, cb)
+
+
+def kqv_value(v, bits, S, cb=None):
+    """Reconstruction of a value row under KQV: rotate, (n-1)-bit scalar codes, plus the
+    sketch estimate of the residual, back."""
+    d = v.shape[-1]
+    R = rotation(d)
+    cb = lloyd_max(bits - 1, d) if cb is None else cb
+    y = R @ v
+    codes, nrm = scalar_encode(y, cb)
+    yh = scalar_decode(codes, nrm, cb)
+    signs, rn = qjl_sketch(y - yh, S)
+    return R @ (yh + qjl_vector(signs, rn, S))

@@ -1,0 +1,105 @@
+"""Pins of the KQV oracle (oracle.kqv): the Lloyd-Max quantizer of the Beta coordinate
+marginal against closed forms and textbook tables, and the QJL sketch against its
+closed-form mean and variance by Monte Carlo over seeded sketch matrices."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import kqv
+
+
+@pytest.mark.parametrize("d", [3, 8, 128, 2049])
+def test_marginal_is_a_symmetric_density(d):
+    L = min(1.0, 14.0 / math.sqrt(d))
+    x = np.linspace(-L, L, 400001)
+    f = kqv.marginal_pdf(x, d)
+    assert abs(np.trapezoid(f, x) - 1.0) < 1e-5   # (d = 3: half a cell lost at each open end)
+    np.testing.assert_allclose(f, f[::-1], rtol=1e-9, atol=1e-12 * f.max())
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3])
+def test_d3_marginal_is_uniform_so_lloyd_max_is_the_uniform_quantizer(bits):
+    # a coordinate of a random unit vector in R^3 is uniform on [-1, 1] (Archimedes)
+    k = 1 << bits
+    want = (2 * np.arange(k) + 1) / k - 1.0
+    np.testing.assert_allclose(kqv.lloyd_max(bits, 3), want, atol=1e-5)
+
+
+@pytest.mark.parametrize("d", [3, 16, 128, 2049])
+def test_one_bit_centroid_is_the_mean_absolute_coordinate(d):
+    # E|x| = Gamma(d/2) / (sqrt(pi) Gamma((d+1)/2))
+    ex = math.exp(math.lgamma(d / 2.0) - math.lgamma(0.5) - math.lgamma((d + 1) / 2.0))
+    c = kqv.lloyd_max(1, d)
+    np.testing.assert_allclose(c, [-ex, ex], rtol=1e-4)
+
+
+def test_large_d_approaches_the_gaussian_lloyd_max_table():
+    # Max (1960), N(0, 1): 1 bit 0.7979; 2 bits 0.4528, 1.510; 3 bits 0.2451, 0.7560,
+    # 1.344, 2.152 (positive halves); the marginal tends to N(0, 1/d)
+    table = {1: [0.7979], 2: [0.4528, 1.510], 3: [0.2451, 0.7560, 1.344, 2.152]}
+    d = 20001
+    for bits, pos in table.items():
+        c = kqv.lloyd_max(bits, d) * math.sqrt(d)
+        np.testing.assert_allclose(c[len(c) // 2:], pos, atol=2e-3)
+        np.testing.assert_allclose(c[: len(c) // 2], -np.array(pos[::-1]), atol=2e-3)
+
+
+def test_lloyd_max_is_a_fixed_point():
+    # centroids are the conditional means of the cells between midpoints
+    c = kqv.lloyd_max(2, 128)
+    np.testing.assert_allclose(kqv.lloyd_max(2, 128, iters=301), c, atol=1e-12)
+
+
+def _sketch_samples(q, r, m, n, seed):
+    rng = np.random.default_rng(seed)
+    S = rng.standard_normal((n, m, q.size))
+    signs = np.where(S @ r >= 0, 1.0, -1.0)
+    return math.sqrt(math.pi / 2) / m * np.linalg.norm(r) * np.einsum("nm,nm->n", S @ q, signs), S, signs
+
+
+@pytest.mark.parametrize("orthogonal", [True, False])
+def test_qjl_inner_product_is_unbiased_with_the_stated_variance(orthogonal):
+    d = m = 64
+    rng = np.random.default_rng(1)
+    r = rng.standard_normal(d) * 0.3
+    q = rng.standard_normal(d)
+    if orthogonal:
+        q -= (q @ r) / (r @ r) * r
+    est, S, signs = _sketch_samples(q, r, m, 4000, 2)
+    # the library-facing function agrees with the vectorized estimate
+    assert est[0] == pytest.approx(kqv.qjl_inner(q, signs[0], np.linalg.norm(r), S[0]), rel=1e-12)
+    var = (math.pi / 2 * (q @ q) * (r @ r) - (q @ r) ** 2) / m
+    if orthogonal:   # the page's pi/2 ||r||^2 / d, for a unit query
+        assert var == pytest.approx(math.pi / 2 * (r @ r) * (q @ q) / d, rel=1e-9)
+    assert abs(est.mean() - q @ r) < 4 * math.sqrt(var / est.size)
+    assert est.var() == pytest.approx(var, rel=0.1)
+
+
+def test_qjl_vector_and_kqv_values_are_unbiased():
+    d = 32
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal(d)
+    n = 3000
+    Ss = rng.standard_normal((n, d, d))
+    cb = kqv.lloyd_max(1, d)
+    recon = np.array([kqv.kqv_value(v, 2, S, cb) for S in Ss])
+    err = recon.mean(axis=0) - v
+    # per-coordinate standard error of the mean of the sketch estimate
+    se = recon.std(axis=0) / math.sqrt(n)
+    assert np.all(np.abs(err) < 5 * se + 1e-12)
+    # one draw: the scalar part alone is biased towards the codebook, the sketch removes it
+    yh_only = kqv.rotation(d) @ kqv.scalar_decode(*kqv.scalar_encode(kqv.rotation(d) @ v, cb), cb)
+    assert np.linalg.norm(recon.mean(axis=0) - v) < 0.25 * np.linalg.norm(yh_only - v)
+
+
+def test_key_codes_reconstruct_within_the_codebook_error():
+    d = 128
+    rng = np.random.default_rng(4)
+    k = rng.standard_normal(d)
+    for bits in (2, 3, 4):
+        kh = kqv.kqv_key(k, bits)
+        rel = np.linalg.norm(kh - k) / np.linalg.norm(k)
+        # Lloyd-Max MSE of a Gaussian: 0.1175 (2 bits), 0.03454 (3), 0.009497 (4), per unit variance
+        mse = {2: 0.1175, 3: 0.03454, 4: 0.009497}[bits]
+        assert rel < 2.0 * math.sqrt(mse)
