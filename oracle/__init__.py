@@ -17,6 +17,8 @@ Sources (web pages, cited by title and section):
   [MIX]   "MixKVQ: Query-Aware Mixed-Precision KV Cache Quantization for
           Long-Context Reasoning"
   [K4V2]  "Quantize What Counts: More for Keys, Less for Values"
+  [TQ]    "Statistical Inference and Quality Measures of KV Cache Quantisations
+          Inspired by TurboQuant"
 
 Parity status of each module is stated in its docstring.  Parts with no pin to
 anything outside the oracle are marked "parity unpinned".
