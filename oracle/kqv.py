@@ -46,11 +46,13 @@ def marginal_pdf(x, d):
     return np.where(inside, np.exp(logc + (d - 3) / 2.0 * np.log1p(-xi * xi)), 0.0)
 
 
-def lloyd_max(bits, d, iters=300, grid=400001):
+def lloyd_max(bits, d, iters=300, grid=400000):
     """Lloyd-Max centroids (2^bits, ascending) of the marginal at dimension d: thresholds at
     midpoints, centroids at the conditional means, by midpoint quadrature on a uniform grid
     over [-L, L], L = min(1, 14 / sqrt(d)) (the mass beyond 14 standard deviations is below
-    1e-40)."""
+    1e-40).  The density is symmetric, so each iteration keeps the centroids symmetric
+    (on a discrete grid an off-centre fixed point, one grid point away, exists as well);
+    an even number of grid points keeps the central threshold 0 off the grid."""
     k = 1 << bits
     L = min(1.0, 14.0 / math.sqrt(d))
     x = (np.arange(grid) + 0.5) / grid * 2.0 * L - L
@@ -64,6 +66,7 @@ def lloyd_max(bits, d, iters=300, grid=400001):
         mass = np.bincount(lab, weights=w, minlength=k)
         mom = np.bincount(lab, weights=w * x, minlength=k)
         c = np.where(mass > 0, mom / np.maximum(mass, 1e-300), c)
+        c = (c - c[::-1]) / 2.0   # the density is symmetric, so is its Lloyd-Max quantizer
     return np.sort(c)
 
 

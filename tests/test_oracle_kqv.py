@@ -23,7 +23,7 @@ def test_d3_marginal_is_uniform_so_lloyd_max_is_the_uniform_quantizer(bits):
     # a coordinate of a random unit vector in R^3 is uniform on [-1, 1] (Archimedes)
     k = 1 << bits
     want = (2 * np.arange(k) + 1) / k - 1.0
-    np.testing.assert_allclose(kqv.lloyd_max(bits, 3), want, atol=1e-5)
+    np.testing.assert_allclose(kqv.lloyd_max(bits, 3), want, atol=1e-9)
 
 
 @pytest.mark.parametrize("d", [3, 16, 128, 2049])
@@ -31,7 +31,7 @@ def test_one_bit_centroid_is_the_mean_absolute_coordinate(d):
     # E|x| = Gamma(d/2) / (sqrt(pi) Gamma((d+1)/2))
     ex = math.exp(math.lgamma(d / 2.0) - math.lgamma(0.5) - math.lgamma((d + 1) / 2.0))
     c = kqv.lloyd_max(1, d)
-    np.testing.assert_allclose(c, [-ex, ex], rtol=1e-4)
+    np.testing.assert_allclose(c, [-ex, ex], rtol=1e-8)
 
 
 def test_large_d_approaches_the_gaussian_lloyd_max_table():
@@ -103,3 +103,20 @@ def test_key_codes_reconstruct_within_the_codebook_error():
         # Lloyd-Max MSE of a Gaussian: 0.1175 (2 bits), 0.03454 (3), 0.009497 (4), per unit variance
         mse = {2: 0.1175, 3: 0.03454, 4: 0.009497}[bits]
         assert rel < 2.0 * math.sqrt(mse)
+
+
+def test_stored_codebooks_are_the_oracle_s():
+    # tests/golden/kqv_codebooks.json is written by tests/golden/make_kqv_codebooks.py
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "kqv_codebooks.json")
+    stored = json.load(open(path))
+    assert stored["d"] == 128
+    for b in ("1", "2", "3"):
+        np.testing.assert_allclose(stored["f64"][b], kqv.lloyd_max(int(b), 128), rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(np.float32(stored["f64"][b]), np.float32(stored["f32"][b]))
+    # symmetric, strictly increasing, inside [-1, 1]
+    for b, c in stored["f64"].items():
+        c = np.array(c)
+        assert c.size == 1 << int(b) and np.all(np.diff(c) > 0) and np.all(np.abs(c) < 1)
+        np.testing.assert_allclose(c, -c[::-1], atol=1e-6)
