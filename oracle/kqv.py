@@ -26,7 +26,8 @@ Readings (the page names the pieces, not their constants):
 Pins (tests/test_oracle_kqv.py): at d = 3 the marginal is uniform and Lloyd-Max is the
 uniform quantizer; the 1-bit centroid is E|x| in closed form at every d; for large d the
 scaled centroids approach the Gaussian Lloyd-Max table; the sketch's mean and variance
-match the closed forms by Monte Carlo over seeded S.
+match the closed forms by Monte Carlo over seeded S; and the page's effect holds at the
+4-bit budget: KQV keys give a lower attention KL divergence than QKQV keys.
 """
 from __future__ import annotations
 
@@ -126,3 +127,10 @@ def kqv_value(v, bits, S, cb=None):
     yh = scalar_decode(codes, nrm, cb)
     signs, rn = qjl_sketch(y - yh, S)
     return R @ (yh + qjl_vector(signs, rn, S))
+
+
+def qkqv_key(k, bits, S, cb=None):
+    """A key row under QKQV (the comparison scheme): (n-1)-bit scalar codes plus the sketch
+    of the residual, like a KQV value.  Its scores q . k^ are the scalar part plus the
+    sketch's unbiased inner-product estimate."""
+    return kqv_value(k, bits, S, cb)

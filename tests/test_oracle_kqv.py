@@ -120,3 +120,28 @@ def test_stored_codebooks_are_the_oracle_s():
         c = np.array(c)
         assert c.size == 1 << int(b) and np.all(np.diff(c) > 0) and np.all(np.abs(c) < 1)
         np.testing.assert_allclose(c, -c[::-1], atol=1e-6)
+
+
+def test_keys_without_the_sketch_give_lower_attention_kl():
+    # [TQ] "Key Contributions" 2: at the 4-bit budget KQV (4-bit scalar keys) has a lower
+    # KL divergence of the attention weights than QKQV (3-bit keys + 1-bit sketch): the
+    # sketch's variance is amplified by the softmax.  The page reports 2.25x on its data.
+    d, T, G = 64, 256, 4
+    cb4, cb3 = kqv.lloyd_max(4, d), kqv.lloyd_max(3, d)
+    for seed in range(3):
+        rng = np.random.default_rng(seed)
+        q = rng.standard_normal((G, d))
+        K = rng.standard_normal((T, d))
+        Kk = np.array([kqv.kqv_key(k, 4, cb4) for k in K])
+        Kq = np.array([kqv.qkqv_key(k, 4, rng.standard_normal((d, d)), cb3) for k in K])
+
+        def probs(Kx):
+            s = (q @ Kx.T) / math.sqrt(d)
+            s -= s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            return p / p.sum(axis=1, keepdims=True)
+
+        p0, pk, pq = probs(K), probs(Kk), probs(Kq)
+        kl_k = float((p0 * np.log(p0 / pk)).sum(axis=1).mean())
+        kl_q = float((p0 * np.log(p0 / pq)).sum(axis=1).mean())
+        assert kl_q > 2.0 * kl_k
