@@ -65,12 +65,27 @@ def attention_lse(q, K, V, scale):
 
 def merge_parts(outs, lses):
     """Attention over disjoint token sets from each set's (out, lse): the softmax weights of
-    the union split into per-set weights exp(lse_r - lse), lse = log sum_r exp(lse_r)."""
+    the union split into per-set weights exp(lse_r - lse), lse = log sum_r exp(lse_r).
+    A set without tokens has lse = -inf and weight 0 (its out is never read).  When no set
+    has tokens (every lse = -inf) the union is empty and carries no softmax mass; the pages
+    do not treat that case, and the reading taken is out = 0, lse = -inf."""
     outs = np.asarray(outs, np.float64)
     lses = np.asarray(lses, np.float64)
-    m = lses.max(axis=0)
-    w = np.exp(lses - m)
-    return (w[..., None] * outs).sum(axis=0) / w.sum(axis=0)[..., None], m + np.log(w.sum(axis=0))
+    n, D = outs.shape[0], outs.shape[-1]
+    o2 = outs.reshape(n, -1, D)
+    l2 = lses.reshape(n, -1)
+    out = np.zeros(o2.shape[1:])
+    lse = np.full(l2.shape[1], -np.inf)
+    for i in range(l2.shape[1]):
+        live = [r for r in range(n) if l2[r, i] != -np.inf]
+        if not live:
+            continue
+        m = max(l2[r, i] for r in live)
+        w = {r: np.exp(l2[r, i] - m) for r in live}
+        tot = sum(w.values())
+        out[i] = sum(w[r] * o2[r, i] for r in live) / tot
+        lse[i] = m + np.log(tot)
+    return out.reshape(outs.shape[1:]), lse.reshape(lses.shape[1:])
 
 
 def kv_slab(fmt, cache, b, h, t_quant, t_res):

@@ -117,3 +117,29 @@ def test_merge_of_disjoint_parts_is_attention_over_the_union():
     # one part is the identity
     one, one_lse = merge_parts([whole], [lse])
     np.testing.assert_allclose(one, whole, rtol=1e-15)
+
+
+def test_merge_with_empty_parts():
+    # a part with no tokens (lse = -inf) has no weight, whatever its out holds; a row whose
+    # every part is empty merges to out = 0, lse = -inf
+    from oracle.attention import attention_lse, merge_parts
+    rng = np.random.default_rng(23)
+    q = rng.standard_normal((3, 16))
+    K = rng.standard_normal((20, 16))
+    V = rng.standard_normal((20, 16))
+    whole, lse = attention_lse(q, K, V, 0.25)
+    a = attention_lse(q, K[:9], V[:9], 0.25)
+    b = attention_lse(q, K[9:], V[9:], 0.25)
+    empty_out = np.full_like(whole, np.nan)
+    empty_lse = np.full_like(lse, -np.inf)
+    merged, mlse = merge_parts([a[0], empty_out, b[0]], [a[1], empty_lse, b[1]])
+    np.testing.assert_allclose(merged, whole, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(mlse, lse, rtol=1e-13)
+    # rows 0 and 2 lose every token: zeros and -inf there, row 1 unchanged
+    la, lb = a[1].copy(), b[1].copy()
+    la[[0, 2]] = -np.inf
+    lb[[0, 2]] = -np.inf
+    merged, mlse = merge_parts([a[0], b[0]], [la, lb])
+    assert np.all(merged[[0, 2]] == 0.0) and np.all(np.isneginf(mlse[[0, 2]]))
+    np.testing.assert_allclose(merged[1], whole[1], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(mlse[1], lse[1], rtol=1e-13)

@@ -76,3 +76,47 @@ def test_fp32_ops_are_single_roundings():
     np.testing.assert_array_equal(fp.sub32(a, b), (a - b).astype(np.float64))
     np.testing.assert_array_equal(fp.add32(a, b), (a + b).astype(np.float64))
     np.testing.assert_array_equal(fp.mul32(a, b), (a * b).astype(np.float64))
+
+
+def _f32_patterns(seed, n):
+    """Finite float32 values from random bit patterns: normals over the whole exponent
+    range, subnormals, exact bf16 ties (low 16 bits 0x8000) and their neighbours, and
+    the overflow edge."""
+    r = np.random.default_rng(seed)
+    bits = r.integers(0, 1 << 32, n, dtype=np.uint64).astype(np.uint32)
+    sub = r.integers(1, 1 << 23, n // 4, dtype=np.uint64).astype(np.uint32)          # subnormal
+    ties = (r.integers(0, 1 << 16, n // 4, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    near = np.concatenate([ties - 1, ties + 1])
+    edge = np.array([0x7F7F7FFF, 0x7F7F8000, 0x7F7F8001, 0x7F7FFFFF, 0x00008000, 0x00018000,
+                     0x00000001, 0x007FFFFF, 0x00800000], np.uint32)
+    allb = np.concatenate([bits, sub, ties, near, edge])
+    allb = np.concatenate([allb, allb ^ np.uint32(0x80000000)])
+    x = allb.view(np.float32)
+    return x[np.isfinite(x)]
+
+
+def test_bf16_nearest_matches_torch():
+    # bf16 round-to-nearest-even against torch's float32 -> bfloat16 conversion (one
+    # rounding: the float32 inputs are exact in float64)
+    torch = pytest.importorskip("torch")
+    x = _f32_patterns(4, 400000)
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(fp.bf16(x.astype(np.float64), "rn"), want)
+
+
+def test_bf16_directed_roundings_bracket():
+    torch = pytest.importorskip("torch")
+    x = _f32_patterns(5, 100000).astype(np.float64)
+    big = float(torch.finfo(torch.bfloat16).max)
+    x = x[np.abs(x) < big]
+    lo, hi = fp.bf16(x, "rd"), fp.bf16(x, "ru")
+    assert np.all(lo <= x) and np.all(x <= hi)
+    # both representable in bf16, adjacent unless exact
+    rt = lambda v: torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(rt(lo), lo)
+    np.testing.assert_array_equal(rt(hi), hi)
+    exact = lo == x
+    assert np.all((lo == hi) == exact)
+    bl = torch.from_numpy(lo).to(torch.bfloat16)
+    up = torch.nextafter(bl, torch.full_like(bl, float("inf"))).to(torch.float64).numpy()
+    assert np.all(exact | (up >= hi))
