@@ -1193,6 +1193,597 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   }
 }
 
+// ==== K4/V2 keys with G <= 4: the lean kernel ============================================
+// Same partition, ring discipline, math encoding and partial-state contract as
+// decode_mma_kernel, arranged so that every lane owns one query head:
+//  - The key product's N columns are (head 0 high, head 0 remainder, head 1 high, ...):
+//    lane (g, j) ends with the high part and the remainder of head j for tokens g and
+//    g + 8 of the tile and adds them in place; the online softmax then runs on two
+//    values per lane and tile, with m, l and W scalars per lane.
+//  - The probabilities of a tile, packed as (p[g][j] s_g, p[g + 8][j] s_{g+8}), become
+//    the value product's B operand with one 8x8 transpose (movmatrix) and one shuffle:
+//    after the transpose lane (2h, j') holds tokens 2j', 2j' + 1 of head h and lane
+//    (2h + 1, j') tokens 2j' + 8, 2j' + 9, so column 2h of the product is head h and
+//    the odd columns carry values that are never read.
+//  - The key-product B operand of a group is built with every (head, channel) product
+//    formed once: lane L forms head L / 8, channels 16 (L % 8) .. + 15, and the fragments
+//    reach their lanes through the warp's scratch.  Each head has its own exponent.
+//  - Stages arrive by 1-D bulk copies (the TMA engine; this GPU's memory only, no
+//    multicast) on one mbarrier per stage, issued by lane 0; waits are bounded.
+constexpr int kQBytes = 4 * 128 * 4;            // pre-scaled queries of up to four heads
+constexpr int kBScratch = 32 * 16 * 4;          // key-operand fragments on their way to lanes
+constexpr int kLeanWarpBytes = kBuffers * kStageBytes + kQBytes + kBScratch;
+constexpr int kWaitLimit = 1 << 20;             // try_wait rounds before a wait gives up
+static_assert(kRecordFloats * 4 <= kBuffers * kStageBytes, "merge record fits the ring");
+static_assert(64 * 8 <= kBScratch, "value scale / zero-point pairs fit the scratch");
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// 1-D bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`
+// (addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of `parity` to complete; false when kWaitLimit rounds pass first.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  bool ok = false;
+  for (int it = 0; it < kWaitLimit && !ok; ++it) ok = mbar_try_wait(bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void mma16816_n(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movtrans_n(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Copies of one half group (key codes, value codes, value scale / zero-point and, when
+// `with_key`, the group's key scale / zero-point) into a stage; lane 0 only.
+__device__ __forceinline__ void issue_half(const MmaArgs& a, uint8_t* buf, uint64_t* bar, int64_t head,
+                                           int gi, int hf, bool with_key) {
+  const int64_t t0 = (int64_t)gi * 128 + 64 * hf;
+  mbar_expect_tx(bar, kHalfK + kHalfV + kHalfVM + (with_key ? kHalfKM : 0));
+  bulk_g2s(buf, a.k_codes + head * a.k_slab_bytes + t0 * 64, kHalfK, bar);
+  bulk_g2s(buf + kHalfK, a.v_codes + head * a.v_slab_bytes + t0 * 32, kHalfV, bar);
+  bulk_g2s(buf + kHalfK + kHalfV, a.v_scale + head * a.C + t0, 128, bar);
+  bulk_g2s(buf + kHalfK + kHalfV + 128, a.v_zero + head * a.C + t0, 128, bar);
+  if (with_key) {
+    const int64_t grp = head * a.ng + gi;
+    bulk_g2s(buf + kHalfK + kHalfV + kHalfVM, a.k_scale + grp * 128, 256, bar);
+    bulk_g2s(buf + kHalfK + kHalfV + kHalfVM + 256, a.k_zero + grp * 128, 256, bar);
+  }
+}
+
+// Copies of raw item r (its sink and / or residual key rows, then value rows at
+// +kRawBytes) into a stage; lane 0 only.
+__device__ __forceinline__ void issue_raw(const MmaArgs& a, uint8_t* buf, uint64_t* bar, int64_t head, int r) {
+  const int rowb = a.src_dtype == KVQ_F32 ? 512 : 256;
+  const int nraw = a.n_sink + a.t_res;
+  const int t0 = r * a.rt, nt = min(a.rt, nraw - t0);
+  const int ns = max(0, min(nt, a.n_sink - t0));   // sink tokens of the item
+  const int nr = nt - ns;                           // residual tokens of the item
+  mbar_expect_tx(bar, (uint32_t)(2 * nt * rowb));
+  if (ns > 0) {
+    const int64_t row = head * a.n_sink + t0;
+    bulk_g2s(buf, reinterpret_cast<const uint8_t*>(a.sink_k) + row * rowb, ns * rowb, bar);
+    bulk_g2s(buf + kRawBytes, reinterpret_cast<const uint8_t*>(a.sink_v) + row * rowb, ns * rowb, bar);
+  }
+  if (nr > 0) {
+    const int64_t row = head * a.res_cap + (t0 + ns - a.n_sink);
+    bulk_g2s(buf + ns * rowb, reinterpret_cast<const uint8_t*>(a.res_k) + row * rowb, nr * rowb, bar);
+    bulk_g2s(buf + kRawBytes + ns * rowb, reinterpret_cast<const uint8_t*>(a.res_v) + row * rowb, nr * rowb,
+             bar);
+  }
+}
+
+// Online-softmax state of lane (g, j) for head j: O[cm][0] and O[cm][2] are channels
+// d0 = 16 g + 8 (cm >> 2) + 2 (cm & 3) and d0 + 1 (elements 1 and 3 belong to columns
+// that are never read); m, l, W the running max, sum and sum of p z (l and W summed
+// over the lanes g of the column at the end).
+struct LeanState {
+  float O[8][4];
+  float m, l, W;
+};
+
+__device__ __forceinline__ void lean_reset(LeanState& st) {
+#pragma unroll
+  for (int cm = 0; cm < 8; ++cm) st.O[cm][0] = st.O[cm][1] = st.O[cm][2] = st.O[cm][3] = 0.0f;
+  st.m = -INFINITY;
+  st.l = st.W = 0.0f;
+}
+
+__device__ __forceinline__ void lean_rescale(LeanState& st, float mnew) {
+  if (__any_sync(0xffffffffu, mnew != st.m)) {
+    const float c = ex2(st.m - mnew);
+#pragma unroll
+    for (int cm = 0; cm < 8; ++cm) {
+      st.O[cm][0] *= c;
+      st.O[cm][2] *= c;
+    }
+    st.l *= c;
+    st.W *= c;
+    st.m = mnew;
+  }
+}
+
+// Writes the state as (o[hh][128], m[hh], l[hh]) for hh < G (o of head hh at o + hh os,
+// m and l at m + hh ms, l + hh ms); the state is not usable afterwards.
+__device__ void lean_emit(LeanState& st, int G, float* o, int64_t os, float* m, float* l, int64_t ms) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
+#pragma unroll
+  for (int s = 4; s < 32; s <<= 1) {
+    st.l += __shfl_xor_sync(0xffffffffu, st.l, s);
+    st.W += __shfl_xor_sync(0xffffffffu, st.W, s);
+  }
+  if (j < G) {
+    float* dst = o + j * os;
+#pragma unroll
+    for (int cm = 0; cm < 8; ++cm) {
+      const int d0 = 16 * g + 8 * (cm >> 2) + 2 * (cm & 3);
+      *reinterpret_cast<float2*>(dst + d0) = make_float2(fmaf(st.O[cm][0], inv_f_lo(cm & 1), st.W),
+                                                         fmaf(st.O[cm][2], inv_f_hi(cm & 1), st.W));
+    }
+    if (g == 0) {
+      m[j * ms] = st.m;
+      l[j * ms] = st.l;
+    }
+  }
+}
+
+// Sixteen consecutive elements (element offset c0, a multiple of 8) of a raw row in
+// shared memory, as fp32.
+__device__ __forceinline__ void load16(const uint8_t* row, int c0, int dtype, float* v) {
+  if (dtype == KVQ_F32) {
+    const float4* p = reinterpret_cast<const float4*>(row) + c0 / 4;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 x = p[u];
+      v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+    }
+    return;
+  }
+  const uint4* p = reinterpret_cast<const uint4*>(row) + c0 / 8;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const uint4 x = p[u];
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (dtype == KVQ_F16) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        v[8 * u + 2 * k] = f.x;
+        v[8 * u + 2 * k + 1] = f.y;
+      } else {
+        v[8 * u + 2 * k] = __uint_as_float(w[k] << 16);
+        v[8 * u + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+      }
+    }
+  }
+}
+
+// Raw tokens (sink + residual, nt <= 8) staged at stg (key rows, value rows at
+// +kRawBytes): fp32 scores on CUDA cores, lane (g, j) over channels 16 g .. 16 g + 15 of
+// head j, summed over the lanes g; the probabilities go into the state's tiles scaled
+// by each row's field factor f / 2^24.
+__device__ void lean_raw(LeanState& st, const uint8_t* stg, int nt, int dtype, const float* qs) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
+  const float lkeep = g == 0 ? 1.0f : 0.0f;   // l is summed over the eight lanes of a column
+  const int rowb = dtype == KVQ_F32 ? 512 : 256;
+  float q[16];
+  {
+    const float4* p = reinterpret_cast<const float4*>(qs + j * 128 + 16 * g);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 x = p[u];
+      q[4 * u] = x.x; q[4 * u + 1] = x.y; q[4 * u + 2] = x.z; q[4 * u + 3] = x.w;
+    }
+  }
+  float sc[8];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    sc[t] = -INFINITY;
+    if (t < nt) {
+      float k[16];
+      load16(stg + t * rowb, 16 * g, dtype, k);
+      float part = q[0] * k[0];
+#pragma unroll
+      for (int c = 1; c < 16; ++c) part = fmaf(q[c], k[c], part);
+      part += __shfl_xor_sync(0xffffffffu, part, 4);
+      part += __shfl_xor_sync(0xffffffffu, part, 8);
+      part += __shfl_xor_sync(0xffffffffu, part, 16);
+      sc[t] = part;
+      mx = fmaxf(mx, part);
+    }
+  }
+  lean_rescale(st, fmaxf(st.m, mx));
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    if (t < nt) {
+      const float p = ex2(sc[t] - st.m);
+      st.l = fmaf(p, lkeep, st.l);
+      const float pe = p * (1.0f / 16777216.0f), po = p * (1.0f / 1048576.0f);
+      const float qe = p * (1.0f / 4194304.0f), qo = p * (1.0f / 262144.0f);
+      float v[16];
+      load16(stg + kRawBytes + t * rowb, 16 * g, dtype, v);
+#pragma unroll
+      for (int cm = 0; cm < 8; ++cm) {
+        const int i0 = 8 * (cm >> 2) + 2 * (cm & 3);
+        st.O[cm][0] = fmaf((cm & 1) ? po : pe, v[i0], st.O[cm][0]);
+        st.O[cm][2] = fmaf((cm & 1) ? qo : qe, v[i0 + 1], st.O[cm][2]);
+      }
+    }
+  }
+}
+
+// The key-product B operand of a group: b[2 kk + r] is register r of k-step kk for
+// column g' = 2 h + part of lane (g', j') (part 0: the fp16 high part, 1: the remainder
+// of q~[h][c] s[c] 2^(24 - e_h) / f_c over the channels 32 j' .. 32 j' + 31 in the order
+// of the key unpack); mult = 2^e_j and bias = sum_c q~[j][c] z[c] of the lane's head j.
+struct LeanKey {
+  uint32_t b[16];
+  float mult, bias;
+};
+
+__device__ __forceinline__ void lean_key_operand(const __half* ks, const __half* kz, const float* qs,
+                                                 uint32_t* scr, LeanKey& ko) {
+  const int lane = threadIdx.x & 31;
+  const int hL = lane >> 3, cb = lane & 7;   // head, 16-channel block formed by this lane
+  float a[16];
+  float amax = 0.0f, dz = 0.0f;
+  {
+    const float4* q4 = reinterpret_cast<const float4*>(qs + hL * 128 + 16 * cb);
+    const uint4* s4 = reinterpret_cast<const uint4*>(ks + 16 * cb);
+    const uint4* z4 = reinterpret_cast<const uint4*>(kz + 16 * cb);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint4 sv = s4[u], zv = z4[u];
+      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w}, zw[4] = {zv.x, zv.y, zv.z, zv.w};
+      const float4 qa = q4[2 * u], qb = q4[2 * u + 1];
+      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[k]));
+        const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&zw[k]));
+        const int i = 8 * u + 2 * k;
+        a[i] = qv[2 * k] * s2.x;
+        a[i + 1] = qv[2 * k + 1] * s2.y;
+        dz = fmaf(qv[2 * k], z2.x, dz);
+        dz = fmaf(qv[2 * k + 1], z2.y, dz);
+        amax = fmaxf(amax, fmaxf(fabsf(a[i]), fabsf(a[i + 1])));
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
+    dz += __shfl_xor_sync(0xffffffffu, dz, s);
+  }
+  // the head's exponent: max |a 2^(24 - e)| < 2^15
+  int ex = 0;
+  if (amax > 0.0f) ex = (int)((__float_as_uint(amax) >> 23) & 0xff) - 127 + 10;
+  ex = max(-100, min(127, ex));
+  const float mult = pow2(ex);
+  const float sc = __uint_as_float((uint32_t)max(1, min(254, 127 + 24 - ex)) << 23);
+  const float sc16 = sc * 0.0625f;   // channels at the odd nibble of a byte (factor 16)
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {   // channel pairs (p, p + 4) of word 2 cb + u
+      const float f = (p & 1) ? sc16 : sc;
+      const float y0 = a[8 * u + p] * f, y1 = a[8 * u + p + 4] * f;
+      split_half2(y0, y1, &hw[p], &lw[p]);
+    }
+    const int W = 2 * cb + u, jd = W >> 2, w = W & 3;
+    *reinterpret_cast<uint4*>(scr + (4 * (2 * hL) + jd) * 16 + 4 * w) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(scr + (4 * (2 * hL + 1) + jd) * 16 + 4 * w) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint4 x = *reinterpret_cast<const uint4*>(scr + lane * 16 + 4 * u);
+    ko.b[4 * u] = x.x; ko.b[4 * u + 1] = x.y; ko.b[4 * u + 2] = x.z; ko.b[4 * u + 3] = x.w;
+  }
+  ko.mult = __shfl_sync(0xffffffffu, mult, 8 * (lane & 3));
+  ko.bias = __shfl_sync(0xffffffffu, dz, 8 * (lane & 3));
+  __syncwarp();
+}
+
+// 64 tokens (one half of a group) held in a stage; szbuf: the warp's scratch, which
+// receives the half's value scale / zero-point as fp32 pairs.
+__device__ __forceinline__ void lean_half(LeanState& st, const uint8_t* stage, const LeanKey& ko, int tvalid,
+                                          float* szbuf) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
+  const uint4* kc4 = reinterpret_cast<const uint4*>(stage);
+  const uint2* vc2 = reinterpret_cast<const uint2*>(stage + kHalfK);
+  const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stage + kHalfK + kHalfV);
+  {   // tokens 2 lane, 2 lane + 1; tokens past tvalid get (0, 0)
+    float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&vsz[lane]));
+    float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&vsz[32 + lane]));
+    if (2 * lane >= tvalid) s2.x = z2.x = 0.0f;
+    if (2 * lane + 1 >= tvalid) s2.y = z2.y = 0.0f;
+    reinterpret_cast<float4*>(szbuf)[lane] = make_float4(s2.x, z2.x, s2.y, z2.y);
+  }
+  // ---- scores of the 64 tokens (4 tiles of 16) ----
+  float S[4][4];
+  uint4 wlo[4], whi[4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    S[mt][0] = S[mt][1] = S[mt][2] = S[mt][3] = 0.0f;
+    wlo[mt] = kc4[(16 * mt + g) * 4 + j];
+    whi[mt] = kc4[(16 * mt + g + 8) * 4 + j];
+  }
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const uint32_t x0 = w == 0 ? wlo[mt].x : w == 1 ? wlo[mt].y : w == 2 ? wlo[mt].z : wlo[mt].w;
+      const uint32_t x1 = w == 0 ? whi[mt].x : w == 1 ? whi[mt].y : w == 2 ? whi[mt].z : whi[mt].w;
+      const uint32_t p0 = odd_bytes_down(x0), p1 = odd_bytes_down(x1);
+      mma16816_n(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u, ko.b[4 * w],
+                 ko.b[4 * w + 1]);
+      mma16816_n(S[mt], p0 & 0x000F000Fu, p1 & 0x000F000Fu, p0 & 0x00F000F0u, p1 & 0x00F000F0u, ko.b[4 * w + 2],
+                 ko.b[4 * w + 3]);
+    }
+  }
+  // ---- online softmax (log2 domain) on head j, tokens g and g + 8 of every tile ----
+  float x[4][2];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    x[mt][0] = S[mt][0] + S[mt][1];
+    x[mt][1] = S[mt][2] + S[mt][3];
+  }
+  if (tvalid < 64) {
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      if (16 * mt + g >= tvalid) x[mt][0] = -INFINITY;
+      if (16 * mt + g + 8 >= tvalid) x[mt][1] = -INFINITY;
+    }
+  }
+  float lm = fmaxf(fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1])),
+                   fmaxf(fmaxf(x[2][0], x[2][1]), fmaxf(x[3][0], x[3][1])));
+  lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 4));
+  lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 8));
+  lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 16));
+  lean_rescale(st, fmaxf(st.m, fmaf(lm, ko.mult, ko.bias)));
+  const float bm = ko.bias - st.m;
+  __syncwarp();   // the scale / zero-point pairs
+  const float2* sz = reinterpret_cast<const float2*>(szbuf);
+  // ---- value product: one 16-token k-step per score tile ----
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const float p0 = ex2(fmaf(x[mt][0], ko.mult, bm)), p1 = ex2(fmaf(x[mt][1], ko.mult, bm));
+    const float2 a0 = sz[16 * mt + g], a1 = sz[16 * mt + g + 8];
+    st.l += p0 + p1;
+    st.W = fmaf(p0, a0.y, fmaf(p1, a1.y, st.W));
+    const uint32_t pb0 = movtrans_n(pack_half2(p0 * a0.x, p1 * a1.x));
+    const uint32_t pb1 = __shfl_xor_sync(0xffffffffu, pb0, 4);
+    const uint2 va = vc2[(8 * mt + j) * 8 + g];
+    const uint2 vb = vc2[(8 * mt + j + 4) * 8 + g];
+    const uint32_t ya = odd_bytes_down(va.x), yb = odd_bytes_down(vb.x);
+    const uint32_t za = odd_bytes_down(va.y), zb = odd_bytes_down(vb.y);
+    // fields at bits 0, 2, 4, 6 of each half: factors 1, 4, 16, 64
+    mma16816_n(st.O[0], va.x & 0x00030003u, va.x & 0x000C000Cu, vb.x & 0x00030003u, vb.x & 0x000C000Cu, pb0, pb1);
+    mma16816_n(st.O[1], va.x & 0x00300030u, va.x & 0x00C000C0u, vb.x & 0x00300030u, vb.x & 0x00C000C0u, pb0, pb1);
+    mma16816_n(st.O[2], ya & 0x00030003u, ya & 0x000C000Cu, yb & 0x00030003u, yb & 0x000C000Cu, pb0, pb1);
+    mma16816_n(st.O[3], ya & 0x00300030u, ya & 0x00C000C0u, yb & 0x00300030u, yb & 0x00C000C0u, pb0, pb1);
+    mma16816_n(st.O[4], va.y & 0x00030003u, va.y & 0x000C000Cu, vb.y & 0x00030003u, vb.y & 0x000C000Cu, pb0, pb1);
+    mma16816_n(st.O[5], va.y & 0x00300030u, va.y & 0x00C000C0u, vb.y & 0x00300030u, vb.y & 0x00C000C0u, pb0, pb1);
+    mma16816_n(st.O[6], za & 0x00030003u, za & 0x000C000Cu, zb & 0x00030003u, zb & 0x000C000Cu, pb0, pb1);
+    mma16816_n(st.O[7], za & 0x00300030u, za & 0x00C000C0u, zb & 0x00300030u, zb & 0x00C000C0u, pb0, pb1);
+  }
+}
+
+template <bool ROT>
+__global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * kCW + warp;
+  const int64_t i0 = item_start(gw, a.I, a.W), i1 = item_start(gw + 1, a.I, a.W);
+  const int U = a.U;
+  uint8_t* ring = smem + (size_t)warp * kLeanWarpBytes;
+  float* qs = reinterpret_cast<float*>(ring + kBuffers * kStageBytes);
+  uint32_t* scr = reinterpret_cast<uint32_t*>(ring + kBuffers * kStageBytes + kQBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kCW * kLeanWarpBytes) + kBuffers * warp;
+  int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * kLeanWarpBytes + kCW * kBuffers * 8);
+  const int nraw = a.n_sink + a.t_res;
+  const int G = a.G;
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kBuffers; ++s) mbar_init(&bars[s], 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
+
+  // load cursor: one work item ahead of the compute cursor (odd raw positions carry none)
+  int64_t lhead = i0 / U, li = i0;
+  int lr = (int)(i0 - lhead * U);
+  int issued = 0;
+  auto advance_load = [&]() {
+    ++li;
+    if (++lr == U) {
+      lr = 0;
+      ++lhead;
+    }
+  };
+  auto issue_next = [&]() {
+    while (li < i1 && lr < a.nrp && (lr & 1)) advance_load();
+    if (li < i1) {
+      if (lane == 0) {
+        const int sb = issued % kBuffers;
+        uint8_t* buf = ring + sb * kStageBytes;
+        if (lr < a.nrp) {
+          issue_raw(a, buf, &bars[sb], lhead, lr >> 1);
+        } else {
+          const int p = lr - a.nrp;
+          issue_half(a, buf, &bars[sb], lhead, p >> 1, p & 1, (p & 1) == 0 || li == i0);
+        }
+      }
+      ++issued;
+      advance_load();
+    }
+  };
+  issue_next();
+
+  LeanState st;
+  lean_reset(st);
+  LeanKey ko;
+  int64_t head = i0 / U, cur_head = -1;
+  int r = (int)(i0 - head * U);
+  bool qbad = false, qrot = false, timed_out = false;
+  int consumed = 0;
+  // this head's queries, pre-scaled, channels 4 lane .. 4 lane + 3 of every head (as given
+  // for raw tokens; in the Walsh-Hadamard basis for the packed keys of a rotating format)
+  auto load_queries = [&](bool rotated) {
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (hh < G) x = load4(a.q, (head * G + hh) * 128 + 4 * lane, a.q_dtype);
+      qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+      if constexpr (ROT) {
+        if (rotated) x = rotate_q(x, lane, a.rot_scale);
+      }
+      reinterpret_cast<float4*>(qs + hh * 128)[lane] =
+          make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale);
+    }
+    __syncwarp();
+  };
+#pragma unroll 1
+  for (int64_t i = i0; i < i1; ++i) {
+    if (head != cur_head) {
+      if (cur_head >= 0) {   // the range crosses into the next head: slot 0 of this one
+        const int64_t row0 = cur_head * G;
+        lean_emit(st, G, a.ws_o + row0 * a.S * 128, (int64_t)a.S * 128, a.ws_m + row0 * a.S,
+                  a.ws_l + row0 * a.S, a.S);
+        lean_reset(st);
+      }
+      cur_head = head;
+      qrot = ROT && r >= a.nrp;
+      load_queries(qrot);
+    }
+    if (r < a.nrp && (r & 1)) {   // second position of a raw item: no work
+      if (++r == U) {
+        r = 0;
+        ++head;
+      }
+      continue;
+    }
+    if (ROT && r >= a.nrp && !qrot) {   // a head's raw items come first: one switch per head
+      qrot = true;
+      load_queries(true);
+    }
+    // the next item goes into the stage consumed last time, then this one is waited for
+    issue_next();
+    const int sb = consumed % kBuffers;
+    if (!mbar_wait(&bars[sb], (uint32_t)(consumed / kBuffers) & 1u)) {
+      timed_out = true;
+      break;
+    }
+    const uint8_t* stg = ring + sb * kStageBytes;
+    if (r < a.nrp) {
+      lean_raw(st, stg, min(a.rt, nraw - (r >> 1) * a.rt), a.src_dtype, qs);
+    } else {
+      const int p = r - a.nrp, gi = p >> 1, hf = p & 1;
+      if (hf == 0 || i == i0) {
+        const __half* ks = reinterpret_cast<const __half*>(stg + kHalfK + kHalfV + kHalfVM);
+        lean_key_operand(ks, ks + 128, qs, scr, ko);
+      }
+      const int tvalid = (int)min((int64_t)64, a.t_quant - (int64_t)gi * 128 - 64 * hf);
+      lean_half(st, stg, ko, tvalid, reinterpret_cast<float*>(scr));
+    }
+    __syncwarp();
+    ++consumed;
+    if (++r == U) {
+      r = 0;
+      ++head;
+    }
+  }
+  if (timed_out) {
+    // let the copies still in flight land before the stages are reused below
+    for (int c = consumed; c < issued; ++c) mbar_wait(&bars[c % kBuffers], (uint32_t)(c / kBuffers) & 1u);
+    if (lane == 0) flag(a.status, KVQ_DEV_TIMEOUT);
+  }
+  if (__any_sync(0xffffffffu, qbad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+
+  // ---- merge of the warps' last heads inside the CTA (as decode_mma_kernel) ----
+  const int lh = i1 > 0 ? (int)((i1 - 1) / U) : -1;
+  float* rec = reinterpret_cast<float*>(ring);
+  if (lh >= 0) lean_emit(st, G, rec, 128, rec + 8 * 128, rec + 8 * 128 + 8, 1);
+  if (lane == 0) last_head[warp] = lh;
+  __syncthreads();
+  int w0 = 0;
+#pragma unroll 1
+  while (w0 < kCW) {
+    const int h = last_head[w0];
+    int w1 = w0;
+    while (w1 + 1 < kCW && last_head[w1 + 1] == h) ++w1;
+    if (h >= 0) {
+      const int64_t ca = first_ending_warp(h, U, a.I, a.W) / kCW;
+      const int slot = 1 + (int)((int64_t)blockIdx.x - ca);
+#pragma unroll 1
+      for (int idx = threadIdx.x; idx < G * 128; idx += kThreads) {
+        const int hh = idx >> 7, d = idx & 127;
+        float M = -INFINITY;
+        for (int w = w0; w <= w1; ++w) {
+          const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * kLeanWarpBytes);
+          M = fmaxf(M, rw[8 * 128 + hh]);
+        }
+        float o = 0.0f, l = 0.0f;
+        for (int w = w0; w <= w1; ++w) {
+          const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * kLeanWarpBytes);
+          const float mw = rw[8 * 128 + hh];
+          if (mw != -INFINITY) {
+            const float f = ex2(mw - M);
+            o = fmaf(f, rw[hh * 128 + d], o);
+            l = fmaf(f, rw[8 * 128 + 8 + hh], l);
+          }
+        }
+        const int64_t sl = ((int64_t)h * G + hh) * a.S + slot;
+        a.ws_o[sl * 128 + d] = o;
+        if (d == 0) {
+          a.ws_m[sl] = M;
+          a.ws_l[sl] = l;
+        }
+      }
+    }
+    w0 = w1 + 1;
+  }
+}
+
+size_t lean_smem() {
+  return (size_t)kCW * kLeanWarpBytes + (size_t)kCW * kBuffers * 8 + kCW * sizeof(int);
+}
+
 // ---- combine for this path: the valid slots of a head follow from the partition ---------
 struct CombArgsMma {
   int G, S;
@@ -1319,11 +1910,18 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.ws_l = ws_l;
   a.ws_o = ws_o;
   a.status = d_status;
-  const size_t smem = mma_smem();
   const bool mix = L.side[0].scheme == KVQ_MIXED;
+  if (!mix && a.G <= 4) {
+    const size_t smem = lean_smem();
+    auto kern = a.k_rotate ? decode_k4v2_kernel<true> : decode_k4v2_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<p.grid_ctas, kThreads, smem, s>>>(a);
+    return cudaGetLastError();
+  }
+  const size_t smem = mma_smem();
   auto kern = mix ? (a.G <= 4 ? decode_mma_kernel<true, false, true> : decode_mma_kernel<false, false, true>)
-            : a.G <= 4 ? (a.k_rotate ? decode_mma_kernel<true, true, false> : decode_mma_kernel<true, false, false>)
-                       : (a.k_rotate ? decode_mma_kernel<false, true, false> : decode_mma_kernel<false, false, false>);
+            : (a.k_rotate ? decode_mma_kernel<false, true, false> : decode_mma_kernel<false, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<p.grid_ctas, kThreads, smem, s>>>(a);
