@@ -330,7 +330,8 @@ kvq_status kvq_decode_combine_lse(const kvq_format* fmt, int32_t batch, int32_t 
 /* Merge of n_parts such results, gathered into outs[n_parts][rows][head_dim] and
  * lses[n_parts][rows] (device fp32, 16-byte aligned; rows = B * Hq): for every row,
  * out = sum_r w_r outs[r] / sum_r w_r with w_r = exp(lses[r] - max_r lses[r]); a part
- * with lse = -inf (no tokens) has weight 0.  out is written in out_dtype; lse_out
+ * with lse = -inf (no tokens) has weight 0, and a row whose every part has lse = -inf
+ * gets out = 0 and lse_out = -inf.  out is written in out_dtype; lse_out
  * (nullable) receives the merged log-denominator.  The gather itself (one all-gather
  * of (head_dim + 1) * 4 bytes per query row and part) belongs to the caller's
  * collective library.  KVQ_ERR_INVALID for n_parts outside [1, 4096], rows outside
@@ -351,10 +352,13 @@ kvq_status kvq_merge_states(int32_t n_parts, int64_t rows, int32_t head_dim, con
  * Nothing is allocated and nothing is freed.  Returns KVQ_ERR_WORKSPACE when the
  * call would need more than KVQ_NOALLOC_SCRATCH_BYTES (see
  * kvq_decode_workspace_bytes).  The first call on a device looks up the array's
- * device address (with that device current) and keeps it for later calls; make that
- * first call outside any stream capture.  All calls on a device share the one array
- * and it keeps the last call's contents: calls that overlap on the GPU (on different
- * streams, or from different host threads) race with one another. */
+ * device address (with that device current) and keeps it, with the context it belongs
+ * to, for later calls; make that first call outside any stream capture.  A later call
+ * in another context of the device (after cudaDeviceReset, say) looks the address up
+ * again, and that call too should come outside any stream capture.  All calls on a
+ * device share the one array and it keeps the last call's contents: calls that overlap
+ * on the GPU (on different streams, or from different host threads) race with one
+ * another. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (16u << 20)
 kvq_status kvq_decode_attention_noalloc(const kvq_format* fmt, const kvq_cache* cache,
                                         const void* q, int32_t q_dtype, int32_t q_heads,

@@ -885,21 +885,32 @@ __device__ __forceinline__ void mma_half(MmaState& st, const uint8_t* stage, con
     st.W[0] = fmaf(p00, z0, fmaf(p10, z1, st.W[0]));
     st.W[1] = fmaf(p01, z0, fmaf(p11, z1, st.W[1]));
     const float sk0 = s0 * keep, sk1 = s1 * keep;
-    const uint32_t pb0 = movtrans(pack_half2(p00 * sk0, p01 * sk0));
-    const uint32_t pb1 = movtrans(pack_half2(p10 * sk1, p11 * sk1));
+    // P = p s_t as an fp16 high part and an fp16 remainder (about 22 bits): two products
+    // with the same value codes into the same accumulators
+    uint32_t h0, l0, h1, l1;
+    split_half2(p00 * sk0, p01 * sk0, &h0, &l0);
+    split_half2(p10 * sk1, p11 * sk1, &h1, &l1);
+    const uint32_t pb0 = movtrans(h0), pb1 = movtrans(h1);
+    const uint32_t pr0 = movtrans(l0), pr1 = movtrans(l1);
     const uint2 va = *reinterpret_cast<const uint2*>(vc + (8 * mt + j) * 16 + 2 * g);
     const uint2 vb = *reinterpret_cast<const uint2*>(vc + (8 * mt + j + 4) * 16 + 2 * g);
     const uint32_t ya = odd_bytes_down(va.x), yb = odd_bytes_down(vb.x);
     const uint32_t za = odd_bytes_down(va.y), zb = odd_bytes_down(vb.y);
     // fields at bits 0, 2, 4, 6 of each half: factors 1, 4, 16, 64
-    mma16816(st.O[0], va.x & 0x00030003u, va.x & 0x000C000Cu, vb.x & 0x00030003u, vb.x & 0x000C000Cu, pb0, pb1);
-    mma16816(st.O[1], va.x & 0x00300030u, va.x & 0x00C000C0u, vb.x & 0x00300030u, vb.x & 0x00C000C0u, pb0, pb1);
-    mma16816(st.O[2], ya & 0x00030003u, ya & 0x000C000Cu, yb & 0x00030003u, yb & 0x000C000Cu, pb0, pb1);
-    mma16816(st.O[3], ya & 0x00300030u, ya & 0x00C000C0u, yb & 0x00300030u, yb & 0x00C000C0u, pb0, pb1);
-    mma16816(st.O[4], va.y & 0x00030003u, va.y & 0x000C000Cu, vb.y & 0x00030003u, vb.y & 0x000C000Cu, pb0, pb1);
-    mma16816(st.O[5], va.y & 0x00300030u, va.y & 0x00C000C0u, vb.y & 0x00300030u, vb.y & 0x00C000C0u, pb0, pb1);
-    mma16816(st.O[6], za & 0x00030003u, za & 0x000C000Cu, zb & 0x00030003u, zb & 0x000C000Cu, pb0, pb1);
-    mma16816(st.O[7], za & 0x00300030u, za & 0x00C000C0u, zb & 0x00300030u, zb & 0x00C000C0u, pb0, pb1);
+    const uint32_t A[8][4] = {
+        {va.x & 0x00030003u, va.x & 0x000C000Cu, vb.x & 0x00030003u, vb.x & 0x000C000Cu},
+        {va.x & 0x00300030u, va.x & 0x00C000C0u, vb.x & 0x00300030u, vb.x & 0x00C000C0u},
+        {ya & 0x00030003u, ya & 0x000C000Cu, yb & 0x00030003u, yb & 0x000C000Cu},
+        {ya & 0x00300030u, ya & 0x00C000C0u, yb & 0x00300030u, yb & 0x00C000C0u},
+        {va.y & 0x00030003u, va.y & 0x000C000Cu, vb.y & 0x00030003u, vb.y & 0x000C000Cu},
+        {va.y & 0x00300030u, va.y & 0x00C000C0u, vb.y & 0x00300030u, vb.y & 0x00C000C0u},
+        {za & 0x00030003u, za & 0x000C000Cu, zb & 0x00030003u, zb & 0x000C000Cu},
+        {za & 0x00300030u, za & 0x00C000C0u, zb & 0x00300030u, zb & 0x00C000C0u}};
+#pragma unroll
+    for (int cm = 0; cm < 8; ++cm) {
+      mma16816(st.O[cm], A[cm][0], A[cm][1], A[cm][2], A[cm][3], pb0, pb1);
+      mma16816(st.O[cm], A[cm][0], A[cm][1], A[cm][2], A[cm][3], pr0, pr1);
+    }
   }
 }
 
@@ -977,26 +988,49 @@ __device__ __forceinline__ void load_raw(const MmaArgs& a, uint8_t* buf, int64_t
 }
 
 // ---- final combine of one query-head row over its valid slots -------------------------
-// Lane owns channels 4 lane .. 4 lane + 3.
+// Lane owns channels 4 lane .. 4 lane + 3.  The slots are read eight at a time, all loads
+// of a batch issued before any of them is used.
 __device__ __forceinline__ void combine_row(const float* m, const float* l, const float* o, int S,
                                             int64_t row, int s_lo, int s_hi, int lane, void* out,
                                             int out_dtype, float* lse) {
   const float* mrow = m + row * S;
   const float* lrow = l + row * S;
-  float M = -INFINITY;
-  for (int s = s_lo; s <= s_hi; ++s) M = fmaxf(M, __ldcg(mrow + s));
-  float L = 0.0f;
+  float M = -INFINITY, L = 0.0f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = s_lo; s <= s_hi; ++s) {
-    const float ms = __ldcg(mrow + s);
-    if (ms == -INFINITY) continue;
-    const float f = ex2(ms - M);
-    L = fmaf(f, __ldcg(lrow + s), L);
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(o + (row * S + s) * 128) + lane);
-    acc.x = fmaf(f, v.x, acc.x);
-    acc.y = fmaf(f, v.y, acc.y);
-    acc.z = fmaf(f, v.z, acc.z);
-    acc.w = fmaf(f, v.w, acc.w);
+  for (int s0 = s_lo; s0 <= s_hi; s0 += 8) {
+    float mv[8], lv[8];
+    float4 ov[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      mv[u] = -INFINITY;
+      lv[u] = 0.0f;
+      ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s <= s_hi) {
+        mv[u] = __ldcg(mrow + s);
+        lv[u] = __ldcg(lrow + s);
+        ov[u] = __ldcg(reinterpret_cast<const float4*>(o + (row * S + s) * 128) + lane);
+      }
+    }
+    float Mc = M;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) Mc = fmaxf(Mc, mv[u]);
+    if (M != -INFINITY && Mc != M) {   // earlier batches were weighted against M
+      const float c = ex2(M - Mc);
+      L *= c;
+      acc.x *= c; acc.y *= c; acc.z *= c; acc.w *= c;
+    }
+    M = Mc;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (mv[u] == -INFINITY) continue;
+      const float f = ex2(mv[u] - M);
+      L = fmaf(f, lv[u], L);
+      acc.x = fmaf(f, ov[u].x, acc.x);
+      acc.y = fmaf(f, ov[u].y, acc.y);
+      acc.z = fmaf(f, ov[u].z, acc.z);
+      acc.w = fmaf(f, ov[u].w, acc.w);
+    }
   }
   const float inv = 1.0f / L;
   const int64_t i = row * 128 + 4 * lane;
@@ -1194,27 +1228,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
 }
 
 // ==== K4/V2 keys with G <= 4: the lean kernel ============================================
-// Same partition, ring discipline, math encoding and partial-state contract as
-// decode_mma_kernel, arranged so that every lane owns one query head:
+// Same partition, math encoding and partial-state contract as decode_mma_kernel, arranged
+// so that every lane owns one query head:
+//  - Each half group (64 tokens: key and value codes, value scale / zero-point and, for
+//    the half that opens a group, the group's key scale / zero-point) arrives in a stage
+//    of the warp's two-stage ring by 1-D bulk copies (the TMA engine; this GPU's memory
+//    only, no multicast) on one mbarrier per stage.  Lane 0 issues the copies of the
+//    next half (predicated, no divergent branch) before the warp waits for the current
+//    one; waits are bounded.
 //  - The key product's N columns are (head 0 high, head 0 remainder, head 1 high, ...):
 //    lane (g, j) ends with the high part and the remainder of head j for tokens g and
 //    g + 8 of the tile and adds them in place; the online softmax then runs on two
 //    values per lane and tile, with m, l and W scalars per lane.
-//  - The probabilities of a tile, packed as (p[g][j] s_g, p[g + 8][j] s_{g+8}), become
-//    the value product's B operand with one 8x8 transpose (movmatrix) and one shuffle:
-//    after the transpose lane (2h, j') holds tokens 2j', 2j' + 1 of head h and lane
-//    (2h + 1, j') tokens 2j' + 8, 2j' + 9, so column 2h of the product is head h and
-//    the odd columns carry values that are never read.
+//  - The value product's B operand carries the probabilities P = p s_t of a tile as an
+//    fp16 high part and an fp16 remainder (about 22 bits): column 2h holds head h's high
+//    parts and column 2h + 1 its remainders.  Packed per lane as (high, remainder) of
+//    token g (and of token g + 8), one 8x8 transpose (movmatrix) each puts exactly the
+//    B fragment in place: lane (2h, j') receives the high parts of tokens 2j', 2j' + 1
+//    of head h, lane (2h + 1, j') their remainders.
 //  - The key-product B operand of a group is built with every (head, channel) product
 //    formed once: lane L forms head L / 8, channels 16 (L % 8) .. + 15, and the fragments
 //    reach their lanes through the warp's scratch.  Each head has its own exponent.
-//  - Stages arrive by 1-D bulk copies (the TMA engine; this GPU's memory only, no
-//    multicast) on one mbarrier per stage, issued by lane 0; waits are bounded.
+//  - A warp's range covers at most two heads; each is a run of raw items (staged with
+//    cp.async in the same stages, the next one in flight) and a run of halves, walked
+//    with 32-bit counters.
 constexpr int kQBytes = 4 * 128 * 4;            // pre-scaled queries of up to four heads
 constexpr int kBScratch = 32 * 16 * 4;          // key-operand fragments on their way to lanes
-constexpr int kLeanWarpBytes = kBuffers * kStageBytes + kQBytes + kBScratch;
-constexpr int kWaitLimit = 1 << 20;             // try_wait rounds before a wait gives up
+constexpr int kKMetaBytes = 2 * 128 * 4;        // the group's key scale / zero-point as fp32
+constexpr int kLeanWarpBytes = kBuffers * kStageBytes + kQBytes + kBScratch + kKMetaBytes;
+constexpr int kWaitRounds = 1000;               // try_wait rounds (each up to 1 ms) before giving up
 static_assert(kRecordFloats * 4 <= kBuffers * kStageBytes, "merge record fits the ring");
+static_assert(2 * kRawBytes <= kStageBytes, "raw item fits a stage");
 static_assert(64 * 8 <= kBScratch, "value scale / zero-point pairs fit the scratch");
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -1223,32 +1267,38 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 __device__ __forceinline__ void mbar_fence_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-// 1-D bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`
-// (addresses 16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+// On lane 0 only (pred != 0): arrive on `bar` expecting `bytes` of transfers.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes, uint32_t pred) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %2, 0;\n @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n}" ::"r"(
+          smem_u32(bar)),
+      "r"(bytes), "r"(pred)
+      : "memory");
+}
+// On lane 0 only: 1-D bulk copy global -> this CTA's shared memory completing `bytes` on
+// `bar` (addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint32_t pred) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n}" ::"r"(
           smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "r"(pred)
       : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
-// Waits for the phase of `parity` to complete; false when kWaitLimit rounds pass first.
+// Waits for the phase of `parity`; false when kWaitRounds rounds pass first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   bool ok = false;
-  for (int it = 0; it < kWaitLimit && !ok; ++it) ok = mbar_try_wait(bar, parity);
+  for (int it = 0; it < kWaitRounds && !ok; ++it) ok = mbar_try_wait(bar, parity);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -1265,49 +1315,53 @@ __device__ __forceinline__ uint32_t movtrans_n(uint32_t x) {
   return y;
 }
 
-// Copies of one half group (key codes, value codes, value scale / zero-point and, when
-// `with_key`, the group's key scale / zero-point) into a stage; lane 0 only.
-__device__ __forceinline__ void issue_half(const MmaArgs& a, uint8_t* buf, uint64_t* bar, int64_t head,
-                                           int gi, int hf, bool with_key) {
-  const int64_t t0 = (int64_t)gi * 128 + 64 * hf;
-  mbar_expect_tx(bar, kHalfK + kHalfV + kHalfVM + (with_key ? kHalfKM : 0));
-  bulk_g2s(buf, a.k_codes + head * a.k_slab_bytes + t0 * 64, kHalfK, bar);
-  bulk_g2s(buf + kHalfK, a.v_codes + head * a.v_slab_bytes + t0 * 32, kHalfV, bar);
-  bulk_g2s(buf + kHalfK + kHalfV, a.v_scale + head * a.C + t0, 128, bar);
-  bulk_g2s(buf + kHalfK + kHalfV + 128, a.v_zero + head * a.C + t0, 128, bar);
+// Copies of half p (key codes, value codes, value scale / zero-point and, when
+// `with_key`, the key scale / zero-point of its group) of head `head` into a stage, on
+// lane 0.
+__device__ __forceinline__ void issue_half(const MmaArgs& a, uint8_t* buf, uint64_t* bar, int64_t head, int p,
+                                           bool with_key) {
+  const uint32_t l0 = (threadIdx.x & 31) == 0;
+  const int64_t t0 = 64 * (int64_t)p;
+  mbar_expect_tx(bar, kHalfK + kHalfV + kHalfVM + (with_key ? kHalfKM : 0), l0);
+  bulk_g2s(buf, a.k_codes + head * a.k_slab_bytes + t0 * 64, kHalfK, bar, l0);
+  bulk_g2s(buf + kHalfK, a.v_codes + head * a.v_slab_bytes + t0 * 32, kHalfV, bar, l0);
+  bulk_g2s(buf + kHalfK + kHalfV, a.v_scale + head * a.C + t0, 128, bar, l0);
+  bulk_g2s(buf + kHalfK + kHalfV + 128, a.v_zero + head * a.C + t0, 128, bar, l0);
   if (with_key) {
-    const int64_t grp = head * a.ng + gi;
-    bulk_g2s(buf + kHalfK + kHalfV + kHalfVM, a.k_scale + grp * 128, 256, bar);
-    bulk_g2s(buf + kHalfK + kHalfV + kHalfVM + 256, a.k_zero + grp * 128, 256, bar);
+    const int64_t grp = head * a.ng + (p >> 1);
+    bulk_g2s(buf + kHalfK + kHalfV + kHalfVM, a.k_scale + grp * 128, 256, bar, l0);
+    bulk_g2s(buf + kHalfK + kHalfV + kHalfVM + 256, a.k_zero + grp * 128, 256, bar, l0);
   }
 }
 
-// Copies of raw item r (its sink and / or residual key rows, then value rows at
-// +kRawBytes) into a stage; lane 0 only.
-__device__ __forceinline__ void issue_raw(const MmaArgs& a, uint8_t* buf, uint64_t* bar, int64_t head, int r) {
-  const int rowb = a.src_dtype == KVQ_F32 ? 512 : 256;
+__device__ __forceinline__ void cp_async16_lean(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// Raw item r of head `head` (its key rows, then its value rows at +kRawBytes) into a
+// stage with cp.async, every lane moving 16-byte chunks; committed as one group.
+__device__ __forceinline__ void stage_raw(const MmaArgs& a, uint8_t* buf, int64_t head, int r) {
+  const int lane = threadIdx.x & 31;
+  const int lg = a.src_dtype == KVQ_F32 ? 5 : 4;   // log2 of the 16-byte chunks per row
+  const int rowb = 16 << lg;
   const int nraw = a.n_sink + a.t_res;
   const int t0 = r * a.rt, nt = min(a.rt, nraw - t0);
-  const int ns = max(0, min(nt, a.n_sink - t0));   // sink tokens of the item
-  const int nr = nt - ns;                           // residual tokens of the item
-  mbar_expect_tx(bar, (uint32_t)(2 * nt * rowb));
-  if (ns > 0) {
-    const int64_t row = head * a.n_sink + t0;
-    bulk_g2s(buf, reinterpret_cast<const uint8_t*>(a.sink_k) + row * rowb, ns * rowb, bar);
-    bulk_g2s(buf + kRawBytes, reinterpret_cast<const uint8_t*>(a.sink_v) + row * rowb, ns * rowb, bar);
+  const int per = nt << lg;
+  for (int c = lane; c < 2 * per; c += 32) {
+    const int kv = c >= per, rem = c - (kv ? per : 0);
+    const int t = rem >> lg, ch = rem & ((1 << lg) - 1);
+    const int tok = t0 + t;
+    const bool sink = tok < a.n_sink;
+    const void* arr = kv ? (sink ? a.sink_v : a.res_v) : (sink ? a.sink_k : a.res_k);
+    const int64_t row = head * (sink ? a.n_sink : a.res_cap) + (sink ? tok : tok - a.n_sink);
+    cp_async16_lean(buf + kv * kRawBytes + t * rowb + ch * 16, reinterpret_cast<const uint8_t*>(arr) + row * rowb + ch * 16);
   }
-  if (nr > 0) {
-    const int64_t row = head * a.res_cap + (t0 + ns - a.n_sink);
-    bulk_g2s(buf + ns * rowb, reinterpret_cast<const uint8_t*>(a.res_k) + row * rowb, nr * rowb, bar);
-    bulk_g2s(buf + kRawBytes + ns * rowb, reinterpret_cast<const uint8_t*>(a.res_v) + row * rowb, nr * rowb,
-             bar);
-  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// Online-softmax state of lane (g, j) for head j: O[cm][0] and O[cm][2] are channels
-// d0 = 16 g + 8 (cm >> 2) + 2 (cm & 3) and d0 + 1 (elements 1 and 3 belong to columns
-// that are never read); m, l, W the running max, sum and sum of p z (l and W summed
-// over the lanes g of the column at the end).
+// Online-softmax state of lane (g, j) for head j: O[cm][0] + O[cm][1] and O[cm][2] +
+// O[cm][3] are channels d0 = 16 g + 8 (cm >> 2) + 2 (cm & 3) and d0 + 1 (the high-part
+// and remainder columns of the value product); m, l, W the running max, sum and sum of
+// p z (l and W summed over the lanes g of the column at the end).
 struct LeanState {
   float O[8][4];
   float m, l, W;
@@ -1326,7 +1380,9 @@ __device__ __forceinline__ void lean_rescale(LeanState& st, float mnew) {
 #pragma unroll
     for (int cm = 0; cm < 8; ++cm) {
       st.O[cm][0] *= c;
+      st.O[cm][1] *= c;
       st.O[cm][2] *= c;
+      st.O[cm][3] *= c;
     }
     st.l *= c;
     st.W *= c;
@@ -1348,8 +1404,9 @@ __device__ void lean_emit(LeanState& st, int G, float* o, int64_t os, float* m, 
 #pragma unroll
     for (int cm = 0; cm < 8; ++cm) {
       const int d0 = 16 * g + 8 * (cm >> 2) + 2 * (cm & 3);
-      *reinterpret_cast<float2*>(dst + d0) = make_float2(fmaf(st.O[cm][0], inv_f_lo(cm & 1), st.W),
-                                                         fmaf(st.O[cm][2], inv_f_hi(cm & 1), st.W));
+      *reinterpret_cast<float2*>(dst + d0) =
+          make_float2(fmaf(st.O[cm][0] + st.O[cm][1], inv_f_lo(cm & 1), st.W),
+                      fmaf(st.O[cm][2] + st.O[cm][3], inv_f_hi(cm & 1), st.W));
     }
     if (g == 0) {
       m[j * ms] = st.m;
@@ -1453,7 +1510,8 @@ struct LeanKey {
   float mult, bias;
 };
 
-__device__ __forceinline__ void lean_key_operand(const __half* ks, const __half* kz, const float* qs,
+// ks, kz: the group's key scale / zero-point as fp32 [128] in shared memory.
+__device__ __forceinline__ void lean_key_operand(const float* ks, const float* kz, const float* qs,
                                                  uint32_t* scr, LeanKey& ko) {
   const int lane = threadIdx.x & 31;
   const int hL = lane >> 3, cb = lane & 7;   // head, 16-channel block formed by this lane
@@ -1461,25 +1519,21 @@ __device__ __forceinline__ void lean_key_operand(const __half* ks, const __half*
   float amax = 0.0f, dz = 0.0f;
   {
     const float4* q4 = reinterpret_cast<const float4*>(qs + hL * 128 + 16 * cb);
-    const uint4* s4 = reinterpret_cast<const uint4*>(ks + 16 * cb);
-    const uint4* z4 = reinterpret_cast<const uint4*>(kz + 16 * cb);
+    const float4* s4 = reinterpret_cast<const float4*>(ks + 16 * cb);
+    const float4* z4 = reinterpret_cast<const float4*>(kz + 16 * cb);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const uint4 sv = s4[u], zv = z4[u];
-      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w}, zw[4] = {zv.x, zv.y, zv.z, zv.w};
-      const float4 qa = q4[2 * u], qb = q4[2 * u + 1];
-      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    for (int u = 0; u < 4; ++u) {
+      const float4 qv = q4[u], sv = s4[u], zv = z4[u];
+      a[4 * u] = qv.x * sv.x;
+      a[4 * u + 1] = qv.y * sv.y;
+      a[4 * u + 2] = qv.z * sv.z;
+      a[4 * u + 3] = qv.w * sv.w;
+      dz = fmaf(qv.x, zv.x, dz);
+      dz = fmaf(qv.y, zv.y, dz);
+      dz = fmaf(qv.z, zv.z, dz);
+      dz = fmaf(qv.w, zv.w, dz);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[k]));
-        const float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&zw[k]));
-        const int i = 8 * u + 2 * k;
-        a[i] = qv[2 * k] * s2.x;
-        a[i + 1] = qv[2 * k + 1] * s2.y;
-        dz = fmaf(qv[2 * k], z2.x, dz);
-        dz = fmaf(qv[2 * k + 1], z2.y, dz);
-        amax = fmaxf(amax, fmaxf(fabsf(a[i]), fabsf(a[i + 1])));
-      }
+      for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fabsf(a[4 * u + k]));
     }
   }
 #pragma unroll
@@ -1518,36 +1572,24 @@ __device__ __forceinline__ void lean_key_operand(const __half* ks, const __half*
   __syncwarp();
 }
 
-// 64 tokens (one half of a group) held in a stage; szbuf: the warp's scratch, which
-// receives the half's value scale / zero-point as fp32 pairs.
-__device__ __forceinline__ void lean_half(LeanState& st, const uint8_t* stage, const LeanKey& ko, int tvalid,
-                                          float* szbuf) {
+// The scores of the half's 64 tokens (4 tiles of 16) from its key codes [64][16] words in
+// shared memory: lane (g, j) takes words 4j .. 4j + 3 of rows 16 mt + g and 16 mt + g + 8.
+__device__ __forceinline__ void lean_scores(float (&S)[4][4], const uint4* kc4, const LeanKey& ko) {
   const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
-  const uint4* kc4 = reinterpret_cast<const uint4*>(stage);
-  const uint2* vc2 = reinterpret_cast<const uint2*>(stage + kHalfK);
-  const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stage + kHalfK + kHalfV);
-  {   // tokens 2 lane, 2 lane + 1; tokens past tvalid get (0, 0)
-    float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&vsz[lane]));
-    float2 z2 = __half22float2(*reinterpret_cast<const __half2*>(&vsz[32 + lane]));
-    if (2 * lane >= tvalid) s2.x = z2.x = 0.0f;
-    if (2 * lane + 1 >= tvalid) s2.y = z2.y = 0.0f;
-    reinterpret_cast<float4*>(szbuf)[lane] = make_float4(s2.x, z2.x, s2.y, z2.y);
-  }
-  // ---- scores of the 64 tokens (4 tiles of 16) ----
-  float S[4][4];
-  uint4 wlo[4], whi[4];
+  uint4 kw[8];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     S[mt][0] = S[mt][1] = S[mt][2] = S[mt][3] = 0.0f;
-    wlo[mt] = kc4[(16 * mt + g) * 4 + j];
-    whi[mt] = kc4[(16 * mt + g + 8) * 4 + j];
+    kw[2 * mt] = kc4[(16 * mt + g) * 4 + j];
+    kw[2 * mt + 1] = kc4[(16 * mt + g + 8) * 4 + j];
   }
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
-      const uint32_t x0 = w == 0 ? wlo[mt].x : w == 1 ? wlo[mt].y : w == 2 ? wlo[mt].z : wlo[mt].w;
-      const uint32_t x1 = w == 0 ? whi[mt].x : w == 1 ? whi[mt].y : w == 2 ? whi[mt].z : whi[mt].w;
+      const uint4 lo = kw[2 * mt], hi = kw[2 * mt + 1];
+      const uint32_t x0 = w == 0 ? lo.x : w == 1 ? lo.y : w == 2 ? lo.z : lo.w;
+      const uint32_t x1 = w == 0 ? hi.x : w == 1 ? hi.y : w == 2 ? hi.z : hi.w;
       const uint32_t p0 = odd_bytes_down(x0), p1 = odd_bytes_down(x1);
       mma16816_n(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u, ko.b[4 * w],
                  ko.b[4 * w + 1]);
@@ -1555,7 +1597,17 @@ __device__ __forceinline__ void lean_half(LeanState& st, const uint8_t* stage, c
                  ko.b[4 * w + 3]);
     }
   }
-  // ---- online softmax (log2 domain) on head j, tokens g and g + 8 of every tile ----
+}
+
+// Online softmax of the half on head j (tokens g and g + 8 of every tile): l and W
+// updated, the probability operands of the half's value product returned in pb (tile mt:
+// pb[mt][0] = the (high, remainder) columns of tokens 2j', 2j' + 1 and pb[mt][1] of tokens
+// 2j' + 8, 2j' + 9, as the B fragment of m16n8k16).  sz: the half's value scale /
+// zero-point as fp32 pairs in shared memory.  The value product of any earlier half must
+// already be in st.O (a new maximum rescales it).
+__device__ __forceinline__ void lean_softmax(LeanState& st, const float (&S)[4][4], const LeanKey& ko,
+                                             int tvalid, const float2* sz, uint32_t (&pb)[4][2]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2;
   float x[4][2];
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
@@ -1576,95 +1628,95 @@ __device__ __forceinline__ void lean_half(LeanState& st, const uint8_t* stage, c
   lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 16));
   lean_rescale(st, fmaxf(st.m, fmaf(lm, ko.mult, ko.bias)));
   const float bm = ko.bias - st.m;
-  __syncwarp();   // the scale / zero-point pairs
-  const float2* sz = reinterpret_cast<const float2*>(szbuf);
-  // ---- value product: one 16-token k-step per score tile ----
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const float p0 = ex2(fmaf(x[mt][0], ko.mult, bm)), p1 = ex2(fmaf(x[mt][1], ko.mult, bm));
     const float2 a0 = sz[16 * mt + g], a1 = sz[16 * mt + g + 8];
     st.l += p0 + p1;
     st.W = fmaf(p0, a0.y, fmaf(p1, a1.y, st.W));
-    const uint32_t pb0 = movtrans_n(pack_half2(p0 * a0.x, p1 * a1.x));
-    const uint32_t pb1 = __shfl_xor_sync(0xffffffffu, pb0, 4);
-    const uint2 va = vc2[(8 * mt + j) * 8 + g];
-    const uint2 vb = vc2[(8 * mt + j + 4) * 8 + g];
+    uint32_t ph, pl;   // high parts and remainders of (P of token g, P of token g + 8)
+    split_half2(p0 * a0.x, p1 * a1.x, &ph, &pl);
+    pb[mt][0] = movtrans_n(__byte_perm(ph, pl, 0x5410));   // (high, remainder) of token g
+    pb[mt][1] = movtrans_n(__byte_perm(ph, pl, 0x7632));   // of token g + 8
+  }
+}
+
+// The value words of a half in this lane's fragment registers: vw[2 mt] = pair g of pair
+// row 8 mt + j, vw[2 mt + 1] = pair g of pair row 8 mt + j + 4 (vc2: [32 pair rows][8]).
+__device__ __forceinline__ void lean_value_words(uint2 (&vw)[8], const uint2* vc2) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, j = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    vw[2 * mt] = vc2[(8 * mt + j) * 8 + g];
+    vw[2 * mt + 1] = vc2[(8 * mt + j + 4) * 8 + g];
+  }
+}
+
+// The value product of a half: st.O += V^T P from its value words and probability operands.
+__device__ __forceinline__ void lean_pv(LeanState& st, const uint2 (&vw)[8], const uint32_t (&pb)[4][2]) {
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const uint2 va = vw[2 * mt], vb = vw[2 * mt + 1];
+    const uint32_t b0 = pb[mt][0], b1 = pb[mt][1];
     const uint32_t ya = odd_bytes_down(va.x), yb = odd_bytes_down(vb.x);
     const uint32_t za = odd_bytes_down(va.y), zb = odd_bytes_down(vb.y);
     // fields at bits 0, 2, 4, 6 of each half: factors 1, 4, 16, 64
-    mma16816_n(st.O[0], va.x & 0x00030003u, va.x & 0x000C000Cu, vb.x & 0x00030003u, vb.x & 0x000C000Cu, pb0, pb1);
-    mma16816_n(st.O[1], va.x & 0x00300030u, va.x & 0x00C000C0u, vb.x & 0x00300030u, vb.x & 0x00C000C0u, pb0, pb1);
-    mma16816_n(st.O[2], ya & 0x00030003u, ya & 0x000C000Cu, yb & 0x00030003u, yb & 0x000C000Cu, pb0, pb1);
-    mma16816_n(st.O[3], ya & 0x00300030u, ya & 0x00C000C0u, yb & 0x00300030u, yb & 0x00C000C0u, pb0, pb1);
-    mma16816_n(st.O[4], va.y & 0x00030003u, va.y & 0x000C000Cu, vb.y & 0x00030003u, vb.y & 0x000C000Cu, pb0, pb1);
-    mma16816_n(st.O[5], va.y & 0x00300030u, va.y & 0x00C000C0u, vb.y & 0x00300030u, vb.y & 0x00C000C0u, pb0, pb1);
-    mma16816_n(st.O[6], za & 0x00030003u, za & 0x000C000Cu, zb & 0x00030003u, zb & 0x000C000Cu, pb0, pb1);
-    mma16816_n(st.O[7], za & 0x00300030u, za & 0x00C000C0u, zb & 0x00300030u, zb & 0x00C000C0u, pb0, pb1);
+    mma16816_n(st.O[0], va.x & 0x00030003u, va.x & 0x000C000Cu, vb.x & 0x00030003u, vb.x & 0x000C000Cu, b0, b1);
+    mma16816_n(st.O[1], va.x & 0x00300030u, va.x & 0x00C000C0u, vb.x & 0x00300030u, vb.x & 0x00C000C0u, b0, b1);
+    mma16816_n(st.O[2], ya & 0x00030003u, ya & 0x000C000Cu, yb & 0x00030003u, yb & 0x000C000Cu, b0, b1);
+    mma16816_n(st.O[3], ya & 0x00300030u, ya & 0x00C000C0u, yb & 0x00300030u, yb & 0x00C000C0u, b0, b1);
+    mma16816_n(st.O[4], va.y & 0x00030003u, va.y & 0x000C000Cu, vb.y & 0x00030003u, vb.y & 0x000C000Cu, b0, b1);
+    mma16816_n(st.O[5], va.y & 0x00300030u, va.y & 0x00C000C0u, vb.y & 0x00300030u, vb.y & 0x00C000C0u, b0, b1);
+    mma16816_n(st.O[6], za & 0x00030003u, za & 0x000C000Cu, zb & 0x00030003u, zb & 0x000C000Cu, b0, b1);
+    mma16816_n(st.O[7], za & 0x00300030u, za & 0x00C000C0u, zb & 0x00300030u, zb & 0x00C000C0u, b0, b1);
   }
+}
+
+// The value scale / zero-point pairs of tokens 2 lane, 2 lane + 1 as fp32 into szbuf
+// (tokens past tvalid get (0, 0)).
+__device__ __forceinline__ void lean_sz(uint32_t s2, uint32_t z2, int tvalid, float* szbuf) {
+  const int lane = threadIdx.x & 31;
+  float2 s = __half22float2(*reinterpret_cast<const __half2*>(&s2));
+  float2 z = __half22float2(*reinterpret_cast<const __half2*>(&z2));
+  if (2 * lane >= tvalid) s.x = z.x = 0.0f;
+  if (2 * lane + 1 >= tvalid) s.y = z.y = 0.0f;
+  reinterpret_cast<float4*>(szbuf)[lane] = make_float4(s.x, z.x, s.y, z.y);
 }
 
 template <bool ROT>
 __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
+  griddep_wait();   // launched with launch_pdl: the cache and q are complete
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = (int64_t)blockIdx.x * kCW + warp;
   const int64_t i0 = item_start(gw, a.I, a.W), i1 = item_start(gw + 1, a.I, a.W);
   const int U = a.U;
   uint8_t* ring = smem + (size_t)warp * kLeanWarpBytes;
-  float* qs = reinterpret_cast<float*>(ring + kBuffers * kStageBytes);
-  uint32_t* scr = reinterpret_cast<uint32_t*>(ring + kBuffers * kStageBytes + kQBytes);
+  float* qs = reinterpret_cast<float*>(ring + kBuffers * kStageBytes);                        // [4][128]
+  uint32_t* scr = reinterpret_cast<uint32_t*>(ring + kBuffers * kStageBytes + kQBytes);      // fragments / pairs
+  float* kmeta = reinterpret_cast<float*>(ring + kBuffers * kStageBytes + kQBytes + kBScratch);   // s, z [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kCW * kLeanWarpBytes) + kBuffers * warp;
   int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * kLeanWarpBytes + kCW * kBuffers * 8);
   const int nraw = a.n_sink + a.t_res;
   const int G = a.G;
+  const int nrp = a.nrp;
+  const uint32_t l0 = lane == 0;
 
-  if (lane == 0) {
+  if (l0) {
 #pragma unroll
-    for (int s = 0; s < kBuffers; ++s) mbar_init(&bars[s], 1);
+    for (int b = 0; b < kBuffers; ++b) mbar_init(&bars[b], 1);
     mbar_fence_init();
   }
   __syncwarp();
 
-  // load cursor: one work item ahead of the compute cursor (odd raw positions carry none)
-  int64_t lhead = i0 / U, li = i0;
-  int lr = (int)(i0 - lhead * U);
-  int issued = 0;
-  auto advance_load = [&]() {
-    ++li;
-    if (++lr == U) {
-      lr = 0;
-      ++lhead;
-    }
-  };
-  auto issue_next = [&]() {
-    while (li < i1 && lr < a.nrp && (lr & 1)) advance_load();
-    if (li < i1) {
-      if (lane == 0) {
-        const int sb = issued % kBuffers;
-        uint8_t* buf = ring + sb * kStageBytes;
-        if (lr < a.nrp) {
-          issue_raw(a, buf, &bars[sb], lhead, lr >> 1);
-        } else {
-          const int p = lr - a.nrp;
-          issue_half(a, buf, &bars[sb], lhead, p >> 1, p & 1, (p & 1) == 0 || li == i0);
-        }
-      }
-      ++issued;
-      advance_load();
-    }
-  };
-  issue_next();
-
   LeanState st;
   lean_reset(st);
-  LeanKey ko;
-  int64_t head = i0 / U, cur_head = -1;
-  int r = (int)(i0 - head * U);
-  bool qbad = false, qrot = false, timed_out = false;
-  int consumed = 0;
+  bool qbad = false, timed_out = false;
+  int nbulk = 0, ncons = 0;   // halves issued to / consumed from the ring, over the whole range
   // this head's queries, pre-scaled, channels 4 lane .. 4 lane + 3 of every head (as given
   // for raw tokens; in the Walsh-Hadamard basis for the packed keys of a rotating format)
-  auto load_queries = [&](bool rotated) {
+  auto load_queries = [&](int64_t head, bool rotated) {
 #pragma unroll
     for (int hh = 0; hh < 4; ++hh) {
       float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1678,61 +1730,110 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
     }
     __syncwarp();
   };
+
+  // The warp's range of positions covers at most two heads (a range never exceeds U).
+  const int64_t hA = i0 / U;
+  const int64_t endA = min(i1, (hA + 1) * (int64_t)U);
 #pragma unroll 1
-  for (int64_t i = i0; i < i1; ++i) {
-    if (head != cur_head) {
-      if (cur_head >= 0) {   // the range crosses into the next head: slot 0 of this one
-        const int64_t row0 = cur_head * G;
-        lean_emit(st, G, a.ws_o + row0 * a.S * 128, (int64_t)a.S * 128, a.ws_m + row0 * a.S,
-                  a.ws_l + row0 * a.S, a.S);
-        lean_reset(st);
+  for (int segi = 0; segi < 2 && !timed_out; ++segi) {
+    const int64_t head = hA + segi;
+    const int64_t sb = segi == 0 ? i0 : (hA + 1) * (int64_t)U;
+    const int64_t se = segi == 0 ? endA : i1;
+    if (se <= sb) continue;
+    const int pb = (int)(sb - head * U), pe = (int)(se - head * U);   // positions in the head's row
+    if (segi == 1) {   // the range crosses into the next head: slot 0 of the first one
+      const int64_t row0 = hA * G;
+      lean_emit(st, G, a.ws_o + row0 * a.S * 128, (int64_t)a.S * 128, a.ws_m + row0 * a.S,
+                a.ws_l + row0 * a.S, a.S);
+      lean_reset(st);
+    }
+    // raw items with work: r with 2 r in [pb, pe) and 2 r < nrp
+    const int ra = (pb + 1) >> 1, rb = (min(pe, nrp) + 1) >> 1;
+    // packed halves: [ha, hb)
+    const int ha = max(pb, nrp) - nrp, hb = max(pe, nrp) - nrp;
+    if (ra < rb) {   // staged with cp.async in the ring, the next item in flight
+      load_queries(head, false);
+      stage_raw(a, ring, head, ra);
+#pragma unroll 1
+      for (int r = ra; r < rb; ++r) {
+        if (r + 1 < rb) stage_raw(a, ring + ((r + 1 - ra) & 1) * kStageBytes, head, r + 1);
+        else asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncwarp();
+        lean_raw(st, ring + ((r - ra) & 1) * kStageBytes, min(a.rt, nraw - r * a.rt), a.src_dtype, qs);
+        __syncwarp();
       }
-      cur_head = head;
-      qrot = ROT && r >= a.nrp;
-      load_queries(qrot);
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      // the ring's next writers are bulk copies (async proxy) after these generic writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
     }
-    if (r < a.nrp && (r & 1)) {   // second position of a raw item: no work
-      if (++r == U) {
-        r = 0;
-        ++head;
+    if (ha < hb) {
+      load_queries(head, ROT);
+      // two halves in flight; a half's stage is released once its value words are in
+      // registers, and its value product runs during the next half's key product
+#pragma unroll 1
+      for (int q = ha; q < min(hb, ha + kBuffers); ++q) {
+        issue_half(a, ring + (nbulk & 1) * kStageBytes, &bars[nbulk & 1], head, q, q == ha || (q & 1) == 0);
+        ++nbulk;
       }
-      continue;
-    }
-    if (ROT && r >= a.nrp && !qrot) {   // a head's raw items come first: one switch per head
-      qrot = true;
-      load_queries(true);
-    }
-    // the next item goes into the stage consumed last time, then this one is waited for
-    issue_next();
-    const int sb = consumed % kBuffers;
-    if (!mbar_wait(&bars[sb], (uint32_t)(consumed / kBuffers) & 1u)) {
-      timed_out = true;
-      break;
-    }
-    const uint8_t* stg = ring + sb * kStageBytes;
-    if (r < a.nrp) {
-      lean_raw(st, stg, min(a.rt, nraw - (r >> 1) * a.rt), a.src_dtype, qs);
-    } else {
-      const int p = r - a.nrp, gi = p >> 1, hf = p & 1;
-      if (hf == 0 || i == i0) {
-        const __half* ks = reinterpret_cast<const __half*>(stg + kHalfK + kHalfV + kHalfVM);
-        lean_key_operand(ks, ks + 128, qs, scr, ko);
+      LeanKey ko;
+      // the pending value product (zero operands before the first half: it adds nothing,
+      // and the two products stay in one block for the scheduler)
+      uint2 vw[8];
+      uint32_t pb[4][2];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) vw[u] = make_uint2(0u, 0u);
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) pb[mt][0] = pb[mt][1] = 0u;
+      bool pend = false;
+#pragma unroll 1
+      for (int p = ha; p < hb; ++p) {
+        const int sb2 = ncons & 1;
+        if (!mbar_wait(&bars[sb2], (uint32_t)(ncons >> 1) & 1u)) {
+          timed_out = true;
+          break;
+        }
+        const uint8_t* stg = ring + sb2 * kStageBytes;
+        if ((p & 1) == 0 || p == ha) {   // the group's key operand
+          const uint2 sv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM)[lane];
+          const uint2 zv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM + 256)[lane];
+          const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
+          const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
+          const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zv.x));
+          const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&zv.y));
+          reinterpret_cast<float4*>(kmeta)[lane] = make_float4(s01.x, s01.y, s23.x, s23.y);
+          reinterpret_cast<float4*>(kmeta + 128)[lane] = make_float4(z01.x, z01.y, z23.x, z23.y);
+          __syncwarp();
+          lean_key_operand(kmeta, kmeta + 128, qs, scr, ko);
+        }
+        const int tvalid = (int)min((int64_t)64, a.t_quant - 64 * (int64_t)p);
+        const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stg + kHalfK + kHalfV);
+        lean_sz(vsz[lane], vsz[32 + lane], tvalid, reinterpret_cast<float*>(scr));
+        float S[4][4];
+        lean_scores(S, reinterpret_cast<const uint4*>(stg), ko);
+        lean_pv(st, vw, pb);   // the previous half's value product
+        __syncwarp();   // the scale / zero-point pairs
+        lean_softmax(st, S, ko, tvalid, reinterpret_cast<const float2*>(scr), pb);
+        lean_value_words(vw, reinterpret_cast<const uint2*>(stg + kHalfK));
+        pend = true;
+        __syncwarp();   // stage and scratch reads done before they are written again
+        ++ncons;
+        if (p + kBuffers < hb) {   // the freed stage takes the half after the next
+          issue_half(a, ring + (nbulk & 1) * kStageBytes, &bars[nbulk & 1], head, p + kBuffers,
+                     ((p + kBuffers) & 1) == 0);
+          ++nbulk;
+        }
       }
-      const int tvalid = (int)min((int64_t)64, a.t_quant - (int64_t)gi * 128 - 64 * hf);
-      lean_half(st, stg, ko, tvalid, reinterpret_cast<float*>(scr));
-    }
-    __syncwarp();
-    ++consumed;
-    if (++r == U) {
-      r = 0;
-      ++head;
+      if (pend && !timed_out) lean_pv(st, vw, pb);
     }
   }
   if (timed_out) {
-    // let the copies still in flight land before the stages are reused below
-    for (int c = consumed; c < issued; ++c) mbar_wait(&bars[c % kBuffers], (uint32_t)(c / kBuffers) & 1u);
-    if (lane == 0) flag(a.status, KVQ_DEV_TIMEOUT);
+    // let the copies still in flight land before the ring is reused below
+    for (int c = ncons; c < nbulk; ++c) mbar_wait(&bars[c & 1], (uint32_t)(c >> 1) & 1u);
+    if (l0) flag(a.status, KVQ_DEV_TIMEOUT);
   }
+  __syncwarp();
   if (__any_sync(0xffffffffu, qbad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
 
   // ---- merge of the warps' last heads inside the CTA (as decode_mma_kernel) ----
@@ -1798,6 +1899,8 @@ struct CombArgsMma {
 
 // One warp per query-head row.
 __global__ void __launch_bounds__(128) combine_mma_kernel(CombArgsMma a) {
+  griddep_wait();   // launched with launch_pdl: the split kernel's states are complete
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= a.rows) return;
@@ -1916,8 +2019,7 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
     auto kern = a.k_rotate ? decode_k4v2_kernel<true> : decode_k4v2_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<p.grid_ctas, kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(p.grid_ctas), dim3(kThreads), smem, s, a);
   }
   const size_t smem = mma_smem();
   auto kern = mix ? (a.G <= 4 ? decode_mma_kernel<true, false, true> : decode_mma_kernel<false, false, true>)
@@ -1944,8 +2046,7 @@ cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, con
   c.out = out;
   c.out_dtype = out_dtype;
   c.lse = lse;
-  combine_mma_kernel<<<(unsigned)((c.rows + 3) / 4), 128, 0, s>>>(c);
-  return cudaGetLastError();
+  return launch_pdl(combine_mma_kernel, dim3((unsigned)((c.rows + 3) / 4)), dim3(128), 0, s, c);
 }
 
 }  // namespace kvq

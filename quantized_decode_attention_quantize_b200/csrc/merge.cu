@@ -43,11 +43,12 @@ __global__ void __launch_bounds__(128) merge_states_kernel(MergeArgs a) {
     for (int j = 0; j < 8; ++j)
       if (j < nj) acc[j] = fmaf(w, o[lane + 32 * j], acc[j]);
   }
-  const float inv = 1.0f / W;
+  // a row that no part has tokens for (every lse = -inf): zeros and lse = -inf
+  const float inv = W > 0.0f ? 1.0f / W : 0.0f;
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     if (j < nj) store_elem(a.out, row * a.D + lane + 32 * j, a.out_dtype, acc[j] * inv);
-  if (a.lse_out && lane == 0) a.lse_out[row] = M + logf(W);
+  if (a.lse_out && lane == 0) a.lse_out[row] = W > 0.0f ? M + logf(W) : -INFINITY;
 }
 
 }  // namespace

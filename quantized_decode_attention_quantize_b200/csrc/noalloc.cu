@@ -9,6 +9,7 @@
 // workspace.  Everything else -- inputs, outputs, kernels -- is the same as
 // kvq_decode_attention.
 #include <atomic>
+#include <mutex>
 
 #include "kvq_internal.cuh"
 
@@ -19,23 +20,53 @@ static __device__ __align__(256) unsigned char kvq_noalloc_scratch[KVQ_NOALLOC_S
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+// The driver's cuCtxGetCurrent, reached through the runtime (no link against libcuda).
+typedef int (*CtxGetCurrentFn)(void**);
 
-// Device address of the scratch on the current device, looked up once per device
-// (with that device current) and then reused.
+CtxGetCurrentFn ctx_get_current() {
+  static std::atomic<CtxGetCurrentFn> fn{nullptr};
+  CtxGetCurrentFn f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && p != nullptr) {
+      f = reinterpret_cast<CtxGetCurrentFn>(p);
+      fn.store(f, std::memory_order_release);
+    }
+  }
+  return f;
+}
+
+constexpr int kMaxDevices = 64;
+// Per device: the context the address was looked up in, and the address.
+std::mutex g_lock;
+void* g_scratch_ctx[kMaxDevices];
+void* g_scratch_addr[kMaxDevices];
+
+// Device address of the scratch on the current device.  It is looked up (with that
+// device current) the first time and again whenever the current context is not the one
+// it was looked up in: after cudaDeviceReset, for instance, the library's device code is
+// loaded anew in a new context, and an address kept from the old one is no longer mapped.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    e = cudaGetSymbolAddress(&p, kvq_noalloc_scratch);
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr) return cudaErrorInitializationError;
+  void* ctx = nullptr;
+  if (get(&ctx) != 0) return cudaErrorInitializationError;
+  std::lock_guard<std::mutex> hold(g_lock);
+  if (ctx == nullptr || g_scratch_addr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, kvq_noalloc_scratch);   // makes the device's context current
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev].store(p, std::memory_order_release);
+    if (get(&ctx) != 0 || ctx == nullptr) return cudaErrorInitializationError;
+    g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
-  *out = p;
+  *out = g_scratch_addr[dev];
   return cudaSuccess;
 }
 

@@ -452,6 +452,8 @@ __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
 // (group, channel block, head), the rest value blocks (token block, head).
 __global__ void __launch_bounds__(kThreads) asym_kv_kernel(AArgs ak, AArgs av, int kgx, int kgy, int nk,
                                                            int vgx) {
+  griddep_wait();   // launched with launch_pdl: earlier work on the stream is complete
+  griddep_launch_dependents();
   const int b = blockIdx.x;
   if (b < nk) {
     asym_keys_block(ak, b % kgx, (b / kgx) % kgy, b / (kgx * kgy));
@@ -522,7 +524,8 @@ cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const voi
   if (L.k_rotate)
     asym_kv_rot_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, (int)nk, vgx);
   else
-    asym_kv_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, kgy, (int)nk, vgx);
+    return launch_pdl(asym_kv_kernel, dim3((unsigned)(nk + nv)), dim3(kThreads), 0, s, ak, av, kgx, kgy,
+                      (int)nk, vgx);
   return cudaGetLastError();
 }
 

@@ -36,11 +36,14 @@ def decode_local(fmt, cache: kvq.Cache, q: torch.Tensor, t_quant: int, t_res: in
     """This rank's part: out [B, Hq, D] fp32 and lse [B, Hq] fp32 over its own tokens."""
     B, Hq, D = q.shape
     need = kvq.decode_workspace_bytes(fmt, B, Hq, cache.H, t_quant, t_res, num_splits)
-    ws = torch.empty(max(16, need), dtype=torch.uint8, device=q.device)
+    # the buffers belong to the stream the kernels run on, so that the caching allocator
+    # does not hand them out again while those kernels may still use them
+    with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream(q.device)):
+        ws = torch.empty(max(16, need), dtype=torch.uint8, device=q.device)
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     kvq.decode_partial(fmt, cache, q, t_quant, t_res, scale, ws, num_splits=num_splits, status=status,
                        stream=stream)
-    out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
-    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     kvq.decode_combine_lse(fmt, B, Hq, cache.H, t_quant, t_res, ws, out, lse, num_splits=num_splits,
                            stream=stream)
     return out, lse

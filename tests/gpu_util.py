@@ -75,6 +75,32 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
+def rel_l2_rows(a, b):
+    """Largest relative L2 error over the query rows (the last axis is the head dimension)."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    a = a.reshape(-1, a.shape[-1])
+    b = b.reshape(-1, b.shape[-1])
+    return float(np.max(np.linalg.norm(a - b, axis=1) / np.linalg.norm(b, axis=1)))
+
+
+# Unit roundoff of the output types: the largest relative error of rounding one value.
+UNIT_ROUNDOFF = {F32: 0.0, F16: 2.0 ** -11, BF16: 2.0 ** -8}
+
+
+def assert_attn(out, ref, tol, out_dtype=F32):
+    """Attention parity: the whole tensor's relative L2 within `tol`, and every query row's
+    relative L2 within `tol` plus the output type's unit roundoff u, so that one bad row
+    cannot hide among good ones.  Rounding each element of a row to the output type alone
+    moves the row by at most u in relative L2 (every element by at most u relative), and
+    the rows of a 16-bit output scatter around the whole-tensor figure by up to that much;
+    for fp32 output the two bars are the same."""
+    whole, worst = rel_l2(out, ref), rel_l2_rows(out, ref)
+    row_bar = tol + UNIT_ROUNDOFF[out_dtype]
+    assert whole <= tol and worst <= row_bar, \
+        f"relative L2 {whole:.3e} (bar {tol:.1e}), worst row {worst:.3e} (bar {row_bar:.2e})"
+
+
 def tolerance(out_dtype):
     """Attention parity bar against the float64 oracle: relative L2 <= 1e-3 for fp32
     output, <= 2e-3 when the output is fp16 / bf16."""

@@ -12,6 +12,11 @@ import synth
 from oracle import formats as of
 from quantized_decode_attention_quantize_b200 import kvq
 
+
+def torch_cuda_available():
+    import torch
+    return torch.cuda.is_available()
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -105,6 +110,13 @@ class _FakeCache:
         return ctypes.byref(self.struct)
 
 
+# The tests below hand made-up device addresses to launching entry points, relying on
+# the host checks to refuse them before any launch.  They run where no GPU is present;
+# on a GPU machine a regressed check would launch kernels on those addresses.
+fake_pointers = pytest.mark.skipif(torch_cuda_available(), reason="made-up device addresses; CPU only")
+
+
+@fake_pointers
 def test_host_validation_rejects_before_launch():
     L = kvq.lib()
     f = _fmt()
@@ -151,6 +163,7 @@ def test_workspace_bytes_with_explicit_splits():
     assert n == 2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4
 
 
+@fake_pointers
 def test_sequence_split_entry_points_validate_on_the_host():
     # nothing is launched: every call below fails validation before touching memory
     L = kvq.lib()
@@ -173,3 +186,22 @@ def test_sequence_split_entry_points_validate_on_the_host():
     assert L.kvq_merge_states(2, 8, 128, outs, lses, out, 9, None, None) == kvq.KVQ_ERR_INVALID
     assert L.kvq_merge_states(2, 8, 128, ctypes.c_void_p(0x600008), lses, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
     assert L.kvq_merge_states(2, 8, 128, outs, None, out, kvq.F32, None, None) == kvq.KVQ_ERR_INVALID
+
+
+def test_noalloc_rejects_oversized_requests():
+    # A workspace need above the library's fixed scratch is refused before anything runs.
+    # Every cache array and the q / out pointers are null: the size check comes first, and
+    # should it ever regress, the null pointers fail the host validation that follows
+    # (KVQ_ERR_INVALID) instead of reaching a launch.
+    fd = dict(head_dim=128, group_tokens=128, src_dtype=of.BF16, k_scheme=of.ASYM, k_bits=4,
+              k_axis=of.CHANNEL, k_outliers=0, v_scheme=of.ASYM, v_bits=2, v_axis=of.TOKEN,
+              v_outliers=0, mixed_hi=0, mixed_mid=0, n_sink=0, residual_cap=0, rope=1,
+              rope_base=10000.0, k_rotate=0)
+    f = kvq.make_format(fd)              # RoPE keys: the generic path, 64 splits per head as asked
+    B, Hq, Hkv, tq = 64, 64, 64, 131072
+    need = kvq.decode_workspace_bytes(f, B, Hq, Hkv, tq, 0, 64)
+    assert need > kvq.NOALLOC_SCRATCH_BYTES
+    cache = kvq.kvq_cache(batch=B, kv_heads=Hkv, capacity=tq)
+    st = kvq.lib().kvq_decode_attention_noalloc(ctypes.byref(f), ctypes.byref(cache), None, kvq.BF16, Hq,
+                                                tq, 0, 0.1, None, kvq.F32, 64, None, None)
+    assert st == kvq.KVQ_ERR_WORKSPACE

@@ -16,7 +16,7 @@ import synth
 from oracle import attention as oatt
 from oracle.formats import BF16, F16, F32, NUQ
 from quantized_decode_attention_quantize_b200 import kvq, seqsplit
-from tests.gpu_util import dev, rel_l2
+from tests.gpu_util import assert_attn, dev, rel_l2
 from tests.test_gpu_decode import build, vals
 
 pytestmark = pytest.mark.gpu
@@ -69,7 +69,7 @@ def test_merged_parts_match_the_oracle_over_the_union(kw, G, spans):
                                       np.concatenate(Vs), scale)
             ref[b, h * G:(h + 1) * G] = o
             ref_lse[b, h * G:(h + 1) * G] = l
-    assert rel_l2(merged.cpu().numpy(), ref) <= 1e-3
+    assert_attn(merged.cpu().numpy(), ref, 1e-3)
     lse_all = torch.empty((B, G * H), dtype=torch.float32, device="cuda")
     kvq.merge_states(torch.stack(outs), torch.stack(lses), kvq.F32, lse_out=lse_all)
     torch.cuda.synchronize()
@@ -105,3 +105,25 @@ def test_empty_part_has_no_weight_and_16_bit_output():
     w0, w2 = np.exp(l[0] - np.maximum(l[0], l[2])), np.exp(l[2] - np.maximum(l[0], l[2]))
     want = (w0[:, None] * o[0] + w2[:, None] * o[2]) / (w0 + w2)[:, None]
     assert np.abs(got.float().cpu().numpy() - want).max() <= 2 ** -7 * np.abs(want).max()
+
+
+def test_rows_without_tokens_merge_to_zero():
+    # every part of rows 1 and 4 is empty (lse = -inf): out = 0 there and lse = -inf,
+    # the other rows as the oracle's merge
+    from oracle.attention import merge_parts
+    rows, D = 6, 128
+    rng = np.random.default_rng(5)
+    outs = rng.standard_normal((2, rows, D)).astype(np.float32)
+    lses = rng.standard_normal((2, rows)).astype(np.float32)
+    lses[:, [1, 4]] = -np.inf
+    outs[:, [1, 4]] = np.nan
+    lse_out = torch.empty(rows, dtype=torch.float32, device="cuda")
+    got = kvq.merge_states(torch.tensor(outs, device="cuda"), torch.tensor(lses, device="cuda"), kvq.F32,
+                           lse_out=lse_out)
+    torch.cuda.synchronize()
+    want, want_lse = merge_parts(outs, lses)
+    g, gl = got.cpu().numpy(), lse_out.cpu().numpy()
+    assert np.all(g[[1, 4]] == 0.0) and np.all(np.isneginf(gl[[1, 4]]))
+    live = [0, 2, 3, 5]
+    assert np.abs(g[live] - want[live]).max() <= 1e-6 * np.abs(want[live]).max()
+    assert np.abs(gl[live] - want_lse[live]).max() <= 1e-6 * max(1.0, np.abs(want_lse[live]).max())

@@ -2,15 +2,15 @@
 cannot allocate device memory (it uses a scratch array inside the library instead of
 a caller workspace).  Collected last on purpose: a run that stops at the first failure
 has run every other test before this one.  Checks the output of two calls in a row
-against kvq_decode_attention on the same inputs, within the decode tolerance."""
+against kvq_decode_attention on the same inputs: both run the same kernels on the same
+inputs, so the outputs are equal bit for bit."""
 import numpy as np
 import pytest
 import torch
 
-import synth
 from oracle.formats import BF16, F16, F32
 from quantized_decode_attention_quantize_b200 import kvq
-from tests.gpu_util import dev, rel_l2, tolerance
+from tests.gpu_util import dev
 from tests.test_gpu_decode import build, fmt, vals
 
 pytestmark = pytest.mark.gpu
@@ -31,23 +31,6 @@ def test_noalloc_matches_workspace_entry_point(G, src, out_dtype):
                                                  status=status))
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-    ref = want.float().cpu().numpy()
     for o in outs:
-        assert rel_l2(o.float().cpu().numpy(), ref) <= tolerance(out_dtype)
+        assert torch.equal(o, want)
 
-
-def test_noalloc_rejects_oversized_requests():
-    # a workspace need above the scratch size is refused before anything runs
-    fd = fmt(src_dtype=BF16, rope=1)        # the generic path: 64 splits per head as asked
-    f = kvq.make_format(fd)
-    B, Hq, Hkv, tq = 64, 64, 64, 131072
-    need = kvq.decode_workspace_bytes(f, B, Hq, Hkv, tq, 0, 64)
-    assert need > kvq.NOALLOC_SCRATCH_BYTES
-    cache = kvq.kvq_cache(batch=B, kv_heads=Hkv, capacity=tq)
-    for i, n in enumerate(kvq.ARRAYS):
-        setattr(cache, n, 0x10000 * (i + 1))
-    import ctypes
-    st = kvq.lib().kvq_decode_attention_noalloc(ctypes.byref(f), ctypes.byref(cache), ctypes.c_void_p(0x100000),
-                                                kvq.BF16, Hq, tq, 0, 0.1, ctypes.c_void_p(0x200000), kvq.F32,
-                                                64, None, None)
-    assert st == kvq.KVQ_ERR_WORKSPACE
