@@ -1,8 +1,9 @@
 """KQV: scalar MSE codes for the keys, scalar codes plus a 1-bit QJL sketch of the
 residual for the values, both after a Walsh-Hadamard rotation.
 
-TEST INFRASTRUCTURE ONLY (see the package docstring).  The library does not implement
-this scheme yet; these definitions are the reference its kernels will be held to.
+TEST INFRASTRUCTURE ONLY (see the package docstring).  The float64 functions below state
+the scheme; the "stored format" section at the end states the fp32 arithmetic the
+library's kernels store codes with, which decides every code and sign bit.
 
 [TQ] "Statistical Inference and Quality Measures of KV Cache Quantisations Inspired by
 TurboQuant", Technical Summary: "Theoretical Framework" (a coordinate of a uniformly
@@ -134,3 +135,76 @@ def qkqv_key(k, bits, S, cb=None):
     of the residual, like a KQV value.  Its scores q . k^ are the scalar part plus the
     sketch's unbiased inner-product estimate."""
     return kqv_value(k, bits, S, cb)
+
+
+# ---- stored format (the library's KVQ_KQV scheme) ------------------------------------
+# The float64 definitions above leave the precision of every decision open.  The stored
+# format fixes it in fp32, each operation one IEEE rounding and no fused multiply-add, so
+# that codes and sign bits are reproducible:
+#   y     = the key-only rotation's fp32 Walsh-Hadamard transform (oracle.rotate.wht_f32);
+#   ||y|| = fl32(sqrt(T(fl32(y_c * y_c)))), T the pairwise tree over the channel index
+#           (level 1 adds elements 2i and 2i + 1, level 2 the results 2i and 2i + 1, ...,
+#           every sum rounded to fp32);
+#   u_c   = fl32(y_c / ||y||)  (0 when ||y|| = 0);
+#   code  = #{j : u_c > m_j},  m_j = fl32(fl32(C_j + C_{j+1}) * 0.5), C the fp32 centroids;
+#   values also: yh_c = fl32(||y|| * C[code_c]), r_c = fl32(y_c - yh_c),
+#           ||r|| = fl32(sqrt(T(fl32(r_c * r_c)))), and sign bit i = (T_c(fl32(S_ic * r_c)) >= 0).
+# Reconstruction (decode, dequantize) is a real-valued formula evaluated in float64 here:
+#   k^ = R (||y|| C[code]),   v^ = R (||y|| C[code] + sqrt(pi/2) / m ||r|| S^T s),
+# R the same orthonormal transform (its own inverse), s_i = +1 for a set bit, -1 otherwise.
+
+
+def tree_sum_f32(a):
+    """Pairwise sum over the last axis (a power of two long) in fp32: each level adds the
+    elements 2i and 2i + 1 of the previous one, every sum rounded to fp32."""
+    a = np.asarray(a, np.float32)
+    while a.shape[-1] > 1:
+        a = (a[..., 0::2] + a[..., 1::2]).astype(np.float32)
+    return a[..., 0]
+
+
+def centroids_f32(cb):
+    """The fp32 centroids and their fp32 midpoints fl32(fl32(C_j + C_{j+1}) * 0.5)."""
+    c = np.asarray(cb, np.float32)
+    mids = ((c[:-1] + c[1:]).astype(np.float32) * np.float32(0.5)).astype(np.float32)
+    return c, mids
+
+
+def stored_encode(x, cb, S=None):
+    """Rows x [n, D] of exact fp32 source values -> (codes [n, D], norms fp32 [n]) for keys;
+    with S (fp32 [D, D], values): also (signs bool [n, D], residual norms fp32 [n])."""
+    from . import rotate
+    x = np.asarray(x, np.float32)
+    y = np.asarray(rotate.wht_f32(x), np.float32)
+    nrm = np.sqrt(tree_sum_f32((y * y).astype(np.float32))).astype(np.float32)
+    safe = np.where(nrm > 0, nrm, np.float32(1.0)).astype(np.float32)
+    u = np.where(nrm[..., None] > 0, (y / safe[..., None]).astype(np.float32), np.float32(0.0))
+    c, mids = centroids_f32(cb)
+    codes = (u[..., None] > mids).sum(axis=-1)
+    if S is None:
+        return codes, nrm
+    yh = (nrm[..., None] * c[codes]).astype(np.float32)
+    r = (y - yh).astype(np.float32)
+    rn = np.sqrt(tree_sum_f32((r * r).astype(np.float32))).astype(np.float32)
+    S = np.asarray(S, np.float32)
+    t = tree_sum_f32((S[None, :, :] * r[:, None, :]).astype(np.float32))   # [n, m]
+    return codes, nrm, t >= 0, rn
+
+
+def stored_key(codes, nrm, cb):
+    """k^ [n, D] float64 from stored key codes and norms."""
+    R = rotation(np.asarray(codes).shape[-1])
+    c = np.asarray(cb, np.float32).astype(np.float64)
+    return (np.asarray(nrm, np.float64)[..., None] * c[codes]) @ R
+
+
+def stored_value(codes, nrm, signs, rn, cb, S):
+    """v^ [n, D] float64 from stored value codes, norms, sign bits and residual norms."""
+    D = np.asarray(codes).shape[-1]
+    R = rotation(D)
+    S = np.asarray(S, np.float32).astype(np.float64)
+    c = np.asarray(cb, np.float32).astype(np.float64)
+    sv = np.where(np.asarray(signs), 1.0, -1.0)
+    yh = np.asarray(nrm, np.float64)[..., None] * c[codes]
+    sk = math.sqrt(math.pi / 2.0) / S.shape[0] * np.asarray(rn, np.float64)[..., None] * (sv @ S)
+    return (yh + sk) @ R

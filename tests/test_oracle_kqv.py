@@ -145,3 +145,78 @@ def test_keys_without_the_sketch_give_lower_attention_kl():
         kl_k = float((p0 * np.log(p0 / pk)).sum(axis=1).mean())
         kl_q = float((p0 * np.log(p0 / pq)).sum(axis=1).mean())
         assert kl_q > 2.0 * kl_k
+
+
+# ---- stored format ---------------------------------------------------------------------
+
+def test_tree_sum_is_the_pairwise_tree():
+    # brute-force recursion over halves, and exact on small integers
+    rng = np.random.default_rng(3)
+    a = rng.standard_normal((5, 128)).astype(np.float32)
+
+    def rec(v):
+        if len(v) == 1:
+            return np.float32(v[0])
+        h = len(v) // 2
+        return np.float32(rec(v[:h]) + rec(v[h:]))
+
+    got = kqv.tree_sum_f32(a)
+    for i in range(5):
+        assert got[i] == rec(a[i])
+    ints = rng.integers(-1000, 1000, (4, 64)).astype(np.float32)
+    np.testing.assert_array_equal(kqv.tree_sum_f32(ints), ints.sum(axis=1))
+
+
+def test_stored_codes_are_the_nearest_centroid_of_the_rotated_direction():
+    # the fp32 decision against a float64 brute force, wherever the float64 distance gap is
+    # wide enough that fp32 rounding cannot swap the two nearest centroids
+    from oracle import rotate
+    rng = np.random.default_rng(4)
+    D = 128
+    x = (rng.standard_t(4, (64, D)) * 2.0).astype(np.float32)
+    cb = kqv.lloyd_max(3, D)
+    codes, nrm = kqv.stored_encode(x, cb)
+    y = np.asarray(rotate.wht_f32(x), np.float64)
+    np.testing.assert_allclose(nrm, np.linalg.norm(y, axis=1), rtol=2 ** -20)
+    u = y / np.linalg.norm(y, axis=1, keepdims=True)
+    c32 = np.asarray(cb, np.float32).astype(np.float64)
+    dist = np.abs(u[..., None] - c32)
+    best = dist.argmin(axis=-1)
+    srt = np.sort(dist, axis=-1)
+    clear = (srt[..., 1] - srt[..., 0]) > 1e-5
+    assert clear.mean() > 0.99
+    np.testing.assert_array_equal(codes[clear], best[clear])
+
+
+def test_stored_value_is_the_float64_scheme_up_to_fp32_rounding():
+    # codes, norms and sketch signs of the stored format reconstruct the float64 KQV value
+    # (kqv_value) to fp32 accuracy; the sketch signs agree wherever S r is not tiny
+    rng = np.random.default_rng(5)
+    D = 128
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    cb = kqv.lloyd_max(3, D)
+    x = rng.standard_normal((16, D)).astype(np.float32)
+    codes, nrm, signs, rn = kqv.stored_encode(x, cb, S)
+    got = kqv.stored_value(codes, nrm, signs, rn, cb, S)
+    want = np.stack([kqv.kqv_value(x[i].astype(np.float64), 4, S.astype(np.float64), cb=cb.astype(np.float32))
+                     for i in range(16)])
+    np.testing.assert_allclose(got, want, rtol=0, atol=2e-5 * np.abs(want).max())
+    from oracle import rotate
+    y = np.asarray(rotate.wht_f32(x), np.float64)
+    yh = nrm.astype(np.float64)[:, None] * np.asarray(cb, np.float32)[codes]
+    t = (y - yh) @ S.astype(np.float64).T
+    big = np.abs(t) > 1e-4 * np.abs(t).max()
+    np.testing.assert_array_equal(signs[big], (t >= 0)[big])
+
+
+def test_stored_key_round_trip_error_matches_lloyd_max():
+    # relative key error of 4-bit KQV keys on Gaussian rows: the Lloyd-Max MSE of the
+    # marginal at d = 128 (about 0.0095 of ||x||^2, Max's table) within sampling noise
+    rng = np.random.default_rng(6)
+    D = 128
+    cb = kqv.lloyd_max(4, D)
+    x = rng.standard_normal((400, D)).astype(np.float32)
+    codes, nrm = kqv.stored_encode(x, cb)
+    kh = kqv.stored_key(codes, nrm, cb)
+    err = np.sum((kh - x) ** 2) / np.sum(x.astype(np.float64) ** 2)
+    assert 0.0075 < err < 0.0115
