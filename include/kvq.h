@@ -55,7 +55,7 @@ extern "C" {
 #endif
 
 #define KVQ_VERSION_MAJOR 0
-#define KVQ_VERSION_MINOR 1
+#define KVQ_VERSION_MINOR 2
 
 typedef enum kvq_status {
   KVQ_OK = 0,
@@ -66,8 +66,10 @@ typedef enum kvq_status {
 } kvq_status;
 
 /* Bits OR-ed into the caller's device status word.  KVQ_DEV_TIMEOUT: a bounded wait
- * inside a kernel ran out (the kernel stopped early; its outputs are unspecified). */
-enum { KVQ_DEV_NONFINITE = 1, KVQ_DEV_RANGE = 2, KVQ_DEV_TIMEOUT = 4 };
+ * inside a kernel ran out (the kernel stopped early; its outputs are unspecified).
+ * KVQ_DEV_BOUNDS: a device-side length or block id was out of range (paged entry
+ * points); the work it named was skipped and the affected outputs are unspecified. */
+enum { KVQ_DEV_NONFINITE = 1, KVQ_DEV_RANGE = 2, KVQ_DEV_TIMEOUT = 4, KVQ_DEV_BOUNDS = 8 };
 
 /* Element types of sources, raw tokens, queries and outputs. */
 enum { KVQ_F32 = 0, KVQ_F16 = 1, KVQ_BF16 = 2 };
@@ -103,8 +105,24 @@ enum { KVQ_F32 = 0, KVQ_F16 = 1, KVQ_BF16 = 2 };
  *              kvq_key_salience); slots [0, mixed_hi) keep the raw 16-bit source,
  *              slots [mixed_hi, mixed_hi + mixed_mid) use KVQ_ASYM 4-bit and the rest
  *              KVQ_ASYM 2-bit, both per channel over the group.
+ *  KVQ_KQV   : the KQV scheme of [TQ] ("Quantization Schemes"), keys and values
+ *              together (both sides KVQ_KQV, axis TOKEN, D = 128, no outliers, rope or
+ *              k_rotate).  Each token row x is rotated, y = the fp32 Walsh-Hadamard
+ *              transform described at k_rotate, and coded by its direction: with the
+ *              pairwise-tree fp32 sum T over the channels (level 1 adds elements 2i and
+ *              2i + 1, every later level the results 2i and 2i + 1 of the one before),
+ *              n = fl32(sqrt(T(fl32(y_c * y_c)))), u_c = fl32(y_c / n) (0 when n = 0),
+ *              code_c = #{ j : u_c > fl32(fl32(C[j] + C[j+1]) * 0.5) } for the 2^b
+ *              ascending fp32 centroids C of the LUT (b = k_bits for keys, v_bits - 1
+ *              for values: v_bits is the value budget including the sketch bit).  Values
+ *              add a one-bit sketch of the residual: yh_c = fl32(n * C[code_c]),
+ *              r_c = fl32(y_c - yh_c), rn = fl32(sqrt(T(fl32(r_c * r_c)))), and for each
+ *              row i of the D x D fp32 matrix S (cache->v_sketch) sign bit
+ *              s_i = (T_c(fl32(S[i][c] * r_c)) >= 0).  Reconstruction (real-valued):
+ *              k^ = H (n C[code]),  v^ = H (n C[code] + sqrt(pi/2) / D * rn * S^T s),
+ *              s_i = +1 for a set bit and -1 otherwise, H the orthonormal transform.
  */
-enum { KVQ_NONE = 0, KVQ_SYM8 = 1, KVQ_ASYM = 2, KVQ_NUQ = 3, KVQ_MIXED = 4 };
+enum { KVQ_NONE = 0, KVQ_SYM8 = 1, KVQ_ASYM = 2, KVQ_NUQ = 3, KVQ_MIXED = 4, KVQ_KQV = 5 };
 
 /* Grouping axes ([AXES]: tensor / token / channel scales). */
 enum { KVQ_AXIS_TENSOR = 0, KVQ_AXIS_TOKEN = 1, KVQ_AXIS_CHANNEL = 2 };
@@ -157,6 +175,11 @@ typedef struct kvq_format {
  *    NUQ (3-bit), keys and values: [C][3*D/32] uint32 per token row: D/16 words of
  *           the low two code bits in the row layout, then D/32 words of the high bit
  *           (channel c at bit c % 32 of word c / 32).
+ *    KQV, keys: [C][b*D/32] uint32 per token row, b = k_bits in {2, 3, 4}: the row
+ *           layout for b = 2 and 4, the NUQ layout (two planes) for b = 3.
+ *    KQV, values: [C][(b + 1)*D/32] uint32 per token row, b = v_bits - 1 in {1, 2, 3}:
+ *           the codes as for keys (b = 1: row layout), then D/32 words of sketch bits
+ *           (bit i at bit i % 32 of word i / 32).
  *    MIXED (keys): [ngroups][g * (2*hi + mid/2 + lo/4)] bytes per group: the raw
  *           plane [g][hi] src_dtype, then the 4-bit plane [g][mid/8] uint32 and the
  *           2-bit plane [g][lo/16] uint32, both in the row layout over slots.
@@ -164,8 +187,10 @@ typedef struct kvq_format {
  *    SYM8   fp32 scale only: TENSOR [ngroups], TOKEN [C], CHANNEL [ngroups][D].
  *    ASYM, NUQ (channel axis)  fp16 [ngroups][D].
  *    MIXED  fp16 [ngroups][D - hi], indexed by slot - hi.
+ *    KQV    k_scale: fp32 [C], the row norms n; no k_zero.
  *  v_scale / v_zero
  *    SYM8   fp32 as for keys.   ASYM, NUQ (token axis): fp16 [C].
+ *    KQV    v_scale: fp32 [C], the row norms n; v_zero: fp32 [C], the residual norms rn.
  *  k_order             MIXED: uint8 [ngroups][D], slot -> channel.
  *  k_out_rowptr        NUQ keys with outliers: int32 [ngroups][g + 1]; CSR row
  *                      pointers by token row of the group, relative to the group's
@@ -176,6 +201,10 @@ typedef struct kvq_format {
  *                      CSR whose row pointer is implicit (k entries per token row),
  *                      sorted by channel within the row.
  *  k_lut / v_lut       NUQ: fp16 [8] ascending centroids in [-1, 1].
+ *                      KQV: fp32 [2^b] ascending centroids (see kvq_kqv_codebook).
+ *  v_sketch            KQV: fp32 [D][D], the sketch matrix S (row i = direction i);
+ *                      one matrix for the whole cache, read by quantize, dequantize
+ *                      and decode (the method's random draw, made by the caller).
  *  sink_k / sink_v     [n_sink][D] src_dtype (raw, pre-RoPE keys).
  *  res_k / res_v       [residual_cap][D] src_dtype (raw, pre-RoPE keys).
  * Unused arrays may be NULL.
@@ -189,6 +218,7 @@ typedef struct kvq_cache {
   void *v_out_col, *v_out_val;
   const void *k_lut, *v_lut;
   void *sink_k, *sink_v, *res_k, *res_v;
+  const void* v_sketch;
 } kvq_cache;
 
 /* Array identifiers for kvq_cache_array_bytes (same order as kvq_cache). */
@@ -199,6 +229,7 @@ enum {
   KVQ_ARR_V_OUT_COL, KVQ_ARR_V_OUT_VAL,
   KVQ_ARR_K_LUT, KVQ_ARR_V_LUT,
   KVQ_ARR_SINK_K, KVQ_ARR_SINK_V, KVQ_ARR_RES_K, KVQ_ARR_RES_V,
+  KVQ_ARR_V_SKETCH,
   KVQ_ARR_COUNT
 };
 
@@ -245,11 +276,24 @@ kvq_status kvq_quantize_kv(const kvq_format* fmt, const kvq_cache* cache, const 
                            int64_t stride_t, int64_t t0, int64_t n, int32_t* d_status,
                            void* stream);
 
+/* The Lloyd-Max centroids of KVQ_KQV ([TQ] "Theoretical Framework": a coordinate of a
+ * uniformly random unit vector in head_dim dimensions has the density
+ * (1 - x^2)^((d - 3) / 2) / B(1/2, (d - 1) / 2) on [-1, 1]): the 2^bits ascending
+ * centroids minimising the mean squared error under that density (thresholds at the
+ * midpoints, centroids at the conditional means, iterated to a fixed point by
+ * quadrature in double and kept symmetric), rounded to fp32.  bits in 1..4, head_dim
+ * in 3..4096.  `centroids` is host memory of 2^bits floats.  Host only; about a tenth
+ * of a second. */
+kvq_status kvq_kqv_codebook(int32_t bits, int32_t head_dim, float* centroids);
+
 /* Reconstruct packed rows [t0, t0 + n) of keys or values (which = KVQ_KEYS/VALUES)
  * into `out` (device, [B][Hkv][n][D] contiguous, out_dtype).  fp32 output is the exact
  * x^ of the scheme; fp16 / bf16 output is that fp32 value rounded to nearest-even.
  * Outlier positions return their stored fp16 value; MIXED raw channels return the
- * stored source value.  No RoPE is applied. */
+ * stored source value.  No RoPE is applied.  KQV rows are the real-valued k^ / v^ of
+ * the scheme evaluated in fp32 (products with the centroids, the sketch sum S^T s in
+ * channel order, the Walsh-Hadamard butterfly), so they match it to fp32 rounding,
+ * not bit for bit. */
 kvq_status kvq_dequantize(const kvq_format* fmt, const kvq_cache* cache, int32_t which,
                           int64_t t0, int64_t n, void* out, int32_t out_dtype,
                           int32_t* d_status, void* stream);
@@ -339,6 +383,64 @@ kvq_status kvq_decode_combine_lse(const kvq_format* fmt, int32_t batch, int32_t 
 kvq_status kvq_merge_states(int32_t n_parts, int64_t rows, int32_t head_dim, const float* outs,
                             const float* lses, void* out, int32_t out_dtype, float* lse_out,
                             void* stream);
+
+/* ---- Paged cache with per-sequence lengths ---------------------------------------
+ * A serving cache grows by whole token groups flushed from each sequence's raw window
+ * ([MIX] Figure 4) and holds sequences of different lengths side by side ([MIX]
+ * Figure 5 measures memory and throughput of such batches).  The pages give no
+ * layout; this one is the plainest:
+ *  - The packed arrays are a pool of num_blocks blocks, each holding one token group of
+ *    every KV head, laid out exactly as a kvq_cache with batch = num_blocks, kv_heads
+ *    and capacity = group_tokens (size each pool array with kvq_cache_array_bytes on
+ *    those numbers; the group's key metadata sits at group 0 of its block).
+ *  - Sequence s owns blocks block_table[s][0 .. ceil(t_quant[s] / group_tokens)), in
+ *    token order; a block may belong to one sequence at a time.
+ *  - The raw sink and residual arrays are per sequence, [num_seqs][kv_heads][...] as in
+ *    kvq_cache.
+ * Every group is quantized on its own, so a sequence's packed bytes are the same as in
+ * a contiguous cache.  Formats: the 4-bit per-channel key / 2-bit per-token value
+ * format with D = 128, group_tokens = 128, no RoPE and no MIXED keys (key rotation
+ * allowed); decode needs q_heads / kv_heads <= 4.  Other combinations return
+ * KVQ_ERR_UNSUPPORTED. */
+typedef struct kvq_paged_cache {
+  kvq_cache pool;             /* batch = num_blocks, capacity = group_tokens; its sink /
+                                 residual pointers are not used                         */
+  int32_t num_seqs;
+  int32_t max_blocks;         /* columns of block_table                                 */
+  const int32_t* block_table; /* device [num_seqs][max_blocks], physical block ids      */
+  void *sink_k, *sink_v;      /* device [num_seqs][kv_heads][n_sink][D] src_dtype        */
+  void *res_k, *res_v;        /* device [num_seqs][kv_heads][residual_cap][D] src_dtype  */
+} kvq_paged_cache;
+
+/* Quantize the first n (1 <= n <= group_tokens) tokens of one new token group of every
+ * sequence into pool block blocks[s] (device int32 [num_seqs]): keys and values, in one
+ * launch.  k_src / v_src: [s][h][t][c] at s*stride_b + h*stride_h + t*stride_t + c
+ * (rules as kvq_quantize_kv).  A block id outside [0, num_blocks) sets KVQ_DEV_BOUNDS and
+ * that sequence is skipped.  The 4-bit / 2-bit asymmetric format above only. */
+kvq_status kvq_quantize_kv_paged(const kvq_format* fmt, const kvq_paged_cache* cache,
+                                 const void* k_src, const void* v_src, int64_t stride_b,
+                                 int64_t stride_h, int64_t stride_t, const int32_t* blocks,
+                                 int64_t n, int32_t* d_status, void* stream);
+
+/* Workspace bytes for kvq_decode_attention_paged with these bounds on the lengths. */
+size_t kvq_decode_paged_workspace_bytes(const kvq_format* fmt, int32_t num_seqs, int32_t q_heads,
+                                        int32_t kv_heads, int64_t max_t_quant, int32_t max_t_res);
+
+/* Decode attention over a paged cache, every sequence over its own tokens: its n_sink
+ * sink tokens, packed tokens [0, t_quant[s]) and residual rows [0, t_res[s]).
+ * t_quant, t_res: device int32 [num_seqs]; max_t_quant / max_t_res are host bounds on
+ * them (max_t_quant <= max_blocks * group_tokens, max_t_res <= residual_cap) that size
+ * the launch and the workspace; a device length beyond its bound is clamped and sets
+ * KVQ_DEV_BOUNDS, and so does a block id outside [0, num_blocks) (its group is then read
+ * from block 0).  A sequence with no tokens at all gets out = 0.  q, out: device
+ * [num_seqs][q_heads][D].  Otherwise as kvq_decode_attention.  One kernel computes the
+ * partial states of chunks of each sequence's tokens, a second merges them. */
+kvq_status kvq_decode_attention_paged(const kvq_format* fmt, const kvq_paged_cache* cache,
+                                      const int32_t* t_quant, const int32_t* t_res,
+                                      int64_t max_t_quant, int32_t max_t_res, const void* q,
+                                      int32_t q_dtype, int32_t q_heads, float softmax_scale,
+                                      void* out, int32_t out_dtype, void* workspace,
+                                      size_t workspace_bytes, int32_t* d_status, void* stream);
 
 /* Decode attention without a caller workspace, for callers that cannot allocate
  * device memory at all -- for example a serving process whose allocator reserved

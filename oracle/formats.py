@@ -132,6 +132,8 @@ def array_bytes(fmt: Format, B: int, H: int, C: int, name: str) -> int:
         return slabs * fmt.n_sink * D * raw
     if name in ("res_k", "res_v"):
         return slabs * fmt.residual_cap * D * raw
+    if name == "v_sketch":
+        return 0   # the KQV scheme's sketch matrix (oracle.kqv); none of these formats has one
     raise KeyError(name)
 
 

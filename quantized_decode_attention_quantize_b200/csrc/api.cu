@@ -2,6 +2,7 @@
 // kernel dispatch.  No allocation, no synchronisation, no global state.
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "kvq_internal.cuh"
 
@@ -47,6 +48,11 @@ kvq_status check_side(const kvq_format* f, int which) {
       if (f->mixed_hi % 8 || f->mixed_mid % 8 || lo % 16) return KVQ_ERR_INVALID;
       return KVQ_OK;
     }
+    case KVQ_KQV:
+      // keys b in {2, 3, 4} bits; values a budget of b in {2, 3, 4} (b - 1 code bits + sketch)
+      if (bits < 2 || bits > 4 || nout != 0) return KVQ_ERR_INVALID;
+      if (axis < KVQ_AXIS_TENSOR || axis > KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID;
+      return axis == KVQ_AXIS_TOKEN ? KVQ_OK : KVQ_ERR_UNSUPPORTED;
     default:
       return KVQ_ERR_INVALID;
   }
@@ -61,6 +67,7 @@ int64_t code_row_bytes(const kvq_format* f, int which) {
     case KVQ_SYM8: return D;
     case KVQ_ASYM: return (int64_t)D * bits / 8;
     case KVQ_NUQ: return 3 * (int64_t)D / 8;
+    case KVQ_KQV: return (int64_t)D * bits / 8;   // values: b - 1 code bits and the sketch bit
     case KVQ_MIXED: {
       const int lo = D - f->mixed_hi - f->mixed_mid;
       return 2 * f->mixed_hi + f->mixed_mid / 2 + lo / 4;
@@ -81,12 +88,24 @@ void meta_elems(const kvq_format* f, int which, int64_t C, int64_t* ns, int64_t*
     *ns = *nz = axis == KVQ_AXIS_CHANNEL ? ng * D : C;
   } else if (scheme == KVQ_MIXED) {
     *ns = *nz = ng * (D - f->mixed_hi);
+  } else if (scheme == KVQ_KQV) {
+    *ns = C;                                  // row norms
+    *nz = which == KVQ_VALUES ? C : 0;        // residual norms
   }
 }
 
 int meta_elem_bytes(const kvq_format* f, int which) {
   const int scheme = which == KVQ_KEYS ? f->k_scheme : f->v_scheme;
-  return scheme == KVQ_SYM8 ? 4 : 2;
+  return scheme == KVQ_SYM8 || scheme == KVQ_KQV ? 4 : 2;
+}
+
+// LUT bytes: NUQ fp16 [8]; KQV fp32 [2^code bits]
+int64_t lut_bytes(const kvq_format* f, int which) {
+  const int scheme = which == KVQ_KEYS ? f->k_scheme : f->v_scheme;
+  const int bits = which == KVQ_KEYS ? f->k_bits : f->v_bits - 1;
+  if (scheme == KVQ_NUQ) return 16;
+  if (scheme == KVQ_KQV) return 4 * ((int64_t)1 << bits);
+  return 0;
 }
 
 }  // namespace
@@ -121,12 +140,69 @@ kvq_status kvq_format_check(const kvq_format* f) {
   if (f->k_rotate && (f->rope || (f->k_scheme != KVQ_SYM8 && f->k_scheme != KVQ_ASYM &&
                                   f->k_scheme != KVQ_NUQ)))
     return KVQ_ERR_UNSUPPORTED;
+  // KQV codes keys and values together, D = 128, its own rotation, no RoPE
+  if ((f->k_scheme == KVQ_KQV) != (f->v_scheme == KVQ_KQV)) return KVQ_ERR_UNSUPPORTED;
+  if (f->k_scheme == KVQ_KQV && (D != 128 || f->rope || f->k_rotate)) return KVQ_ERR_UNSUPPORTED;
   kvq_status a = check_side(f, KVQ_KEYS);
   if (a == KVQ_ERR_INVALID) return a;
   kvq_status b = check_side(f, KVQ_VALUES);
   if (b == KVQ_ERR_INVALID) return b;
   if (a != KVQ_OK) return a;
   return b;
+}
+
+kvq_status kvq_kqv_codebook(int32_t bits, int32_t d, float* centroids) {
+  if (bits < 1 || bits > 4 || d < 3 || d > 4096 || !centroids) return KVQ_ERR_INVALID;
+  // midpoint quadrature on [-R, R], R = min(1, 14 / sqrt(d)): the density beyond 14
+  // standard deviations (1 / sqrt(d)) carries no mass at double precision
+  const int N = 400000, K = 1 << bits;
+  const double R = std::fmin(1.0, 14.0 / std::sqrt((double)d));
+  const double logc = std::lgamma(d / 2.0) - std::lgamma(0.5) - std::lgamma((d - 1) / 2.0);
+  std::vector<double> x(N), w(N);
+  double tot = 0.0;
+  for (int i = 0; i < N; ++i) {
+    x[i] = ((i + 0.5) / N) * 2.0 * R - R;
+    w[i] = std::fabs(x[i]) < 1.0 ? std::exp(logc + (d - 3) / 2.0 * std::log1p(-x[i] * x[i])) : 0.0;
+    tot += w[i];
+  }
+  for (int i = 0; i < N; ++i) w[i] /= tot;
+  // start at the quantiles (k + 1/2) / K of the grid's distribution, linearly interpolated
+  double c[16], t[15];
+  {
+    double cdf = 0.0, prev_cdf = 0.0;
+    int k = 0, i = 0;
+    while (k < K) {
+      const double target = (k + 0.5) / K;
+      while (i < N && cdf < target) {
+        prev_cdf = cdf;
+        cdf += w[i++];
+      }
+      if (i == 0) {
+        c[k] = x[0];
+      } else if (cdf <= prev_cdf) {
+        c[k] = x[i - 1];
+      } else {
+        const double f = (target - prev_cdf) / (cdf - prev_cdf);
+        c[k] = i >= 2 ? x[i - 2] + f * (x[i - 1] - x[i - 2]) : x[i - 1];
+      }
+      ++k;
+    }
+  }
+  for (int it = 0; it < 300; ++it) {
+    for (int j = 0; j + 1 < K; ++j) t[j] = 0.5 * (c[j] + c[j + 1]);
+    double mass[16] = {0}, mom[16] = {0};
+    int cell = 0;
+    for (int i = 0; i < N; ++i) {
+      while (cell < K - 1 && t[cell] < x[i]) ++cell;   // cell = #{ j : t_j < x }
+      mass[cell] += w[i];
+      mom[cell] += w[i] * x[i];
+    }
+    double nc[16];
+    for (int j = 0; j < K; ++j) nc[j] = mass[j] > 0.0 ? mom[j] / mass[j] : c[j];
+    for (int j = 0; j < K; ++j) c[j] = 0.5 * (nc[j] - nc[K - 1 - j]);   // symmetric density
+  }
+  for (int j = 0; j < K; ++j) centroids[j] = (float)c[j];
+  return KVQ_OK;
 }
 
 size_t kvq_cache_array_bytes(const kvq_format* f, int32_t B, int32_t H, int64_t C, int32_t id) {
@@ -141,17 +217,18 @@ size_t kvq_cache_array_bytes(const kvq_format* f, int32_t B, int32_t H, int64_t 
     case KVQ_ARR_K_CODES: return slabs * C * code_row_bytes(f, KVQ_KEYS);
     case KVQ_ARR_V_CODES: return slabs * C * code_row_bytes(f, KVQ_VALUES);
     case KVQ_ARR_K_SCALE: meta_elems(f, KVQ_KEYS, C, &ns, &nz); return slabs * ns * meta_elem_bytes(f, KVQ_KEYS);
-    case KVQ_ARR_K_ZERO: meta_elems(f, KVQ_KEYS, C, &ns, &nz); return slabs * nz * 2;
+    case KVQ_ARR_K_ZERO: meta_elems(f, KVQ_KEYS, C, &ns, &nz); return slabs * nz * meta_elem_bytes(f, KVQ_KEYS);
     case KVQ_ARR_V_SCALE: meta_elems(f, KVQ_VALUES, C, &ns, &nz); return slabs * ns * meta_elem_bytes(f, KVQ_VALUES);
-    case KVQ_ARR_V_ZERO: meta_elems(f, KVQ_VALUES, C, &ns, &nz); return slabs * nz * 2;
+    case KVQ_ARR_V_ZERO: meta_elems(f, KVQ_VALUES, C, &ns, &nz); return slabs * nz * meta_elem_bytes(f, KVQ_VALUES);
     case KVQ_ARR_K_ORDER: return f->k_scheme == KVQ_MIXED ? slabs * ng * D : 0;
     case KVQ_ARR_K_OUT_ROWPTR: return kout ? slabs * ng * (g + 1) * 4 : 0;
     case KVQ_ARR_K_OUT_COL: return kout ? slabs * ng * D * f->k_outliers : 0;
     case KVQ_ARR_K_OUT_VAL: return kout ? slabs * ng * D * f->k_outliers * 2 : 0;
     case KVQ_ARR_V_OUT_COL: return vout ? slabs * C * f->v_outliers : 0;
     case KVQ_ARR_V_OUT_VAL: return vout ? slabs * C * f->v_outliers * 2 : 0;
-    case KVQ_ARR_K_LUT: return f->k_scheme == KVQ_NUQ ? 16 : 0;
-    case KVQ_ARR_V_LUT: return f->v_scheme == KVQ_NUQ ? 16 : 0;
+    case KVQ_ARR_K_LUT: return lut_bytes(f, KVQ_KEYS);
+    case KVQ_ARR_V_LUT: return lut_bytes(f, KVQ_VALUES);
+    case KVQ_ARR_V_SKETCH: return f->v_scheme == KVQ_KQV ? D * D * 4 : 0;
     case KVQ_ARR_SINK_K:
     case KVQ_ARR_SINK_V: return slabs * f->n_sink * D * raw;
     case KVQ_ARR_RES_K:
@@ -208,7 +285,11 @@ kvq_status make_layout(const kvq_format* f, const kvq_cache* c, Layout* L) {
     if (ns && (!s.scale || !aligned16(s.scale))) return KVQ_ERR_INVALID;
     if (nz && (!s.zero || !aligned16(s.zero))) return KVQ_ERR_INVALID;
     if (s.scheme == KVQ_NUQ && (!s.lut || !aligned16(s.lut))) return KVQ_ERR_INVALID;
+    s.lutf = reinterpret_cast<const float*>(w == 0 ? c->k_lut : c->v_lut);
+    if (s.scheme == KVQ_KQV && (!s.lutf || !aligned16(s.lutf))) return KVQ_ERR_INVALID;
   }
+  L->sketch = reinterpret_cast<const float*>(c->v_sketch);
+  if (f->v_scheme == KVQ_KQV && (!L->sketch || !aligned16(L->sketch))) return KVQ_ERR_INVALID;
   L->k_order = reinterpret_cast<uint8_t*>(c->k_order);
   if (f->k_scheme == KVQ_MIXED && (!L->k_order || !aligned16(L->k_order))) return KVQ_ERR_INVALID;
   if (f->k_scheme == KVQ_NUQ && f->k_outliers > 0) {
@@ -343,6 +424,7 @@ static kvq_status decode_args(const kvq_format* f, int32_t B, int32_t Hq, int32_
   if (s != KVQ_OK) return s;
   if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv) return KVQ_ERR_INVALID;
   if ((int64_t)(Hq / Hkv) * f->head_dim > 2048 || Hq / Hkv > 16) return KVQ_ERR_UNSUPPORTED;
+  if (f->k_scheme == KVQ_KQV && Hq / Hkv > 8) return KVQ_ERR_UNSUPPORTED;
   if (t_quant < 0 || t_res < 0 || t_res > f->residual_cap || num_splits < 0)
     return KVQ_ERR_INVALID;
   if (f->n_sink + t_quant + t_res <= 0) return KVQ_ERR_INVALID;
@@ -477,6 +559,112 @@ kvq_status kvq_decode_attention(const kvq_format* f, const kvq_cache* c, const v
                                 num_splits, d_status, stream, &L, &p);
   if (s != KVQ_OK) return s;
   cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+
+static kvq_status paged_layout(const kvq_format* f, const kvq_paged_cache* pc, Layout* L) {
+  if (!pc) return KVQ_ERR_INVALID;
+  kvq_status st = make_layout(f, &pc->pool, L);
+  if (st != KVQ_OK) return st;
+  if (pc->pool.capacity != f->group_tokens) return KVQ_ERR_INVALID;
+  if (pc->num_seqs < 1 || pc->max_blocks < 1 || !pc->block_table ||
+      (reinterpret_cast<uintptr_t>(pc->block_table) & 3))
+    return KVQ_ERR_INVALID;
+  return KVQ_OK;
+}
+
+kvq_status kvq_quantize_kv_paged(const kvq_format* f, const kvq_paged_cache* pc, const void* k_src,
+                                 const void* v_src, int64_t sb, int64_t sh, int64_t st, const int32_t* blocks,
+                                 int64_t n, int32_t* d_status, void* stream) {
+  Layout L;
+  kvq_status s = paged_layout(f, pc, &L);
+  if (s != KVQ_OK) return s;
+  if (!(asym_fast_ok(L, KVQ_KEYS) && asym_fast_ok(L, KVQ_VALUES))) return KVQ_ERR_UNSUPPORTED;
+  if (n < 1 || n > L.g) return KVQ_ERR_INVALID;
+  if (!blocks || (reinterpret_cast<uintptr_t>(blocks) & 3)) return KVQ_ERR_INVALID;
+  if (!k_src || !v_src || !aligned16(k_src) || !aligned16(v_src)) return KVQ_ERR_INVALID;
+  const int64_t eb = dtype_bytes(L.src_dtype);
+  if (st < L.D || sb < 0 || sh < 0) return KVQ_ERR_INVALID;
+  if ((st * eb) % 16 || (sh * eb) % 16 || (sb * eb) % 16) return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  const int num_blocks = L.B;
+  Layout Ls = L;
+  Ls.B = pc->num_seqs;   // the grid covers the sequences; destinations go through `blocks`
+  cudaError_t e = launch_quantize_asym_kv(Ls, k_src, v_src, sb, sh, st, 0, n, d_status,
+                                          reinterpret_cast<cudaStream_t>(stream), blocks, num_blocks);
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+static size_t paged_ws_bytes(const Layout& L, int num_seqs, int Hq, int S) {
+  const size_t rows = (size_t)num_seqs * Hq * S;
+  const size_t a16 = (rows * 4 + 15) & ~(size_t)15;
+  return 2 * a16 + ((rows * L.D * 4 + 15) & ~(size_t)15);
+}
+
+static kvq_status paged_args(const kvq_format* f, int32_t num_seqs, int32_t Hq, int32_t Hkv, int64_t max_tq,
+                             int32_t max_tr, Layout* L) {
+  kvq_status s = kvq_format_check(f);
+  if (s != KVQ_OK) return s;
+  if (num_seqs < 1 || Hkv < 1 || Hq < 1 || Hq % Hkv) return KVQ_ERR_INVALID;
+  if (max_tq < 0 || max_tr < 0 || max_tr > f->residual_cap || f->n_sink + max_tq + max_tr < 1)
+    return KVQ_ERR_INVALID;
+  plan_layout(f, 1, Hkv, L);
+  L->src_dtype = f->src_dtype;
+  if (!paged_path_ok(*L, Hq)) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+size_t kvq_decode_paged_workspace_bytes(const kvq_format* f, int32_t num_seqs, int32_t Hq, int32_t Hkv,
+                                        int64_t max_tq, int32_t max_tr) {
+  Layout L;
+  if (paged_args(f, num_seqs, Hq, Hkv, max_tq, max_tr, &L) != KVQ_OK) return 0;
+  return paged_ws_bytes(L, num_seqs, Hq, paged_slots(L, max_tq, max_tr));
+}
+
+kvq_status kvq_decode_attention_paged(const kvq_format* f, const kvq_paged_cache* pc, const int32_t* t_quant,
+                                      const int32_t* t_res, int64_t max_tq, int32_t max_tr, const void* q,
+                                      int32_t q_dtype, int32_t Hq, float scale, void* out, int32_t out_dtype,
+                                      void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  Layout L;
+  kvq_status s = paged_layout(f, pc, &L);
+  if (s != KVQ_OK) return s;
+  Layout Lp;
+  s = paged_args(f, pc->num_seqs, Hq, L.Hkv, max_tq, max_tr, &Lp);
+  if (s != KVQ_OK) return s;
+  if (max_tq > (int64_t)pc->max_blocks * L.g) return KVQ_ERR_INVALID;
+  if (!t_quant || !t_res || (reinterpret_cast<uintptr_t>(t_quant) & 3) || (reinterpret_cast<uintptr_t>(t_res) & 3))
+    return KVQ_ERR_INVALID;
+  if (!q || !aligned16(q) || !valid_dtype(q_dtype) || !(scale > 0.0f)) return KVQ_ERR_INVALID;
+  if (!out || !aligned16(out) || !valid_dtype(out_dtype)) return KVQ_ERR_INVALID;
+  if (L.n_sink && (!pc->sink_k || !pc->sink_v || !aligned16(pc->sink_k) || !aligned16(pc->sink_v)))
+    return KVQ_ERR_INVALID;
+  if (max_tr && (!pc->res_k || !pc->res_v || !aligned16(pc->res_k) || !aligned16(pc->res_v)))
+    return KVQ_ERR_INVALID;
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return KVQ_ERR_INVALID;
+  const int S = paged_slots(L, max_tq, max_tr);
+  if ((int64_t)S > 65535 || (int64_t)pc->num_seqs * L.Hkv > 65535) return KVQ_ERR_UNSUPPORTED;
+  if (!ws || !aligned16(ws)) return KVQ_ERR_INVALID;
+  if (ws_bytes < paged_ws_bytes(L, pc->num_seqs, Hq, S)) return KVQ_ERR_WORKSPACE;
+  const size_t rows = (size_t)pc->num_seqs * Hq * S;
+  const size_t a16 = (rows * 4 + 15) & ~(size_t)15;
+  float* ws_m = reinterpret_cast<float*>(ws);
+  float* ws_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + a16);
+  float* ws_o = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * a16);
+  PagedDecode pd;
+  pd.table = pc->block_table;
+  pd.t_quant = t_quant;
+  pd.t_res = t_res;
+  pd.num_seqs = pc->num_seqs;
+  pd.max_blocks = pc->max_blocks;
+  pd.max_t_quant = max_tq;
+  pd.max_t_res = max_tr;
+  pd.sink[0] = pc->sink_k;
+  pd.sink[1] = pc->sink_v;
+  pd.res[0] = pc->res_k;
+  pd.res[1] = pc->res_v;
+  cudaError_t e = launch_decode_paged(L, pd, S, q, q_dtype, Hq, scale, ws_m, ws_l, ws_o, out, out_dtype, d_status,
+                                      reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

@@ -31,6 +31,14 @@ cudaError_t launch_decode_cc(const Layout& L, const DecodePlan& p, const void* q
                              int64_t t_quant, int t_res, float scale, float* ws_m, float* ws_l,
                              float* ws_o, int32_t* d_status, cudaStream_t s);
 
+// KQV caches (decode_kqv.cu)
+size_t kqv_workspace_bytes(const Layout& L, int Hq, const DecodePlan& p);
+cudaError_t launch_decode_kqv(const Layout& L, const DecodePlan& p, const void* q, int q_dtype, int Hq,
+                              int64_t t_quant, int t_res, float scale, void* ws, int32_t* d_status,
+                              cudaStream_t s);
+cudaError_t launch_combine_kqv(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
+                               int out_dtype, float* lse, cudaStream_t s);
+
 namespace {
 
 constexpr int kWarps = 4;
@@ -479,6 +487,7 @@ DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int 
 
 // m [rows], l [rows], o [rows][D] (rows = B * Hq * S).
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p) {
+  if (L.side[0].scheme == KVQ_KQV) return kqv_workspace_bytes(L, Hq, p);
   const size_t rows = (size_t)L.B * Hq * p.S;
   return align16(rows * 4) * 2 + align16(rows * L.D * 4);
 }
@@ -486,6 +495,8 @@ size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p) {
 cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
                                   int Hq, int64_t t_quant, int t_res, float scale, void* ws,
                                   int32_t* d_status, cudaStream_t s) {
+  if (L.side[0].scheme == KVQ_KQV)
+    return launch_decode_kqv(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws, d_status, s);
   const size_t rows = (size_t)L.B * Hq * p.S;
   float* ws_m = reinterpret_cast<float*>(ws);
   float* ws_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align16(rows * 4));
@@ -520,6 +531,7 @@ cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const vo
 
 cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const void* ws, void* out,
                            int out_dtype, float* lse, cudaStream_t s) {
+  if (L.side[0].scheme == KVQ_KQV) return launch_combine_kqv(L, Hq, p, ws, out, out_dtype, lse, s);
   const size_t rows = (size_t)L.B * Hq * p.S;
   const float* m = reinterpret_cast<const float*>(ws);
   const float* l = reinterpret_cast<const float*>(reinterpret_cast<const char*>(ws) + align16(rows * 4));

@@ -46,6 +46,7 @@
 // Waits.  A warp only waits for its own copies (cp.async.wait_group) and, once, at
 // the CTA barrier before the merge, which every warp reaches.
 #include <algorithm>
+#include <cstring>
 #include <cstdint>
 
 #include "kvq_internal.cuh"
@@ -1032,7 +1033,7 @@ __device__ __forceinline__ void combine_row(const float* m, const float* l, cons
       acc.w = fmaf(f, ov[u].w, acc.w);
     }
   }
-  const float inv = 1.0f / L;
+  const float inv = L > 0.0f ? 1.0f / L : 0.0f;   // L = 0: a row with no tokens
   const int64_t i = row * 128 + 4 * lane;
   // natural log of the row's softmax denominator (scores were kept as log2 units)
   if (lse && lane == 0) lse[row] = (M + __log2f(L)) * 0.6931471805599453f;
@@ -1315,9 +1316,8 @@ __device__ __forceinline__ uint32_t movtrans_n(uint32_t x) {
   return y;
 }
 
-// Copies of half p (key codes, value codes, value scale / zero-point and, when
-// `with_key`, the key scale / zero-point of its group) of head `head` into a stage, on
-// lane 0.
+// Copies of half p of slab `head` (key codes, value codes, value scale / zero-point
+// and, when `with_key`, the key scale / zero-point of its group) into a stage, on lane 0.
 __device__ __forceinline__ void issue_half(const MmaArgs& a, uint8_t* buf, uint64_t* bar, int64_t head, int p,
                                            bool with_key) {
   const uint32_t l0 = (threadIdx.x & 31) == 0;
@@ -1337,13 +1337,13 @@ __device__ __forceinline__ void issue_half(const MmaArgs& a, uint8_t* buf, uint6
 __device__ __forceinline__ void cp_async16_lean(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-// Raw item r of head `head` (its key rows, then its value rows at +kRawBytes) into a
-// stage with cp.async, every lane moving 16-byte chunks; committed as one group.
-__device__ __forceinline__ void stage_raw(const MmaArgs& a, uint8_t* buf, int64_t head, int r) {
+// Raw item r of raw head `head` (nraw raw tokens: its key rows, then its value rows at
+// +kRawBytes) into a stage with cp.async, every lane moving 16-byte chunks; committed as
+// one group.
+__device__ __forceinline__ void stage_raw(const MmaArgs& a, uint8_t* buf, int64_t head, int r, int nraw) {
   const int lane = threadIdx.x & 31;
   const int lg = a.src_dtype == KVQ_F32 ? 5 : 4;   // log2 of the 16-byte chunks per row
   const int rowb = 16 << lg;
-  const int nraw = a.n_sink + a.t_res;
   const int t0 = r * a.rt, nt = min(a.rt, nraw - t0);
   const int per = nt << lg;
   for (int c = lane; c < 2 * per; c += 32) {
@@ -1683,6 +1683,178 @@ __device__ __forceinline__ void lean_sz(uint32_t s2, uint32_t z2, int tvalid, fl
   reinterpret_cast<float4*>(szbuf)[lane] = make_float4(s.x, z.x, s.y, z.y);
 }
 
+// The head's queries, pre-scaled, channels 4 lane .. 4 lane + 3 of heads 0..3 (rows
+// qhead * G + hh of q; as given for raw tokens, in the Walsh-Hadamard basis for the
+// packed keys of a rotating format) into qs [4][128].
+template <bool ROT>
+__device__ __forceinline__ void lean_load_queries(const MmaArgs& a, int64_t qhead, bool rotated, float* qs,
+                                                  bool& qbad) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int hh = 0; hh < 4; ++hh) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (hh < a.G) x = load4(a.q, (qhead * a.G + hh) * 128 + 4 * lane, a.q_dtype);
+    qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+    if constexpr (ROT) {
+      if (rotated) x = rotate_q(x, lane, a.rot_scale);
+    }
+    reinterpret_cast<float4*>(qs + hh * 128)[lane] =
+        make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale);
+  }
+  __syncwarp();
+}
+
+// The warp's shared-memory areas and ring counters.
+struct LeanWarp {
+  uint8_t* ring;      // kBuffers stages
+  float* qs;          // [4][128] queries
+  uint32_t* scr;      // key-operand fragments / value scale and zero-point pairs
+  float* kmeta;       // the group's key scale / zero-point as fp32, [2][128]
+  uint64_t* bars;     // one mbarrier per stage
+  int nbulk, ncons;   // halves issued to / consumed from the ring
+};
+
+// One warp's run over one KV head: raw items [ra, rb) (nraw raw tokens in all, rows of
+// raw head `rawhead`), then packed halves [ha, hb) of the head's tq packed tokens.
+// Queries are rows qhead * G + hh of q.  slab_of(p, &slab, &ph) names the slab holding
+// half p and the half's index in it (the contiguous cache: the head's slab and p; a
+// paged pool: the block's slab and p & 1).  Returns false when a wait ran out.
+template <bool ROT, typename SlabOf>
+__device__ __forceinline__ bool lean_run(const MmaArgs& a, LeanState& st, LeanWarp& w, int64_t qhead,
+                                         int64_t rawhead, int nraw, int64_t tq, int ra, int rb, int ha, int hb,
+                                         const SlabOf& slab_of, bool& qbad) {
+  const int lane = threadIdx.x & 31;
+  if (ra < rb) {   // staged with cp.async in the ring, the next item in flight
+    lean_load_queries<ROT>(a, qhead, false, w.qs, qbad);
+    stage_raw(a, w.ring, rawhead, ra, nraw);
+#pragma unroll 1
+    for (int r = ra; r < rb; ++r) {
+      if (r + 1 < rb) stage_raw(a, w.ring + ((r + 1 - ra) & 1) * kStageBytes, rawhead, r + 1, nraw);
+      else asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      __syncwarp();
+      lean_raw(st, w.ring + ((r - ra) & 1) * kStageBytes, min(a.rt, nraw - r * a.rt), a.src_dtype, w.qs);
+      __syncwarp();
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // the ring's next writers are bulk copies (async proxy) after these generic writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+  }
+  if (ha >= hb) return true;
+  lean_load_queries<ROT>(a, qhead, ROT, w.qs, qbad);
+  // two halves in flight; a half's stage is released once its value words are in
+  // registers, and its value product runs during the next half's key product
+  auto issue = [&](int q) {
+    int64_t slab;
+    int ph;
+    slab_of(q, &slab, &ph);
+    issue_half(a, w.ring + (w.nbulk & 1) * kStageBytes, &w.bars[w.nbulk & 1], slab, ph, q == ha || (q & 1) == 0);
+    ++w.nbulk;
+  };
+#pragma unroll 1
+  for (int q = ha; q < min(hb, ha + kBuffers); ++q) issue(q);
+  LeanKey ko;
+  // the pending value product (zero operands before the first half: it adds nothing, and
+  // the two products stay in one block for the scheduler)
+  uint2 vw[8];
+  uint32_t pb[4][2];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) vw[u] = make_uint2(0u, 0u);
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) pb[mt][0] = pb[mt][1] = 0u;
+#pragma unroll 1
+  for (int p = ha; p < hb; ++p) {
+    const int sb2 = w.ncons & 1;
+    if (!mbar_wait(&w.bars[sb2], (uint32_t)(w.ncons >> 1) & 1u)) return false;
+    const uint8_t* stg = w.ring + sb2 * kStageBytes;
+    if ((p & 1) == 0 || p == ha) {   // the group's key operand
+      const uint2 sv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM)[lane];
+      const uint2 zv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM + 256)[lane];
+      const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
+      const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
+      const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zv.x));
+      const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&zv.y));
+      reinterpret_cast<float4*>(w.kmeta)[lane] = make_float4(s01.x, s01.y, s23.x, s23.y);
+      reinterpret_cast<float4*>(w.kmeta + 128)[lane] = make_float4(z01.x, z01.y, z23.x, z23.y);
+      __syncwarp();
+      lean_key_operand(w.kmeta, w.kmeta + 128, w.qs, w.scr, ko);
+    }
+    const int tvalid = (int)min((int64_t)64, tq - 64 * (int64_t)p);
+    const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stg + kHalfK + kHalfV);
+    lean_sz(vsz[lane], vsz[32 + lane], tvalid, reinterpret_cast<float*>(w.scr));
+    float S[4][4];
+    lean_scores(S, reinterpret_cast<const uint4*>(stg), ko);
+    lean_pv(st, vw, pb);   // the previous half's value product
+    __syncwarp();          // the scale / zero-point pairs
+    lean_softmax(st, S, ko, tvalid, reinterpret_cast<const float2*>(w.scr), pb);
+    lean_value_words(vw, reinterpret_cast<const uint2*>(stg + kHalfK));
+    __syncwarp();          // stage and scratch reads done before they are written again
+    ++w.ncons;
+    if (p + kBuffers < hb) issue(p + kBuffers);   // the freed stage takes the half after the next
+  }
+  lean_pv(st, vw, pb);
+  return true;
+}
+
+// Waits for the copies still in flight (after a wait ran out) so that the ring can be
+// reused, then flags the timeout.
+__device__ __forceinline__ void lean_drain(const MmaArgs& a, LeanWarp& w) {
+  for (int c = w.ncons; c < w.nbulk; ++c) mbar_wait(&w.bars[c & 1], (uint32_t)(c >> 1) & 1u);
+  if ((threadIdx.x & 31) == 0) flag(a.status, KVQ_DEV_TIMEOUT);
+}
+
+// The warp areas of warp `warp` in a CTA of nw warps (stages, queries, scratch, key
+// metadata per warp, then the mbarriers of every warp).
+__device__ __forceinline__ LeanWarp lean_warp(uint8_t* smem, int warp, int nw) {
+  LeanWarp w;
+  w.ring = smem + (size_t)warp * kLeanWarpBytes;
+  w.qs = reinterpret_cast<float*>(w.ring + kBuffers * kStageBytes);
+  w.scr = reinterpret_cast<uint32_t*>(w.ring + kBuffers * kStageBytes + kQBytes);
+  w.kmeta = reinterpret_cast<float*>(w.ring + kBuffers * kStageBytes + kQBytes + kBScratch);
+  w.bars = reinterpret_cast<uint64_t*>(smem + (size_t)nw * kLeanWarpBytes) + kBuffers * warp;
+  w.nbulk = w.ncons = 0;
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int b = 0; b < kBuffers; ++b) mbar_init(&w.bars[b], 1);
+    mbar_fence_init();
+  }
+  __syncwarp();
+  return w;
+}
+
+// Merges the records of warps [w0, w1] of the CTA (each warp's ring: o[G][128], m[G],
+// l[G] of one head) and writes the merged state of query rows h G + hh into slot `slot`.
+__device__ __forceinline__ void lean_merge(const MmaArgs& a, uint8_t* smem, int w0, int w1, int64_t h, int slot,
+                                           int nthreads) {
+  const int G = a.G;
+#pragma unroll 1
+  for (int idx = threadIdx.x; idx < G * 128; idx += nthreads) {
+    const int hh = idx >> 7, d = idx & 127;
+    float M = -INFINITY;
+    for (int w = w0; w <= w1; ++w) {
+      const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * kLeanWarpBytes);
+      M = fmaxf(M, rw[8 * 128 + hh]);
+    }
+    float o = 0.0f, l = 0.0f;
+    for (int w = w0; w <= w1; ++w) {
+      const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * kLeanWarpBytes);
+      const float mw = rw[8 * 128 + hh];
+      if (mw != -INFINITY) {
+        const float f = ex2(mw - M);
+        o = fmaf(f, rw[hh * 128 + d], o);
+        l = fmaf(f, rw[8 * 128 + 8 + hh], l);
+      }
+    }
+    const int64_t sl = (h * G + hh) * a.S + slot;
+    a.ws_o[sl * 128 + d] = o;
+    if (d == 0) {
+      a.ws_m[sl] = M;
+      a.ws_l[sl] = l;
+    }
+  }
+}
+
 template <bool ROT>
 __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -1692,45 +1864,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   const int64_t gw = (int64_t)blockIdx.x * kCW + warp;
   const int64_t i0 = item_start(gw, a.I, a.W), i1 = item_start(gw + 1, a.I, a.W);
   const int U = a.U;
-  uint8_t* ring = smem + (size_t)warp * kLeanWarpBytes;
-  float* qs = reinterpret_cast<float*>(ring + kBuffers * kStageBytes);                        // [4][128]
-  uint32_t* scr = reinterpret_cast<uint32_t*>(ring + kBuffers * kStageBytes + kQBytes);      // fragments / pairs
-  float* kmeta = reinterpret_cast<float*>(ring + kBuffers * kStageBytes + kQBytes + kBScratch);   // s, z [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kCW * kLeanWarpBytes) + kBuffers * warp;
+  LeanWarp w = lean_warp(smem, warp, kCW);
   int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * kLeanWarpBytes + kCW * kBuffers * 8);
   const int nraw = a.n_sink + a.t_res;
   const int G = a.G;
   const int nrp = a.nrp;
-  const uint32_t l0 = lane == 0;
-
-  if (l0) {
-#pragma unroll
-    for (int b = 0; b < kBuffers; ++b) mbar_init(&bars[b], 1);
-    mbar_fence_init();
-  }
-  __syncwarp();
 
   LeanState st;
   lean_reset(st);
   bool qbad = false, timed_out = false;
-  int nbulk = 0, ncons = 0;   // halves issued to / consumed from the ring, over the whole range
-  // this head's queries, pre-scaled, channels 4 lane .. 4 lane + 3 of every head (as given
-  // for raw tokens; in the Walsh-Hadamard basis for the packed keys of a rotating format)
-  auto load_queries = [&](int64_t head, bool rotated) {
-#pragma unroll
-    for (int hh = 0; hh < 4; ++hh) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (hh < G) x = load4(a.q, (head * G + hh) * 128 + 4 * lane, a.q_dtype);
-      qbad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
-      if constexpr (ROT) {
-        if (rotated) x = rotate_q(x, lane, a.rot_scale);
-      }
-      reinterpret_cast<float4*>(qs + hh * 128)[lane] =
-          make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale);
-    }
-    __syncwarp();
-  };
-
   // The warp's range of positions covers at most two heads (a range never exceeds U).
   const int64_t hA = i0 / U;
   const int64_t endA = min(i1, (hA + 1) * (int64_t)U);
@@ -1747,98 +1889,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
                 a.ws_l + row0 * a.S, a.S);
       lean_reset(st);
     }
-    // raw items with work: r with 2 r in [pb, pe) and 2 r < nrp
+    // raw items with work: r with 2 r in [pb, pe) and 2 r < nrp; packed halves [ha, hb)
     const int ra = (pb + 1) >> 1, rb = (min(pe, nrp) + 1) >> 1;
-    // packed halves: [ha, hb)
     const int ha = max(pb, nrp) - nrp, hb = max(pe, nrp) - nrp;
-    if (ra < rb) {   // staged with cp.async in the ring, the next item in flight
-      load_queries(head, false);
-      stage_raw(a, ring, head, ra);
-#pragma unroll 1
-      for (int r = ra; r < rb; ++r) {
-        if (r + 1 < rb) stage_raw(a, ring + ((r + 1 - ra) & 1) * kStageBytes, head, r + 1);
-        else asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-        __syncwarp();
-        lean_raw(st, ring + ((r - ra) & 1) * kStageBytes, min(a.rt, nraw - r * a.rt), a.src_dtype, qs);
-        __syncwarp();
-      }
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      // the ring's next writers are bulk copies (async proxy) after these generic writes
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-    }
-    if (ha < hb) {
-      load_queries(head, ROT);
-      // two halves in flight; a half's stage is released once its value words are in
-      // registers, and its value product runs during the next half's key product
-#pragma unroll 1
-      for (int q = ha; q < min(hb, ha + kBuffers); ++q) {
-        issue_half(a, ring + (nbulk & 1) * kStageBytes, &bars[nbulk & 1], head, q, q == ha || (q & 1) == 0);
-        ++nbulk;
-      }
-      LeanKey ko;
-      // the pending value product (zero operands before the first half: it adds nothing,
-      // and the two products stay in one block for the scheduler)
-      uint2 vw[8];
-      uint32_t pb[4][2];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) vw[u] = make_uint2(0u, 0u);
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) pb[mt][0] = pb[mt][1] = 0u;
-      bool pend = false;
-#pragma unroll 1
-      for (int p = ha; p < hb; ++p) {
-        const int sb2 = ncons & 1;
-        if (!mbar_wait(&bars[sb2], (uint32_t)(ncons >> 1) & 1u)) {
-          timed_out = true;
-          break;
-        }
-        const uint8_t* stg = ring + sb2 * kStageBytes;
-        if ((p & 1) == 0 || p == ha) {   // the group's key operand
-          const uint2 sv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM)[lane];
-          const uint2 zv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM + 256)[lane];
-          const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
-          const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
-          const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zv.x));
-          const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&zv.y));
-          reinterpret_cast<float4*>(kmeta)[lane] = make_float4(s01.x, s01.y, s23.x, s23.y);
-          reinterpret_cast<float4*>(kmeta + 128)[lane] = make_float4(z01.x, z01.y, z23.x, z23.y);
-          __syncwarp();
-          lean_key_operand(kmeta, kmeta + 128, qs, scr, ko);
-        }
-        const int tvalid = (int)min((int64_t)64, a.t_quant - 64 * (int64_t)p);
-        const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stg + kHalfK + kHalfV);
-        lean_sz(vsz[lane], vsz[32 + lane], tvalid, reinterpret_cast<float*>(scr));
-        float S[4][4];
-        lean_scores(S, reinterpret_cast<const uint4*>(stg), ko);
-        lean_pv(st, vw, pb);   // the previous half's value product
-        __syncwarp();   // the scale / zero-point pairs
-        lean_softmax(st, S, ko, tvalid, reinterpret_cast<const float2*>(scr), pb);
-        lean_value_words(vw, reinterpret_cast<const uint2*>(stg + kHalfK));
-        pend = true;
-        __syncwarp();   // stage and scratch reads done before they are written again
-        ++ncons;
-        if (p + kBuffers < hb) {   // the freed stage takes the half after the next
-          issue_half(a, ring + (nbulk & 1) * kStageBytes, &bars[nbulk & 1], head, p + kBuffers,
-                     ((p + kBuffers) & 1) == 0);
-          ++nbulk;
-        }
-      }
-      if (pend && !timed_out) lean_pv(st, vw, pb);
-    }
+    auto slab_of = [&](int p, int64_t* slab, int* ph) {
+      *slab = head;
+      *ph = p;
+    };
+    timed_out = !lean_run<ROT>(a, st, w, head, head, nraw, a.t_quant, ra, rb, ha, hb, slab_of, qbad);
   }
-  if (timed_out) {
-    // let the copies still in flight land before the ring is reused below
-    for (int c = ncons; c < nbulk; ++c) mbar_wait(&bars[c & 1], (uint32_t)(c >> 1) & 1u);
-    if (l0) flag(a.status, KVQ_DEV_TIMEOUT);
-  }
+  if (timed_out) lean_drain(a, w);
   __syncwarp();
   if (__any_sync(0xffffffffu, qbad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
 
   // ---- merge of the warps' last heads inside the CTA (as decode_mma_kernel) ----
   const int lh = i1 > 0 ? (int)((i1 - 1) / U) : -1;
-  float* rec = reinterpret_cast<float*>(ring);
+  float* rec = reinterpret_cast<float*>(w.ring);
   if (lh >= 0) lean_emit(st, G, rec, 128, rec + 8 * 128, rec + 8 * 128 + 8, 1);
   if (lane == 0) last_head[warp] = lh;
   __syncthreads();
@@ -1850,35 +1916,118 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
     while (w1 + 1 < kCW && last_head[w1 + 1] == h) ++w1;
     if (h >= 0) {
       const int64_t ca = first_ending_warp(h, U, a.I, a.W) / kCW;
-      const int slot = 1 + (int)((int64_t)blockIdx.x - ca);
-#pragma unroll 1
-      for (int idx = threadIdx.x; idx < G * 128; idx += kThreads) {
-        const int hh = idx >> 7, d = idx & 127;
-        float M = -INFINITY;
-        for (int w = w0; w <= w1; ++w) {
-          const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * kLeanWarpBytes);
-          M = fmaxf(M, rw[8 * 128 + hh]);
-        }
-        float o = 0.0f, l = 0.0f;
-        for (int w = w0; w <= w1; ++w) {
-          const float* rw = reinterpret_cast<const float*>(smem + (size_t)w * kLeanWarpBytes);
-          const float mw = rw[8 * 128 + hh];
-          if (mw != -INFINITY) {
-            const float f = ex2(mw - M);
-            o = fmaf(f, rw[hh * 128 + d], o);
-            l = fmaf(f, rw[8 * 128 + 8 + hh], l);
-          }
-        }
-        const int64_t sl = ((int64_t)h * G + hh) * a.S + slot;
-        a.ws_o[sl * 128 + d] = o;
-        if (d == 0) {
-          a.ws_m[sl] = M;
-          a.ws_l[sl] = l;
-        }
-      }
+      lean_merge(a, smem, w0, w1, h, 1 + (int)((int64_t)blockIdx.x - ca), kThreads);
     }
     w0 = w1 + 1;
   }
+}
+
+// ==== paged cache with per-sequence lengths ==============================================
+// Grid (chunk, sequence x KV head).  Each KV head of a sequence is a row of positions as
+// above (two per raw item, one per packed half), with the sequence's own lengths; CTA
+// (c, head) takes positions [c kPagedChunk, (c + 1) kPagedChunk) of that row, its kPagedWarps
+// warps a contiguous quarter each, and writes one partial state per query row into slot c
+// (m = -inf for an empty chunk).  Half p of a sequence lives in block block_table[s][p / 2],
+// at half p % 2 of that block's slab; a warp reads the block ids of its groups once, and
+// every id is checked against the pool before any copy uses it.
+constexpr int kPagedWarps = 4;
+constexpr int kPagedThreads = kPagedWarps * 32;
+constexpr int kPagedChunk = 64;   // positions per CTA
+static_assert(kPagedChunk % kPagedWarps == 0, "chunk splits over the warps");
+static_assert(kPagedChunk / kPagedWarps / 2 + 1 <= 32, "a warp's block ids fit its lanes");
+
+struct PagedArgs {
+  MmaArgs a;                 // pool arrays as slabs of one group (C = g, ng = 1); raw arrays per sequence
+  const int32_t* table;      // [num_seqs][max_blocks]
+  const int32_t* t_quant;    // [num_seqs]
+  const int32_t* t_res;      // [num_seqs]
+  int max_blocks, num_blocks;
+  int64_t max_t_quant;
+  int max_t_res;
+};
+
+// Positions of a head row: two per raw item of rt tokens, then one per packed half.
+__device__ __forceinline__ int row_positions(int nraw, int rt, int64_t tq, int* nrp) {
+  *nrp = 2 * ((nraw + rt - 1) / rt);
+  if (tq <= 0) return *nrp;
+  const int64_t ngv = (tq + 127) / 128, rem = tq - (ngv - 1) * 128;
+  return *nrp + (int)(2 * (ngv - 1) + (rem > 64 ? 2 : 1));
+}
+
+template <bool ROT>
+__global__ void __launch_bounds__(kPagedThreads, 1) decode_paged_kernel(PagedArgs pa) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  griddep_wait();   // launched with launch_pdl: the cache, tables and q are complete
+  griddep_launch_dependents();
+  const MmaArgs& a = pa.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const int64_t head = blockIdx.y;   // sequence s, KV head kvh
+  const int s = (int)(head / a.Hkv), kvh = (int)(head % a.Hkv);
+  LeanWarp w = lean_warp(smem, warp, kPagedWarps);
+
+  // the sequence's lengths, clamped to the bounds the launch was sized for
+  int64_t tq = pa.t_quant[s];
+  int tr = pa.t_res[s];
+  bool oob = false;
+  const int64_t tq_cap = min(pa.max_t_quant, (int64_t)pa.max_blocks * 128);
+  if (tq < 0 || tq > tq_cap) { oob = true; tq = tq < 0 ? 0 : tq_cap; }
+  if (tr < 0 || tr > pa.max_t_res) { oob = true; tr = tr < 0 ? 0 : pa.max_t_res; }
+  const int nraw = a.n_sink + tr;
+  int nrp;
+  const int U = row_positions(nraw, a.rt, tq, &nrp);
+  const int per = kPagedChunk / kPagedWarps;
+  const int p0 = min(U, c * kPagedChunk + warp * per), p1 = min(U, c * kPagedChunk + (warp + 1) * per);
+
+  LeanState st;
+  lean_reset(st);
+  bool qbad = false;
+  if (p0 < p1) {
+    const int ra = (p0 + 1) >> 1, rb = (min(p1, nrp) + 1) >> 1;
+    const int ha = max(p0, nrp) - nrp, hb = max(p1, nrp) - nrp;
+    // the block ids of the warp's groups, lane i holding group (ha / 2) + i
+    const int g0 = ha >> 1;
+    int blk = 0;
+    if (ha < hb && g0 + lane <= (hb - 1) >> 1) {
+      const int gi = g0 + lane;
+      blk = pa.table[(int64_t)s * pa.max_blocks + gi];
+      if (blk < 0 || blk >= pa.num_blocks) { oob = true; blk = 0; }
+    }
+    auto slab_of = [&](int p, int64_t* slab, int* ph) {
+      const int b = __shfl_sync(0xffffffffu, blk, (p >> 1) - g0);
+      *slab = (int64_t)b * a.Hkv + kvh;
+      *ph = p & 1;
+    };
+    if (!lean_run<ROT>(a, st, w, head, head, nraw, tq, ra, rb, ha, hb, slab_of, qbad)) lean_drain(a, w);
+  }
+  __syncwarp();
+  if (__any_sync(0xffffffffu, qbad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+  if (__any_sync(0xffffffffu, oob) && lane == 0) flag(a.status, KVQ_DEV_BOUNDS);
+  // every warp's state (empty ones: m = -inf) into its record, then one slot per CTA
+  float* rec = reinterpret_cast<float*>(w.ring);
+  lean_emit(st, a.G, rec, 128, rec + 8 * 128, rec + 8 * 128 + 8, 1);
+  __syncthreads();
+  lean_merge(a, smem, 0, kPagedWarps - 1, head, c, kPagedThreads);
+}
+
+// The merge of a row's slots for the paged path (slots with m = -inf are empty; a row
+// with no tokens at all gets zeros).
+struct CombArgsPaged {
+  int S;
+  int64_t rows;
+  const float* m;
+  const float* l;
+  const float* o;
+  void* out;
+  int out_dtype;
+};
+__global__ void __launch_bounds__(128) combine_paged_kernel(CombArgsPaged a) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (row >= a.rows) return;
+  combine_row(a.m, a.l, a.o, a.S, row, 0, a.S - 1, lane, a.out, a.out_dtype, nullptr);
 }
 
 size_t lean_smem() {
@@ -2028,6 +2177,87 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   if (e != cudaSuccess) return e;
   kern<<<p.grid_ctas, kThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+bool paged_path_ok(const Layout& L, int Hq) {
+  const Side& K = L.side[0];
+  const Side& V = L.side[1];
+  const int G = Hq / L.Hkv;
+  return L.D == 128 && L.g == 128 && K.scheme == KVQ_ASYM && K.bits == 4 && K.axis == KVQ_AXIS_CHANNEL &&
+         V.scheme == KVQ_ASYM && V.bits == 2 && V.axis == KVQ_AXIS_TOKEN && L.rope == 0 && G >= 1 && G <= 4;
+}
+
+int paged_slots(const Layout& L, int64_t max_t_quant, int max_t_res) {
+  const int rt = kRawBytes / (128 * (L.src_dtype == KVQ_F32 ? 4 : 2));
+  const int nraw = L.n_sink + max_t_res;
+  int64_t U = 2 * ((nraw + rt - 1) / rt);
+  if (max_t_quant > 0) {
+    const int64_t ngv = (max_t_quant + 127) / 128, rem = max_t_quant - (ngv - 1) * 128;
+    U += 2 * (ngv - 1) + (rem > 64 ? 2 : 1);
+  }
+  return (int)std::max<int64_t>(1, (U + kPagedChunk - 1) / kPagedChunk);
+}
+
+cudaError_t launch_decode_paged(const Layout& L, const PagedDecode& pd, int S, const void* q, int q_dtype, int Hq,
+                                float scale, float* ws_m, float* ws_l, float* ws_o, void* out, int out_dtype,
+                                int32_t* d_status, cudaStream_t s) {
+  PagedArgs pa;
+  MmaArgs& a = pa.a;
+  std::memset(&pa, 0, sizeof(pa));
+  a.k_codes = reinterpret_cast<const uint8_t*>(L.side[0].codes);
+  a.v_codes = reinterpret_cast<const uint8_t*>(L.side[1].codes);
+  a.k_scale = reinterpret_cast<const __half*>(L.side[0].scale);
+  a.k_zero = reinterpret_cast<const __half*>(L.side[0].zero);
+  a.v_scale = reinterpret_cast<const __half*>(L.side[1].scale);
+  a.v_zero = reinterpret_cast<const __half*>(L.side[1].zero);
+  a.k_slab_bytes = L.side[0].code_slab_bytes;   // one group per slab
+  a.v_slab_bytes = L.side[1].code_slab_bytes;
+  a.C = L.C;
+  a.ng = L.ng;
+  a.Hkv = L.Hkv;
+  a.Hq = Hq;
+  a.G = Hq / L.Hkv;
+  a.n_sink = L.n_sink;
+  a.res_cap = L.res_cap;
+  a.src_dtype = L.src_dtype;
+  a.sink_k = pd.sink[0];
+  a.sink_v = pd.sink[1];
+  a.res_k = pd.res[0];
+  a.res_v = pd.res[1];
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.qscale = scale * kLog2e;
+  a.k_rotate = L.k_rotate;
+  a.rot_scale = L.rot_scale;
+  a.rt = kRawBytes / (128 * (L.src_dtype == KVQ_F32 ? 4 : 2));
+  a.S = S;
+  a.ws_m = ws_m;
+  a.ws_l = ws_l;
+  a.ws_o = ws_o;
+  a.status = d_status;
+  pa.table = pd.table;
+  pa.t_quant = pd.t_quant;
+  pa.t_res = pd.t_res;
+  pa.max_blocks = pd.max_blocks;
+  pa.num_blocks = L.B;
+  pa.max_t_quant = pd.max_t_quant;
+  pa.max_t_res = pd.max_t_res;
+  const size_t smem = (size_t)kPagedWarps * kLeanWarpBytes + (size_t)kPagedWarps * kBuffers * 8;
+  auto kern = L.k_rotate ? decode_paged_kernel<true> : decode_paged_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kern, dim3((unsigned)S, (unsigned)((int64_t)pd.num_seqs * L.Hkv)), dim3(kPagedThreads), smem, s,
+                 pa);
+  if (e != cudaSuccess) return e;
+  CombArgsPaged c;
+  c.S = S;
+  c.rows = (int64_t)pd.num_seqs * Hq;
+  c.m = ws_m;
+  c.l = ws_l;
+  c.o = ws_o;
+  c.out = out;
+  c.out_dtype = out_dtype;
+  return launch_pdl(combine_paged_kernel, dim3((unsigned)((c.rows + 3) / 4)), dim3(128), 0, s, c);
 }
 
 cudaError_t launch_combine_mma(const Layout& L, const DecodePlan& p, int Hq, const float* ws_m,

@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DqArgs a) {
 cudaError_t launch_dequantize(const Layout& L, int which, int64_t t0, int64_t n, void* out,
                               int out_dtype, int32_t* d_status, cudaStream_t s) {
   (void)d_status;
+  if (L.side[which].scheme == KVQ_KQV) return launch_dequantize_kqv(L, which, t0, n, out, out_dtype, s);
   DqArgs a;
   a.L = L;
   a.which = which;

@@ -24,6 +24,7 @@ struct Side {
   void* scale;
   void* zero;
   const __half* lut;
+  const float* lutf;         // KQV: fp32 centroids
 };
 
 struct Layout {
@@ -45,6 +46,7 @@ struct Layout {
   void* sink[2];
   void* res[2];
   int raw_bytes;             // element size of src_dtype
+  const float* sketch;       // KQV: the D x D sketch matrix
 };
 
 // Host helpers (api.cpp)
@@ -58,11 +60,18 @@ bool asym_fast_ok(const Layout& L, int which);
 cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, int64_t sb,
                                  int64_t sh, int64_t st, int64_t t0, int64_t n,
                                  int32_t* d_status, cudaStream_t s);
+// blocks (nullable): a paged pool, sequence b's group going to block blocks[b] (L: the
+// pool as one group per slab, L.B = the number of sequences, num_blocks the pool's blocks)
 cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const void* vsrc, int64_t sb,
                                     int64_t sh, int64_t st, int64_t t0, int64_t n, int32_t* d_status,
-                                    cudaStream_t s);
+                                    cudaStream_t s, const int32_t* blocks = nullptr, int num_blocks = 0);
 cudaError_t launch_dequantize(const Layout& L, int which, int64_t t0, int64_t n, void* out,
                               int out_dtype, int32_t* d_status, cudaStream_t s);
+// KQV (quantize_kqv.cu)
+cudaError_t launch_quantize_kqv(const Layout& L, int which, const void* src, int64_t sb, int64_t sh,
+                                int64_t st, int64_t t0, int64_t n, int32_t* d_status, cudaStream_t s);
+cudaError_t launch_dequantize_kqv(const Layout& L, int which, int64_t t0, int64_t n, void* out, int out_dtype,
+                                  cudaStream_t s);
 cudaError_t launch_salience(const Layout& L, const void* q, int64_t qsb, int64_t qsh,
                             int64_t qst, const void* k, int64_t ksb, int64_t ksh, int64_t kst,
                             int B, int Hq, int Hkv, int R, double* sal, uint8_t* order,
@@ -90,6 +99,24 @@ cudaError_t launch_combine(const Layout& L, int Hq, const DecodePlan& p, const v
 cudaError_t launch_merge_states(int n, int64_t rows, int D, const float* outs, const float* lses,
                                 void* out, int out_dtype, float* lse_out, cudaStream_t s);
 int device_sm_count();
+
+// Paged cache (the 4-bit / 2-bit tensor-core format, G <= 4): the pool layout L has one
+// group per slab (C = g, B = num_blocks).
+struct PagedDecode {
+  const int32_t* table;
+  const int32_t* t_quant;
+  const int32_t* t_res;
+  int num_seqs, max_blocks;
+  int64_t max_t_quant;
+  int max_t_res;
+  const void* sink[2];
+  const void* res[2];
+};
+bool paged_path_ok(const Layout& L, int Hq);
+int paged_slots(const Layout& L, int64_t max_t_quant, int max_t_res);
+cudaError_t launch_decode_paged(const Layout& L, const PagedDecode& pd, int S, const void* q, int q_dtype, int Hq,
+                                float scale, float* ws_m, float* ws_l, float* ws_o, void* out, int out_dtype,
+                                int32_t* d_status, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Device helpers

@@ -665,6 +665,7 @@ cudaError_t launch_quantize(const Layout& L, int which, const void* src, int64_t
                             int64_t st, int64_t t0, int64_t n, int32_t* d_status,
                             cudaStream_t s) {
   if (asym_fast_ok(L, which)) return launch_quantize_asym(L, which, src, sb, sh, st, t0, n, d_status, s);
+  if (L.side[which].scheme == KVQ_KQV) return launch_quantize_kqv(L, which, src, sb, sh, st, t0, n, d_status, s);
   QArgs a;
   a.L = L;
   a.which = which;

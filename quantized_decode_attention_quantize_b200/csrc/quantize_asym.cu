@@ -21,7 +21,28 @@ struct AArgs {
   const void* src;
   int64_t sb, sh, st, t0, n;
   int32_t* status;
+  // paged destination: sequence b's group goes to pool block blocks[b] (slab blocks[b] *
+  // Hkv + h of a layout with one group per slab); null for a contiguous cache
+  const int32_t* blocks;
+  int num_blocks;
 };
+
+// The destination slab of source head `head` = (b, h): the head itself, or in a paged
+// pool the slab of its block (false, with KVQ_DEV_BOUNDS raised once, when the block id
+// is out of range).
+__device__ __forceinline__ bool dest_slab(const AArgs& a, int head, int b, int h, int64_t* slab) {
+  if (a.blocks == nullptr) {
+    *slab = head;
+    return true;
+  }
+  const int blk = a.blocks[b];
+  if (blk < 0 || blk >= a.num_blocks) {
+    if (threadIdx.x == 0) flag(a.status, KVQ_DEV_BOUNDS);
+    return false;
+  }
+  *slab = (int64_t)blk * a.L.Hkv + h;
+  return true;
+}
 
 // 8 consecutive elements (16 bytes for 16-bit sources, two 16-byte loads for fp32)
 __device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, float* out) {
@@ -77,6 +98,8 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
   const int cb = by * kCB;
   const int head = bz;
   const int b = head / L.Hkv, h = head % L.Hkv;
+  int64_t slab;
+  if (!dest_slab(a, head, b, h, &slab)) return;   // uniform over the CTA
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int v = lane & 3, rs = warp * 8 + (lane >> 2);
   if (threadIdx.x == 0) flags = 0;
@@ -133,7 +156,7 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
     }
     __half s, z;
     if (!asym_params(m0, m1, bits, &s, &z)) atomicOr(&flags, 2);
-    const int64_t mi = ((int64_t)head * L.ng + gi) * D + cb + c;
+    const int64_t mi = (slab * L.ng + gi) * D + cb + c;
     reinterpret_cast<__half*>(S.scale)[mi] = s;
     reinterpret_cast<__half*>(S.zero)[mi] = z;
     sf[c] = __half2float(s);
@@ -146,7 +169,7 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
     s8[c] = sf[8 * v + c];
     z8[c] = zf[8 * v + c];
   }
-  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
   const int rowb = D * bits / 8;   // bytes per code row
 #pragma unroll
   for (int k = 0; k < kMaxKeyRows; ++k) {
@@ -183,6 +206,8 @@ __device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by
   const int nt = (int)min((int64_t)kTB, a.t0 + a.n - tb);
   const int head = by;
   const int b = head / L.Hkv, h = head % L.Hkv;
+  int64_t slab;
+  if (!dest_slab(a, head, b, h, &slab)) return;   // uniform over the CTA
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nvec = D / 8, rpp = 32 / nvec, sub = lane / nvec, vl = lane % nvec;
   const int passes = (4 + rpp - 1) / rpp;
@@ -196,7 +221,7 @@ __device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by
   }
   __syncthreads();   // flags initialised
   int bad = 0, rbad = 0;
-  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
   uint32_t half_prev = 0;   // 2- and 4-bit, one token per pass: the even token's half words
   uint32_t half_prev2 = 0;
 #pragma unroll
@@ -222,8 +247,8 @@ __device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by
     const bool good = asym_params(mn, mx, bits, &s, &z);
     if (ok && vl == 0) {
       rbad |= !good;
-      reinterpret_cast<__half*>(S.scale)[(int64_t)head * L.C + tb + t] = s;
-      reinterpret_cast<__half*>(S.zero)[(int64_t)head * L.C + tb + t] = z;
+      reinterpret_cast<__half*>(S.scale)[slab * L.C + tb + t] = s;
+      reinterpret_cast<__half*>(S.zero)[slab * L.C + tb + t] = z;
     }
     float s8[8], z8[8];
     const float sv = __half2float(s), zv = __half2float(z);
@@ -311,6 +336,8 @@ __device__ __forceinline__ void asym_keys_rot_block(const AArgs& a, int bx, int 
   const int ln = (int)min((int64_t)g, a.t0 + a.n - ts);
   const int gi = (int)(ts / g);
   const int b = head / L.Hkv, h = head % L.Hkv;
+  int64_t slab;
+  if (!dest_slab(a, head, b, h, &slab)) return;   // uniform over the CTA
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) flags = 0;
   float x[kRotRows][4];
@@ -380,7 +407,7 @@ __device__ __forceinline__ void asym_keys_rot_block(const AArgs& a, int bx, int 
     }
     __half sh, zh;
     if (!asym_params(m0, m1, bits, &sh, &zh)) atomicOr(&flags, 2);
-    const int64_t mi = ((int64_t)head * L.ng + gi) * 128 + c;
+    const int64_t mi = (slab * L.ng + gi) * 128 + c;
     reinterpret_cast<__half*>(S.scale)[mi] = sh;
     reinterpret_cast<__half*>(S.zero)[mi] = zh;
     sf[c] = __half2float(sh);
@@ -394,7 +421,7 @@ __device__ __forceinline__ void asym_keys_rot_block(const AArgs& a, int bx, int 
     z4[j] = zf[4 * lane + j];
   }
   const int maxc = (1 << bits) - 1;
-  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + (int64_t)head * S.code_slab_bytes;
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
   const int rowb = 128 * bits / 8;
 #pragma unroll
   for (int k = 0; k < kRotRows; ++k) {
@@ -487,6 +514,8 @@ cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, in
   a.t0 = t0;
   a.n = n;
   a.status = d_status;
+  a.blocks = nullptr;
+  a.num_blocks = 0;
   if (which == KVQ_KEYS && L.k_rotate) {
     dim3 grid((unsigned)((n + L.g - 1) / L.g), L.B * L.Hkv);
     asym_keys_rot_kernel<<<grid, kThreads, 0, s>>>(a);
@@ -506,8 +535,10 @@ namespace kvq {
 
 cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const void* vsrc, int64_t sb,
                                     int64_t sh, int64_t st, int64_t t0, int64_t n, int32_t* d_status,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, const int32_t* blocks, int num_blocks) {
   AArgs ak, av;
+  ak.blocks = av.blocks = blocks;
+  ak.num_blocks = av.num_blocks = num_blocks;
   ak.L = av.L = L;
   ak.src = ksrc;
   av.src = vsrc;

@@ -16,9 +16,9 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 # enums of include/kvq.h
 KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA, KVQ_ERR_WORKSPACE = range(5)
-KVQ_DEV_NONFINITE, KVQ_DEV_RANGE = 1, 2
+KVQ_DEV_NONFINITE, KVQ_DEV_RANGE, KVQ_DEV_TIMEOUT, KVQ_DEV_BOUNDS = 1, 2, 4, 8
 F32, F16, BF16 = 0, 1, 2
-NONE, SYM8, ASYM, NUQ, MIXED = range(5)
+NONE, SYM8, ASYM, NUQ, MIXED, KQV = range(6)
 TENSOR, TOKEN, CHANNEL = range(3)
 KEYS, VALUES = 0, 1
 
@@ -29,6 +29,7 @@ ARRAYS = [
     "v_out_col", "v_out_val",
     "k_lut", "v_lut",
     "sink_k", "sink_v", "res_k", "res_v",
+    "v_sketch",
 ]
 
 TORCH_DTYPE = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
@@ -49,6 +50,12 @@ class kvq_cache(ctypes.Structure):
                 ("capacity", ctypes.c_int64)] + [(n, ctypes.c_void_p) for n in ARRAYS]
 
 
+class kvq_paged_cache(ctypes.Structure):
+    _fields_ = [("pool", kvq_cache), ("num_seqs", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
+                ("block_table", ctypes.c_void_p), ("sink_k", ctypes.c_void_p), ("sink_v", ctypes.c_void_p),
+                ("res_k", ctypes.c_void_p), ("res_v", ctypes.c_void_p)]
+
+
 class KvqError(RuntimeError):
     def __init__(self, fn, status):
         super().__init__(f"{fn}: {status_string(status)} ({status})")
@@ -67,11 +74,13 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         FP, CP = ctypes.POINTER(kvq_format), ctypes.POINTER(kvq_cache)
+        PP = ctypes.POINTER(kvq_paged_cache)
         sig = {
             "kvq_version": (I32, []),
             "kvq_status_string": (ctypes.c_char_p, [I32]),
             "kvq_format_check": (I32, [FP]),
             "kvq_cache_array_bytes": (SZ, [FP, I32, I32, I64, I32]),
+            "kvq_kqv_codebook": (I32, [I32, I32, ctypes.POINTER(ctypes.c_float)]),
             "kvq_quantize_keys": (I32, [FP, CP, P, I64, I64, I64, I64, I64, P, P]),
             "kvq_quantize_values": (I32, [FP, CP, P, I64, I64, I64, I64, I64, P, P]),
             "kvq_quantize_kv": (I32, [FP, CP, P, P, I64, I64, I64, I64, I64, P, P]),
@@ -89,6 +98,10 @@ def lib():
             "kvq_merge_states": (I32, [I32, I64, I32, P, P, P, I32, P, P]),
             "kvq_decode_attention_noalloc": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float,
                                                    P, I32, I32, P, P]),
+            "kvq_quantize_kv_paged": (I32, [FP, PP, P, P, I64, I64, I64, P, I64, P, P]),
+            "kvq_decode_paged_workspace_bytes": (SZ, [FP, I32, I32, I32, I64, I32]),
+            "kvq_decode_attention_paged": (I32, [FP, PP, P, P, I64, I32, P, I32, I32, ctypes.c_float, P,
+                                                 I32, P, SZ, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -131,11 +144,20 @@ def cache_array_bytes(fmt: kvq_format, B, H, C, array_id) -> int:
     return lib().kvq_cache_array_bytes(ctypes.byref(fmt), B, H, C, array_id)
 
 
+def kqv_codebook(bits: int, head_dim: int):
+    """kvq_kqv_codebook: the 2^bits fp32 Lloyd-Max centroids (a list of floats)."""
+    out = (ctypes.c_float * (1 << bits))()
+    _check("kvq_kqv_codebook", lib().kvq_kqv_codebook(bits, head_dim, out))
+    return list(out)
+
+
 class Cache:
-    """Device arrays of a packed cache (torch uint8 tensors), owned by this object."""
+    """Device arrays of a packed cache (torch uint8 tensors), owned by this object.
+    k_lut / v_lut: the codebooks (NUQ: stored as fp16, KQV: fp32); sketch: the KQV sketch
+    matrix [D][D] (stored as fp32)."""
 
     def __init__(self, fmt: kvq_format, B: int, H: int, C: int, device="cuda", k_lut=None,
-                 v_lut=None):
+                 v_lut=None, sketch=None):
         self.fmt, self.B, self.H, self.C = fmt, B, H, C
         self.tensors = {}
         self.struct = kvq_cache(batch=B, kv_heads=H, capacity=C)
@@ -145,9 +167,12 @@ class Cache:
                 t = torch.zeros(n, dtype=torch.uint8, device=device)
                 self.tensors[name] = t
                 setattr(self.struct, name, t.data_ptr())
-        for name, lut in (("k_lut", k_lut), ("v_lut", v_lut)):
+        for name, lut, scheme in (("k_lut", k_lut, fmt.k_scheme), ("v_lut", v_lut, fmt.v_scheme)):
             if name in self.tensors and lut is not None:
-                self.tensors[name].copy_(torch.tensor(lut, dtype=torch.float16).view(torch.uint8))
+                dt = torch.float32 if scheme == KQV else torch.float16
+                self.tensors[name].copy_(torch.tensor(lut, dtype=dt).reshape(-1).view(torch.uint8))
+        if "v_sketch" in self.tensors and sketch is not None:
+            self.tensors["v_sketch"].copy_(torch.as_tensor(sketch, dtype=torch.float32).reshape(-1).view(torch.uint8))
 
     def array(self, name):
         return self.tensors[name]
@@ -290,4 +315,61 @@ def decode_attention_noalloc(fmt, cache: Cache, q: torch.Tensor, t_quant: int, t
                                             _ptr(out), out_dtype, num_splits, _ptr(status),
                                             _stream(stream))
     _check("kvq_decode_attention_noalloc", st)
+    return out
+
+
+class PagedCache:
+    """A paged cache: a pool of num_blocks blocks (one token group of every KV head each,
+    the layout of a Cache with batch = num_blocks and capacity = group_tokens), per-sequence
+    sink / residual arrays and a device block table [num_seqs][max_blocks] (int32, -1)."""
+
+    def __init__(self, fmt: kvq_format, kv_heads: int, num_blocks: int, num_seqs: int, max_blocks: int,
+                 device="cuda"):
+        self.fmt, self.H, self.num_blocks = fmt, kv_heads, num_blocks
+        self.num_seqs, self.max_blocks = num_seqs, max_blocks
+        self.pool = Cache(fmt, num_blocks, kv_heads, fmt.group_tokens, device=device)
+        raw = Cache(fmt, num_seqs, kv_heads, fmt.group_tokens, device=device)
+        self.raw = {n: raw.tensors[n] for n in ("sink_k", "sink_v", "res_k", "res_v") if n in raw.tensors}
+        self.block_table = torch.full((num_seqs, max_blocks), -1, dtype=torch.int32, device=device)
+        self.struct = kvq_paged_cache(pool=self.pool.struct, num_seqs=num_seqs, max_blocks=max_blocks,
+                                      block_table=self.block_table.data_ptr())
+        for n, t in self.raw.items():
+            setattr(self.struct, n, t.data_ptr())
+
+    def array(self, name):
+        return self.raw[name] if name in self.raw else self.pool.tensors[name]
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+def quantize_kv_paged(fmt, cache: PagedCache, k_src: torch.Tensor, v_src: torch.Tensor, blocks: torch.Tensor,
+                      n: int, status=None, stream=None):
+    """kvq_quantize_kv_paged: k_src, v_src [num_seqs, H, n, D]; blocks int32 [num_seqs] (device)."""
+    if k_src.stride() != v_src.stride():
+        raise ValueError("k_src and v_src must have the same strides")
+    st = lib().kvq_quantize_kv_paged(ctypes.byref(fmt), cache.ref(), _ptr(k_src), _ptr(v_src), k_src.stride(0),
+                                     k_src.stride(1), k_src.stride(2), _ptr(blocks), n, _ptr(status),
+                                     _stream(stream))
+    _check("kvq_quantize_kv_paged", st)
+
+
+def decode_paged_workspace_bytes(fmt, num_seqs, Hq, Hkv, max_t_quant, max_t_res) -> int:
+    return lib().kvq_decode_paged_workspace_bytes(ctypes.byref(fmt), num_seqs, Hq, Hkv, max_t_quant, max_t_res)
+
+
+def decode_attention_paged(fmt, cache: PagedCache, t_quant: torch.Tensor, t_res: torch.Tensor, max_t_quant: int,
+                           max_t_res: int, q: torch.Tensor, scale: float, out_dtype=F32, out=None, workspace=None,
+                           status=None, stream=None):
+    """kvq_decode_attention_paged: t_quant, t_res int32 [num_seqs] (device); q [num_seqs, Hq, D]."""
+    S, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((S, Hq, D), dtype=TORCH_DTYPE[out_dtype], device=q.device)
+    need = decode_paged_workspace_bytes(fmt, S, Hq, cache.H, max_t_quant, max_t_res)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().kvq_decode_attention_paged(ctypes.byref(fmt), cache.ref(), _ptr(t_quant), _ptr(t_res), max_t_quant,
+                                          max_t_res, _ptr(q), KVQ_DTYPE[q.dtype], Hq, scale, _ptr(out), out_dtype,
+                                          _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _check("kvq_decode_attention_paged", st)
     return out

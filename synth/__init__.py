@@ -31,7 +31,7 @@ from __future__ import annotations
 import numpy as np
 
 F32, F16, BF16 = 0, 1, 2
-NONE, SYM8, ASYM, NUQ, MIXED = 0, 1, 2, 3, 4
+NONE, SYM8, ASYM, NUQ, MIXED, KQV = 0, 1, 2, 3, 4, 5
 TENSOR, TOKEN, CHANNEL = 0, 1, 2
 
 TAGS = {"k": 1, "v": 2, "q": 3, "qwin": 4, "kchan": 5, "qchan": 6, "toy": 7}

@@ -32,7 +32,7 @@ def test_library_exports_every_declared_function():
     lib = kvq.lib()
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.kvq_version() == (0 << 16) | 1
+    assert lib.kvq_version() == (0 << 16) | 2
 
 
 def test_status_strings():
@@ -205,3 +205,21 @@ def test_noalloc_rejects_oversized_requests():
     st = kvq.lib().kvq_decode_attention_noalloc(ctypes.byref(f), ctypes.byref(cache), None, kvq.BF16, Hq,
                                                 tq, 0, 0.1, None, kvq.F32, 64, None, None)
     assert st == kvq.KVQ_ERR_WORKSPACE
+
+
+def test_paged_entry_points_validate_on_the_host():
+    # null pools, tables and lengths are refused before anything runs (all pointers null)
+    L = kvq.lib()
+    f = _fmt(k_bits=4, v_bits=2)
+    pc = kvq.kvq_paged_cache()
+    pc.pool = kvq.kvq_cache(batch=4, kv_heads=2, capacity=128)
+    pc.num_seqs, pc.max_blocks = 2, 3
+    assert L.kvq_decode_attention_paged(ctypes.byref(f), ctypes.byref(pc), None, None, 256, 0, None, kvq.BF16, 8,
+                                        0.1, None, kvq.F32, None, 0, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_quantize_kv_paged(ctypes.byref(f), ctypes.byref(pc), None, None, 0, 0, 128, None, 16, None,
+                                   None) == kvq.KVQ_ERR_INVALID
+    # workspace sizing: unsupported head groups and formats give 0
+    assert L.kvq_decode_paged_workspace_bytes(ctypes.byref(f), 2, 16, 2, 256, 0) == 0     # G = 8
+    assert L.kvq_decode_paged_workspace_bytes(ctypes.byref(f), 2, 8, 2, 256, 0) > 0
+    f8 = _fmt(k_bits=8)
+    assert L.kvq_decode_paged_workspace_bytes(ctypes.byref(f8), 2, 8, 2, 256, 0) == 0

@@ -170,3 +170,54 @@ def test_rejects_nonfinite_source():
     K[0, 0, 3, 4] = np.nan
     with pytest.raises(quant.RejectedInput):
         quantize(f, c, KEYS, K, 0, 16)
+
+
+def test_paged_decode_equals_contiguous_per_sequence():
+    # A paged cache whose sequences own scattered blocks gives each sequence the attention
+    # over its own tokens: the same output as a contiguous cache holding that sequence
+    # alone, whatever the block placement (lengths with ragged last groups, one group, none)
+    from oracle import attention as oatt
+    from oracle import cache as ocache
+    from oracle import paged
+    from oracle.formats import Format
+
+    def vals(shape):
+        return fp.f16(rng.standard_normal(shape))
+    fd = dict(head_dim=32, group_tokens=16, src_dtype=F16, n_sink=1, residual_cap=8)
+    f = Format(**fd)
+    H, G, g = 2, 2, 16
+    t_quant = [37, 16, 5, 0]
+    t_res = [3, 0, 8, 2]
+    S = len(t_quant)
+    rng = np.random.default_rng(8)
+    pc = paged.PagedCache(f, H, num_blocks=9, num_seqs=S, max_blocks=3)
+    perm = rng.permutation(9)
+    contig, used = [], 0
+    for s in range(S):
+        ng = -(-t_quant[s] // g)
+        c = ocache.Cache(f, 1, H, max(1, ng) * g)
+        K = vals((1, H, max(1, ng) * g, 32))
+        V = vals((1, H, max(1, ng) * g, 32))
+        for gi in range(ng):
+            n = min(g, t_quant[s] - gi * g)
+            blk = int(perm[used]); used += 1
+            pc.block_table[s, gi] = blk
+            paged.quantize_group(pc, KEYS, K[0, :, gi * g:gi * g + n], blk, n)
+            paged.quantize_group(pc, VALUES, V[0, :, gi * g:gi * g + n], blk, n)
+            ocache.quantize(f, c, KEYS, K[:, :, gi * g:gi * g + n], gi * g, n)
+            ocache.quantize(f, c, VALUES, V[:, :, gi * g:gi * g + n], gi * g, n)
+        for name, shape in (("sink_k", 1), ("sink_v", 1), ("res_k", 8), ("res_v", 8)):
+            raw = ocache.raw_encode(vals((H, shape, 32)), F16)
+            pc.raw[name][s] = raw
+            c[name][0] = raw
+        contig.append(c)
+    q = vals((S, H * G, 32))
+    got = paged.decode_attention(pc, q, t_quant, t_res)
+    for s in range(S):
+        want = oatt.decode_attention(f, contig[s], q[s:s + 1], t_quant[s], t_res[s])[0]
+        np.testing.assert_array_equal(got[s], want)
+        # and the gathered cache holds the same packed bytes as the contiguous one
+        gc = paged.sequence_cache(pc, s, t_quant[s])
+        for name in ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero"):
+            n_rows = gc[name].shape[2]
+            np.testing.assert_array_equal(gc[name][0][:, :n_rows], contig[s][name][0][:, :n_rows])
