@@ -5,10 +5,11 @@ decode attention over the packed cache, on synthetic data shaped like the worklo
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config llama3_8b]
 
-One step = kvq_quantize_kv (keys and values) of one 128-token group (the flush of
-the raw window into the packed cache) + kvq_decode_partial (split kernel)
-+ kvq_decode_combine over all T tokens.  Every step is timed with CUDA events on the
-launching stream; the L2 is flushed between steps, outside the events, by a 512 MiB write and
+One step = kvq_append_decode_attention: the append (kvq_quantize_kv, keys and values)
+of one 128-token group (the flush of the raw window into the packed cache), then the
+split kernel and the combine over all T tokens.  Every step is timed with CUDA events on
+the launching stream, one pair around each step; the per-kernel breakdown comes from a
+separate pass of separate calls with an event between every two launches; the L2 is flushed between steps, outside the events, by a 512 MiB write and
 then a 512 MiB read of another buffer (so that no dirty line of the flush is left
 for the step to write back).  `value` is the effective HBM throughput of the whole step: the format's
 algorithmic bytes (codes, scales, zero-points, raw sink / residual tokens, the new
@@ -37,6 +38,9 @@ METRIC = "Decode-attn effective HBM GB/s over packed KV (% of 8 TB/s); quantize 
 L2_FLUSH_BYTES = 512 << 20
 LAUNCHES_PER_STEP = 3   # quantize K+V (one launch on the K4/V2 path), split kernel, combine
 PATH_DTYPE = {
+    "decode_k4v2_kernel": "f16 tensor-core operands (codes as exact f16 subnormals, probabilities as f16 "
+                          "hi + lo pairs), f32 accumulation",
+    "decode_kqv_kernel": "f32 on CUDA cores (fp32 centroids, sketch signs)",
     "decode_mma_kernel": "f16 tensor-core operands (codes as exact f16 subnormals), f32 accumulation",
     "decode_cc_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
     "decode_generic_kernel": "f32 on CUDA cores (codes reconstructed to f32)",
@@ -49,6 +53,10 @@ def decode_path(cfg):
     G = cfg["Hq"] // cfg["Hkv"]
     mix = f["k_scheme"] == synth.MIXED and f["mixed_hi"] == 8 and f["mixed_mid"] == 24 and \
         f["src_dtype"] == synth.BF16 and f["v_scheme"] == synth.ASYM and f["v_bits"] == 2 and not f["rope"]
+    if f["k_scheme"] == synth.KQV:
+        return "decode_kqv_kernel"
+    if is_k4v2(cfg) and f["head_dim"] == 128 and f["group_tokens"] == 128 and 1 <= G <= 4:
+        return "decode_k4v2_kernel"
     if (is_k4v2(cfg) or mix) and f["head_dim"] == 128 and f["group_tokens"] == 128 and 1 <= G <= 8:
         return "decode_mma_kernel"
     k_ok = (f["k_scheme"] == synth.NUQ) or (f["k_scheme"] == synth.ASYM and f["k_bits"] in (2, 4)) or \
@@ -66,7 +74,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="llama3_8b",
-                    choices=["llama3_8b", "llama2_7b", "kvquant_nuq3", "mixkvq_14b", "llama3_8b_wht"])
+                    choices=list(synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -352,6 +360,10 @@ def run_reference(args, world, rank):
     cfg = synth.CONFIGS[args.config]
     if rank != 0:
         return
+    if cfg["fmt"]["k_scheme"] == synth.KQV:
+        print(json.dumps({"impl": "reference", "unavailable": "the oracle's timed path covers the cache "
+                          "schemes of oracle.cache, not KQV"}), flush=True)
+        return
     per_step = max(0.02, 120.0 / max(1, args.steps + args.warmup))
     smp = oracle_sized(cfg, per_step)
     with single_thread():
@@ -376,8 +388,11 @@ def workload_config(cfg):
     ns, tq, tr = synth.split_tokens(cfg)
     f = cfg["fmt"]
     names = {synth.NONE: "raw", synth.SYM8: "INT8 sym", synth.ASYM: "asym", synth.NUQ: "nuq", synth.MIXED: "mixed"}
+    names[synth.KQV] = "KQV"
     kdesc = (f"mixed {f['mixed_hi']} raw / {f['mixed_mid']} 4-bit / rest 2-bit by salience"
-             if f["k_scheme"] == synth.MIXED else f"{names[f['k_scheme']]}{f['k_bits']} per-channel")
+             if f["k_scheme"] == synth.MIXED else
+             f"KQV {f['k_bits']}-bit Lloyd-Max codes of the rotated direction per token"
+             if f["k_scheme"] == synth.KQV else f"{names[f['k_scheme']]}{f['k_bits']} per-channel")
     if f.get("k_rotate"):
         kdesc += " after a Walsh-Hadamard rotation of each key"
     extra = []
@@ -388,7 +403,9 @@ def workload_config(cfg):
     n_app = cfg.get("append", f["group_tokens"])
     return {"workload": f"{cfg['name']}: B={cfg['B']} Hq={cfg['Hq']} Hkv={cfg['Hkv']} D={cfg['D']} "
                         f"T={cfg['T']} (sink {ns}, packed {tq}, residual {tr}); K {kdesc} "
-                        f"g{f['group_tokens']} + V {names[f['v_scheme']]}{f['v_bits']} per-token"
+                        + (f"+ V KQV {f['v_bits'] - 1}-bit codes + 1-bit sketch per token"
+                           if f["v_scheme"] == synth.KQV else
+                           f"g{f['group_tokens']} + V {names[f['v_scheme']]}{f['v_bits']} per-token")
                         + ("; " + ", ".join(extra) if extra else ""),
             "B": cfg["B"], "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "D": cfg["D"], "T": cfg["T"],
             "step": f"append of {n_app} tokens (quantize K, V" +
@@ -421,11 +438,16 @@ def main():
     # ---- build the cache on the device (data drawn on the device, same recipe)
     K = synth.device_kv(cfg, "k", device=dev, seed_offset=rank)
     V = synth.device_kv(cfg, "v", device=dev, seed_offset=rank)
-    luts = (None, None)
+    luts, sketch = (None, None), None
     if fd["k_scheme"] == synth.NUQ:
         cb = json.load(open(os.path.join(ROOT, "tests", "golden", "nuq3_codebook.json")))
         luts = (cb["k"], cb["v"])
-    cache = kvq.Cache(fmt, B, Hkv, C, device=dev, k_lut=luts[0], v_lut=luts[1])
+    if fd["k_scheme"] == synth.KQV:   # the library's Lloyd-Max codebooks, a seeded N(0, 1) sketch
+        luts = (kvq.kqv_codebook(fd["k_bits"], D), kvq.kqv_codebook(fd["v_bits"] - 1, D))
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(cfg["seed"] * 1000 + 55)
+        sketch = torch.randn((D, D), device=dev, generator=gen)
+    cache = kvq.Cache(fmt, B, Hkv, C, device=dev, k_lut=luts[0], v_lut=luts[1], sketch=sketch)
     mixed = fd["k_scheme"] == synth.MIXED
     qwin = None
     if mixed:   # salience windows: query rows at every packed position (device-drawn)
@@ -485,26 +507,32 @@ def main():
 
     order = cache.array("k_order") if mixed else None
 
-    def append(k_src, v_src, w_src):
+    def salience(k_src, w_src):
         if mixed:
             for j in range(n_app // g):
                 kvq.key_salience(fmt, w_src[:, :, j * g:(j + 1) * g], k_src[:, :, j * g:(j + 1) * g],
                                  order[(gi_f + j) * D:], Hkv * (C // g) * D, (C // g) * D,
                                  status=status, stream=stream)
-        kvq.quantize_kv(fmt, cache, k_src, v_src, a0, n_app, status=status, stream=stream)
+
+    def fused(k_src, v_src, w_src, qq):
+        # the public one-call step: append then decode (kvq_append_decode_attention)
+        salience(k_src, w_src)
+        kvq.append_decode_attention(fmt, cache, k_src, v_src, a0, n_app, qq, tq, tr, scale, kvq.F32, out=out,
+                                    workspace=ws, status=status, stream=stream)
 
     def step(evs=None):
-        if evs:
-            evs[0].record(stream)
-        append(newk, newv, neww)
-        if evs:
-            evs[1].record(stream)
+        if not evs:
+            fused(newk, newv, neww, q)
+            return
+        # the same work as separate calls, an event between every two
+        evs[0].record(stream)
+        salience(newk, neww)
+        kvq.quantize_kv(fmt, cache, newk, newv, a0, n_app, status=status, stream=stream)
+        evs[1].record(stream)
         kvq.decode_partial(fmt, cache, q, tq, tr, scale, ws, status=status, stream=stream)
-        if evs:
-            evs[2].record(stream)
+        evs[2].record(stream)
         kvq.decode_combine(fmt, B, Hq, Hkv, tq, tr, ws, out, stream=stream)
-        if evs:
-            evs[3].record(stream)
+        evs[3].record(stream)
 
     for i in range(args.warmup):
         flush_l2(i)
@@ -515,7 +543,9 @@ def main():
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # the timed steps: one event pair around each step (events between the launches
+    # would stop each kernel from starting while its predecessor drains)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -524,19 +554,24 @@ def main():
     time.sleep(0.15)
     for i in range(args.steps):
         flush_l2(i)
-        step(evs[i])
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    t_quant = [e[0].elapsed_time(e[1]) for e in evs]
-    t_part = [e[1].elapsed_time(e[2]) for e in evs]
-    t_comb = [e[2].elapsed_time(e[3]) for e in evs]
-    t_step = [e[0].elapsed_time(e[3]) for e in evs]
-    ms_step = statistics.mean(t_step)
-    ms_part = statistics.mean(t_part)
-    ms_comb = statistics.mean(t_comb)
-    ms_quant = statistics.mean(t_quant)
+    ms_step = statistics.mean([e[0].elapsed_time(e[1]) for e in evs])
+    # the breakdown: a separate pass with an event between every two launches
+    nb = min(args.steps, 50)
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
+    for i in range(nb):
+        flush_l2(i)
+        step(bevs[i])
+    torch.cuda.synchronize(dev)
+    ms_quant = statistics.mean([e[0].elapsed_time(e[1]) for e in bevs])
+    ms_part = statistics.mean([e[1].elapsed_time(e[2]) for e in bevs])
+    ms_comb = statistics.mean([e[2].elapsed_time(e[3]) for e in bevs])
     ms_step, ms_part, ms_comb, ms_quant = max_over_ranks([ms_step, ms_part, ms_comb, ms_quant], dev)
 
     # ---- end to end through the public API with host buffers
@@ -565,9 +600,7 @@ def main():
         dq.copy_(hq, non_blocking=True)
         if mixed:
             dw.copy_(hw, non_blocking=True)
-        append(dk, dv, dw)
-        kvq.decode_attention(fmt, cache, dq, tq, tr, scale, kvq.F32, out=out, workspace=ws,
-                             status=status, stream=stream)
+        fused(dk, dv, dw, dq)
         hout.copy_(out, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -626,7 +659,8 @@ def main():
         "pct_of_8tbs": 100.0 * value / world / 8000.0,
         "decode_gbs": decode_gbs, "quantize_gbs": quant_gbs,
         "tokens_heads_per_s": world * B * Hq * cfg["T"] / ((ms_part + ms_comb) * 1e-3),
-        "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb},
+        "ms_breakdown": {"quantize": ms_quant, "decode_split": ms_part, "combine": ms_comb,
+                         "note": "a separate pass with an event between every two launches"},
         "full_cache_quantize": full_quant,
         "roofline": {"kernel": f"{path} (kvq_decode_partial)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
@@ -638,10 +672,13 @@ def main():
         * args.steps,
         "clocks": clocks,
     }
-    if path != "decode_mma_kernel":
+    if path not in ("decode_mma_kernel", "decode_k4v2_kernel"):
         line["roofline"]["traffic"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg)
+        if fd["k_scheme"] == synth.KQV:   # the oracle times the cache schemes of oracle.cache only
+            line["cpu_baseline"] = None
+        else:
+            line["cpu_baseline"] = cpu_baseline(cfg)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

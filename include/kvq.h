@@ -337,6 +337,23 @@ kvq_status kvq_decode_attention(const kvq_format* fmt, const kvq_cache* cache,
                                 size_t workspace_bytes, int32_t num_splits,
                                 int32_t* d_status, void* stream);
 
+/* One decode step with its append ([MIX] Figure 4: the full recent window is quantized
+ * into the packed cache and the step then attends over all tokens; [KVQ] "Approach"):
+ * the same as kvq_quantize_kv(fmt, cache, k_src, v_src, stride_b, stride_h, stride_t, t0,
+ * n) followed by kvq_decode_attention(fmt, cache, q, ...) on the same stream, with the
+ * same results bit for bit.  Every argument of both is checked before anything is
+ * launched; n = 0 appends nothing.  When the format's append is one kernel and the
+ * tensor-core split kernel decodes it, the split kernel starts while the append still
+ * runs and waits for it only where it reaches the appended groups' rows. */
+kvq_status kvq_append_decode_attention(const kvq_format* fmt, const kvq_cache* cache,
+                                       const void* k_src, const void* v_src, int64_t stride_b,
+                                       int64_t stride_h, int64_t stride_t, int64_t t0, int64_t n,
+                                       const void* q, int32_t q_dtype, int32_t q_heads,
+                                       int64_t t_quant, int32_t t_residual, float softmax_scale,
+                                       void* out, int32_t out_dtype, void* workspace,
+                                       size_t workspace_bytes, int32_t num_splits,
+                                       int32_t* d_status, void* stream);
+
 /* The two halves of kvq_decode_attention, for callers that time, overlap or
  * distribute them (for instance a sequence split over several GPUs that gathers the
  * partial states before merging them).  kvq_decode_partial runs the split kernel and

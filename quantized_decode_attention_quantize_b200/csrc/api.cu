@@ -472,10 +472,11 @@ int32_t kvq_decode_partial_slots(const kvq_format* f, int32_t B, int32_t Hq, int
   return plan_decode(L, Hq, t_quant, t_res, num_splits).S;
 }
 
-static kvq_status partial_common(const kvq_format* f, const kvq_cache* c, const void* q,
+// Validation and plan of a decode call; nothing is launched.
+static kvq_status decode_prepare(const kvq_format* f, const kvq_cache* c, const void* q,
                                  int32_t q_dtype, int32_t Hq, int64_t t_quant, int32_t t_res,
                                  float scale, void* ws, size_t ws_bytes, int32_t num_splits,
-                                 int32_t* d_status, void* stream, Layout* L, DecodePlan* p) {
+                                 int32_t* d_status, Layout* L, DecodePlan* p) {
   kvq_status s = make_layout(f, c, L);
   if (s != KVQ_OK) return s;
   s = decode_args(f, L->B, Hq, L->Hkv, t_quant, t_res, num_splits);
@@ -490,6 +491,16 @@ static kvq_status partial_common(const kvq_format* f, const kvq_cache* c, const 
   *p = plan_decode(*L, Hq, t_quant, t_res, num_splits);
   if (!ws || !aligned16(ws)) return KVQ_ERR_INVALID;
   if (ws_bytes < workspace_bytes(*L, Hq, *p)) return KVQ_ERR_WORKSPACE;
+  return KVQ_OK;
+}
+
+static kvq_status partial_common(const kvq_format* f, const kvq_cache* c, const void* q,
+                                 int32_t q_dtype, int32_t Hq, int64_t t_quant, int32_t t_res,
+                                 float scale, void* ws, size_t ws_bytes, int32_t num_splits,
+                                 int32_t* d_status, void* stream, Layout* L, DecodePlan* p) {
+  kvq_status s = decode_prepare(f, c, q, q_dtype, Hq, t_quant, t_res, scale, ws, ws_bytes, num_splits,
+                                d_status, L, p);
+  if (s != KVQ_OK) return s;
   cudaError_t e = launch_decode_partial(*L, *p, q, q_dtype, Hq, t_quant, t_res, scale, ws, d_status,
                                         reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -544,6 +555,47 @@ kvq_status kvq_merge_states(int32_t n_parts, int64_t rows, int32_t head_dim, con
     return KVQ_ERR_INVALID;
   cudaError_t e = launch_merge_states(n_parts, rows, head_dim, outs, lses, out, out_dtype, lse_out,
                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_append_decode_attention(const kvq_format* f, const kvq_cache* c, const void* k_src,
+                                       const void* v_src, int64_t sb, int64_t sh, int64_t st, int64_t t0,
+                                       int64_t n, const void* q, int32_t q_dtype, int32_t Hq, int64_t t_quant,
+                                       int32_t t_res, float scale, void* out, int32_t out_dtype, void* ws,
+                                       size_t ws_bytes, int32_t num_splits, int32_t* d_status, void* stream) {
+  // every argument of both halves is checked before anything is launched
+  if (!out || !aligned16(out) || !valid_dtype(out_dtype)) return KVQ_ERR_INVALID;
+  Layout L;
+  DecodePlan p;
+  kvq_status s = decode_prepare(f, c, q, q_dtype, Hq, t_quant, t_res, scale, ws, ws_bytes, num_splits, d_status,
+                                &L, &p);
+  if (s != KVQ_OK) return s;
+  if (n < 0 || t0 < 0 || t0 % L.g || t0 + n > L.C) return KVQ_ERR_INVALID;
+  if (n > 0) {
+    if (!k_src || !v_src || !aligned16(k_src) || !aligned16(v_src)) return KVQ_ERR_INVALID;
+    const int64_t eb = dtype_bytes(L.src_dtype);
+    if (st < L.D || sb < 0 || sh < 0) return KVQ_ERR_INVALID;
+    if ((st * eb) % 16 || (sh * eb) % 16 || (sb * eb) % 16) return KVQ_ERR_INVALID;
+  }
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (n > 0) {
+    if (asym_fast_ok(L, KVQ_KEYS) && asym_fast_ok(L, KVQ_VALUES)) {
+      // one append kernel directly before the split kernel: the split kernel reads the
+      // rows the append does not touch without waiting for it
+      if (launch_quantize_asym_kv(L, k_src, v_src, sb, sh, st, t0, n, d_status, cs) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+      p.defer = 1;
+      p.dep_lo = t0;
+      p.dep_hi = t0 + n;
+    } else {
+      if (launch_quantize(L, KVQ_KEYS, k_src, sb, sh, st, t0, n, d_status, cs) != cudaSuccess ||
+          launch_quantize(L, KVQ_VALUES, v_src, sb, sh, st, t0, n, d_status, cs) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    }
+  }
+  if (launch_decode_partial(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws, d_status, cs) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  cudaError_t e = launch_combine(L, Hq, p, ws, out, out_dtype, nullptr, cs);
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

@@ -110,6 +110,11 @@ struct MmaArgs {
   float* ws_l;
   float* ws_o;
   int32_t* status;
+  // defer = 1: the kernel before this one on the stream writes packed rows [dep_lo, dep_hi)
+  // (an append) and nothing else that this kernel reads; a warp waits for it only before
+  // it first copies a group meeting those rows, and every thread waits before it exits.
+  int defer;
+  int64_t dep_lo, dep_hi;
 };
 
 // ---- partition of the items over the warps (shared with the combine kernel) ------------
@@ -1712,6 +1717,7 @@ struct LeanWarp {
   float* kmeta;       // the group's key scale / zero-point as fp32, [2][128]
   uint64_t* bars;     // one mbarrier per stage
   int nbulk, ncons;   // halves issued to / consumed from the ring
+  bool dep_done;      // the preceding kernel is known to be complete
 };
 
 // One warp's run over one KV head: raw items [ra, rb) (nraw raw tokens in all, rows of
@@ -1746,6 +1752,13 @@ __device__ __forceinline__ bool lean_run(const MmaArgs& a, LeanState& st, LeanWa
   // two halves in flight; a half's stage is released once its value words are in
   // registers, and its value product runs during the next half's key product
   auto issue = [&](int q) {
+    if (a.defer && !w.dep_done) {   // the group of half q (codes and metadata) meets the append
+      const int64_t g0 = 128 * (int64_t)(q >> 1);
+      if (g0 < a.dep_hi && g0 + 128 > a.dep_lo) {
+        griddep_wait();
+        w.dep_done = true;
+      }
+    }
     int64_t slab;
     int ph;
     slab_of(q, &slab, &ph);
@@ -1814,6 +1827,7 @@ __device__ __forceinline__ LeanWarp lean_warp(uint8_t* smem, int warp, int nw) {
   w.kmeta = reinterpret_cast<float*>(w.ring + kBuffers * kStageBytes + kQBytes + kBScratch);
   w.bars = reinterpret_cast<uint64_t*>(smem + (size_t)nw * kLeanWarpBytes) + kBuffers * warp;
   w.nbulk = w.ncons = 0;
+  w.dep_done = false;
   if ((threadIdx.x & 31) == 0) {
 #pragma unroll
     for (int b = 0; b < kBuffers; ++b) mbar_init(&w.bars[b], 1);
@@ -1858,7 +1872,9 @@ __device__ __forceinline__ void lean_merge(const MmaArgs& a, uint8_t* smem, int 
 template <bool ROT>
 __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  griddep_wait();   // launched with launch_pdl: the cache and q are complete
+  // launched with launch_pdl: without a deferred wait the cache and q are complete from
+  // here on; with one (an append just before), see MmaArgs::defer
+  if (!a.defer) griddep_wait();
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = (int64_t)blockIdx.x * kCW + warp;
@@ -1901,6 +1917,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   if (timed_out) lean_drain(a, w);
   __syncwarp();
   if (__any_sync(0xffffffffu, qbad) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+  // this grid completes only after the one before it, so that the kernels after it on
+  // the stream find the append done as well
+  if (a.defer) griddep_wait();
 
   // ---- merge of the warps' last heads inside the CTA (as decode_mma_kernel) ----
   const int lh = i1 > 0 ? (int)((i1 - 1) / U) : -1;
@@ -2162,6 +2181,9 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.ws_l = ws_l;
   a.ws_o = ws_o;
   a.status = d_status;
+  a.defer = p.defer;
+  a.dep_lo = p.dep_lo;
+  a.dep_hi = p.dep_hi;
   const bool mix = L.side[0].scheme == KVQ_MIXED;
   if (!mix && a.G <= 4) {
     const size_t smem = lean_smem();

@@ -85,6 +85,10 @@ struct DecodePlan {
   int raw_pieces;       // fast path: raw positions per head (two per raw item)
   int fast;             // 1 when the tensor-core K4/V2 kernel runs the packed region
   int grid_ctas;        // CTAs of the split kernel
+  // set by the append-and-decode entry point: the split kernel follows the append of
+  // packed rows [dep_lo, dep_hi) directly and may read the other rows before it completes
+  int defer = 0;
+  int64_t dep_lo = 0, dep_hi = 0;
 };
 DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int num_splits);
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p);
@@ -159,6 +163,20 @@ __device__ __forceinline__ bool asym_params(float mn, float mx, int bits, __half
 
 __device__ __forceinline__ int asym_code(float x, float s, float z, int maxc) {
   float q = __fdiv_rn(__fsub_rn(x, z), s);
+  float r = rintf(q);
+  r = fminf(fmaxf(r, 0.0f), (float)maxc);
+  return (int)r;
+}
+
+// The same code without a division in the common case, given rs = fl32(1 / s): for the
+// in-range quotients of a group (|q| <= 2^8) q1 = fl32(fl32(x - z) * rs) is within
+// 2^-22 |q| + 2^-24 |q| < 2^-13 of the exact quotient, so q1 and fl32(fl32(x - z) / s)
+// round to the same integer unless q1 lies within 2^-12 of a half-integer; there the
+// quotient is taken exactly.  Out-of-range quotients clip to the same end either way.
+__device__ __forceinline__ int asym_code_r(float x, float s, float rs, float z, int maxc) {
+  const float u = __fsub_rn(x, z);
+  float q = __fmul_rn(u, rs);
+  if (fabsf(q - floorf(q) - 0.5f) < 0x1p-12f) q = __fdiv_rn(u, s);
   float r = rintf(q);
   r = fminf(fmaxf(r, 0.0f), (float)maxc);
   return (int)r;

@@ -68,17 +68,19 @@ __device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, fl
 }
 
 // 8 codes of `bits` bits packed LSB-first (bits = 2: 16 bits, 4: 32 bits; 8: two words)
-__device__ __forceinline__ uint2 pack8(const float* x, const float* s, const float* z, int bits) {
+__device__ __forceinline__ uint2 pack8(const float* x, const float* s, const float* rs, const float* z,
+                                       int bits) {
   const int maxc = (1 << bits) - 1;
   uint32_t lo = 0, hi = 0;
   if (bits == 8) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) lo |= (uint32_t)asym_code(x[j], s[j], z[j], maxc) << (8 * j);
+    for (int j = 0; j < 4; ++j) lo |= (uint32_t)asym_code_r(x[j], s[j], rs[j], z[j], maxc) << (8 * j);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) hi |= (uint32_t)asym_code(x[4 + j], s[4 + j], z[4 + j], maxc) << (8 * j);
+    for (int j = 0; j < 4; ++j)
+      hi |= (uint32_t)asym_code_r(x[4 + j], s[4 + j], rs[4 + j], z[4 + j], maxc) << (8 * j);
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) lo |= (uint32_t)asym_code(x[j], s[j], z[j], maxc) << (bits * j);
+    for (int j = 0; j < 8; ++j) lo |= (uint32_t)asym_code_r(x[j], s[j], rs[j], z[j], maxc) << (bits * j);
   }
   return make_uint2(lo, hi);
 }
@@ -87,7 +89,7 @@ __device__ __forceinline__ uint2 pack8(const float* x, const float* s, const flo
 // rs, rs + 64, ... with rs = 8 w + lane / 4.
 __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, int bz) {
   __shared__ float pmin[8][kCB], pmax[8][kCB];
-  __shared__ float sf[kCB], zf[kCB];
+  __shared__ float sf[kCB], zf[kCB], rf[kCB];
   __shared__ int flags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_KEYS];
@@ -161,13 +163,15 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
     reinterpret_cast<__half*>(S.zero)[mi] = z;
     sf[c] = __half2float(s);
     zf[c] = __half2float(z);
+    rf[c] = __frcp_rn(sf[c]);
   }
   __syncthreads();
-  float s8[8], z8[8];
+  float s8[8], z8[8], r8[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     s8[c] = sf[8 * v + c];
     z8[c] = zf[8 * v + c];
+    r8[c] = rf[8 * v + c];
   }
   uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
   const int rowb = D * bits / 8;   // bytes per code row
@@ -176,7 +180,7 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
     const int r = rs + 64 * k;
     const bool ok = r < ln;
     uint2 w = make_uint2(0u, 0u);
-    if (ok) w = pack8(x[k], s8, z8, bits);
+    if (ok) w = pack8(x[k], s8, r8, z8, bits);
     uint8_t* row = codes + (ts + r) * rowb;
     if (bits == 8) {
       if (ok) *reinterpret_cast<uint2*>(row + cb + 8 * v) = w;
@@ -250,15 +254,16 @@ __device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by
       reinterpret_cast<__half*>(S.scale)[slab * L.C + tb + t] = s;
       reinterpret_cast<__half*>(S.zero)[slab * L.C + tb + t] = z;
     }
-    float s8[8], z8[8];
-    const float sv = __half2float(s), zv = __half2float(z);
+    float s8[8], z8[8], r8[8];
+    const float sv = __half2float(s), zv = __half2float(z), rv = __frcp_rn(sv);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       s8[j] = sv;
       z8[j] = zv;
+      r8[j] = rv;
     }
     uint2 w = make_uint2(0u, 0u);
-    if (ok) w = pack8(x[p], s8, z8, bits);
+    if (ok) w = pack8(x[p], s8, r8, z8, bits);
     if (bits == 8) {
       if (ok) *reinterpret_cast<uint2*>(codes + (tb + t) * D + 8 * vl) = w;
       continue;
@@ -414,11 +419,12 @@ __device__ __forceinline__ void asym_keys_rot_block(const AArgs& a, int bx, int 
     zf[c] = __half2float(zh);
   }
   __syncthreads();
-  float s4[4], z4[4];
+  float s4[4], z4[4], r4[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     s4[j] = sf[4 * lane + j];
     z4[j] = zf[4 * lane + j];
+    r4[j] = __frcp_rn(s4[j]);
   }
   const int maxc = (1 << bits) - 1;
   uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
@@ -429,7 +435,7 @@ __device__ __forceinline__ void asym_keys_rot_block(const AArgs& a, int bx, int 
     if (r < ln) {   // warp-uniform
       uint32_t v = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v |= (uint32_t)asym_code(x[k][j], s4[j], z4[j], maxc) << (bits * j);
+      for (int j = 0; j < 4; ++j) v |= (uint32_t)asym_code_r(x[k][j], s4[j], r4[j], z4[j], maxc) << (bits * j);
       uint8_t* row = codes + (ts + r) * rowb;
       if (bits == 8) {
         *reinterpret_cast<uint32_t*>(row + 4 * lane) = v;

@@ -90,6 +90,8 @@ def lib():
             "kvq_decode_workspace_bytes": (SZ, [FP, I32, I32, I32, I64, I32, I32]),
             "kvq_decode_attention": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, I32,
                                            P, SZ, I32, P, P]),
+            "kvq_append_decode_attention": (I32, [FP, CP, P, P, I64, I64, I64, I64, I64, P, I32, I32, I64, I32,
+                                                  ctypes.c_float, P, I32, P, SZ, I32, P, P]),
             "kvq_decode_partial_slots": (I32, [FP, I32, I32, I32, I64, I32, I32]),
             "kvq_decode_partial": (I32, [FP, CP, P, I32, I32, I64, I32, ctypes.c_float, P, SZ, I32,
                                          P, P]),
@@ -252,6 +254,27 @@ def decode_attention(fmt, cache: Cache, q: torch.Tensor, t_quant: int, t_res: in
                                     _ptr(workspace), workspace.numel(), num_splits, _ptr(status),
                                     _stream(stream))
     _check("kvq_decode_attention", st)
+    return out
+
+
+def append_decode_attention(fmt, cache: Cache, k_src: torch.Tensor, v_src: torch.Tensor, t0: int, n: int,
+                            q: torch.Tensor, t_quant: int, t_res: int, scale: float, out_dtype=F32, out=None,
+                            workspace=None, num_splits=0, status=None, stream=None):
+    """kvq_append_decode_attention: quantize_kv(k_src, v_src, t0, n) then decode_attention(q)."""
+    if k_src.stride() != v_src.stride():
+        raise ValueError("k_src and v_src must have the same strides")
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=TORCH_DTYPE[out_dtype], device=q.device)
+    need = decode_workspace_bytes(fmt, B, Hq, cache.H, t_quant, t_res, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().kvq_append_decode_attention(ctypes.byref(fmt), cache.ref(), _ptr(k_src), _ptr(v_src),
+                                           k_src.stride(0), k_src.stride(1), k_src.stride(2), t0, n,
+                                           _ptr(q), KVQ_DTYPE[q.dtype], Hq, t_quant, t_res, scale, _ptr(out),
+                                           out_dtype, _ptr(workspace), workspace.numel(), num_splits,
+                                           _ptr(status), _stream(stream))
+    _check("kvq_append_decode_attention", st)
     return out
 
 

@@ -57,6 +57,12 @@ CONFIGS = {
     "llama3_8b_wht": dict(name="llama3_8b_wht", recipe="llama3_8b", B=8, Hq=32, Hkv=8, D=128,
                           T=32768, seed=7, q_dtype=BF16,
                           fmt=_fmt(src_dtype=BF16, n_sink=1, residual_cap=128, k_rotate=1)),
+    # the Llama-3-8B workload under KQV at a 4-bit budget (same data recipe): K 4-bit scalar
+    # codes, V 3-bit codes plus the one-bit sketch, both after the Walsh-Hadamard rotation
+    "llama3_8b_kqv": dict(name="llama3_8b_kqv", recipe="llama3_8b", B=8, Hq=32, Hkv=8, D=128,
+                          T=32768, seed=7, q_dtype=BF16,
+                          fmt=_fmt(src_dtype=BF16, n_sink=1, residual_cap=128, k_scheme=KQV, k_bits=4,
+                                   k_axis=TOKEN, v_scheme=KQV, v_bits=4, v_axis=TOKEN)),
     "kvquant_nuq3": dict(name="kvquant_nuq3", B=1, Hq=32, Hkv=32, D=128, T=131072, seed=7,
                          q_dtype=F16,
                          fmt=_fmt(src_dtype=F16, k_scheme=NUQ, k_bits=3, k_outliers=2,

@@ -44,7 +44,8 @@ def test_headline_figures():
 
 
 def test_decode_path_matches_the_planner_rules():
-    assert bench.decode_path(synth.CONFIGS["llama3_8b"]) == "decode_mma_kernel"
+    assert bench.decode_path(synth.CONFIGS["llama3_8b"]) == "decode_k4v2_kernel"
+    assert bench.decode_path(synth.CONFIGS["llama3_8b_kqv"]) == "decode_kqv_kernel"
     assert bench.decode_path(synth.CONFIGS["mixkvq_14b"]) == "decode_mma_kernel"
     assert bench.decode_path(synth.CONFIGS["kvquant_nuq3"]) == "decode_cc_kernel"
     assert bench.fused_kv(synth.CONFIGS["llama3_8b_wht"])

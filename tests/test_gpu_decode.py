@@ -10,6 +10,7 @@ import torch
 
 import synth
 from oracle import attention as oatt
+from oracle import cache as ocache
 from oracle import salience
 from oracle.formats import BF16, F16, F32, KEYS, MIXED, NUQ, VALUES
 from quantized_decode_attention_quantize_b200 import kvq
@@ -254,6 +255,51 @@ def test_decode_attention_matches_partial_then_combine(B, H, G, tq, ns, tr, spli
     kvq.decode_combine(p.fmt, B, G * H, H, tq, tr, ws, two, num_splits=splits)
     torch.cuda.synchronize()
     assert torch.equal(one, two)
+    ref = oatt.decode_attention(p.of, p.ora, q.float().cpu().numpy().astype(np.float64), tq, tr)
+    assert_attn(one.cpu().numpy(), ref, 1e-3)
+    assert p.status_bits() == 0
+
+
+def clone_cache(p, luts=(None, None)):
+    c = kvq.Cache(p.fmt, p.B, p.H, p.C, k_lut=luts[0], v_lut=luts[1])
+    for name, t in p.gpu.tensors.items():
+        c.tensors[name].copy_(t)
+    return c
+
+
+@pytest.mark.parametrize("kw,G,t0,n", [
+    (dict(), 4, 7 * 128, 128),                      # tensor-core split kernel, deferred wait
+    (dict(), 4, 7 * 128, 37),                       # a partial group
+    (dict(), 2, 3 * 128, 256),                      # two groups inside the cache
+    (dict(k_rotate=1), 4, 7 * 128, 128),            # rotated keys: a plain append launch
+    (dict(), 8, 7 * 128, 128),                      # G = 8: the general tensor-core kernel
+    (dict(), 4, 7 * 128, 0),                        # nothing appended
+    (dict(k_scheme=NUQ, k_bits=3, v_scheme=NUQ, v_bits=3, v_axis=1, k_outliers=2, v_outliers=2), 4, 7 * 128, 128),
+])
+def test_append_decode_matches_separate_calls(kw, G, t0, n):
+    # kvq_append_decode_attention == kvq_quantize_kv then kvq_decode_attention, bit for bit,
+    # cache bytes included; and the result is the oracle's attention over the updated cache
+    fd = fmt(src_dtype=BF16, n_sink=1, residual_cap=128, **kw)
+    luts = (LUT["k"], LUT["v"]) if fd["k_scheme"] == NUQ else (None, None)
+    B, H, tq, tr = 2, 3, 8 * 128 - 5, 20
+    p = build(fd, B, H, G * H, tq, tr, seed=300 + G + n, luts=luts)
+    other = clone_cache(p, luts)
+    Kn = vals(301, (B, H, max(n, 1), 128), BF16, heavy=True)[:, :, :n]
+    Vn = vals(302, (B, H, max(n, 1), 128), BF16)[:, :, :n]
+    q = dev(vals(303, (B, G * H, 128), BF16), BF16)
+    scale = 1.0 / np.sqrt(128.0)
+    kd, vd = dev(Kn, BF16), dev(Vn, BF16)
+    one = kvq.append_decode_attention(p.fmt, p.gpu, kd, vd, t0, n, q, tq, tr, scale, F32, status=p.status)
+    if n:
+        kvq.quantize_kv(p.fmt, other, kd, vd, t0, n, status=p.status)
+    two = kvq.decode_attention(p.fmt, other, q, tq, tr, scale, F32, status=p.status)
+    torch.cuda.synchronize()
+    assert torch.equal(one, two)
+    for name, t in p.gpu.tensors.items():
+        assert torch.equal(t, other.tensors[name]), name
+    if n:
+        ocache.quantize(p.of, p.ora, KEYS, Kn.astype(np.float64), t0, n)
+        ocache.quantize(p.of, p.ora, VALUES, Vn.astype(np.float64), t0, n)
     ref = oatt.decode_attention(p.of, p.ora, q.float().cpu().numpy().astype(np.float64), tq, tr)
     assert_attn(one.cpu().numpy(), ref, 1e-3)
     assert p.status_bits() == 0
