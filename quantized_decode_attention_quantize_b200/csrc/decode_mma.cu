@@ -1451,6 +1451,11 @@ __device__ __forceinline__ void load16(const uint8_t* row, int c0, int dtype, fl
   }
 }
 
+// Shared-memory rows of 128 channels (queries, key scale / zero-point) keep channel quad
+// c / 4 = 4 b + u (16-channel block b, quad u inside it) at float4 slot 8 u + b: the eight
+// lanes of a load phase that read quad u of blocks 0..7 then read one contiguous 128 bytes.
+__device__ __forceinline__ int qslot(int quad) { return 8 * (quad & 3) + (quad >> 2); }
+
 // Raw tokens (sink + residual, nt <= 8) staged at stg (key rows, value rows at
 // +kRawBytes): fp32 scores on CUDA cores, lane (g, j) over channels 16 g .. 16 g + 15 of
 // head j, summed over the lanes g; the probabilities go into the state's tiles scaled
@@ -1461,10 +1466,10 @@ __device__ void lean_raw(LeanState& st, const uint8_t* stg, int nt, int dtype, c
   const int rowb = dtype == KVQ_F32 ? 512 : 256;
   float q[16];
   {
-    const float4* p = reinterpret_cast<const float4*>(qs + j * 128 + 16 * g);
+    const float4* p = reinterpret_cast<const float4*>(qs + j * 128);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float4 x = p[u];
+      const float4 x = p[8 * u + g];
       q[4 * u] = x.x; q[4 * u + 1] = x.y; q[4 * u + 2] = x.z; q[4 * u + 3] = x.w;
     }
   }
@@ -1515,7 +1520,8 @@ struct LeanKey {
   float mult, bias;
 };
 
-// ks, kz: the group's key scale / zero-point as fp32 [128] in shared memory.
+// ks, kz: the group's key scale / zero-point as fp32 [128] in shared memory, qs the queries
+// [4][128]; channel quads at qslot().
 __device__ __forceinline__ void lean_key_operand(const float* ks, const float* kz, const float* qs,
                                                  uint32_t* scr, LeanKey& ko) {
   const int lane = threadIdx.x & 31;
@@ -1523,12 +1529,12 @@ __device__ __forceinline__ void lean_key_operand(const float* ks, const float* k
   float a[16];
   float amax = 0.0f, dz = 0.0f;
   {
-    const float4* q4 = reinterpret_cast<const float4*>(qs + hL * 128 + 16 * cb);
-    const float4* s4 = reinterpret_cast<const float4*>(ks + 16 * cb);
-    const float4* z4 = reinterpret_cast<const float4*>(kz + 16 * cb);
+    const float4* q4 = reinterpret_cast<const float4*>(qs + hL * 128);
+    const float4* s4 = reinterpret_cast<const float4*>(ks);
+    const float4* z4 = reinterpret_cast<const float4*>(kz);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float4 qv = q4[u], sv = s4[u], zv = z4[u];
+      const float4 qv = q4[8 * u + cb], sv = s4[8 * u + cb], zv = z4[8 * u + cb];
       a[4 * u] = qv.x * sv.x;
       a[4 * u + 1] = qv.y * sv.y;
       a[4 * u + 2] = qv.z * sv.z;
@@ -1562,14 +1568,16 @@ __device__ __forceinline__ void lean_key_operand(const float* ks, const float* k
       const float y0 = a[8 * u + p] * f, y1 = a[8 * u + p + 4] * f;
       split_half2(y0, y1, &hw[p], &lw[p]);
     }
+    // register quad w of reader lane R sits at uint4 slot 32 w + R (a read phase of eight
+    // lanes is then one contiguous 128 bytes)
     const int W = 2 * cb + u, jd = W >> 2, w = W & 3;
-    *reinterpret_cast<uint4*>(scr + (4 * (2 * hL) + jd) * 16 + 4 * w) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4*>(scr + (4 * (2 * hL + 1) + jd) * 16 + 4 * w) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    *reinterpret_cast<uint4*>(scr + (32 * w + 4 * (2 * hL) + jd) * 4) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(scr + (32 * w + 4 * (2 * hL + 1) + jd) * 4) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
   __syncwarp();
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const uint4 x = *reinterpret_cast<const uint4*>(scr + lane * 16 + 4 * u);
+    const uint4 x = *reinterpret_cast<const uint4*>(scr + (32 * u + lane) * 4);
     ko.b[4 * u] = x.x; ko.b[4 * u + 1] = x.y; ko.b[4 * u + 2] = x.z; ko.b[4 * u + 3] = x.w;
   }
   ko.mult = __shfl_sync(0xffffffffu, mult, 8 * (lane & 3));
@@ -1703,7 +1711,7 @@ __device__ __forceinline__ void lean_load_queries(const MmaArgs& a, int64_t qhea
     if constexpr (ROT) {
       if (rotated) x = rotate_q(x, lane, a.rot_scale);
     }
-    reinterpret_cast<float4*>(qs + hh * 128)[lane] =
+    reinterpret_cast<float4*>(qs + hh * 128)[qslot(lane)] =
         make_float4(x.x * a.qscale, x.y * a.qscale, x.z * a.qscale, x.w * a.qscale);
   }
   __syncwarp();
@@ -1712,7 +1720,7 @@ __device__ __forceinline__ void lean_load_queries(const MmaArgs& a, int64_t qhea
 // The warp's shared-memory areas and ring counters.
 struct LeanWarp {
   uint8_t* ring;      // kBuffers stages
-  float* qs;          // [4][128] queries
+  float* qs;          // [4][128] queries, channel quads at qslot()
   uint32_t* scr;      // key-operand fragments / value scale and zero-point pairs
   float* kmeta;       // the group's key scale / zero-point as fp32, [2][128]
   uint64_t* bars;     // one mbarrier per stage
@@ -1782,8 +1790,11 @@ __device__ __forceinline__ bool lean_run(const MmaArgs& a, LeanState& st, LeanWa
     if (!mbar_wait(&w.bars[sb2], (uint32_t)(w.ncons >> 1) & 1u)) return false;
     const uint8_t* stg = w.ring + sb2 * kStageBytes;
     if ((p & 1) == 0 || p == ha) {   // the group's key operand
-      const uint2 sv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM)[lane];
-      const uint2 zv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM + 256)[lane];
+      // lane L takes the channel quad stored at slot L (qslot of quad 4 (L & 7) + L / 8): the
+      // stores below are then one contiguous 512 bytes
+      const int quad = 4 * (lane & 7) + (lane >> 3);
+      const uint2 sv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM)[quad];
+      const uint2 zv = reinterpret_cast<const uint2*>(stg + kHalfK + kHalfV + kHalfVM + 256)[quad];
       const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
       const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
       const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zv.x));
