@@ -64,7 +64,11 @@ constexpr int kThreads = kCW * 32;
 constexpr int kHalfK = 64 * 64, kHalfV = 32 * 64, kHalfVM = 2 * 64 * 2, kHalfKM = 2 * 128 * 2;
 constexpr int kStageBytes = kHalfK + kHalfV + kHalfVM + kHalfKM;
 constexpr int kRawBytes = 2048;               // raw item: key rows, then value rows at +kRawBytes
-constexpr int kScratchBytes = 2 * 32 * 16 * 4;  // per warp: hi and lo B fragments
+// per warp: hi and lo B fragments (4 KiB); with MixKVQ keys the slot products [GM][kAv]
+// (rows padded to kAv floats so that the lanes of a fragment read spread over the banks) and,
+// for G <= 4, the queries [4][128] in the last 2 KiB
+constexpr int kScratchBytes = 2 * 32 * 16 * 4 + 512;
+constexpr int kAv = 132;
 constexpr int kRecordFloats = 8 * 130;        // merge record: o[G][128], m[G], l[G]
 constexpr float kLog2e = 1.4426950408889634f;
 // MIXED keys (8 raw bf16 / 24 4-bit / 96 2-bit slots per token) in the key region of a
@@ -407,6 +411,14 @@ struct QVec<false, GM> {
 // (l, l ^ 1) fill the two halves of the same four words; one shuffle gives each of them
 // two whole words (even lane: k-step kk0 = 2 ((l & 7) >> 1), odd lane: kk0 + 1), stored
 // as one 64-bit word pair.
+// Scratch word of k-step kk of consumer lane R's fragments: R's four 16-byte quads sit at
+// slots 4 R + (q ^ frag_swz(R)) (q = kk / 2), so that both the pair stores of the
+// producers and the quad loads of the consumers fall on distinct banks.
+__device__ __forceinline__ int frag_swz(int R) { return (R >> 1) & 3; }
+__device__ __forceinline__ int frag_word(int R, int kk) {
+  return 4 * (4 * R + ((kk >> 1) ^ frag_swz(R))) + 2 * (kk & 1);
+}
+
 template <bool DUAL, int GM>
 __device__ __forceinline__ void key_operand(const MmaArgs& a, const __half* ks, const __half* kz,
                                             uint32_t* scratch, const QVec<DUAL, GM>& qv, KeyOp& ko) {
@@ -462,9 +474,9 @@ __device__ __forceinline__ void key_operand(const MmaArgs& a, const __half* ks, 
       const uint2 wl = odd ? make_uint2(__byte_perm(rl, ml, 0x5410), __byte_perm(rl, ml, 0x7632))
                            : make_uint2(__byte_perm(ml, rl, 0x5410), __byte_perm(ml, rl, 0x7632));
       const int dl = 4 * hh + (lane >> 3);   // consumer lane
-      *reinterpret_cast<uint2*>(scratch + dl * 16 + 2 * kk0) = wh;
-      if (DUAL) *reinterpret_cast<uint2*>(scratch + (dl + 16) * 16 + 2 * kk0) = wl;   // column hh + 4
-      else *reinterpret_cast<uint2*>(scratch + 32 * 16 + dl * 16 + 2 * kk0) = wl;
+      *reinterpret_cast<uint2*>(scratch + frag_word(dl, kk0)) = wh;
+      if (DUAL) *reinterpret_cast<uint2*>(scratch + frag_word(dl + 16, kk0)) = wl;   // column hh + 4
+      else *reinterpret_cast<uint2*>(scratch + 32 * 16 + frag_word(dl, kk0)) = wl;
     }
   }
   // butterfly reduction of the per-head sums q~ . z over the warp
@@ -511,14 +523,14 @@ __device__ __forceinline__ void key_operand(const MmaArgs& a, const __half* ks, 
     const uint4* src = reinterpret_cast<const uint4*>(scratch) + lane * 4;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint4 x = src[u];
+      const uint4 x = src[u ^ frag_swz(lane)];
       ko.bh[2 * u][0] = x.x; ko.bh[2 * u][1] = x.y; ko.bh[2 * u + 1][0] = x.z; ko.bh[2 * u + 1][1] = x.w;
     }
     if (!DUAL) {
       const uint4* srl = reinterpret_cast<const uint4*>(scratch) + 32 * 4 + lane * 4;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint4 x = srl[u];
+        const uint4 x = srl[u ^ frag_swz(lane)];
         ko.bl[2 * u][0] = x.x; ko.bl[2 * u][1] = x.y; ko.bl[2 * u + 1][0] = x.z; ko.bl[2 * u + 1][1] = x.w;
       }
     }
@@ -611,7 +623,7 @@ __device__ __forceinline__ void key_operand_mixed(const MmaArgs& a, const uint8_
   const uint8_t* ord = stage + kMixOrd;
   const __half* ks = reinterpret_cast<const __half*>(stage + kHalfK + kHalfV + kHalfVM);
   const __half* kz = ks + 128;
-  float* av = reinterpret_cast<float*>(scratch);   // [GM][128] slot products, slot order
+  float* av = reinterpret_cast<float*>(scratch);   // [GM][kAv] slot products, slot order
   int ch[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) ch[i] = ord[4 * lane + i] & 127;   // a channel of the head
@@ -623,12 +635,12 @@ __device__ __forceinline__ void key_operand_mixed(const MmaArgs& a, const uint8_
       for (int i = 0; i < 4; ++i) qs[hh][i] = qv.s[hh * 128 + ch[i]];
   } else {   // the queries live in registers by channel: go through the scratch once
 #pragma unroll
-    for (int hh = 0; hh < GM; ++hh) *reinterpret_cast<float4*>(av + hh * 128 + 4 * lane) = qv.get(hh);
+    for (int hh = 0; hh < GM; ++hh) *reinterpret_cast<float4*>(av + hh * kAv + 4 * lane) = qv.get(hh);
     __syncwarp();
 #pragma unroll
     for (int hh = 0; hh < GM; ++hh)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) qs[hh][i] = av[hh * 128 + ch[i]];
+      for (int i = 0; i < 4; ++i) qs[hh][i] = av[hh * kAv + ch[i]];
     __syncwarp();
   }
   float sv[4], zv[4];
@@ -662,14 +674,14 @@ __device__ __forceinline__ void key_operand_mixed(const MmaArgs& a, const uint8_
                              : __uint_as_float((uint32_t)max(1, min(254, 127 - ex)) << 23);
 #pragma unroll
   for (int hh = 0; hh < GM; ++hh)
-    *reinterpret_cast<float4*>(av + hh * 128 + 4 * lane) =
+    *reinterpret_cast<float4*>(av + hh * kAv + 4 * lane) =
         make_float4(qs[hh][0] * sc, qs[hh][1] * sc, qs[hh][2] * sc, qs[hh][3] * sc);
   head_sums<DUAL, GM>(dz, &ko.bias0, &ko.bias1);
   __syncwarp();
   const int hd = DUAL ? (g & 3) : g;
   const bool live = hd < G;
   const bool low_lane = DUAL && g >= 4;   // columns 4..7 carry the low parts
-  const float* ah = av + (live ? hd : 0) * 128;
+  const float* ah = av + (live ? hd : 0) * kAv;
   auto put = [&](int k, float v0, float v1, float v2, float v3) {
     uint32_t h0, l0, h1, l1;
     split_half2(v0, v1, &h0, &l0);
@@ -1107,7 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(MmaArgs a) {
   MmaState st;
   state_reset(st);
   QVec<DUAL, GM> qv;
-  if constexpr (DUAL) qv.s = reinterpret_cast<float*>(my_scratch) + 512;   // upper 2 KiB
+  if constexpr (DUAL) qv.s = reinterpret_cast<float*>(my_scratch) + (kScratchBytes / 4 - 512);   // last 2 KiB
   KeyOpT<MIX> ko;
   int64_t head = i0 / U, cur_head = -1;
   int r = (int)(i0 - head * U);
@@ -1568,16 +1580,18 @@ __device__ __forceinline__ void lean_key_operand(const float* ks, const float* k
       const float y0 = a[8 * u + p] * f, y1 = a[8 * u + p + 4] * f;
       split_half2(y0, y1, &hw[p], &lw[p]);
     }
-    // register quad w of reader lane R sits at uint4 slot 32 w + R (a read phase of eight
-    // lanes is then one contiguous 128 bytes)
-    const int W = 2 * cb + u, jd = W >> 2, w = W & 3;
-    *reinterpret_cast<uint4*>(scr + (32 * w + 4 * (2 * hL) + jd) * 4) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4*>(scr + (32 * w + 4 * (2 * hL + 1) + jd) * 4) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    // register quad w of reader lane R sits at uint4 slot 32 w + (R ^ 4 (w / 2)): a read
+    // phase of eight lanes is one contiguous 128 bytes, and the two stores of a lane pair
+    // (w, w + 2) land in different bank groups
+    const int W = 2 * cb + u, jd = W >> 2, w = W & 3, sw = 4 * (w >> 1);
+    *reinterpret_cast<uint4*>(scr + (32 * w + ((4 * (2 * hL) + jd) ^ sw)) * 4) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(scr + (32 * w + ((4 * (2 * hL + 1) + jd) ^ sw)) * 4) =
+        make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
   __syncwarp();
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const uint4 x = *reinterpret_cast<const uint4*>(scr + (32 * u + lane) * 4);
+    const uint4 x = *reinterpret_cast<const uint4*>(scr + (32 * u + (lane ^ (4 * (u >> 1)))) * 4);
     ko.b[4 * u] = x.x; ko.b[4 * u + 1] = x.y; ko.b[4 * u + 2] = x.z; ko.b[4 * u + 3] = x.w;
   }
   ko.mult = __shfl_sync(0xffffffffu, mult, 8 * (lane & 3));
