@@ -636,7 +636,7 @@ def main():
         pass
     peak = peaks.get("hbm_gbs", 6650.0)
     traffic = None
-    prof = os.path.join(ROOT, "profiles", "decode_mma_llama3_8b.json")
+    prof = os.path.join(ROOT, "profiles", "decode_k4v2_llama3_8b.json")
     if os.path.exists(prof):
         try:
             pj = json.load(open(prof))
