@@ -12,8 +12,7 @@ namespace kvq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kCB = 32;     // channels per key block
-constexpr int kTB = 32;     // tokens per value block
+constexpr int kCB = 32;     // channels per key block (64 when g <= 128 and D % 64 == 0)
 constexpr int kMaxKeyRows = 4;   // rows per thread: g <= 256 over 64 row slices
 
 struct AArgs {
@@ -67,29 +66,53 @@ __device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, fl
   }
 }
 
-// 8 codes of `bits` bits packed LSB-first (bits = 2: 16 bits, 4: 32 bits; 8: two words)
+// 8 codes of `bits` bits packed LSB-first (bits = 2: 16 bits, 4: 32 bits; 8: two words).
+// Each code is rint_even(fl32(fl32(x - z) / s)) clipped to [0, 2^bits - 1], found as
+// asym_code_r does: from q = fl32(fl32(x - z) * rs), rs = fl32(1 / s), which is within
+// 2^-13 of the exact quotient for in-range codes, so that q and the IEEE quotient round to
+// the same integer unless q lies within 2^-12 of a half-integer.  Such elements (rare) take
+// the quotient instead, behind one branch per eight codes.
 __device__ __forceinline__ uint2 pack8(const float* x, const float* s, const float* rs, const float* z,
                                        int bits) {
-  const int maxc = (1 << bits) - 1;
+  const float maxc = (float)((1 << bits) - 1);
+  float q[8];
+  bool near = false;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    q[j] = __fmul_rn(__fsub_rn(x[j], z[j]), rs[j]);
+    near |= fabsf(q[j] - rintf(q[j])) > 0.5f - 0x1p-12f;
+  }
+  if (near) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (fabsf(q[j] - rintf(q[j])) > 0.5f - 0x1p-12f) q[j] = __fdiv_rn(__fsub_rn(x[j], z[j]), s[j]);
+  }
+  uint32_t c[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) c[j] = (uint32_t)fminf(fmaxf(rintf(q[j]), 0.0f), maxc);
   uint32_t lo = 0, hi = 0;
   if (bits == 8) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) lo |= (uint32_t)asym_code_r(x[j], s[j], rs[j], z[j], maxc) << (8 * j);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      hi |= (uint32_t)asym_code_r(x[4 + j], s[4 + j], rs[4 + j], z[4 + j], maxc) << (8 * j);
+    for (int j = 0; j < 4; ++j) {
+      lo |= c[j] << (8 * j);
+      hi |= c[4 + j] << (8 * j);
+    }
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) lo |= (uint32_t)asym_code_r(x[j], s[j], rs[j], z[j], maxc) << (bits * j);
+    for (int j = 0; j < 8; ++j) lo |= c[j] << (bits * j);
   }
   return make_uint2(lo, hi);
 }
 
-// Keys.  Thread (warp w, lane): vector v = lane & 3 (channels cb + 8 v .. + 7) of rows
-// rs, rs + 64, ... with rs = 8 w + lane / 4.
+// Keys over a block of CB channels (32 or 64).  Thread t of the CTA: vector v = t mod VPC
+// (channels cb + 8 v .. + 7, VPC = CB / 8) of rows rs, rs + NS, ... with rs = t / VPC over
+// NS = 256 / VPC row slices (CB = 64: g <= 4 NS = 128; CB = 32: g <= 256).  The min / max
+// of a channel meet first over the lanes of a warp with equal v, then over the 8 warps.
+template <int CB>
 __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, int bz) {
-  __shared__ float pmin[8][kCB], pmax[8][kCB];
-  __shared__ float sf[kCB], zf[kCB], rf[kCB];
+  constexpr int VPC = CB / 8, NS = kThreads / VPC;
+  __shared__ float pmin[8][CB], pmax[8][CB];
+  __shared__ float sf[CB], zf[CB], rf[CB];
   __shared__ int flags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_KEYS];
@@ -97,19 +120,21 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
   const int64_t ts = a.t0 + (int64_t)bx * g;
   const int ln = (int)min((int64_t)g, a.t0 + a.n - ts);
   const int gi = (int)(ts / g);
-  const int cb = by * kCB;
+  const int cb = by * CB;
   const int head = bz;
   const int b = head / L.Hkv, h = head % L.Hkv;
   int64_t slab;
   if (!dest_slab(a, head, b, h, &slab)) return;   // uniform over the CTA
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int v = lane & 3, rs = warp * 8 + (lane >> 2);
+  const int v = threadIdx.x % VPC, rs = threadIdx.x / VPC;
   if (threadIdx.x == 0) flags = 0;
   float x[kMaxKeyRows][8];
   const int64_t base = (int64_t)b * a.sb + (int64_t)h * a.sh + (ts - a.t0) * a.st + cb + 8 * v;
 #pragma unroll
   for (int k = 0; k < kMaxKeyRows; ++k) {
-    const int r = rs + 64 * k;
+    const int r = rs + NS * k;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[k][c] = 0.0f;
     if (r < ln) load8(a.src, base + r * a.st, L.src_dtype, x[k]);
   }
   int bad = 0;
@@ -119,27 +144,29 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
     mn[c] = INFINITY;
     mx[c] = -INFINITY;
   }
+  float fin = 0.0f;   // x * 0 is 0 for finite x and NaN otherwise
 #pragma unroll
   for (int k = 0; k < kMaxKeyRows; ++k) {
-    if (rs + 64 * k < ln) {
+    if (rs + NS * k < ln) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        bad |= !isfinite(x[k][c]);
+        fin = fmaf(x[k][c], 0.0f, fin);
         mn[c] = fminf(mn[c], x[k][c]);
         mx[c] = fmaxf(mx[c], x[k][c]);
       }
     }
   }
-  // over the 8 row slices of the warp (lanes with equal v)
+  bad = !(fin == 0.0f);
+  // over the row slices of the warp (lanes with equal v)
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1)
+  for (int o = VPC; o < 32; o <<= 1)
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       mn[c] = fminf(mn[c], __shfl_xor_sync(0xffffffffu, mn[c], o));
       mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], o));
     }
   __syncthreads();   // flags initialised
-  if (lane < 4) {
+  if (lane < VPC) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       pmin[warp][8 * v + c] = mn[c];
@@ -148,7 +175,7 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&flags, 1);
   __syncthreads();
-  if (threadIdx.x < kCB) {
+  if (threadIdx.x < CB) {
     const int c = threadIdx.x;
     float m0 = pmin[0][c], m1 = pmax[0][c];
 #pragma unroll
@@ -177,10 +204,10 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
   const int rowb = D * bits / 8;   // bytes per code row
 #pragma unroll
   for (int k = 0; k < kMaxKeyRows; ++k) {
-    const int r = rs + 64 * k;
+    const int r = rs + NS * k;
+    if (NS * k >= g) break;   // uniform: no slice has a row k
     const bool ok = r < ln;
-    uint2 w = make_uint2(0u, 0u);
-    if (ok) w = pack8(x[k], s8, r8, z8, bits);
+    const uint2 w = pack8(x[k], s8, r8, z8, bits);
     uint8_t* row = codes + (ts + r) * rowb;
     if (bits == 8) {
       if (ok) *reinterpret_cast<uint2*>(row + cb + 8 * v) = w;
@@ -196,127 +223,103 @@ __device__ __forceinline__ void asym_keys_block(const AArgs& a, int bx, int by, 
     flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
 }
 
-// Values.  A warp takes 4 consecutive tokens of the block; lane (sub, vl) holds vector
-// vl (channels 8 vl .. 8 vl + 7) of one token, sub = lane / nvec, nvec = D / 8 lanes per
-// token, so a pass covers 32 / nvec tokens and a warp ceil(4 nvec / 32) passes.
+// Values.  LPT = D / 32 lanes per token, each holding 32 consecutive channels; a warp takes
+// 32 / LPT consecutive tokens and the CTA's 8 warps value_tokens(D) = 256 / LPT tokens.
+// A token's min / max meet over its LPT lanes; its scale / zero-point, computed by every
+// lane of the token alike, is stored by the first.  In the pair layout (b < 8) the partner
+// token of a pair sits in lane ^ LPT.
+__host__ __device__ __forceinline__ int value_tokens(int D) { return 256 * 32 / D; }
+
 __device__ __forceinline__ void asym_values_block(const AArgs& a, int bx, int by) {
-  constexpr int kPass = 4;   // at most 4 passes (D = 256)
   __shared__ int vflags;
   int& flags = vflags;
   const Layout& L = a.L;
   const Side& S = L.side[KVQ_VALUES];
   const int D = L.D, bits = S.bits;
-  const int64_t tb = a.t0 + (int64_t)bx * kTB;
-  const int nt = (int)min((int64_t)kTB, a.t0 + a.n - tb);
+  const int LPT = D / 32, TPC = value_tokens(D);
+  const int64_t tb = a.t0 + (int64_t)bx * TPC;
+  const int nt = (int)min((int64_t)TPC, a.t0 + a.n - tb);
   const int head = by;
   const int b = head / L.Hkv, h = head % L.Hkv;
   int64_t slab;
   if (!dest_slab(a, head, b, h, &slab)) return;   // uniform over the CTA
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nvec = D / 8, rpp = 32 / nvec, sub = lane / nvec, vl = lane % nvec;
-  const int passes = (4 + rpp - 1) / rpp;
+  const int lane = threadIdx.x & 31;
+  const int t = threadIdx.x / LPT;   // token within the block
+  const int part = threadIdx.x % LPT, c0 = 32 * part;
+  const bool ok = t < nt;
   if (threadIdx.x == 0) flags = 0;
-  float x[kPass][8];
-  const int64_t base = (int64_t)b * a.sb + (int64_t)h * a.sh + (tb - a.t0) * a.st + 8 * vl;
+  float x[4][8];
 #pragma unroll
-  for (int p = 0; p < kPass; ++p) {
-    const int t = warp * 4 + p * rpp + sub;   // token within the block
-    if (p < passes && p * rpp + sub < 4 && t < nt) load8(a.src, base + t * a.st, L.src_dtype, x[p]);
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[k][c] = 0.0f;
+    if (ok) load8(a.src, (int64_t)b * a.sb + (int64_t)h * a.sh + (tb - a.t0 + t) * a.st + c0 + 8 * k,
+                  L.src_dtype, x[k]);
+  }
+  float mn = INFINITY, mx = -INFINITY, fin = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      fin = fmaf(x[k][c], 0.0f, fin);
+      mn = fminf(mn, x[k][c]);
+      mx = fmaxf(mx, x[k][c]);
+    }
+  for (int o = 1; o < LPT; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
   __syncthreads();   // flags initialised
-  int bad = 0, rbad = 0;
-  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
-  uint32_t half_prev = 0;   // 2- and 4-bit, one token per pass: the even token's half words
-  uint32_t half_prev2 = 0;
+  __half sh, zh;
+  const bool good = asym_params(mn, mx, bits, &sh, &zh);
+  if (ok && part == 0) {
+    reinterpret_cast<__half*>(S.scale)[slab * L.C + tb + t] = sh;
+    reinterpret_cast<__half*>(S.zero)[slab * L.C + tb + t] = zh;
+  }
+  const float sv = __half2float(sh), zv = __half2float(zh), rv = __frcp_rn(sv);
+  float s8[8], z8[8], r8[8];
 #pragma unroll
-  for (int p = 0; p < kPass; ++p) {
-    if (p >= passes) break;
-    const int tl = p * rpp + sub;        // token within the warp's 4
-    const int t = warp * 4 + tl;
-    const bool ok = tl < 4 && t < nt;
-    float mn = INFINITY, mx = -INFINITY;
+  for (int j = 0; j < 8; ++j) {
+    s8[j] = sv;
+    z8[j] = zv;
+    r8[j] = rv;
+  }
+  uint2 w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w[k] = pack8(x[k], s8, r8, z8, bits);
+  uint8_t* codes = reinterpret_cast<uint8_t*>(S.codes) + slab * S.code_slab_bytes;
+  if (bits == 8) {
     if (ok) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        bad |= !isfinite(x[p][j]);
-        mn = fminf(mn, x[p][j]);
-        mx = fmaxf(mx, x[p][j]);
-      }
+      for (int k = 0; k < 4; ++k) *reinterpret_cast<uint2*>(codes + (tb + t) * D + c0 + 8 * k) = w[k];
     }
-    for (int o = 1; o < nvec; o <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    __half s, z;
-    const bool good = asym_params(mn, mx, bits, &s, &z);
-    if (ok && vl == 0) {
-      rbad |= !good;
-      reinterpret_cast<__half*>(S.scale)[slab * L.C + tb + t] = s;
-      reinterpret_cast<__half*>(S.zero)[slab * L.C + tb + t] = z;
-    }
-    float s8[8], z8[8], r8[8];
-    const float sv = __half2float(s), zv = __half2float(z), rv = __frcp_rn(sv);
+  } else {
+    // pair layout: word j of pair u holds 16 / bits channels of token 2u (low half) and of
+    // token 2u + 1 (high half); the lane's 32 channels are 2 bits half words
+    uint32_t hw[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      s8[j] = sv;
-      z8[j] = zv;
-      r8[j] = rv;
-    }
-    uint2 w = make_uint2(0u, 0u);
-    if (ok) w = pack8(x[p], s8, r8, z8, bits);
-    if (bits == 8) {
-      if (ok) *reinterpret_cast<uint2*>(codes + (tb + t) * D + 8 * vl) = w;
-      continue;
-    }
-    // pair layout: word j of pair u holds 16 / bits channels of token 2u (low 16 bits)
-    // and token 2u + 1 (high 16 bits); this lane's 8 channels are one half word (2-bit)
-    // or two (4-bit: channels 8 vl .. + 3 and + 4 .. + 7)
-    const uint32_t h0 = w.x & 0xffffu;
-    const uint32_t h1 = bits == 2 ? 0u : (w.x >> 16);
-    uint32_t o0, o1;
-    bool even;
-    if (rpp >= 2) {   // partner token in lane ^ nvec of the same pass
-      o0 = __shfl_xor_sync(0xffffffffu, h0, nvec);
-      o1 = __shfl_xor_sync(0xffffffffu, h1, nvec);
-      even = (sub & 1) == 0;
-    } else {          // one token per pass: partner in the neighbouring pass of this lane
-      o0 = half_prev;
-      o1 = half_prev2;
-      even = (p & 1) == 0;
-      half_prev = h0;
-      half_prev2 = h1;
-    }
-    const int64_t u = (tb + t) / 2;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(codes) + u * (D * bits / 16);
-    const bool last_odd = (t + 1 == nt) && even;   // a lone last token: high half zero
-    if (rpp >= 2) {
-      if (ok && even) {
-        const uint32_t hi0 = last_odd ? 0u : o0, hi1 = last_odd ? 0u : o1;
-        if (bits == 2) dst[vl] = h0 | (hi0 << 16);
-        else {
-          dst[2 * vl] = h0 | (hi0 << 16);
-          dst[2 * vl + 1] = h1 | (hi1 << 16);
-        }
+    for (int k = 0; k < 4; ++k) {
+      if (bits == 2) {
+        hw[k] = w[k].x & 0xffffu;
+      } else {
+        hw[2 * k] = w[k].x & 0xffffu;
+        hw[2 * k + 1] = w[k].x >> 16;
       }
-    } else {
-      // store at the odd pass (or at an even pass whose token is the block's last)
-      if (ok && !even) {
-        if (bits == 2) dst[vl] = o0 | (h0 << 16);
-        else {
-          dst[2 * vl] = o0 | (h0 << 16);
-          dst[2 * vl + 1] = o1 | (h1 << 16);
-        }
-      } else if (ok && last_odd) {
-        if (bits == 2) dst[vl] = h0;
-        else {
-          dst[2 * vl] = h0;
-          dst[2 * vl + 1] = h1;
-        }
+    }
+    const int nh = 2 * bits;   // half words of the lane
+    const bool even = (tb + t) % 2 == 0;
+    const bool lone = even && t + 1 >= nt;   // no partner: its half stays zero
+    uint32_t* dst = reinterpret_cast<uint32_t*>(codes) + ((tb + t) / 2) * (D * bits / 16) + part * nh;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k < nh) {
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, hw[k], LPT);
+        if (ok && even) dst[k] = hw[k] | ((lone ? 0u : other) << 16);
       }
     }
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&flags, 1);
-  if (__any_sync(0xffffffffu, rbad) && lane == 0) atomicOr(&flags, 2);
+  if (__any_sync(0xffffffffu, ok && (!(fin == 0.0f))) && lane == 0) atomicOr(&flags, 1);
+  if (__any_sync(0xffffffffu, ok && !good) && lane == 0) atomicOr(&flags, 2);
   __syncthreads();
   if (threadIdx.x == 0 && flags)
     flag(a.status, ((flags & 1) ? KVQ_DEV_NONFINITE : 0) | ((flags & 2) ? KVQ_DEV_RANGE : 0));
@@ -473,8 +476,9 @@ __global__ void __launch_bounds__(kThreads) asym_kv_rot_kernel(AArgs ak, AArgs a
   }
 }
 
+template <int CB>
 __global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
-  asym_keys_block(a, blockIdx.x, blockIdx.y, blockIdx.z);
+  asym_keys_block<CB>(a, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
@@ -483,18 +487,23 @@ __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
 
 // Keys and values of one append in one launch: blocks [0, nk) are key blocks
 // (group, channel block, head), the rest value blocks (token block, head).
+template <int CB>
 __global__ void __launch_bounds__(kThreads) asym_kv_kernel(AArgs ak, AArgs av, int kgx, int kgy, int nk,
                                                            int vgx) {
   griddep_wait();   // launched with launch_pdl: earlier work on the stream is complete
   griddep_launch_dependents();
   const int b = blockIdx.x;
   if (b < nk) {
-    asym_keys_block(ak, b % kgx, (b / kgx) % kgy, b / (kgx * kgy));
+    asym_keys_block<CB>(ak, b % kgx, (b / kgx) % kgy, b / (kgx * kgy));
   } else {
     const int v = b - nk;
     asym_values_block(av, v % vgx, v / vgx);
   }
 }
+
+// Channels per key block: 64 halves the blocks and the shuffle levels of the min / max
+// when its 32 row slices cover the group.
+int key_cb(const Layout& L) { return (L.g <= 128 && L.D % 64 == 0) ? 64 : kCB; }
 
 }  // namespace
 
@@ -526,10 +535,13 @@ cudaError_t launch_quantize_asym(const Layout& L, int which, const void* src, in
     dim3 grid((unsigned)((n + L.g - 1) / L.g), L.B * L.Hkv);
     asym_keys_rot_kernel<<<grid, kThreads, 0, s>>>(a);
   } else if (which == KVQ_KEYS) {
-    dim3 grid((unsigned)((n + L.g - 1) / L.g), L.D / kCB, L.B * L.Hkv);
-    asym_keys_kernel<<<grid, kThreads, 0, s>>>(a);
+    const int cb = key_cb(L);
+    dim3 grid((unsigned)((n + L.g - 1) / L.g), L.D / cb, L.B * L.Hkv);
+    if (cb == 64) asym_keys_kernel<64><<<grid, kThreads, 0, s>>>(a);
+    else asym_keys_kernel<kCB><<<grid, kThreads, 0, s>>>(a);
   } else {
-    dim3 grid((unsigned)((n + kTB - 1) / kTB), L.B * L.Hkv);
+    const int tpc = value_tokens(L.D);
+    dim3 grid((unsigned)((n + tpc - 1) / tpc), L.B * L.Hkv);
     asym_values_kernel<<<grid, kThreads, 0, s>>>(a);
   }
   return cudaGetLastError();
@@ -554,14 +566,16 @@ cudaError_t launch_quantize_asym_kv(const Layout& L, const void* ksrc, const voi
   ak.t0 = av.t0 = t0;
   ak.n = av.n = n;
   ak.status = av.status = d_status;
-  const int kgx = (int)((n + L.g - 1) / L.g), kgy = L.k_rotate ? 1 : L.D / kCB, heads = L.B * L.Hkv;
-  const int vgx = (int)((n + kTB - 1) / kTB);
+  const int cb = key_cb(L);
+  const int kgx = (int)((n + L.g - 1) / L.g), kgy = L.k_rotate ? 1 : L.D / cb, heads = L.B * L.Hkv;
+  const int vgx = (int)((n + value_tokens(L.D) - 1) / value_tokens(L.D));
   const int64_t nk = (int64_t)kgx * kgy * heads, nv = (int64_t)vgx * heads;
   if (nk + nv > 0x7fffffff) return cudaErrorInvalidConfiguration;
   if (L.k_rotate)
     asym_kv_rot_kernel<<<(unsigned)(nk + nv), kThreads, 0, s>>>(ak, av, kgx, (int)nk, vgx);
   else
-    return launch_pdl(asym_kv_kernel, dim3((unsigned)(nk + nv)), dim3(kThreads), 0, s, ak, av, kgx, kgy,
+    return launch_pdl(cb == 64 ? asym_kv_kernel<64> : asym_kv_kernel<kCB>, dim3((unsigned)(nk + nv)),
+                      dim3(kThreads), 0, s, ak, av, kgx, kgy,
                       (int)nk, vgx);
   return cudaGetLastError();
 }
