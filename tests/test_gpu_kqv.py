@@ -236,3 +236,66 @@ def test_decode_kqv_long_context_splits():
              vals(rng, (1, 2, t, D), BF16), 0)
     out, ref = run_decode(p, 4, t, 1, 128, F32, 400)
     assert_attn(out, ref, KQV_TOL)
+
+
+@pytest.mark.timeout(1800)
+def test_full_size_llama3_8b_kqv():
+    # the Llama-3-8B KQV workload at full size, built and decoded as the benchmark does; two
+    # sampled (batch, KV-head) slabs take host-generated values and are checked against the
+    # oracle byte for byte and on their query heads' outputs
+    cfg = synth.CONFIGS["llama3_8b_kqv"]
+    fd = cfg["fmt"]
+    B, Hq, H, g = cfg["B"], cfg["Hq"], cfg["Hkv"], fd["group_tokens"]
+    G = Hq // H
+    ns, tq, tr = synth.split_tokens(cfg)
+    C = -(-tq // g) * g
+    ck, cv = codebook(fd["k_bits"]), codebook(fd["v_bits"] - 1)
+    S = np.random.default_rng(77).standard_normal((D, D)).astype(np.float32)
+    fmt = kvq.make_format(fd)
+    cache = kvq.Cache(fmt, B, H, C, k_lut=ck, v_lut=cv, sketch=S)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K = synth.device_kv(cfg, "k")
+    V = synth.device_kv(cfg, "v")
+    slabs = [(0, 0), (7, 7)]
+    host = {}
+    for b, h in slabs:
+        hk, hv = synth.kv_slab(cfg, b, h, which="k"), synth.kv_slab(cfg, b, h, which="v")
+        K[b, h] = torch.from_numpy(np.ascontiguousarray(hk)).to(K)
+        V[b, h] = torch.from_numpy(np.ascontiguousarray(hv)).to(V)
+        host[(b, h)] = (hk, hv)
+    kvq.quantize_kv(fmt, cache, K[:, :, ns:ns + tq], V[:, :, ns:ns + tq], 0, tq, status=status)
+    a0 = (tq // g) * g - g   # the step's flush of one group
+    kvq.quantize_kv(fmt, cache, K[:, :, ns + a0:ns + a0 + g].contiguous(), V[:, :, ns + a0:ns + a0 + g].contiguous(),
+                    a0, g, status=status)
+    cache.array("sink_k").copy_(K[:, :, :ns].contiguous().view(-1).view(torch.uint8))
+    cache.array("sink_v").copy_(V[:, :, :ns].contiguous().view(-1).view(torch.uint8))
+    cache.array("res_k").copy_(K[:, :, ns + tq:].contiguous().view(-1).view(torch.uint8))
+    cache.array("res_v").copy_(V[:, :, ns + tq:].contiguous().view(-1).view(torch.uint8))
+    del K, V
+    q = synth.device_queries(cfg)
+    out = kvq.decode_attention(fmt, cache, q, tq, tr, 1.0 / np.sqrt(D), F32, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got_out = out.cpu().numpy()
+    kw, vw = fd["k_bits"] * D // 32, fd["v_bits"] * D // 32
+    for (b, h), (hk, hv) in host.items():
+        Kp, Vp = hk[ns:ns + tq], hv[ns:ns + tq]
+        kc, kn = okqv.stored_encode(Kp, ck)
+        parts = [okqv.stored_encode(Vp[i:i + 512], cv, S) for i in range(0, tq, 512)]
+        vc, vn, sg, rn = (np.concatenate([x[j] for x in parts]) for j in range(4))
+        pk = opack.pack_3bit(kc) if fd["k_bits"] == 3 else opack.pack_row(kc, fd["k_bits"])
+        pv = np.concatenate([opack.pack_3bit(vc) if fd["v_bits"] == 4 else opack.pack_row(vc, fd["v_bits"] - 1),
+                             opack.pack_row(sg.astype(np.int64), 1)], axis=-1)
+        sl = b * H + h
+        got_k = cache.array("k_codes").view(torch.int32).view(B * H, C, kw)[sl, :tq].cpu().numpy().view(np.uint32)
+        got_v = cache.array("v_codes").view(torch.int32).view(B * H, C, vw)[sl, :tq].cpu().numpy().view(np.uint32)
+        np.testing.assert_array_equal(got_k, pk)
+        np.testing.assert_array_equal(got_v, pv)
+        for name, want in (("k_scale", kn), ("v_scale", vn), ("v_zero", rn)):
+            got = cache.array(name).view(torch.float32).view(B * H, C)[sl, :tq].cpu().numpy()
+            np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+        Kh = np.concatenate([hk[:ns], okqv.stored_key(kc, kn, ck), hk[ns + tq:]])
+        Vh = np.concatenate([hv[:ns], okqv.stored_value(vc, vn, sg, rn, cv, S), hv[ns + tq:]])
+        qh = np.stack([synth.query(cfg, b, hq) for hq in range(h * G, (h + 1) * G)]).astype(np.float64)
+        ref = oatt.attention(qh, Kh.astype(np.float64), Vh, 1.0 / np.sqrt(D))
+        assert_attn(got_out[b, h * G:(h + 1) * G], ref, KQV_TOL)
