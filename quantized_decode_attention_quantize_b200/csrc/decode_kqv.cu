@@ -12,9 +12,10 @@
 // rotates its o at the end so that every split's state is in the same basis.
 //
 // Work split and partial-state workspace as the generic kernel (split = a run of token
-// groups of one KV head, or the raw tokens; four warps, token t to warp t mod 4), lane l
-// owning channels (and sketch coordinates) 4 l .. 4 l + 3; four tokens' scores are
-// reduced together, then one softmax update per head.  The workspace also carries a copy
+// groups of one KV head, or the raw tokens; four warps); a warp takes 32-token chunks
+// k = warp, warp + 4, ... staged through its own two-stage cp.async ring, lane l owning
+// channels (and sketch coordinates) 4 l .. 4 l + 3; four tokens' scores are reduced
+// together, then one softmax update per head.  The workspace also carries a copy
 // of S (written by the first CTA), so the combine needs nothing but the workspace.
 #include <cmath>
 
@@ -29,6 +30,11 @@ constexpr int kW = 4;
 constexpr int kB = 4;
 constexpr int kD = 128;
 constexpr int kRec = 2 * kD + 4;     // per warp and head: o[128], u[128], m, l, padding
+// A warp's 32-token chunk staged in shared memory: key rows, value rows (at most 16 words
+// each), then the fp32 key norms, value norms and residual norms.
+constexpr int kChunk = 32;
+constexpr int kStK = 0, kStV = kChunk * 64, kStKn = 2 * kChunk * 64, kStVn = kStKn + 4 * kChunk,
+              kStVr = kStVn + 4 * kChunk, kStBytes = kStVr + 4 * kChunk;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kKappa = 0.009791516697777345f;   // sqrt(pi / 2) / 128
 
@@ -97,6 +103,15 @@ __device__ __forceinline__ void row_centroids(const uint32_t* row, int b, int la
   for (int j = 0; j < 4; ++j) x[j] = __shfl_sync(0xffffffffu, clane, code[j]);
 }
 
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void stage_bytes(uint8_t* dst, const void* src, int bytes, int lane) {
+  for (int o = 16 * lane; o < bytes; o += 512) cp16(dst + o, reinterpret_cast<const uint8_t*>(src) + o);
+}
+
 template <int GM>
 struct KqvState {
   float q[GM][4], o[GM][4], u[GM][4];
@@ -105,7 +120,7 @@ struct KqvState {
 
 template <int GM>
 __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
-  extern __shared__ __align__(16) float smem[];   // [kW][GM][kRec] records, then [GM][D] tile
+  extern __shared__ __align__(16) float smem[];   // [kW][GM][kRec] records, [GM][D] tile, [kW][2] stages
   const Layout& L = a.L;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -158,22 +173,52 @@ __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
     const int64_t g0 = (int64_t)split * a.split_groups;
     const int64_t tb = g0 * L.g;
     const int64_t te = min(a.t_quant, min(ngv, g0 + a.split_groups) * L.g);
-    for (int64_t t0 = tb + warp; t0 < te; t0 += kW * kB) {
+    // the warp's 32-token chunks k = warp, warp + kW, ... through a two-stage cp.async ring
+    // (a chunk's rows past te stay inside the capacity, a multiple of g)
+    uint8_t* ring = reinterpret_cast<uint8_t*>(smem + (size_t)kW * GM * kRec + (size_t)GM * kD) +
+                    (size_t)warp * 2 * kStBytes;
+    const int64_t nchunk = (te - tb + kChunk - 1) / kChunk;
+    auto issue = [&](int64_t k, int bufi) {
+      if (k < nchunk) {
+        uint8_t* stg = ring + bufi * kStBytes;
+        const int64_t t0 = tb + kChunk * k;
+        stage_bytes(stg + kStK, kbase + t0 * kw, kChunk * kw * 4, lane);
+        stage_bytes(stg + kStV, vbase + t0 * vw, kChunk * vw * 4, lane);
+        stage_bytes(stg + kStKn, kn + t0, 4 * kChunk, lane);
+        stage_bytes(stg + kStVn, vn + t0, 4 * kChunk, lane);
+        stage_bytes(stg + kStVr, vr + t0, 4 * kChunk, lane);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    issue(warp, 0);
+    int bufi = 0;
+    for (int64_t k = warp; k < nchunk; k += kW) {
+      issue(k + kW, bufi ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      __syncwarp();
+      const uint8_t* stg = ring + bufi * kStBytes;
+      const uint32_t* krows = reinterpret_cast<const uint32_t*>(stg + kStK);
+      const uint32_t* vrows = reinterpret_cast<const uint32_t*>(stg + kStV);
+      const float* skn = reinterpret_cast<const float*>(stg + kStKn);
+      const float* svn = reinterpret_cast<const float*>(stg + kStVn);
+      const float* svr = reinterpret_cast<const float*>(stg + kStVr);
+      const int nt = (int)min((int64_t)kChunk, te - (tb + kChunk * k));
+    for (int r0 = 0; r0 < nt; r0 += kB) {
       float kf[kB][4], vf[kB][4], nk[kB], nv[kB], rv[kB];
       uint32_t sg[kB];
       bool ok[kB];
 #pragma unroll
       for (int e = 0; e < kB; ++e) {
-        const int64_t t = t0 + (int64_t)e * kW;
-        ok[e] = t < te;
-        const int64_t tt = ok[e] ? t : tb;   // a valid row for the loads of unused slots
-        row_centroids(kbase + tt * kw, kb, lane, klane, kf[e]);
-        const uint32_t* vrow = vbase + tt * vw;
+        const int r = r0 + e;
+        ok[e] = r < nt;
+        const int rr = ok[e] ? r : 0;   // a valid row for the reads of unused slots
+        row_centroids(krows + rr * kw, kb, lane, klane, kf[e]);
+        const uint32_t* vrow = vrows + rr * vw;
         row_centroids(vrow, vb, lane, vlane, vf[e]);
         sg[e] = vrow[vb * kD / 32 + (lane >> 3)] >> (4 * (lane & 7));
-        nk[e] = kn[tt];
-        nv[e] = vn[tt];
-        rv[e] = vr[tt];
+        nk[e] = skn[rr];
+        nv[e] = svn[rr];
+        rv[e] = svr[rr];
       }
       float sc[kB][GM];
 #pragma unroll
@@ -224,6 +269,10 @@ __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
         }
       }
     }
+      __syncwarp();   // the stage's reads are done before it is refilled
+      bufi ^= 1;
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
   } else if (split == a.raw_slot) {
     const int nraw = L.n_sink + a.t_res;
     for (int r = warp; r < nraw; r += kW) {
@@ -343,7 +392,7 @@ size_t a16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 template <int GM>
 cudaError_t launch_g(const KqvDec& a, cudaStream_t s) {
-  const size_t smem = ((size_t)kW * GM * kRec + (size_t)GM * kD) * sizeof(float);
+  const size_t smem = ((size_t)kW * GM * kRec + (size_t)GM * kD) * sizeof(float) + (size_t)kW * 2 * kStBytes;
   cudaError_t e = cudaFuncSetAttribute(decode_kqv_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
