@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
       const float* svr = reinterpret_cast<const float*>(stg + kStVr);
       const int nt = (int)min((int64_t)kChunk, te - (tb + kChunk * k));
     for (int r0 = 0; r0 < nt; r0 += kB) {
-      float kf[kB][4], vf[kB][4], nk[kB], nv[kB], rv[kB];
+      float kf[kB][4], vf[kB][4], nk[kB], nv[kB], rv[kB], sgf[kB][4];
       uint32_t sg[kB];
       bool ok[kB];
 #pragma unroll
@@ -216,6 +216,9 @@ __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
         const uint32_t* vrow = vrows + rr * vw;
         row_centroids(vrow, vb, lane, vlane, vf[e]);
         sg[e] = vrow[vb * kD / 32 + (lane >> 3)] >> (4 * (lane & 7));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)   // sketch bit j as +1.0f (set) or -1.0f
+          sgf[e][j] = __uint_as_float(0xBF800000u ^ ((sg[e] << (31 - j)) & 0x80000000u));
         nk[e] = skn[rr];
         nv[e] = svn[rr];
         rv[e] = svr[rr];
@@ -245,12 +248,14 @@ __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
             sc[e][hh] *= nk[e];
             if (ok[e]) mn = fmaxf(mn, sc[e][hh]);
           }
-          const float corr = exp2f(st.m[hh] - mn);   // 0 when m = -inf
-          st.l[hh] *= corr;
+          if (mn > st.m[hh]) {   // uniform over the warp (reduced scores); a factor 1 changes nothing
+            const float corr = exp2f(st.m[hh] - mn);   // 0 when m = -inf
+            st.l[hh] *= corr;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            st.o[hh][j] *= corr;
-            st.u[hh][j] *= corr;
+            for (int j = 0; j < 4; ++j) {
+              st.o[hh][j] *= corr;
+              st.u[hh][j] *= corr;
+            }
           }
 #pragma unroll
           for (int e = 0; e < kB; ++e) {
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 st.o[hh][j] = fmaf(pv, vf[e][j], st.o[hh][j]);
-                st.u[hh][j] += ((sg[e] >> j) & 1u) ? pr : -pr;
+                st.u[hh][j] = fmaf(pr, sgf[e][j], st.u[hh][j]);   // u + (+-pr), one rounding
               }
             }
           }
