@@ -27,7 +27,7 @@ namespace kvq {
 namespace {
 
 constexpr int kW = 4;
-constexpr int kB = 4;
+constexpr int kB = 2;   // tokens per score reduction
 constexpr int kD = 128;
 constexpr int kRec = 2 * kD + 4;     // per warp and head: o[128], u[128], m, l, padding
 // A warp's 32-token chunk staged in shared memory: key rows, value rows (at most 16 words
@@ -119,7 +119,7 @@ struct KqvState {
 };
 
 template <int GM>
-__global__ void __launch_bounds__(kW * 32) decode_kqv_kernel(KqvDec a) {
+__global__ void __launch_bounds__(kW * 32, GM <= 4 ? 4 : 2) decode_kqv_kernel(KqvDec a) {
   extern __shared__ __align__(16) float smem[];   // [kW][GM][kRec] records, [GM][D] tile, [kW][2] stages
   const Layout& L = a.L;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
