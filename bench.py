@@ -360,9 +360,9 @@ def run_reference(args, world, rank):
     cfg = synth.CONFIGS[args.config]
     if rank != 0:
         return
-    if cfg["fmt"]["k_scheme"] == synth.KQV:
-        print(json.dumps({"impl": "reference", "unavailable": "the oracle's timed path covers the cache "
-                          "schemes of oracle.cache, not KQV"}), flush=True)
+    if cfg["fmt"]["k_scheme"] == synth.KQV or cfg.get("paged"):
+        print(json.dumps({"impl": "reference", "unavailable": "the oracle's timed sample covers the "
+                          "contiguous cache schemes of oracle.cache"}), flush=True)
         return
     per_step = max(0.02, 120.0 / max(1, args.steps + args.warmup))
     smp = oracle_sized(cfg, per_step)
@@ -414,6 +414,136 @@ def workload_config(cfg):
             "parallelism": "replicas (one independent cache per GPU)"}
 
 
+def main_paged(args, cfg, world, rank, dev):
+    """The paged cache with per-sequence lengths: one step = the flush of one group per
+    sequence into its block (kvq_quantize_kv_paged) + kvq_decode_attention_paged over every
+    sequence's own tokens."""
+    import torch
+    from quantized_decode_attention_quantize_b200 import kvq
+    fd = cfg["fmt"]
+    fmt = kvq.make_format(fd)
+    S, Hq, Hkv, D, g = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["D"], fd["group_tokens"]
+    ns = fd["n_sink"]
+    tqs, trs = synth.paged_lengths(cfg)
+    ngs = [-(-t // g) for t in tqs]
+    nblocks = sum(ngs)
+    max_blocks = max(ngs)
+    scale = 1.0 / float(np.sqrt(D))
+    cache = kvq.PagedCache(fmt, Hkv, nblocks, S, max_blocks, device=dev)
+    # every block's group drawn with the workload's recipe, quantized into the pool at once
+    K = synth.device_kv(cfg, "k", T=g, B=nblocks, device=dev, seed_offset=rank)
+    V = synth.device_kv(cfg, "v", T=g, B=nblocks, device=dev, seed_offset=rank)
+    kvq.quantize_kv(fmt, cache.pool, K, V, 0, g)
+    del K, V
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(cfg["seed"] * 1000 + 66 + rank)
+    perm = torch.randperm(nblocks, generator=gen)
+    table = torch.full((S, max_blocks), -1, dtype=torch.int32)
+    o = 0
+    for s_, n in enumerate(ngs):
+        table[s_, :n] = perm[o:o + n].to(torch.int32)
+        o += n
+    cache.block_table.copy_(table)
+    for name in ("sink_k", "sink_v", "res_k", "res_v"):
+        t = cache.array(name)
+        t.copy_(torch.randn(t.numel() // 2, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+                .to(torch.bfloat16).view(torch.uint8))
+    tq_d = torch.tensor(tqs, dtype=torch.int32, device=dev)
+    tr_d = torch.tensor(trs, dtype=torch.int32, device=dev)
+    # the step's flush: the last full group of each sequence, rewritten from new values
+    last = torch.tensor([int(table[s_, tqs[s_] // g - 1]) for s_ in range(S)], dtype=torch.int32, device=dev)
+    newk = synth.device_kv(cfg, "k", T=g, B=S, device=dev, seed_offset=rank + 1)
+    newv = synth.device_kv(cfg, "v", T=g, B=S, device=dev, seed_offset=rank + 1)
+    q = synth.device_queries(cfg, B=S, device=dev)
+    out = torch.empty((S, Hq, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(kvq.decode_paged_workspace_bytes(fmt, S, Hq, Hkv, max(tqs), max(trs)), dtype=torch.uint8,
+                     device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        flush_r.sum()
+
+    def append():
+        kvq.quantize_kv_paged(fmt, cache, newk, newv, last, g, status=status, stream=stream)
+
+    def decode():
+        kvq.decode_attention_paged(fmt, cache, tq_d, tr_d, max(tqs), max(trs), q, scale, kvq.F32, out=out,
+                                   workspace=ws, status=status, stream=stream)
+
+    for i in range(args.warmup):
+        flush_l2(i)
+        append()
+        decode()
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(dev.index))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.15)
+    for i in range(args.steps):
+        flush_l2(i)
+        evs[i][0].record(stream)
+        append()
+        evs[i][1].record(stream)
+        decode()
+        evs[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms_step = statistics.mean([e[0].elapsed_time(e[2]) for e in evs])
+    ms_app = statistics.mean([e[0].elapsed_time(e[1]) for e in evs])
+    ms_dec = statistics.mean([e[1].elapsed_time(e[2]) for e in evs])
+    ms_step, ms_app, ms_dec = max_over_ranks([ms_step, ms_app, ms_dec], dev)
+    assert int(status.item()) == 0 and bool(torch.isfinite(out).all())
+    # algorithmic bytes: per sequence its packed rows (64 + 32 + 4 B per token and KV head),
+    # the key scale / zero-point of its groups (512 B each), its raw tokens (2 D bf16 K and
+    # V), q and the fp32 out; the append reads the bf16 group and writes its codes
+    dec_bytes = sum(Hkv * (t * 100 + n * 512 + (ns + r) * 2 * D * 2) for t, n, r in zip(tqs, ngs, trs))
+    dec_bytes += S * Hq * D * (2 + 4)
+    app_bytes = S * Hkv * (g * D * 2 * 2 + g * 100 + 512)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        pass
+    peak = peaks.get("hbm_gbs", 6650.0)
+    achieved = dec_bytes / (ms_dec * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": world * (dec_bytes + app_bytes) / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": PATH_DTYPE["decode_k4v2_kernel"], "data": "synthetic (device-drawn, recipe of synth/)",
+        "config": {"workload": f"{cfg['name']}: paged pool of {nblocks} blocks (one 128-token group of "
+                               f"{Hkv} KV heads each, shuffled), {S} sequences of {tqs} packed + 1 sink + "
+                               f"{trs} residual tokens, Hq={Hq}, D={D}; K asym4 per-channel g128 + V asym2 "
+                               "per-token",
+                   "step": "flush of one group per sequence into its block + paged decode attention",
+                   "l2": "flushed between steps outside the timed events",
+                   "parallelism": "replicas (one independent cache per GPU)"},
+        "ms_breakdown": {"append": ms_app, "decode": ms_dec},
+        "roofline": {"kernel": "decode_paged_kernel + combine_paged_kernel (kvq_decode_attention_paged)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "algorithmic_bytes": dec_bytes,
+                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks else "fallback"},
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks, "cpu_baseline": None,
+    }
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     import torch
@@ -428,6 +558,9 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     cfg = synth.CONFIGS[args.config]
+    if cfg.get("paged"):
+        main_paged(args, cfg, world, rank, dev)
+        return
     fd = cfg["fmt"]
     fmt = kvq.make_format(fd)
     B, Hq, Hkv, D, g = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["D"], fd["group_tokens"]

@@ -63,6 +63,12 @@ CONFIGS = {
                           T=32768, seed=7, q_dtype=BF16,
                           fmt=_fmt(src_dtype=BF16, n_sink=1, residual_cap=128, k_scheme=KQV, k_bits=4,
                                    k_axis=TOKEN, v_scheme=KQV, v_bits=4, v_axis=TOKEN)),
+    # the Llama-3-8B format as a paged cache with a length mix: 8 sequences of 32k, 28k, ...,
+    # 4k tokens (sink 1, residual windows of 128, 112, ..., 16 tokens), their groups in
+    # blocks of a shared pool in shuffled order
+    "llama3_8b_paged": dict(name="llama3_8b_paged", recipe="llama3_8b", B=8, Hq=32, Hkv=8, D=128,
+                            T=32768, seed=7, q_dtype=BF16, paged=True,
+                            fmt=_fmt(src_dtype=BF16, n_sink=1, residual_cap=128)),
     "kvquant_nuq3": dict(name="kvquant_nuq3", B=1, Hq=32, Hkv=32, D=128, T=131072, seed=7,
                          q_dtype=F16,
                          fmt=_fmt(src_dtype=F16, k_scheme=NUQ, k_bits=3, k_outliers=2,
@@ -255,3 +261,16 @@ def device_queries(cfg, B=None, Hq=None, device="cuda"):
     Hq = cfg["Hq"] if Hq is None else Hq
     q = torch.tensor(queries(cfg, B, Hq), device=device)
     return q.to({F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}[cfg["q_dtype"]])
+
+
+def paged_lengths(cfg):
+    """(t_quant, t_residual) per sequence of a paged workload: T (8 - s) / 8 tokens for
+    sequence s, sink n_sink, residual window 128 - 16 s."""
+    ns = cfg["fmt"]["n_sink"]
+    tqs, trs = [], []
+    for s in range(cfg["B"]):
+        T = cfg["T"] * (cfg["B"] - s) // cfg["B"]
+        tr = 128 - 16 * s
+        tqs.append(T - ns - tr)
+        trs.append(tr)
+    return tqs, trs
