@@ -1576,8 +1576,17 @@ __device__ __forceinline__ void lean_key_operand(const float* ks, const float* k
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {   // channel pairs (p, p + 4) of word 2 cb + u
-      const float f = (p & 1) ? sc16 : sc;
-      const float y0 = a[8 * u + p] * f, y1 = a[8 * u + p + 4] * f;
+      // odd p: the A element is a whole byte, c_p-1 + 16 c_p, weighted a_p sc / 16; even p:
+      // the A element c_p alone, weighted a_p sc - a_p+1 sc / 16, so that each channel
+      // still enters with its own weight
+      float y0, y1;
+      if (p & 1) {
+        y0 = a[8 * u + p] * sc16;
+        y1 = a[8 * u + p + 4] * sc16;
+      } else {
+        y0 = fmaf(-a[8 * u + p + 1], sc16, a[8 * u + p] * sc);
+        y1 = fmaf(-a[8 * u + p + 5], sc16, a[8 * u + p + 4] * sc);
+      }
       split_half2(y0, y1, &hw[p], &lw[p]);
     }
     // register quad w of reader lane R sits at uint4 slot 32 w + (R ^ 4 (w / 2)): a read
@@ -1618,10 +1627,10 @@ __device__ __forceinline__ void lean_scores(float (&S)[4][4], const uint4* kc4, 
       const uint32_t x0 = w == 0 ? lo.x : w == 1 ? lo.y : w == 2 ? lo.z : lo.w;
       const uint32_t x1 = w == 0 ? hi.x : w == 1 ? hi.y : w == 2 ? hi.z : hi.w;
       const uint32_t p0 = odd_bytes_down(x0), p1 = odd_bytes_down(x1);
-      mma16816_n(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x00F000F0u, ko.b[4 * w],
+      // low nibble alone, then the whole byte (low + 16 high; the byte of p as it stands)
+      mma16816_n(S[mt], x0 & 0x000F000Fu, x1 & 0x000F000Fu, x0 & 0x00FF00FFu, x1 & 0x00FF00FFu, ko.b[4 * w],
                  ko.b[4 * w + 1]);
-      mma16816_n(S[mt], p0 & 0x000F000Fu, p1 & 0x000F000Fu, p0 & 0x00F000F0u, p1 & 0x00F000F0u, ko.b[4 * w + 2],
-                 ko.b[4 * w + 3]);
+      mma16816_n(S[mt], p0 & 0x000F000Fu, p1 & 0x000F000Fu, p0, p1, ko.b[4 * w + 2], ko.b[4 * w + 3]);
     }
   }
 }
