@@ -120,6 +120,19 @@ def fused_kv(cfg):
     return is_k4v2(cfg) and (not f.get("k_rotate", 0) or (f["head_dim"] == 128 and f["group_tokens"] <= 128))
 
 
+def step_launches(cfg, n_app):
+    """Kernels one timed step launches: the split kernel appends a single group of a
+    K4/V2 cache itself (unrotated keys, 16-bit sources, G <= 4), else the append is one
+    launch (two for separate key and value kernels, one more per MixKVQ salience window)."""
+    f = cfg["fmt"]
+    g = f["group_tokens"]
+    if (is_k4v2(cfg) and not f.get("k_rotate", 0) and f["src_dtype"] in (synth.F16, synth.BF16)
+            and cfg["Hq"] // cfg["Hkv"] <= 4 and n_app <= g):
+        return 2
+    mixed = f["k_scheme"] == synth.MIXED
+    return LAUNCHES_PER_STEP + (0 if fused_kv(cfg) else 1) + (n_app // g if mixed else 0)
+
+
 def cache_read_bytes(cache, cfg, tq, tr):
     """Algorithmic decode bytes of any format: every cache array the decode reads (codes,
     metadata, slot order, outliers: sized for the packed capacity, i.e. t_quant rounded up
@@ -844,8 +857,7 @@ def main():
                 "mode": "pipelined: step i+1's host-to-device copies on a copy stream overlap step i",
                 "serial": {"value": world * step_bytes / (ms_e2e_serial * 1e-3) / 1e9,
                            "ms_per_step": ms_e2e_serial}},
-        "gpu_launches": (LAUNCHES_PER_STEP + (0 if fused_kv(cfg) else 1) + (n_app // g if mixed else 0))
-        * args.steps,
+        "gpu_launches": step_launches(cfg, n_app) * args.steps,
         "clocks": clocks,
     }
     if path not in ("decode_mma_kernel", "decode_k4v2_kernel"):

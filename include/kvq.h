@@ -342,9 +342,13 @@ kvq_status kvq_decode_attention(const kvq_format* fmt, const kvq_cache* cache,
  * the same as kvq_quantize_kv(fmt, cache, k_src, v_src, stride_b, stride_h, stride_t, t0,
  * n) followed by kvq_decode_attention(fmt, cache, q, ...) on the same stream, with the
  * same results bit for bit.  Every argument of both is checked before anything is
- * launched; n = 0 appends nothing.  When the format's append is one kernel and the
- * tensor-core split kernel decodes it, the split kernel starts while the append still
- * runs and waits for it only where it reaches the appended groups' rows. */
+ * launched; n = 0 appends nothing.  For one group (t0 a multiple of 128, n <= 128) of a
+ * K4-per-channel / V2-per-token cache with unrotated keys and 16-bit sources decoded by
+ * the G <= 4 tensor-core split kernel, that kernel quantizes the group itself before its
+ * decode (warp-sized units, each announced by a flag in the workspace; a warp waits for
+ * its head's flags before it copies that group).  Otherwise, when the format's append is
+ * one kernel and the tensor-core split kernel decodes it, the split kernel starts while
+ * the append still runs and waits for it only where it reaches the appended rows. */
 kvq_status kvq_append_decode_attention(const kvq_format* fmt, const kvq_cache* cache,
                                        const void* k_src, const void* v_src, int64_t stride_b,
                                        int64_t stride_h, int64_t stride_t, int64_t t0, int64_t n,

@@ -6,6 +6,9 @@
 
 #include "kvq_internal.cuh"
 
+#include <atomic>
+#include <chrono>
+
 using namespace kvq;
 
 namespace {
@@ -558,6 +561,18 @@ kvq_status kvq_merge_states(int32_t n_parts, int64_t rows, int32_t head_dim, con
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+// A value per call of the fused append that the flags of an earlier call (or a fresh
+// workspace) do not hold: a per-process counter from a clock-seeded start, never 0.
+static uint32_t next_epoch() {
+  static std::atomic<uint32_t> counter{(uint32_t)std::chrono::steady_clock::now().time_since_epoch().count() |
+                                       1u};
+  uint32_t e;
+  do {
+    e = counter.fetch_add(1, std::memory_order_relaxed);
+  } while (e == 0);
+  return e;
+}
+
 kvq_status kvq_append_decode_attention(const kvq_format* f, const kvq_cache* c, const void* k_src,
                                        const void* v_src, int64_t sb, int64_t sh, int64_t st, int64_t t0,
                                        int64_t n, const void* q, int32_t q_dtype, int32_t Hq, int64_t t_quant,
@@ -579,7 +594,19 @@ kvq_status kvq_append_decode_attention(const kvq_format* f, const kvq_cache* c, 
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (n > 0) {
-    if (asym_fast_ok(L, KVQ_KEYS) && asym_fast_ok(L, KVQ_VALUES)) {
+    if (fused_append_ok(L, Hq, p, t0, n)) {
+      // the split kernel quantizes the group itself before its decode (no append launch)
+      p.fuse = 1;
+      p.dep_lo = t0;
+      p.dep_hi = t0 + n;
+      p.app_n = (int)n;
+      p.app_k = k_src;
+      p.app_v = v_src;
+      p.app_sb = sb;
+      p.app_sh = sh;
+      p.app_st = st;
+      p.epoch = next_epoch();
+    } else if (asym_fast_ok(L, KVQ_KEYS) && asym_fast_ok(L, KVQ_VALUES)) {
       // one append kernel directly before the split kernel: the split kernel reads the
       // rows the append does not touch without waiting for it
       if (launch_quantize_asym_kv(L, k_src, v_src, sb, sh, st, t0, n, d_status, cs) != cudaSuccess)

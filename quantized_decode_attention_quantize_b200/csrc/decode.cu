@@ -489,7 +489,9 @@ DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int 
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p) {
   if (L.side[0].scheme == KVQ_KQV) return kqv_workspace_bytes(L, Hq, p);
   const size_t rows = (size_t)L.B * Hq * p.S;
-  return align16(rows * 4) * 2 + align16(rows * L.D * 4);
+  // the fast path keeps 32 flags per KV head after the partial states (fused append)
+  const size_t flags = p.fast ? align16((size_t)L.B * L.Hkv * 32 * 4) : 0;
+  return align16(rows * 4) * 2 + align16(rows * L.D * 4) + flags;
 }
 
 cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q, int q_dtype,
@@ -501,8 +503,12 @@ cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const vo
   float* ws_m = reinterpret_cast<float*>(ws);
   float* ws_l = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align16(rows * 4));
   float* ws_o = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4));
-  if (p.fast)
-    return launch_decode_mma(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
+  if (p.fast) {
+    DecodePlan pf = p;
+    pf.flags = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 2 * align16(rows * 4) +
+                                           align16(rows * L.D * 4));
+    return launch_decode_mma(L, pf, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
+  }
   if (cc_path_ok(L, Hq))
     return launch_decode_cc(L, p, q, q_dtype, Hq, t_quant, t_res, scale, ws_m, ws_l, ws_o, d_status, s);
   DecArgs a;

@@ -119,6 +119,18 @@ struct MmaArgs {
   // it first copies a group meeting those rows, and every thread waits before it exits.
   int defer;
   int64_t dep_lo, dep_hi;
+  // fuse = 1 (contiguous cache, K4 per channel / V2 per token, 16-bit sources): this
+  // kernel writes packed rows [dep_lo, dep_lo + app_n) of one group of every head itself,
+  // before its decode, in warp-sized units (fused_append); each unit then sets its flag to
+  // `epoch`, and a warp waits for a head's 32 flags before it first copies that group.
+  int fuse;
+  int app_n;
+  const void* app_k;
+  const void* app_v;
+  int64_t app_sb, app_sh, app_st;
+  uint32_t* flags;   // [heads][32]
+  uint32_t epoch;
+  int64_t heads;
 };
 
 // ---- partition of the items over the warps (shared with the combine kernel) ------------
@@ -1351,6 +1363,171 @@ __device__ __forceinline__ void issue_half(const MmaArgs& a, uint8_t* buf, uint6
   }
 }
 
+// ---- the fused append: one group of every head, in warp-sized units -------------------
+// Unit j of a head (kFusedUnits of them, flags at head * 32 + j): j < 16 takes key channels
+// 8 j .. 8 j + 7 of the group's rows (lane l: rows l, l + 32, l + 64, l + 96; the channel
+// statistics meet over the warp), j >= 16 value rows 16 (j - 16) .. + 15 (two lanes per row,
+// 64 channels each).  Same rules, arithmetic and
+// layouts as the append kernels: asym_params for the metadata, pack8 for the codes, the
+// pair layout for the 2-bit value rows ([KVQ] "Approach"; [K4V2]).
+constexpr int kFusedUnits = 32;
+__device__ void fused_key_unit(const MmaArgs& a, int64_t head, int j) {
+  const int lane = threadIdx.x & 31;
+  const int64_t b = head / a.Hkv, h = head % a.Hkv;
+  const int c0 = 8 * j;
+  float x[4][8], mn[8], mx[8];
+  float fin = 0.0f;   // x * 0 is 0 for finite x and NaN otherwise
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    mn[c] = INFINITY;
+    mx[c] = -INFINITY;
+  }
+  const int64_t base = b * a.app_sb + h * a.app_sh + c0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = lane + 32 * k;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[k][c] = 0.0f;
+    if (r < a.app_n) {
+      load8(a.app_k, base + r * a.app_st, a.src_dtype, x[k]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        fin = fmaf(x[k][c], 0.0f, fin);
+        mn[c] = fminf(mn[c], x[k][c]);
+        mx[c] = fmaxf(mx[c], x[k][c]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      mn[c] = fminf(mn[c], __shfl_xor_sync(0xffffffffu, mn[c], o));
+      mx[c] = fmaxf(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], o));
+    }
+  // lane c < 8 forms channel c's scale / zero-point and stores them; all lanes get all eight
+  float m0 = mn[0], m1 = mx[0];
+#pragma unroll
+  for (int c = 1; c < 8; ++c)
+    if (lane == c) {
+      m0 = mn[c];
+      m1 = mx[c];
+    }
+  __half s, z;
+  const bool good = asym_params(m0, m1, 4, &s, &z);
+  if (lane < 8) {
+    const int64_t mi = (head * a.ng + a.dep_lo / 128) * 128 + c0 + lane;
+    const_cast<__half*>(a.k_scale)[mi] = s;
+    const_cast<__half*>(a.k_zero)[mi] = z;
+  }
+  const float sf = __half2float(s), zf = __half2float(z), rf = __frcp_rn(sf);
+  float s8[8], z8[8], r8[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    s8[c] = __shfl_sync(0xffffffffu, sf, c);
+    z8[c] = __shfl_sync(0xffffffffu, zf, c);
+    r8[c] = __shfl_sync(0xffffffffu, rf, c);
+  }
+  uint8_t* codes = const_cast<uint8_t*>(a.k_codes) + head * a.k_slab_bytes + a.dep_lo * 64 + c0 / 2;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = lane + 32 * k;
+    if (r < a.app_n) *reinterpret_cast<uint32_t*>(codes + r * 64) = pack8(x[k], s8, r8, z8, 4).x;
+  }
+  if (__any_sync(0xffffffffu, !(fin == 0.0f)) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+  if (__any_sync(0xffffffffu, lane < 8 && !good) && lane == 0) flag(a.status, KVQ_DEV_RANGE);
+}
+
+__device__ void fused_value_unit(const MmaArgs& a, int64_t head, int j) {
+  const int lane = threadIdx.x & 31;
+  const int64_t b = head / a.Hkv, h = head % a.Hkv;
+  const int r = 8 * j + (lane >> 2), part = lane & 3, c0 = 32 * part;   // row in the group
+  const bool ok = r < a.app_n;
+  float x[4][8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[k][c] = 0.0f;
+    if (ok) load8(a.app_v, b * a.app_sb + h * a.app_sh + r * a.app_st + c0 + 8 * k, a.src_dtype, x[k]);
+  }
+  float mn = INFINITY, mx = -INFINITY, fin = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      fin = fmaf(x[k][c], 0.0f, fin);
+      mn = fminf(mn, x[k][c]);
+      mx = fmaxf(mx, x[k][c]);
+    }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  __half sh, zh;
+  const bool good = asym_params(mn, mx, 2, &sh, &zh);
+  const int64_t t = a.dep_lo + r;
+  if (ok && part == 0) {
+    const_cast<__half*>(a.v_scale)[head * a.C + t] = sh;
+    const_cast<__half*>(a.v_zero)[head * a.C + t] = zh;
+  }
+  const float sv = __half2float(sh), zv = __half2float(zh), rv = __frcp_rn(sv);
+  float s8[8], z8[8], r8[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    s8[c] = sv;
+    z8[c] = zv;
+    r8[c] = rv;
+  }
+  const bool even = (t & 1) == 0;
+  const bool lone = even && r + 1 >= a.app_n;
+  uint32_t* dst = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.v_codes) + head * a.v_slab_bytes) +
+                  (t / 2) * 16 + part * 4;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t hw = pack8(x[k], s8, r8, z8, 2).x & 0xffffu;
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, hw, 4);
+    if (ok && even) dst[k] = hw | ((lone ? 0u : other) << 16);
+  }
+  if (__any_sync(0xffffffffu, ok && !(fin == 0.0f)) && lane == 0) flag(a.status, KVQ_DEV_NONFINITE);
+  if (__any_sync(0xffffffffu, ok && !good) && lane == 0) flag(a.status, KVQ_DEV_RANGE);
+}
+
+// Warp gw's units (gw, gw + W, ...), each announced by its flag once its rows are visible
+// to the other SMs' bulk copies.
+__device__ void fused_append(const MmaArgs& a, int64_t gw) {
+  const int64_t units = a.heads * kFusedUnits;
+#pragma unroll 1
+  for (int64_t u = gw; u < units; u += a.W) {
+    const int64_t head = u / kFusedUnits;
+    const int j = (int)(u % kFusedUnits);
+    if (j < 16) fused_key_unit(a, head, j);
+    else fused_value_unit(a, head, j - 16);
+    __threadfence();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) atomicExch(a.flags + head * 32 + j, a.epoch);
+  }
+}
+
+// Waits (bounded) until the kFusedUnits units of `head` are done; a wait that runs out sets
+// KVQ_DEV_TIMEOUT and goes on.
+constexpr int kFlagRounds = 1 << 22;   // polls, each followed by a sleep of about 0.25 us
+__device__ __noinline__ void fused_wait(const uint32_t* flags, uint32_t epoch, int32_t* status, int64_t head) {
+  const uint32_t* f = flags + head * 32 + (threadIdx.x & 31);
+#pragma unroll 1
+  for (int it = 0; it < kFlagRounds; ++it) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (__all_sync(0xffffffffu, v == epoch || (threadIdx.x & 31) >= kFusedUnits)) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      return;
+    }
+    __nanosleep(256);
+  }
+  if ((threadIdx.x & 31) == 0) flag(status, KVQ_DEV_TIMEOUT);
+}
+
 __device__ __forceinline__ void cp_async16_lean(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
@@ -1756,7 +1933,7 @@ struct LeanWarp {
 // Queries are rows qhead * G + hh of q.  slab_of(p, &slab, &ph) names the slab holding
 // half p and the half's index in it (the contiguous cache: the head's slab and p; a
 // paged pool: the block's slab and p & 1).  Returns false when a wait ran out.
-template <bool ROT, typename SlabOf>
+template <bool ROT, typename SlabOf, bool FUSE = false>
 __device__ __forceinline__ bool lean_run(const MmaArgs& a, LeanState& st, LeanWarp& w, int64_t qhead,
                                          int64_t rawhead, int nraw, int64_t tq, int ra, int rb, int ha, int hb,
                                          const SlabOf& slab_of, bool& qbad) {
@@ -1782,11 +1959,14 @@ __device__ __forceinline__ bool lean_run(const MmaArgs& a, LeanState& st, LeanWa
   lean_load_queries<ROT>(a, qhead, ROT, w.qs, qbad);
   // two halves in flight; a half's stage is released once its value words are in
   // registers, and its value product runs during the next half's key product
+  if constexpr (FUSE) w.dep_done = false;   // fused append: its flags are per head
   auto issue = [&](int q) {
-    if (a.defer && !w.dep_done) {   // the group of half q (codes and metadata) meets the append
+    if ((FUSE || a.defer) && !w.dep_done) {   // the group of half q (codes and metadata) meets the append
       const int64_t g0 = 128 * (int64_t)(q >> 1);
       if (g0 < a.dep_hi && g0 + 128 > a.dep_lo) {
-        griddep_wait();
+        // fused: the head's units are done (the contiguous cache: slab = head = qhead)
+        if constexpr (FUSE) fused_wait(a.flags, a.epoch, a.status, qhead);
+        else griddep_wait();
         w.dep_done = true;
       }
     }
@@ -1903,7 +2083,7 @@ __device__ __forceinline__ void lean_merge(const MmaArgs& a, uint8_t* smem, int 
   }
 }
 
-template <bool ROT>
+template <bool ROT, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   // launched with launch_pdl: without a deferred wait the cache and q are complete from
@@ -1914,6 +2094,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
   const int64_t gw = (int64_t)blockIdx.x * kCW + warp;
   const int64_t i0 = item_start(gw, a.I, a.W), i1 = item_start(gw + 1, a.I, a.W);
   const int U = a.U;
+  if constexpr (FUSE) fused_append(a, gw);
   LeanWarp w = lean_warp(smem, warp, kCW);
   int* last_head = reinterpret_cast<int*>(smem + (size_t)kCW * kLeanWarpBytes + kCW * kBuffers * 8);
   const int nraw = a.n_sink + a.t_res;
@@ -1946,7 +2127,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_k4v2_kernel(MmaArgs a) {
       *slab = head;
       *ph = p;
     };
-    timed_out = !lean_run<ROT>(a, st, w, head, head, nraw, a.t_quant, ra, rb, ha, hb, slab_of, qbad);
+    timed_out = !lean_run<ROT, decltype(slab_of), FUSE>(a, st, w, head, head, nraw, a.t_quant, ra, rb, ha, hb,
+                                                        slab_of, qbad);
   }
   if (timed_out) lean_drain(a, w);
   __syncwarp();
@@ -2147,6 +2329,15 @@ bool mma_path_ok(const Layout& L, int Hq) {
          V.axis == KVQ_AXIS_TOKEN && L.rope == 0 && G >= 1 && G <= 8;
 }
 
+bool fused_append_ok(const Layout& L, int Hq, const DecodePlan& p, int64_t t0, int64_t n) {
+  const Side& K = L.side[0];
+  const Side& V = L.side[1];
+  return p.fast && mma_path_ok(L, Hq) && Hq / L.Hkv <= 4 && K.scheme == KVQ_ASYM && K.bits == 4 &&
+         K.axis == KVQ_AXIS_CHANNEL && !L.k_rotate && V.scheme == KVQ_ASYM && V.bits == 2 &&
+         (L.src_dtype == KVQ_F16 || L.src_dtype == KVQ_BF16) && n >= 1 && n <= 128 && t0 % 128 == 0 &&
+         t0 + n <= L.C;
+}
+
 // Partition of the fast path (t_quant >= 1): CTAs, slots per query head.  At least one
 // warp per head, so that no warp range is longer than a head's row of items.
 void plan_mma(const Layout& L, int64_t t_quant, int t_res, int max_ctas, DecodePlan& p) {
@@ -2218,10 +2409,22 @@ cudaError_t launch_decode_mma(const Layout& L, const DecodePlan& p, const void* 
   a.defer = p.defer;
   a.dep_lo = p.dep_lo;
   a.dep_hi = p.dep_hi;
+  a.fuse = p.fuse;
+  a.app_n = p.app_n;
+  a.app_k = p.app_k;
+  a.app_v = p.app_v;
+  a.app_sb = p.app_sb;
+  a.app_sh = p.app_sh;
+  a.app_st = p.app_st;
+  a.flags = p.flags;
+  a.epoch = p.epoch;
+  a.heads = (int64_t)L.B * L.Hkv;
   const bool mix = L.side[0].scheme == KVQ_MIXED;
   if (!mix && a.G <= 4) {
     const size_t smem = lean_smem();
-    auto kern = a.k_rotate ? decode_k4v2_kernel<true> : decode_k4v2_kernel<false>;
+    // the fused append takes no rotated keys (fused_append_ok)
+    auto kern = a.fuse ? decode_k4v2_kernel<false, true>
+              : (a.k_rotate ? decode_k4v2_kernel<true, false> : decode_k4v2_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(p.grid_ctas), dim3(kThreads), smem, s, a);

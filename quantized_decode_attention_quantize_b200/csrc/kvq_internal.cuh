@@ -89,10 +89,23 @@ struct DecodePlan {
   // packed rows [dep_lo, dep_hi) directly and may read the other rows before it completes
   int defer = 0;
   int64_t dep_lo = 0, dep_hi = 0;
+  // set by the append-and-decode entry point when the split kernel does the append itself
+  // (fused_append_ok): one group at dep_lo of app_n rows from these sources, flags in the
+  // workspace, a fresh epoch per call
+  int fuse = 0;
+  int app_n = 0;
+  const void* app_k = nullptr;
+  const void* app_v = nullptr;
+  int64_t app_sb = 0, app_sh = 0, app_st = 0;
+  uint32_t* flags = nullptr;
+  uint32_t epoch = 0;
 };
 DecodePlan plan_decode(const Layout& L, int Hq, int64_t t_quant, int t_res, int num_splits);
 size_t workspace_bytes(const Layout& L, int Hq, const DecodePlan& p);
 bool fast_path_ok(const Layout& L, int Hq);
+// The split kernel can take the append of n rows at t0 itself (one group; K4 per channel,
+// V2 per token, not rotated, 16-bit sources, the G <= 4 tensor-core kernel).
+bool fused_append_ok(const Layout& L, int Hq, const DecodePlan& p, int64_t t0, int64_t n);
 cudaError_t launch_decode_partial(const Layout& L, const DecodePlan& p, const void* q,
                                   int q_dtype, int Hq, int64_t t_quant, int t_res, float scale,
                                   void* ws, int32_t* d_status, cudaStream_t s);
@@ -230,6 +243,68 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// ---- append-time code packing (the append kernels and the split kernel's fused append) ----
+// 8 consecutive elements (16 bytes for 16-bit sources, two 16-byte loads for fp32)
+__device__ __forceinline__ void load8(const void* base, int64_t i, int dtype, float* out) {
+  if (dtype == KVQ_F32) {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i + 4);
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (dtype == KVQ_F16) {
+        out[2 * j] = half_bits_to_float((uint16_t)(w[j] & 0xffffu));
+        out[2 * j + 1] = half_bits_to_float((uint16_t)(w[j] >> 16));
+      } else {
+        out[2 * j] = __uint_as_float(w[j] << 16);
+        out[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    }
+  }
+}
+
+// 8 codes of `bits` bits packed LSB-first (bits = 2: 16 bits, 4: 32 bits; 8: two words).
+// Each code is rint_even(fl32(fl32(x - z) / s)) clipped to [0, 2^bits - 1], found as
+// asym_code_r does: from q = fl32(fl32(x - z) * rs), rs = fl32(1 / s), which is within
+// 2^-13 of the exact quotient for in-range codes, so that q and the IEEE quotient round to
+// the same integer unless q lies within 2^-12 of a half-integer.  Such elements (rare) take
+// the quotient instead, behind one branch per eight codes.
+__device__ __forceinline__ uint2 pack8(const float* x, const float* s, const float* rs, const float* z,
+                                       int bits) {
+  const float maxc = (float)((1 << bits) - 1);
+  float q[8];
+  bool near = false;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    q[j] = __fmul_rn(__fsub_rn(x[j], z[j]), rs[j]);
+    near |= fabsf(q[j] - rintf(q[j])) > 0.5f - 0x1p-12f;
+  }
+  if (near) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (fabsf(q[j] - rintf(q[j])) > 0.5f - 0x1p-12f) q[j] = __fdiv_rn(__fsub_rn(x[j], z[j]), s[j]);
+  }
+  uint32_t c[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) c[j] = (uint32_t)fminf(fmaxf(rintf(q[j]), 0.0f), maxc);
+  uint32_t lo = 0, hi = 0;
+  if (bits == 8) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      lo |= c[j] << (8 * j);
+      hi |= c[4 + j] << (8 * j);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) lo |= c[j] << (bits * j);
+  }
+  return make_uint2(lo, hi);
 }
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -268,9 +268,11 @@ def clone_cache(p, luts=(None, None)):
 
 
 @pytest.mark.parametrize("kw,G,t0,n", [
-    (dict(), 4, 7 * 128, 128),                      # tensor-core split kernel, deferred wait
-    (dict(), 4, 7 * 128, 37),                       # a partial group
-    (dict(), 2, 3 * 128, 256),                      # two groups inside the cache
+    (dict(), 4, 7 * 128, 128),                      # the split kernel appends the group itself
+    (dict(), 4, 7 * 128, 37),                       # a partial group, appended the same way
+    (dict(), 2, 3 * 128, 128),                      # a group inside the decoded rows (fused)
+    (dict(), 1, 0, 5),                              # the first rows of the first group (fused)
+    (dict(), 2, 3 * 128, 256),                      # two groups: append launch, deferred wait
     (dict(k_rotate=1), 4, 7 * 128, 128),            # rotated keys: a plain append launch
     (dict(), 8, 7 * 128, 128),                      # G = 8: the general tensor-core kernel
     (dict(), 4, 7 * 128, 0),                        # nothing appended

@@ -150,6 +150,22 @@ def test_paged_long_sequence_spans_chunks():
         assert_attn(out[s], ref[s], tolerance(F32))
 
 
+@pytest.mark.parametrize("S,H,tq_max,seed", [(300, 8, 200, 250), (20, 2, 10, 260)])
+def test_paged_many_short_sequences(S, H, tq_max, seed):
+    # many short rows next to one of the longest: most chunks past a sequence's end are
+    # empty, and (20 sequences of a few tokens) most sequences take a single chunk
+    rng = np.random.default_rng(seed)
+    fd = fmt(src_dtype=BF16, n_sink=1, residual_cap=16)
+    t_quant = [int(x) for x in rng.integers(0, tq_max + 1, S)]
+    t_res = [int(x) for x in rng.integers(0, 17, S)]
+    t_quant[0], t_res[0] = tq_max, 16
+    gpu, ora, table = build(fd, H, t_quant, t_res, num_blocks=sum(-(-t // g) for t in t_quant) + 2, seed=seed)
+    out, ref, st = run(gpu, ora, fd, t_quant, t_res, 4, BF16, F32, seed + 1)
+    assert st == 0
+    for s in range(S):
+        assert_attn(out[s], ref[s], tolerance(F32))
+
+
 def test_paged_bounds_are_flagged_not_followed():
     # a block id outside the pool and a length past its bound: KVQ_DEV_BOUNDS, no fault;
     # the other sequences' outputs are unaffected

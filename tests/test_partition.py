@@ -96,6 +96,12 @@ MIXED_SHAPES = [
 ]
 
 
+def flag_bytes(B, Hkv):
+    """The tensor-core path's workspace ends with 32 flags (4 bytes each) per KV head, 16-byte
+    aligned, for the append that its split kernel can take over."""
+    return (B * Hkv * 32 * 4 + 15) // 16 * 16
+
+
 @pytest.mark.parametrize("B,Hkv,G,tq,ns,tr,splits,src", MIXED_SHAPES)
 def test_mixed_tiers_plan_like_k4v2(B, Hkv, G, tq, ns, tr, splits, src):
     # every host planning helper sees the tiers: the slot count, the workspace of the
@@ -108,7 +114,7 @@ def test_mixed_tiers_plan_like_k4v2(B, Hkv, G, tq, ns, tr, splits, src):
     assert kvq.decode_partial_slots(f, B, G * Hkv, Hkv, tq, tr, splits) == want
     rows = B * G * Hkv * want
     assert kvq.decode_workspace_bytes(f, B, G * Hkv, Hkv, tq, tr, splits) == \
-        2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4
+        2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4 + flag_bytes(B, Hkv)
 
 
 @pytest.mark.parametrize("B,Hkv,G,tq,ns,tr,splits,src", SHAPES)
@@ -121,4 +127,4 @@ def test_planned_slots_match_the_partition_model(B, Hkv, G, tq, ns, tr, splits, 
     assert kvq.decode_partial_slots(f, B, G * Hkv, Hkv, tq, tr, splits) == want
     rows = B * G * Hkv * want
     assert kvq.decode_workspace_bytes(f, B, G * Hkv, Hkv, tq, tr, splits) == \
-        2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4
+        2 * ((rows * 4 + 15) // 16 * 16) + rows * 128 * 4 + flag_bytes(B, Hkv)
