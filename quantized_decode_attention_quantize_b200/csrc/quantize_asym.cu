@@ -426,8 +426,10 @@ __global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
 
 // Keys and values of one append in one launch: blocks [0, nk) are key blocks
 // (group, channel block, head), the rest value blocks (token block, head).
+// Four CTAs per SM (64 registers): a full-cache quantize streams at about 1.7 TB/s against
+// 1.15 TB/s with two CTAs per SM (92 registers).
 template <int CB>
-__global__ void __launch_bounds__(kThreads) asym_kv_kernel(AArgs ak, AArgs av, int kgx, int kgy, int nk,
+__global__ void __launch_bounds__(kThreads, 4) asym_kv_kernel(AArgs ak, AArgs av, int kgx, int kgy, int nk,
                                                            int vgx) {
   griddep_wait();   // launched with launch_pdl: earlier work on the stream is complete
   griddep_launch_dependents();
