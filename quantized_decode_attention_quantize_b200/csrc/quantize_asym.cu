@@ -416,11 +416,12 @@ __global__ void __launch_bounds__(kThreads) asym_kv_rot_kernel(AArgs ak, AArgs a
 }
 
 template <int CB>
-__global__ void __launch_bounds__(kThreads) asym_keys_kernel(AArgs a) {
+// Four CTAs per SM, as asym_kv_kernel.
+__global__ void __launch_bounds__(kThreads, 4) asym_keys_kernel(AArgs a) {
   asym_keys_block<CB>(a, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
-__global__ void __launch_bounds__(kThreads) asym_values_kernel(AArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) asym_values_kernel(AArgs a) {
   asym_values_block(a, blockIdx.x, blockIdx.y);
 }
 
